@@ -1,0 +1,126 @@
+"""Whole-path compositions of the oracle: CSA prefill, CSA decode step, HCA decode step.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+The order of the stages is the operator graph of "DeepSeek V4 结构速览",
+section "CSA（c4a 路线）": compressor -> (index-key compressor + quantiser) ->
+lightning indexer -> top-k -> concatenation with the raw sliding window ->
+shared-latent MQA with sink.  HCA (section "HCA（c128a 路线）") drops the
+indexer and attends to every visible entry.
+
+Every argument is a numpy array holding the values the caller feeds the
+library (bf16 inputs given as float64 on the bf16 grid).  ``idx_dtype`` picks
+the index-path number format: "f32" (no quantisation), "fp8" (E4M3, one fp32
+scale per row of d_I) or "nvfp4" (E2M1, one UE4M3 scale per 16 elements).
+"""
+
+import numpy as np
+
+from . import codecs
+from . import csa
+
+
+def round_out(x, dtype):
+    """Round float64 results to the library's storage type ("bf16" or "f32")."""
+    if dtype == "bf16":
+        return codecs.round_to_bf16(x)
+    if dtype == "f32":
+        return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+    raise ValueError(dtype)
+
+
+def quantize_rows(x, idx_dtype):
+    """Quantise rows (last axis) of the index path and return the dequantised float64 values.
+
+    The quantiser consumes float32 values (the compressor's output precision),
+    so the float64 input is first rounded to float32.
+    Returns (dequantised values, raw pieces tuple).
+    """
+    x32 = np.asarray(x, dtype=np.float64).astype(np.float32)
+    if idx_dtype == "f32":
+        return x32.astype(np.float64), (x32,)
+    if idx_dtype == "fp8":
+        codes, scales = codecs.quant_fp8_rows(x32)
+        return codecs.dequant_fp8_rows(codes, scales), (codes, scales)
+    if idx_dtype == "nvfp4":
+        packed, sc = codecs.quant_nvfp4(x32)
+        return codecs.dequant_nvfp4(packed, sc), (packed, sc)
+    raise ValueError(idx_dtype)
+
+
+def csa_prefill(main, index, q, q_I, w, sink, *, m, d_rope, theta, eps, k, n_w, scale,
+                kv_dtype, idx_dtype, score_dtype, query_rows=None):
+    """CSA prefill of one sequence: every token t = 0..n-1 is a query.
+
+    main / index: dicts with C_a, Z_a, B_a, C_b, Z_b, B_b ([n][c], [m][c]).
+    q [n][H][d]; q_I [n][H_I][d_I] (unquantised); w [n][H_I]; sink [H].
+    The raw window rows are the main branch's C_a (the uncompressed latent).
+    ``query_rows`` restricts the queries evaluated (all entries are still
+    compressed, as every query may select any visible entry).
+    Returns a dict of every intermediate.
+    """
+    n = main["C_a"].shape[0]
+    E = n // m
+    kv = csa.compress_range(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
+                            main["B_b"], m, True, 0, E, d_rope, theta, eps)
+    kv_st = round_out(kv, kv_dtype)
+    kI = csa.compress_range(index["C_a"], index["Z_a"], index["B_a"], index["C_b"], index["Z_b"],
+                            index["B_b"], m, True, 0, E, d_rope, theta, eps)
+    kI_deq, _ = quantize_rows(kI, idx_dtype)
+    rows = np.arange(n) if query_rows is None else np.asarray(query_rows, dtype=np.int64)
+    qI_deq, _ = quantize_rows(np.asarray(q_I)[rows], idx_dtype)
+    scores = csa.index_scores(qI_deq, np.asarray(w)[rows], kI_deq, rows, m, score_dtype)
+    idx, cnt = csa.topk(scores, rows, m, k)
+    o, lse = csa.sparse_attn(np.asarray(q)[rows], kv_st, idx, cnt, main["C_a"], rows, sink, n_w, scale)
+    return dict(kv=kv, kv_stored=kv_st, kI=kI, kI_deq=kI_deq, qI_deq=qI_deq, scores=scores,
+                idx=idx, cnt=cnt, out=round_out(o, kv_dtype), out_f64=o, lse=lse, rows=rows)
+
+
+def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k, n_w, scale,
+                   kv_dtype, idx_dtype):
+    """One CSA decode step of one sequence with L tokens of context.
+
+    The new token is t = L - 1; it completes block E - 1 (E = L / m), so the
+    step compresses that entry (main and index branch) and then scores all E
+    entries, selects k of them and attends over them plus the window.  The
+    earlier entries of the caches are the compressor's outputs for their own
+    blocks (the state the decode step reads), computed here the same way.
+    q [H][d]; q_I [H_I][d_I]; w [H_I].
+    """
+    E = L // m
+    t = L - 1
+    kI = csa.compress_range(index["C_a"], index["Z_a"], index["B_a"], index["C_b"], index["Z_b"],
+                            index["B_b"], m, True, 0, E, d_rope, theta, eps)
+    kI_deq, _ = quantize_rows(kI, idx_dtype)
+    qI_deq, _ = quantize_rows(np.asarray(q_I)[None], idx_dtype)
+    scores = csa.index_scores(qI_deq, np.asarray(w)[None], kI_deq, np.array([t]), m, "bf16")
+    idx, cnt = csa.topk(scores, np.array([t]), m, k)
+    sel = idx[0, :cnt[0]].astype(np.int64)
+    kv_sel = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
+                                  main["B_b"], m, True, sel, d_rope, theta, eps)
+    kv_sel_st = round_out(kv_sel, kv_dtype)
+    rows = np.concatenate([kv_sel_st, np.asarray(main["C_a"])[csa.window_rows(t, n_w)]], axis=0)
+    o, lse = csa.attend(np.asarray(q), rows, sink, scale)
+    new_entry = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
+                                     main["B_b"], m, True, [E - 1], d_rope, theta, eps)[0]
+    return dict(kI=kI, kI_deq=kI_deq, qI_deq=qI_deq, scores=scores[0], idx=idx[0], cnt=int(cnt[0]),
+                kv_sel=kv_sel, new_entry=new_entry, new_kI=kI[E - 1],
+                out=round_out(o, kv_dtype), out_f64=o, lse=lse)
+
+
+def hca_decode_seq(main, q, sink, *, L, m, d_rope, theta, eps, n_w, scale, kv_dtype,
+                   entries_needed=None):
+    """One HCA decode step of one sequence: compress the completed block, attend densely.
+
+    main holds C_a, Z_a, B_a (no previous-block branch in c128a).  The new
+    token t = L - 1 completes entry E - 1; every entry 0..E-1 is visible.
+    """
+    E = L // m
+    t = L - 1
+    kv = csa.compress_range(main["C_a"], main["Z_a"], main["B_a"], None, None, None, m, False,
+                            0, E, d_rope, theta, eps)
+    kv_st = round_out(kv, kv_dtype)
+    rows = np.concatenate([kv_st, np.asarray(main["C_a"])[csa.window_rows(t, n_w)]], axis=0)
+    o, lse = csa.attend(np.asarray(q), rows, sink, scale)
+    return dict(kv=kv, kv_stored=kv_st, new_entry=kv[E - 1], out=round_out(o, kv_dtype),
+                out_f64=o, lse=lse)
