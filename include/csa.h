@@ -1,0 +1,334 @@
+/*
+ * csa.h -- C ABI of the Compressed Sparse Attention (CSA) / Heavily Compressed
+ * Attention (HCA) hot path on NVIDIA B200 (sm_100a).
+ *
+ * The method (DeepSeek-V4 attention, as described on the pages "DeepSeek V4
+ * 结构速览", "DeepSeek Technical Reports", "DeepSeek-V4技术报告解读" and
+ * "DeepSeek-V4 技术解读") has four stages, each one entry point here:
+ *
+ *   csa_compress      KV compressor: per-channel softmax pooling of 2m raw rows
+ *                     at stride m (c4a) or m rows (c128a), RMSNorm, partial
+ *                     RoPE, optional FP8 / NVFP4 quantisation of index keys.
+ *   csa_index_scores  lightning indexer I[t,s] = sum_j w[t,j] ReLU(q[t,j].k[s]).
+ *   csa_topk          causal top-k of the scores of each query.
+ *   csa_sparse_attn   shared-latent MQA (K = V) with a per-head sink over the
+ *                     selected entries plus a raw sliding window; dense over all
+ *                     visible entries when no index list is given (HCA).
+ *
+ * plus csa_quantize (the index-path quantiser on its own) and the fused
+ * drivers csa_decode and csa_prefill that chain the stages on one stream.
+ *
+ * Conventions for every call:
+ *  - Pointers named as tensors are DEVICE pointers, allocated and owned by the
+ *    caller; the library allocates nothing and keeps no state between calls.
+ *  - Every call is asynchronous on the caller's stream; results are ready when
+ *    the stream reaches them.  No call synchronises the device.
+ *  - Layouts are row-major, batch outermost, last dimension contiguous.  Base
+ *    pointers must be 16-byte aligned.
+ *  - Indices are int32; -1 pads unused top-k slots.
+ *  - Argument errors are detected on the host before any launch and returned
+ *    as CSA_ERR_INVALID_ARG (nothing is launched); a launch failure reported
+ *    by the CUDA runtime is CSA_ERR_CUDA.  No call aborts the process.
+ *
+ * Storage types (csa_dtype):
+ *  - CSA_F32, CSA_BF16: plain element arrays.
+ *  - CSA_FP8_E4M3: one byte per element (OCP E4M3FN), plus one float32 scale
+ *    per row: value = decode(code) * scale, scale = amax(row) / 448.
+ *  - CSA_NVFP4: two E2M1 codes per byte (element 2j in bits 0-3, 2j+1 in bits
+ *    4-7), plus one UE4M3 scale byte per 16 consecutive elements:
+ *    value = decode(code) * decode(scale), scale = e4m3(amax(block) / 6).
+ */
+#ifndef CSA_H_
+#define CSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1,   /* bad shape, pointer, alignment or type; nothing launched */
+  CSA_ERR_UNSUPPORTED = 2,   /* a valid combination this build has no kernel for */
+  CSA_ERR_CUDA = 3,          /* the CUDA runtime reported a launch error */
+  CSA_ERR_TIMEOUT = 4        /* a bounded device-side wait gave up */
+} csa_status;
+
+typedef enum {
+  CSA_F32 = 0,
+  CSA_BF16 = 1,
+  CSA_FP8_E4M3 = 2,
+  CSA_NVFP4 = 3
+} csa_dtype;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* csa_status_string(csa_status s);
+
+/* Library version as major * 10000 + minor * 100 + patch. */
+int csa_version(void);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 1: KV compressor                                                    */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Source: "DeepSeek V4 结构速览", section "C4A Compressor" (per-channel softmax
+ * over the stacked logits of the previous and the current block plus a
+ * positional bias, weighted sum of the stacked contents, RMSNorm, RoPE; block
+ * 0 pads its previous half with zero content and -inf logits); section
+ * "核心设计" item 1 (c4a: 8 rows at stride 4; c128a: 128 rows at stride 128);
+ * "DeepSeek-V4技术报告解读", section "Compressed Sparse Attention (CSA)"
+ * (compression formula with bias B).
+ *
+ * Entry i of sequence s, channel ch (R = 2m rows with overlap, m without):
+ *   rows r <  m (overlap only): logit Z_b[s][m(i-1)+r][ch] + B_b[r][ch],
+ *                               content C_b[s][m(i-1)+r][ch]  (i = 0: -inf, 0)
+ *   rows r >= m (or all rows without overlap):
+ *                               logit Z_a[s][mi+r'][ch] + B_a[r'][ch],
+ *                               content C_a[s][mi+r'][ch]     (r' = r - m or r)
+ *   x[ch]  = sum_r softmax_r(logit)[r] * content[r]            (float32)
+ *   x      = x / sqrt(mean(x^2) + eps)                          (if apply_norm)
+ *   pairs (x[c-d_rope+2j], x[c-d_rope+2j+1]) rotated by p * theta^(-2j/d_rope),
+ *   p = m * i, the angle formed in float64.
+ */
+typedef struct {
+  int m;              /* compression rate (>= 1) */
+  int overlap;        /* 1: previous block from the b-branch joins; 0: current block only */
+  int c;              /* channels per entry; multiple of 8 (of 16 for NVFP4 output) */
+  int d_rope;         /* rotary dims at the end of each entry; even, <= c; 0 = none */
+  double rope_theta;  /* RoPE base (10000) */
+  float eps;          /* RMSNorm epsilon (1e-6) */
+  int apply_norm;     /* 1: RMSNorm with unit gain; 0: skip (identity checks) */
+  int in_dtype;       /* CSA_F32 or CSA_BF16: type of C_* and Z_* */
+  int out_dtype;      /* CSA_F32, CSA_BF16, CSA_FP8_E4M3 or CSA_NVFP4 */
+} csa_compress_params;
+
+/*
+ * Compresses entries [entry_begin, entry_begin + entry_count) of each of the b
+ * sequences.
+ *   C_a, Z_a   [b][n][c] (in_dtype)     current-block branch
+ *   C_b, Z_b   [b][n][c] (in_dtype)     previous-block branch; NULL when !overlap
+ *   B_a, B_b   [m][c] float32           positional biases; B_b NULL when !overlap
+ *   n          tokens per sequence; requires m * (entry_begin + entry_count) <= n
+ *   out        [b][out_entries_per_seq][row] with row = c elements (F32/BF16),
+ *              c bytes (FP8) or c/2 bytes (NVFP4); entry i of sequence s is
+ *              written at row s * out_entries_per_seq + i (caches are updated
+ *              in place, other rows untouched)
+ *   out_scales FP8: float32 [b][out_entries_per_seq]; NVFP4: uint8
+ *              [b][out_entries_per_seq][c/16]; NULL for F32/BF16
+ */
+csa_status csa_compress(const csa_compress_params* p,
+                        const void* C_a, const void* Z_a, const float* B_a,
+                        const void* C_b, const void* Z_b, const float* B_b,
+                        int b, int n, int entry_begin, int entry_count, int out_entries_per_seq,
+                        void* out, void* out_scales, cudaStream_t stream);
+
+/*
+ * Index-path quantiser on its own ("DeepSeek V4 结构速览", section "Lightning
+ * Indexer": the QK path of the indexer runs in FP4 end to end).  Quantises
+ * `rows` rows of `d` elements of x (CSA_F32 or CSA_BF16) to out_dtype
+ * CSA_FP8_E4M3 (codes [rows][d], scales float32 [rows]) or CSA_NVFP4 (codes
+ * [rows][d/2], scales uint8 [rows][d/16]).  d must be a multiple of 16.  The
+ * divisions are IEEE float32 and the conversions round to nearest even with
+ * saturation, so results are bit-identical to any exact implementation.
+ */
+csa_status csa_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
+                        void* codes, void* scales, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 2: lightning indexer                                                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Source: "DeepSeek Technical Reports", section DSA (I[t,s] = sum_j w[t,j] *
+ * ReLU(q_I[t,j] . k_I[s])); "DeepSeek V4 结构速览", section "Lightning
+ * Indexer" (FP4 QK path, ReLU, per-head weighted sum, scores kept in BF16,
+ * causal range).  With quantised operands, q and k are their dequantised
+ * values.  Entry s is visible to query position t iff m(s+1)-1 <= t; the
+ * scores of invisible entries are -inf.
+ */
+typedef struct {
+  int H_I;          /* indexer heads */
+  int d_I;          /* index-key dim; multiple of 16 */
+  int m;            /* compression rate (visibility rule) */
+  int qk_dtype;     /* CSA_F32, CSA_FP8_E4M3 or CSA_NVFP4 (q_I and k_I alike) */
+  int score_dtype;  /* CSA_F32 or CSA_BF16 */
+} csa_index_params;
+
+/*
+ *   q_I       [b][T][H_I][row]  codes (row as in csa_compress for qk_dtype)
+ *   q_scales  FP8: float32 [b][T][H_I]; NVFP4: uint8 [b][T][H_I][d_I/16]; F32: NULL
+ *   w         [b][T][H_I] float32 head weights
+ *   k_I       [b][E_cap][row] codes;  k_scales like q_scales per entry
+ *   q_pos     [b][T] int32 position t of each query
+ *   scores    [b][T][E] (score_dtype), E <= E_cap entries scored per query
+ */
+csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const void* q_scales,
+                            const float* w, const void* k_I, const void* k_scales,
+                            const int32_t* q_pos, int b, int T, int E_cap, int E,
+                            void* scores, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 3: causal top-k                                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Source: "DeepSeek Technical Reports", section DSA (Top-k(I[t,:]));
+ * "DeepSeek V4 结构速览", sections "核心设计" item 2 and "Lightning
+ * Indexer" (k = 512 / 1024 among causally visible entries).
+ * For each query: the k largest scores among entries s < E(t) =
+ * min(E, floor((t+1)/m)); equal scores go to the lower s; if E(t) <= k all
+ * visible entries are kept.  idx [b][T][k] lists the kept entries in
+ * ascending order, padded with -1; count [b][T] holds how many.  The result
+ * is exact (a radix select on the stored score bits).
+ *   scores  [b][T][E] (CSA_F32 or CSA_BF16)
+ *   ws      unused by this build (may be NULL, ws_bytes 0)
+ */
+csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b, int T,
+                    int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                    cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Stage 4: shared-latent MQA over selected entries + window, with sink      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Source: "DeepSeek Technical Reports", section DSA (u_t = Attn(h_t,
+ * {c_s | I[t,s] in Top-k})) and section CSA (window of n_w = 128 uncompressed
+ * tokens); "DeepSeek V4 结构速览", sections "CSA（c4a 路线）" (the window
+ * rows are concatenated with the selected entries; one 512-dim latent is
+ * both K and V for 64 heads) and "HCA（c128a 路线）" (dense over all entries,
+ * attention sink); "DeepSeek-V4 技术解读", section 2.1 (shared KV MQA).
+ *
+ * For query t of sequence s and head h, over the rows
+ *   S = { kv_comp[s][idx[j]] : j < count }  (or all j < E(t) when idx == NULL)
+ *     + { kv_win[s][u] : max(0, t-n_w+1) <= u <= t }
+ *   l_r = scale * q[h] . row_r
+ *   out[h] = sum_r e^{l_r} row_r / (e^{sink[h]} + sum_r e^{l_r})
+ *   lse[h] = log(e^{sink[h]} + sum_r e^{l_r})
+ */
+typedef struct {
+  int H;          /* query heads */
+  int d;          /* head dim = latent dim */
+  int n_w;        /* window length (raw tokens, inclusive of t) */
+  float scale;    /* logit scale */
+  int m;          /* compression rate (dense mode: E(t) = floor((t+1)/m)) */
+  int k;          /* idx row length (ignored when idx == NULL) */
+  int dtype;      /* CSA_F32 or CSA_BF16: q, kv_comp, kv_win and out */
+} csa_attn_params;
+
+/*
+ *   q        [b][T][H][d]
+ *   kv_comp  [b][E_cap][d] compressed entries
+ *   idx      [b][T][k] int32 selected entries (ascending, -1 padded) or NULL
+ *   count    [b][T] int32 valid entries of each idx row (NULL iff idx NULL)
+ *   kv_win   [b][n][d] raw rows for the window (n tokens per sequence)
+ *   q_pos    [b][T] int32 positions; requires q_pos < n
+ *   sink     [H] float32
+ *   out      [b][T][H][d];  lse [b][T][H] float32 or NULL
+ *   ws       device scratch of at least csa_sparse_attn_workspace_size() bytes
+ */
+csa_status csa_sparse_attn(const csa_attn_params* p, const void* q, const void* kv_comp, int E_cap,
+                           const int32_t* idx, const int32_t* count, const void* kv_win, int n,
+                           const int32_t* q_pos, const float* sink, int b, int T, void* out,
+                           float* lse, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+size_t csa_sparse_attn_workspace_size(const csa_attn_params* p, int b, int T, int E_cap);
+
+/* ------------------------------------------------------------------------ */
+/* Fused drivers                                                             */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One decode step for b sequences of L tokens each (the operator graph of
+ * "DeepSeek V4 结构速览", section "CSA（c4a 路线）"; HCA per section
+ * "HCA（c128a 路线）").  The new token is t = L-1; it completes entry E-1
+ * (E = L/m, L a multiple of m), which the step compresses from the raw rows
+ * of its block (and of the previous block for c4a) into the caches in
+ * place.  CSA then quantises q_I, scores all E entries, selects k and attends
+ * over them plus the window; HCA attends over all E entries plus the window.
+ */
+typedef struct {
+  int b, L, m, c, H;       /* sequences, context, compression rate, latent dim, heads */
+  int c_I, H_I;            /* index-key dim and indexer heads (CSA only) */
+  int d_rope, d_rope_I;    /* rotary dims of latent entries and of index keys */
+  double rope_theta;
+  float eps;
+  int k, n_w;              /* top-k (CSA) and window */
+  float scale;             /* attention logit scale */
+  int kv_dtype;            /* CSA_BF16 or CSA_F32 */
+  int idx_dtype;           /* CSA_FP8_E4M3, CSA_NVFP4 or CSA_F32 (CSA only) */
+  int hca;                 /* 1: HCA (no indexer, no previous block, dense attention) */
+  int E_cap;               /* entries each cache row-block holds (>= L/m) */
+} csa_decode_params;
+
+typedef struct {
+  const void *C_a, *Z_a, *C_b, *Z_b;   /* [b][L][c]; C_b/Z_b NULL for HCA */
+  const float *B_a, *B_b;              /* [m][c] */
+  const void *CI_a, *ZI_a, *CI_b, *ZI_b; /* [b][L][c_I] (CSA) */
+  const float *BI_a, *BI_b;            /* [m][c_I] (CSA) */
+  void* kv_cache;                      /* [b][E_cap][c] kv_dtype; entry E-1 written */
+  void* kI_cache;                      /* [b][E_cap][row] idx_dtype codes; entry E-1 written */
+  void* kI_scales;                     /* FP8: float32 [b][E_cap]; NVFP4: uint8 [b][E_cap][c_I/16] */
+  const void* kv_win;                  /* [b][L][c] raw window rows */
+  const void* q;                       /* [b][H][c] */
+  const void* q_I;                     /* [b][H_I][c_I] unquantised (kv_dtype) */
+  const float* w;                      /* [b][H_I] */
+  const float* sink;                   /* [H] */
+  void* out;                           /* [b][H][c] kv_dtype */
+  float* lse;                          /* [b][H] or NULL */
+  int32_t* idx_out;                    /* [b][k] selected entries or NULL (CSA) */
+  int32_t* count_out;                  /* [b] or NULL (CSA) */
+} csa_decode_tensors;
+
+csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, void* ws,
+                      size_t ws_bytes, cudaStream_t stream);
+size_t csa_decode_workspace_size(const csa_decode_params* p);
+
+/*
+ * CSA prefill of b sequences of n tokens; every token t = 0..n-1 is a query.
+ * Compresses all E = n/m entries (latent and index branch) into the caches,
+ * quantises q_I, scores every (t, s) pair, selects k per query and attends.
+ */
+typedef struct {
+  int b, n, m, c, H, c_I, H_I, d_rope, d_rope_I;
+  double rope_theta;
+  float eps;
+  int k, n_w;
+  float scale;
+  int kv_dtype;            /* CSA_BF16 or CSA_F32 */
+  int idx_dtype;           /* CSA_FP8_E4M3, CSA_NVFP4 or CSA_F32 */
+  int score_dtype;         /* CSA_BF16 or CSA_F32 */
+} csa_prefill_params;
+
+typedef struct {
+  const void *C_a, *Z_a, *C_b, *Z_b;   /* [b][n][c] */
+  const float *B_a, *B_b;              /* [m][c] */
+  const void *CI_a, *ZI_a, *CI_b, *ZI_b; /* [b][n][c_I] */
+  const float *BI_a, *BI_b;            /* [m][c_I] */
+  const void* kv_win;                  /* [b][n][c] */
+  const void* q;                       /* [b][n][H][c] */
+  const void* q_I;                     /* [b][n][H_I][c_I] unquantised (kv_dtype) */
+  const float* w;                      /* [b][n][H_I] */
+  const float* sink;                   /* [H] */
+  void* kv_cache;                      /* out: [b][n/m][c] */
+  void* kI_cache;                      /* out: [b][n/m][row] */
+  void* kI_scales;                     /* out: as in csa_decode_tensors with E_cap = n/m */
+  void* out;                           /* [b][n][H][c] */
+  float* lse;                          /* [b][n][H] or NULL */
+  int32_t* idx_out;                    /* [b][n][k] or NULL */
+  int32_t* count_out;                  /* [b][n] or NULL */
+} csa_prefill_tensors;
+
+csa_status csa_prefill(const csa_prefill_params* p, const csa_prefill_tensors* x, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
+size_t csa_prefill_workspace_size(const csa_prefill_params* p);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif  /* CSA_H_ */

@@ -1,0 +1,340 @@
+// Host side of the C ABI declared in include/csa.h: argument checks, kernel
+// selection, launches, and the fused decode / prefill drivers.
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+
+using namespace csa;
+
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t dtype_row_bytes(int dt, int d) {
+  switch (dt) {
+    case CSA_F32: return (size_t)d * 4;
+    case CSA_BF16: return (size_t)d * 2;
+    case CSA_FP8_E4M3: return (size_t)d;
+    case CSA_NVFP4: return (size_t)d / 2;
+  }
+  return 0;
+}
+
+inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Bump allocator over a caller-provided workspace.
+// With a NULL base it only measures (every take() returns NULL).
+struct Carve {
+  char* base; size_t cap; size_t used = 0; bool ok = true;
+  Carve(void* b, size_t c) : base(static_cast<char*>(b)), cap(c) {}
+  void* take(size_t bytes) {
+    size_t off = align256(used);
+    used = off + bytes;
+    if (!base) return nullptr;
+    if (used > cap) { ok = false; return nullptr; }
+    return base + off;
+  }
+};
+
+}  // namespace
+
+extern "C" {
+
+const char* csa_status_string(csa_status s) {
+  switch (s) {
+    case CSA_OK: return "CSA_OK";
+    case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG: invalid argument";
+    case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED: no kernel for this combination";
+    case CSA_ERR_CUDA: return "CSA_ERR_CUDA: CUDA launch error";
+    case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT: bounded device wait gave up";
+  }
+  return "CSA_ERR_UNKNOWN";
+}
+
+int csa_version(void) { return 100; }
+
+csa_status csa_compress(const csa_compress_params* p, const void* C_a, const void* Z_a,
+                        const float* B_a, const void* C_b, const void* Z_b, const float* B_b,
+                        int b, int n, int entry_begin, int entry_count, int out_entries_per_seq,
+                        void* out, void* out_scales, cudaStream_t stream) {
+  if (!p) return CSA_ERR_INVALID_ARG;
+  if (p->m < 1 || p->c < 8 || p->c % 8 || p->d_rope < 0 || p->d_rope % 2 || p->d_rope > p->c)
+    return CSA_ERR_INVALID_ARG;
+  if (p->in_dtype != CSA_F32 && p->in_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (p->out_dtype < CSA_F32 || p->out_dtype > CSA_NVFP4) return CSA_ERR_INVALID_ARG;
+  if (p->out_dtype == CSA_NVFP4 && p->c % 16) return CSA_ERR_INVALID_ARG;
+  if (p->in_dtype == CSA_F32 && p->c % 4) return CSA_ERR_INVALID_ARG;
+  if (b < 0 || n < 0 || entry_begin < 0 || entry_count < 0) return CSA_ERR_INVALID_ARG;
+  if ((long long)p->m * (entry_begin + entry_count) > n) return CSA_ERR_INVALID_ARG;
+  if (entry_begin + entry_count > out_entries_per_seq) return CSA_ERR_INVALID_ARG;
+  if (b == 0 || entry_count == 0) return CSA_OK;
+  if (!C_a || !Z_a || !B_a || !out) return CSA_ERR_INVALID_ARG;
+  if (p->overlap && (!C_b || !Z_b || !B_b)) return CSA_ERR_INVALID_ARG;
+  if ((p->out_dtype == CSA_FP8_E4M3 || p->out_dtype == CSA_NVFP4) && !out_scales)
+    return CSA_ERR_INVALID_ARG;
+  if (!aligned16(C_a) || !aligned16(Z_a) || (p->overlap && (!aligned16(C_b) || !aligned16(Z_b))))
+    return CSA_ERR_INVALID_ARG;
+  CompressArgs a{};
+  a.C_a = C_a; a.Z_a = Z_a; a.B_a = B_a; a.C_b = C_b; a.Z_b = Z_b; a.B_b = B_b;
+  a.n = n; a.m = p->m; a.overlap = p->overlap ? 1 : 0; a.c = p->c; a.d_rope = p->d_rope;
+  a.apply_norm = p->apply_norm; a.out_dtype = p->out_dtype; a.entry_begin = entry_begin;
+  a.out_E = out_entries_per_seq; a.theta = p->rope_theta; a.eps = p->eps;
+  a.out = out; a.out_scales = out_scales;
+  return launch_compress(a, p->in_dtype, b, entry_count, stream);
+}
+
+csa_status csa_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d, void* codes,
+                        void* scales, cudaStream_t stream) {
+  if (in_dtype != CSA_F32 && in_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (out_dtype != CSA_FP8_E4M3 && out_dtype != CSA_NVFP4) return CSA_ERR_INVALID_ARG;
+  if (rows < 0 || d <= 0 || d % 16) return CSA_ERR_INVALID_ARG;
+  if (rows == 0) return CSA_OK;
+  if (!x || !codes || !scales || !aligned16(codes)) return CSA_ERR_INVALID_ARG;
+  return launch_quantize(in_dtype, out_dtype, x, rows, d, codes, scales, stream);
+}
+
+csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const void* q_scales,
+                            const float* w, const void* k_I, const void* k_scales,
+                            const int32_t* q_pos, int b, int T, int E_cap, int E, void* scores,
+                            cudaStream_t stream) {
+  if (!p) return CSA_ERR_INVALID_ARG;
+  if (p->H_I < 1 || p->d_I < 16 || p->d_I % 16 || p->m < 1) return CSA_ERR_INVALID_ARG;
+  if (p->qk_dtype < CSA_F32 || p->qk_dtype > CSA_NVFP4 || p->qk_dtype == CSA_BF16)
+    return CSA_ERR_INVALID_ARG;
+  if (p->score_dtype != CSA_F32 && p->score_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (b < 0 || T < 0 || E < 0 || E > E_cap) return CSA_ERR_INVALID_ARG;
+  if (b == 0 || T == 0 || E == 0) return CSA_OK;
+  if (!q_I || !w || !k_I || !q_pos || !scores) return CSA_ERR_INVALID_ARG;
+  if (p->qk_dtype != CSA_F32 && (!q_scales || !k_scales)) return CSA_ERR_INVALID_ARG;
+  IndexArgs a{};
+  a.q = q_I; a.q_scales = q_scales; a.w = w; a.k = k_I; a.k_scales = k_scales; a.q_pos = q_pos;
+  a.T = T; a.H = p->H_I; a.d = p->d_I; a.m = p->m; a.qk_dtype = p->qk_dtype;
+  a.score_dtype = p->score_dtype; a.E_cap = E_cap; a.E = E; a.scores = scores;
+  csa_status st = launch_index_scores_tc(a, b, stream);
+  if (st != CSA_ERR_UNSUPPORTED) return st;
+  return launch_index_scores_simt(a, b, stream);
+}
+
+csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b, int T,
+                    int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                    cudaStream_t stream) {
+  (void)ws; (void)ws_bytes;
+  if (score_dtype != CSA_F32 && score_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (m < 1 || b < 0 || T < 0 || E < 0 || k < 1) return CSA_ERR_INVALID_ARG;
+  if (b == 0 || T == 0) return CSA_OK;
+  if (!scores || !q_pos || !idx || !count) return CSA_ERR_INVALID_ARG;
+  return launch_topk(scores, score_dtype, q_pos, m, b * T, E, k, idx, count, stream);
+}
+
+size_t csa_sparse_attn_workspace_size(const csa_attn_params* p, int b, int T, int E_cap) {
+  if (!p) return 0;
+  return attn_tc_workspace_bytes(p->H, p->d, p->k, p->n_w, b, T, E_cap, p->dtype);
+}
+
+csa_status csa_sparse_attn(const csa_attn_params* p, const void* q, const void* kv_comp, int E_cap,
+                           const int32_t* idx, const int32_t* count, const void* kv_win, int n,
+                           const int32_t* q_pos, const float* sink, int b, int T, void* out,
+                           float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (!p) return CSA_ERR_INVALID_ARG;
+  if (p->H < 1 || p->d < 8 || p->d % 8 || p->n_w < 0 || p->m < 1) return CSA_ERR_INVALID_ARG;
+  if (p->dtype != CSA_F32 && p->dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (b < 0 || T < 0 || E_cap < 0 || n < 1) return CSA_ERR_INVALID_ARG;
+  if (idx && (p->k < 1 || !count)) return CSA_ERR_INVALID_ARG;
+  if (b == 0 || T == 0) return CSA_OK;
+  if (!q || !kv_win || !q_pos || !sink || !out) return CSA_ERR_INVALID_ARG;
+  if (E_cap > 0 && !kv_comp) return CSA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(kv_win) || (kv_comp && !aligned16(kv_comp)) || !aligned16(out))
+    return CSA_ERR_INVALID_ARG;
+  AttnArgs a{};
+  a.q = q; a.kv = kv_comp; a.idx = idx; a.count = count; a.win = kv_win; a.q_pos = q_pos;
+  a.sink = sink; a.T = T; a.H = p->H; a.d = p->d; a.n_w = p->n_w; a.m = p->m; a.k = p->k;
+  a.E_cap = E_cap; a.n = n; a.scale = p->scale; a.out = out; a.lse = lse;
+  csa_status st = launch_attn_tc(a, b, p->dtype, ws, ws_bytes, stream);
+  if (st != CSA_ERR_UNSUPPORTED) return st;
+  return launch_attn_simt(a, b, p->dtype, stream);
+}
+
+// ---------------------------------------------------------------------------
+// decode
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct DecodeWs {
+  void* qI_codes; void* qI_scales; void* scores; int32_t* idx; int32_t* count; int32_t* qpos;
+  void* attn_ws; size_t attn_ws_bytes;
+};
+
+size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs* o) {
+  Carve cv(ws, cap);
+  DecodeWs d{};
+  const int b = p->b;
+  d.qpos = static_cast<int32_t*>(cv.take((size_t)b * 4));
+  if (!p->hca) {
+    const int E = p->L / p->m;
+    if (p->idx_dtype != CSA_F32) {
+      d.qI_codes = cv.take((size_t)b * p->H_I * dtype_row_bytes(p->idx_dtype, p->c_I));
+      d.qI_scales = cv.take(p->idx_dtype == CSA_FP8_E4M3 ? (size_t)b * p->H_I * 4
+                                                          : (size_t)b * p->H_I * (p->c_I / 16));
+    }
+    d.scores = cv.take((size_t)b * E * 2);
+    d.idx = static_cast<int32_t*>(cv.take((size_t)b * p->k * 4));
+    d.count = static_cast<int32_t*>(cv.take((size_t)b * 4));
+  }
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype};
+  d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, b, 1, p->E_cap);
+  d.attn_ws = cv.take(d.attn_ws_bytes);
+  if (o) *o = d;
+  return cv.ok ? align256(cv.used) : 0;
+}
+
+}  // namespace
+
+size_t csa_decode_workspace_size(const csa_decode_params* p) {
+  if (!p) return 0;
+  return decode_layout(p, nullptr, 0, nullptr);
+}
+
+csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, void* ws,
+                      size_t ws_bytes, cudaStream_t stream) {
+  if (!p || !x) return CSA_ERR_INVALID_ARG;
+  if (p->b < 0 || p->m < 1 || p->L < p->m || p->L % p->m) return CSA_ERR_INVALID_ARG;
+  const int E = p->L / p->m;
+  if (E > p->E_cap) return CSA_ERR_INVALID_ARG;
+  if (!p->hca && (p->k < 1 || p->c_I < 16 || p->H_I < 1)) return CSA_ERR_INVALID_ARG;
+  if (p->b == 0) return CSA_OK;
+  DecodeWs d{};
+  const size_t need = decode_layout(p, ws, ws_bytes, &d);
+  if (need == 0 || !ws || ws_bytes < csa_decode_workspace_size(p)) return CSA_ERR_INVALID_ARG;
+  const int b = p->b;
+  const int t = p->L - 1;
+  csa_status st = launch_fill_i32(d.qpos, b, t, stream);
+  if (st) return st;
+
+  // 1. compress the entry the new token completes (latent, then index key)
+  csa_compress_params cp{p->m, p->hca ? 0 : 1, p->c, p->d_rope, p->rope_theta, p->eps, 1,
+                         p->kv_dtype, p->kv_dtype};
+  st = csa_compress(&cp, x->C_a, x->Z_a, x->B_a, x->C_b, x->Z_b, x->B_b, b, p->L, E - 1, 1,
+                    p->E_cap, x->kv_cache, nullptr, stream);
+  if (st) return st;
+  const int32_t* idx = nullptr;
+  const int32_t* cnt = nullptr;
+  if (!p->hca) {
+    csa_compress_params ci{p->m, 1, p->c_I, p->d_rope_I, p->rope_theta, p->eps, 1, p->kv_dtype,
+                           p->idx_dtype};
+    st = csa_compress(&ci, x->CI_a, x->ZI_a, x->BI_a, x->CI_b, x->ZI_b, x->BI_b, b, p->L, E - 1, 1,
+                      p->E_cap, x->kI_cache, x->kI_scales, stream);
+    if (st) return st;
+    // 2. quantise the index queries, score all entries
+    const void* qI = x->q_I;
+    const void* qs = nullptr;
+    if (p->idx_dtype != CSA_F32) {
+      st = csa_quantize(p->kv_dtype, p->idx_dtype, x->q_I, b * p->H_I, p->c_I, d.qI_codes,
+                        d.qI_scales, stream);
+      if (st) return st;
+      qI = d.qI_codes; qs = d.qI_scales;
+    } else if (p->kv_dtype != CSA_F32) {
+      return CSA_ERR_UNSUPPORTED;
+    }
+    csa_index_params ip{p->H_I, p->c_I, p->m, p->idx_dtype, CSA_BF16};
+    st = csa_index_scores(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, 1, p->E_cap, E,
+                          d.scores, stream);
+    if (st) return st;
+    // 3. top-k
+    int32_t* io = x->idx_out ? x->idx_out : d.idx;
+    int32_t* co = x->count_out ? x->count_out : d.count;
+    st = csa_topk(d.scores, CSA_BF16, d.qpos, p->m, b, 1, E, p->k, io, co, nullptr, 0, stream);
+    if (st) return st;
+    idx = io; cnt = co;
+  }
+  // 4. attention over the selection (or all entries) plus the window
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype};
+  return csa_sparse_attn(&ap, x->q, x->kv_cache, p->E_cap, idx, cnt, x->kv_win, p->L, d.qpos,
+                         x->sink, b, 1, x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream);
+}
+
+// ---------------------------------------------------------------------------
+// prefill
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct PrefillWs {
+  void* qI_codes; void* qI_scales; void* scores; int32_t* idx; int32_t* count; int32_t* qpos;
+  void* attn_ws; size_t attn_ws_bytes;
+};
+
+size_t prefill_layout(const csa_prefill_params* p, void* ws, size_t cap, PrefillWs* o) {
+  Carve cv(ws, cap);
+  PrefillWs d{};
+  const size_t rows = (size_t)p->b * p->n;
+  const int E = p->n / p->m;
+  d.qpos = static_cast<int32_t*>(cv.take(rows * 4));
+  if (p->idx_dtype != CSA_F32) {
+    d.qI_codes = cv.take(rows * p->H_I * dtype_row_bytes(p->idx_dtype, p->c_I));
+    d.qI_scales = cv.take(p->idx_dtype == CSA_FP8_E4M3 ? rows * p->H_I * 4
+                                                        : rows * p->H_I * (p->c_I / 16));
+  }
+  d.scores = cv.take(rows * E * (p->score_dtype == CSA_F32 ? 4 : 2));
+  d.idx = static_cast<int32_t*>(cv.take(rows * p->k * 4));
+  d.count = static_cast<int32_t*>(cv.take(rows * 4));
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype};
+  d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, p->b, p->n, E);
+  d.attn_ws = cv.take(d.attn_ws_bytes);
+  if (o) *o = d;
+  return cv.ok ? align256(cv.used) : 0;
+}
+
+}  // namespace
+
+size_t csa_prefill_workspace_size(const csa_prefill_params* p) {
+  if (!p) return 0;
+  return prefill_layout(p, nullptr, 0, nullptr);
+}
+
+csa_status csa_prefill(const csa_prefill_params* p, const csa_prefill_tensors* x, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+  if (!p || !x) return CSA_ERR_INVALID_ARG;
+  if (p->b < 0 || p->m < 1 || p->n < p->m || p->k < 1) return CSA_ERR_INVALID_ARG;
+  if (p->b == 0) return CSA_OK;
+  PrefillWs d{};
+  const size_t need = prefill_layout(p, ws, ws_bytes, &d);
+  if (need == 0 || !ws || ws_bytes < csa_prefill_workspace_size(p)) return CSA_ERR_INVALID_ARG;
+  const int b = p->b, n = p->n, E = n / p->m;
+  csa_status st = launch_iota_positions(d.qpos, b, n, stream);
+  if (st) return st;
+  csa_compress_params cp{p->m, 1, p->c, p->d_rope, p->rope_theta, p->eps, 1, p->kv_dtype,
+                         p->kv_dtype};
+  st = csa_compress(&cp, x->C_a, x->Z_a, x->B_a, x->C_b, x->Z_b, x->B_b, b, n, 0, E, E,
+                    x->kv_cache, nullptr, stream);
+  if (st) return st;
+  csa_compress_params ci{p->m, 1, p->c_I, p->d_rope_I, p->rope_theta, p->eps, 1, p->kv_dtype,
+                         p->idx_dtype};
+  st = csa_compress(&ci, x->CI_a, x->ZI_a, x->BI_a, x->CI_b, x->ZI_b, x->BI_b, b, n, 0, E, E,
+                    x->kI_cache, x->kI_scales, stream);
+  if (st) return st;
+  const void* qI = x->q_I;
+  const void* qs = nullptr;
+  if (p->idx_dtype != CSA_F32) {
+    st = csa_quantize(p->kv_dtype, p->idx_dtype, x->q_I, b * n * p->H_I, p->c_I, d.qI_codes,
+                      d.qI_scales, stream);
+    if (st) return st;
+    qI = d.qI_codes; qs = d.qI_scales;
+  } else if (p->kv_dtype != CSA_F32) {
+    return CSA_ERR_UNSUPPORTED;
+  }
+  csa_index_params ip{p->H_I, p->c_I, p->m, p->idx_dtype, p->score_dtype};
+  st = csa_index_scores(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, n, E, E, d.scores,
+                        stream);
+  if (st) return st;
+  int32_t* io = x->idx_out ? x->idx_out : d.idx;
+  int32_t* co = x->count_out ? x->count_out : d.count;
+  st = csa_topk(d.scores, p->score_dtype, d.qpos, p->m, b, n, E, p->k, io, co, nullptr, 0, stream);
+  if (st) return st;
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype};
+  return csa_sparse_attn(&ap, x->q, x->kv_cache, E, io, co, x->kv_win, n, d.qpos, x->sink, b, n,
+                         x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,306 @@
+// KV compressor (pool -> RMSNorm -> partial RoPE -> store / quantise) and the
+// stand-alone index-path quantiser.
+//
+// Method: "DeepSeek V4 结构速览", section "C4A Compressor"; section "核心设计"
+// item 1 (c4a 8 rows at stride 4, c128a 128 rows at stride 128);
+// "DeepSeek-V4技术报告解读", section "Compressed Sparse Attention (CSA)".
+//
+// Layout of the work: one CTA per (entry, sequence).  Threads are split into
+// `cols` column threads (16 bytes of channels each) x `rg` row groups; each
+// row group streams every rg-th row of the 2m (or m) stacked rows with an
+// online per-channel softmax in float32, then the row groups are merged
+// through shared memory.  Every raw row is read exactly once per entry; the
+// overlap of c4a reads C_b/Z_b for the previous block and C_a/Z_a for the
+// current one, which are different tensors, so no row is read twice overall.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace csa {
+
+template <typename InT>
+struct Vec16;  // 16 bytes of InT
+template <> struct Vec16<float> { static constexpr int N = 4; };
+template <> struct Vec16<__nv_bfloat16> { static constexpr int N = 8; };
+
+template <typename InT>
+__device__ __forceinline__ void load16(const InT* p, float* dst) {
+  uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+  if constexpr (sizeof(InT) == 4) {
+    dst[0] = __uint_as_float(v.x); dst[1] = __uint_as_float(v.y);
+    dst[2] = __uint_as_float(v.z); dst[3] = __uint_as_float(v.w);
+  } else {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      dst[2 * i] = __uint_as_float(w[i] << 16);
+      dst[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+    }
+  }
+}
+
+constexpr int kUnroll = 4;
+
+template <typename InT>
+__global__ void __launch_bounds__(512) compress_kernel(CompressArgs a) {
+  constexpr int VEC = Vec16<InT>::N;
+  extern __shared__ float smem[];
+  const int c = a.c;
+  const int cols = c / VEC;
+  const int rg = blockDim.x / cols;
+  const int tid = threadIdx.x;
+  const int cc = tid % cols;
+  const int g = tid / cols;
+  const int i = a.entry_begin + blockIdx.x;
+  const int s = blockIdx.y;
+  const int m = a.m;
+  const int R = a.overlap ? 2 * m : m;
+
+  const InT* Ca = reinterpret_cast<const InT*>(a.C_a) + (size_t)s * a.n * c;
+  const InT* Za = reinterpret_cast<const InT*>(a.Z_a) + (size_t)s * a.n * c;
+  const InT* Cb = a.overlap ? reinterpret_cast<const InT*>(a.C_b) + (size_t)s * a.n * c : nullptr;
+  const InT* Zb = a.overlap ? reinterpret_cast<const InT*>(a.Z_b) + (size_t)s * a.n * c : nullptr;
+
+  float mx[VEC], sum[VEC], acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) { mx[v] = -INFINITY; sum[v] = 0.f; acc[v] = 0.f; }
+
+  if (g < rg) {
+    for (int r0 = g; r0 < R; r0 += rg * kUnroll) {
+      float zv[kUnroll][VEC], cv[kUnroll][VEC], bv[kUnroll][VEC];
+      bool live[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int r = r0 + u * rg;
+        live[u] = r < R;
+        const InT *Z = nullptr, *C = nullptr;
+        const float* B = nullptr;
+        int row = 0;
+        if (live[u]) {
+          if (a.overlap && r < m) {
+            if (i == 0) { live[u] = false; }
+            else { row = m * (i - 1) + r; Z = Zb; C = Cb; B = a.B_b + (size_t)r * c; }
+          } else {
+            const int rr = a.overlap ? r - m : r;
+            row = m * i + rr; Z = Za; C = Ca; B = a.B_a + (size_t)rr * c;
+          }
+        }
+        if (live[u]) {
+          load16<InT>(Z + (size_t)row * c + cc * VEC, zv[u]);
+          load16<InT>(C + (size_t)row * c + cc * VEC, cv[u]);
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) bv[u][v] = __ldg(B + cc * VEC + v);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (!live[u]) continue;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          const float x = zv[u][v] + bv[u][v];
+          if (x > mx[v]) {
+            const float sc = expf(mx[v] - x);
+            sum[v] = sum[v] * sc + 1.f;
+            acc[v] = acc[v] * sc + cv[u][v];
+            mx[v] = x;
+          } else {
+            const float e = expf(x - mx[v]);
+            sum[v] += e;
+            acc[v] = fmaf(e, cv[u][v], acc[v]);
+          }
+        }
+      }
+    }
+  }
+
+  // merge the row groups
+  float* s_mx = smem;                 // [rg][c]
+  float* s_sum = s_mx + rg * c;       // [rg][c]
+  float* s_acc = s_sum + rg * c;      // [rg][c]
+  float* s_x = s_acc + rg * c;        // [c]
+  float* s_red = s_x + c;             // [32]
+  if (g < rg) {
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      s_mx[g * c + cc * VEC + v] = mx[v];
+      s_sum[g * c + cc * VEC + v] = sum[v];
+      s_acc[g * c + cc * VEC + v] = acc[v];
+    }
+  }
+  __syncthreads();
+  float ss = 0.f;
+  for (int ch = tid; ch < c; ch += blockDim.x) {
+    float M = -INFINITY;
+    for (int q = 0; q < rg; ++q) M = fmaxf(M, s_mx[q * c + ch]);
+    float S = 0.f, A = 0.f;
+    for (int q = 0; q < rg; ++q) {
+      const float mq = s_mx[q * c + ch];
+      if (mq == -INFINITY) continue;
+      const float e = expf(mq - M);
+      S = fmaf(s_sum[q * c + ch], e, S);
+      A = fmaf(s_acc[q * c + ch], e, A);
+    }
+    const float x = A / S;
+    s_x[ch] = x;
+    ss = fmaf(x, x, ss);
+  }
+  float inv = 1.f;
+  if (a.apply_norm) {
+    const float tot = block_sum(ss, s_red);
+    inv = 1.f / sqrtf(tot / (float)c + a.eps);
+  }
+  __syncthreads();
+  // RMSNorm + RoPE (angle in float64), result back into s_x
+  const int rope0 = c - a.d_rope;
+  for (int pj = tid; pj < c / 2; pj += blockDim.x) {
+    const int ch = 2 * pj;
+    float x0 = s_x[ch] * inv, x1 = s_x[ch + 1] * inv;
+    if (ch >= rope0 && a.d_rope > 0) {
+      const int j = (ch - rope0) / 2;
+      const double freq = pow(a.theta, -2.0 * (double)j / (double)a.d_rope);
+      const double ang = (double)((long long)m * i) * freq;
+      double sn, cs;
+      sincos(ang, &sn, &cs);
+      const double y0 = (double)x0 * cs - (double)x1 * sn;
+      const double y1 = (double)x0 * sn + (double)x1 * cs;
+      x0 = (float)y0; x1 = (float)y1;
+    }
+    s_x[ch] = x0; s_x[ch + 1] = x1;
+  }
+  __syncthreads();
+
+  const size_t orow = (size_t)s * a.out_E + i;
+  if (a.out_dtype == CSA_F32) {
+    float* o = reinterpret_cast<float*>(a.out) + orow * c;
+    for (int ch = tid; ch < c; ch += blockDim.x) o[ch] = s_x[ch];
+  } else if (a.out_dtype == CSA_BF16) {
+    __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + orow * c;
+    for (int ch = tid; ch < c; ch += blockDim.x) o[ch] = __float2bfloat16_rn(s_x[ch]);
+  } else if (a.out_dtype == CSA_FP8_E4M3) {
+    float am = 0.f;
+    for (int ch = tid; ch < c; ch += blockDim.x) am = fmaxf(am, fabsf(s_x[ch]));
+    am = block_max(am, s_red);
+    const float scale = am / 448.f;
+    uint8_t* o = reinterpret_cast<uint8_t*>(a.out) + orow * c;
+    for (int ch = tid; ch < c; ch += blockDim.x)
+      o[ch] = scale > 0.f ? f32_to_e4m3(s_x[ch] / scale) : (uint8_t)0;
+    if (tid == 0) reinterpret_cast<float*>(a.out_scales)[orow] = scale;
+  } else {  // CSA_NVFP4
+    uint8_t* o = reinterpret_cast<uint8_t*>(a.out) + orow * (c / 2);
+    uint8_t* so = reinterpret_cast<uint8_t*>(a.out_scales) + orow * (c / 16);
+    for (int blk = tid; blk < c / 16; blk += blockDim.x) {
+      float am = 0.f;
+#pragma unroll
+      for (int e = 0; e < 16; ++e) am = fmaxf(am, fabsf(s_x[blk * 16 + e]));
+      const uint8_t sc = f32_to_e4m3(am / 6.f);
+      const float sv = e4m3_to_f32(sc);
+#pragma unroll
+      for (int e = 0; e < 16; e += 2) {
+        o[blk * 8 + e / 2] = sv > 0.f
+            ? f32x2_to_e2m1x2(s_x[blk * 16 + e] / sv, s_x[blk * 16 + e + 1] / sv)
+            : (uint8_t)0;
+      }
+      so[blk] = sc;
+    }
+  }
+}
+
+// One warp per row: FP8 (per-row scale) or NVFP4 (per-16 scale) codes.
+template <typename InT>
+__global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int out_dtype,
+                                uint8_t* __restrict__ codes, void* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  const InT* xr = x + (size_t)row * d;
+  float am_row = 0.f;
+  for (int base = 0; base < d; base += 128) {
+    const int e0 = base + lane * 4;
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      if (e0 + e < d) am_row = fmaxf(am_row, fabsf(to_f32(xr[e0 + e])));
+  }
+  if (out_dtype == CSA_FP8_E4M3) {
+    am_row = warp_max(am_row);
+    const float scale = am_row / 448.f;
+    for (int base = 0; base < d; base += 128) {
+      const int e0 = base + lane * 4;
+      if (e0 < d) {
+        uint32_t packed = 0;
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t cde = scale > 0.f ? f32_to_e4m3(to_f32(xr[e0 + e]) / scale) : 0u;
+          packed |= cde << (8 * e);
+        }
+        *reinterpret_cast<uint32_t*>(codes + (size_t)row * d + e0) = packed;
+      }
+    }
+    if (lane == 0) reinterpret_cast<float*>(scales)[row] = scale;
+  } else {
+    // NVFP4: 4 lanes x 4 elements = one 16-element block
+    for (int base = 0; base < d; base += 128) {
+      const int e0 = base + lane * 4;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      float am = 0.f;
+      if (e0 < d) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) { v[e] = to_f32(xr[e0 + e]); am = fmaxf(am, fabsf(v[e])); }
+      }
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      const uint8_t sc = f32_to_e4m3(am / 6.f);
+      const float sv = e4m3_to_f32(sc);
+      if (e0 < d) {
+        uint8_t p0 = sv > 0.f ? f32x2_to_e2m1x2(v[0] / sv, v[1] / sv) : (uint8_t)0;
+        uint8_t p1 = sv > 0.f ? f32x2_to_e2m1x2(v[2] / sv, v[3] / sv) : (uint8_t)0;
+        uint8_t* cr = codes + (size_t)row * (d / 2) + e0 / 2;
+        cr[0] = p0; cr[1] = p1;
+        if ((lane & 3) == 0)
+          reinterpret_cast<uint8_t*>(scales)[(size_t)row * (d / 16) + e0 / 16] = sc;
+      }
+    }
+  }
+}
+
+csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry_count,
+                           cudaStream_t st) {
+  const int vec = in_dtype == CSA_F32 ? 4 : 8;
+  const int cols = a.c / vec;
+  const int R = a.overlap ? 2 * a.m : a.m;
+  int nt = R >= 64 ? 512 : 256;
+  if (cols > nt) return CSA_ERR_UNSUPPORTED;
+  // as many whole row groups as fit, at most one row group per row
+  int rg = nt / cols;
+  if (rg > R) rg = R;
+  nt = rg * cols;
+  if (nt % 32) nt = ((nt + 31) / 32) * 32;   // idle tail threads take no rows (g >= rg)
+  const size_t smem = (size_t)(3 * (nt / cols) * a.c + a.c + 32) * sizeof(float);
+  if (smem > 200 * 1024) return CSA_ERR_UNSUPPORTED;
+  dim3 grid(entry_count, b);
+  if (in_dtype == CSA_F32) {
+    cudaFuncSetAttribute(compress_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    compress_kernel<float><<<grid, nt, smem, st>>>(a);
+  } else {
+    cudaFuncSetAttribute(compress_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    compress_kernel<__nv_bfloat16><<<grid, nt, smem, st>>>(a);
+  }
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
+                           void* codes, void* scales, cudaStream_t st) {
+  if (rows == 0) return CSA_OK;
+  const int warps = 8;
+  dim3 grid((rows + warps - 1) / warps);
+  if (in_dtype == CSA_F32)
+    quantize_kernel<float><<<grid, warps * 32, 0, st>>>(
+        reinterpret_cast<const float*>(x), rows, d, out_dtype, reinterpret_cast<uint8_t*>(codes), scales);
+  else
+    quantize_kernel<__nv_bfloat16><<<grid, warps * 32, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), rows, d, out_dtype,
+        reinterpret_cast<uint8_t*>(codes), scales);
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+}  // namespace csa

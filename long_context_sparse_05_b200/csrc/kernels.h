@@ -1,0 +1,54 @@
+// Internal launch interface between the C ABI (api.cu) and the kernel files.
+#pragma once
+
+#include "csa.h"
+
+namespace csa {
+
+struct CompressArgs {
+  const void* C_a; const void* Z_a; const float* B_a;
+  const void* C_b; const void* Z_b; const float* B_b;
+  int n, m, overlap, c, d_rope, apply_norm, out_dtype, entry_begin, out_E;
+  double theta;
+  float eps;
+  void* out;
+  void* out_scales;
+};
+
+struct IndexArgs {
+  const void* q; const void* q_scales; const float* w;
+  const void* k; const void* k_scales; const int32_t* q_pos;
+  int T, H, d, m, qk_dtype, score_dtype, E_cap, E;
+  void* scores;
+};
+
+struct AttnArgs {
+  const void* q; const void* kv; const int32_t* idx; const int32_t* count;
+  const void* win; const int32_t* q_pos; const float* sink;
+  int T, H, d, n_w, m, k, E_cap, n;
+  float scale;
+  void* out; float* lse;
+};
+
+csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry_count,
+                           cudaStream_t st);
+csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
+                           void* codes, void* scales, cudaStream_t st);
+csa_status launch_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int rows,
+                       int E, int k, int32_t* idx, int32_t* count, cudaStream_t st);
+
+// CUDA-core kernels: any shape.
+csa_status launch_index_scores_simt(const IndexArgs& a, int b, cudaStream_t st);
+csa_status launch_attn_simt(const AttnArgs& a, int b, int dtype, cudaStream_t st);
+
+// Tensor-core (tcgen05) kernels: return CSA_ERR_UNSUPPORTED for shapes they do not cover.
+csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st);
+csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t ws_bytes,
+                          cudaStream_t st);
+size_t attn_tc_workspace_bytes(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype);
+
+// Small helpers.
+csa_status launch_fill_i32(int32_t* p, int count, int value, cudaStream_t st);
+csa_status launch_iota_positions(int32_t* p, int b, int n, cudaStream_t st);
+
+}  // namespace csa

@@ -1,0 +1,72 @@
+"""Comparison helpers shared by the parity tests."""
+
+import numpy as np
+import torch
+
+from oracle import codecs
+
+
+def f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def rel_close(gpu, ref, rtol):
+    """Element-wise |gpu - ref| <= rtol * (|ref| + rms(ref)) (the reading of 'relative')."""
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    rms = np.sqrt(np.mean(ref[np.isfinite(ref)] ** 2)) if np.any(np.isfinite(ref)) else 0.0
+    err = np.abs(gpu - ref)
+    bound = rtol * (np.abs(ref) + rms)
+    bad = ~(err <= bound)
+    same_inf = np.isinf(gpu) & np.isinf(ref) & (np.sign(gpu) == np.sign(ref))
+    bad &= ~same_inf
+    return (not np.any(bad)), (float(np.max(np.where(np.isfinite(err), err, 0))) if err.size else 0.0), \
+        int(np.sum(bad))
+
+
+def assert_rel_close(gpu, ref, rtol, what=""):
+    ok, mx, nbad = rel_close(gpu, ref, rtol)
+    assert ok, "%s: %d elements beyond rtol %g (max abs err %g)" % (what, nbad, rtol, mx)
+
+
+def assert_abs_close(gpu, ref, atol, what=""):
+    gpu = np.asarray(gpu, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    err = np.max(np.abs(gpu - ref)) if gpu.size else 0.0
+    assert err <= atol, "%s: max abs err %g > %g" % (what, err, atol)
+
+
+def bf16_ulp(x):
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    _, ex = np.frexp(np.where(x > 0, x, 1.0))
+    return np.ldexp(1.0, np.maximum(ex - 1, -126) - 7)
+
+
+def topk_band_check(gpu_idx, gpu_cnt, exact_scores, ev, k, rel_band=1e-3):
+    """Validate a GPU selection against the oracle's exact (pre-rounding) scores.
+
+    Exact match except for entries whose exact score lies within
+    max(rel_band * |tau|, one bf16 ulp of tau) of the k-th largest exact
+    score tau.  Also checks count, ordering, range and uniqueness.  Returns the
+    number of entries that differ from the oracle's own choice.
+    """
+    gpu_idx = np.asarray(gpu_idx)
+    cnt = int(gpu_cnt)
+    assert cnt == min(k, ev), (cnt, k, ev)
+    sel = gpu_idx[:cnt]
+    assert np.all(gpu_idx[cnt:] == -1)
+    assert np.all(np.diff(sel) > 0), "not strictly ascending"
+    assert cnt == 0 or (sel[0] >= 0 and sel[-1] < ev), "out of the causal range"
+    if ev <= k:
+        assert np.array_equal(sel, np.arange(ev))
+        return 0
+    sc = np.asarray(exact_scores[:ev], dtype=np.float64)
+    order = np.lexsort((np.arange(ev), -sc))
+    ref = set(order[:k].tolist())
+    tau = sc[order[k - 1]]
+    band = max(rel_band * abs(tau), float(bf16_ulp(tau)))
+    diff = ref.symmetric_difference(set(sel.tolist()))
+    for s in diff:
+        assert abs(sc[s] - tau) <= band, "entry %d score %r outside the tie band of tau %r" % (
+            s, sc[s], tau)
+    return len(diff) // 2

@@ -1,0 +1,125 @@
+"""Host-side checks of the C ABI: the library loads, exports every declared
+symbol, its structs match the ctypes mirrors, and argument errors come back as
+CSA_ERR_INVALID_ARG before any CUDA call (so these run without a GPU)."""
+
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import long_context_sparse_05_b200 as csa
+from long_context_sparse_05_b200 import _lib as L
+from long_context_sparse_05_b200 import runner, workloads
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    from long_context_sparse_05_b200 import build
+    build.build()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\*?(csa_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert len(names) >= 12, names
+    lib = ctypes.CDLL(L.LIB_PATH)
+    missing = [n for n in names if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_binding_covers_every_declared_symbol():
+    assert set(declared_functions()) <= set(L._SIGS), set(declared_functions()) - set(L._SIGS)
+
+
+def test_struct_layouts_match_c():
+    structs = {"csa_compress_params": L.CompressParams, "csa_index_params": L.IndexParams,
+               "csa_attn_params": L.AttnParams, "csa_decode_params": L.DecodeParams,
+               "csa_decode_tensors": L.DecodeTensors, "csa_prefill_params": L.PrefillParams,
+               "csa_prefill_tensors": L.PrefillTensors}
+    prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "csa.h"', "int main(void){"]
+    for cname, py in structs.items():
+        prog.append('printf("%s %%zu\\n", sizeof(%s));' % (cname, cname))
+        for fname, _ in py._fields_:
+            prog.append('printf("%s.%s %%zu\\n", offsetof(%s, %s));' % (cname, fname, cname, fname))
+    prog.append("return 0;}")
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write("\n".join(prog))
+        subprocess.check_call(["gcc", "-I", os.path.join(ROOT, "include"), "-I",
+                               "/usr/local/cuda/include", c, "-o", exe])
+        out = subprocess.check_output([exe], text=True).split("\n")
+    got = dict(line.split() for line in out if line)
+    for cname, py in structs.items():
+        assert int(got[cname]) == ctypes.sizeof(py), cname
+        for fname, _ in py._fields_:
+            assert int(got["%s.%s" % (cname, fname)]) == getattr(py, fname).offset, (cname, fname)
+
+
+def test_status_strings():
+    assert csa.csa_status_string(0) == "CSA_OK"
+    assert "INVALID" in csa.csa_status_string(1)
+    assert L.lib().csa_version() >= 100
+
+
+def test_invalid_arguments_rejected_on_host():
+    lib = L.lib()
+    p = L.CompressParams(m=0, overlap=1, c=64, d_rope=16, rope_theta=1e4, eps=1e-6, apply_norm=1,
+                         in_dtype=0, out_dtype=0)
+    fake = 1 << 20   # never dereferenced: validation fails first
+    assert lib.csa_compress(ctypes.byref(p), fake, fake, fake, fake, fake, fake, 1, 64, 0, 16, 16,
+                            fake, None, None) == 1
+    p.m = 4
+    p.d_rope = 7   # odd rotary width
+    assert lib.csa_compress(ctypes.byref(p), fake, fake, fake, fake, fake, fake, 1, 64, 0, 16, 16,
+                            fake, None, None) == 1
+    p.d_rope = 16
+    # more entries than the raw rows can complete
+    assert lib.csa_compress(ctypes.byref(p), fake, fake, fake, fake, fake, fake, 1, 64, 0, 17, 17,
+                            fake, None, None) == 1
+    # unaligned pointer
+    assert lib.csa_compress(ctypes.byref(p), fake + 2, fake, fake, fake, fake, fake, 1, 64, 0, 16,
+                            16, fake, None, None) == 1
+    # zero work is a no-op success
+    assert lib.csa_compress(ctypes.byref(p), None, None, None, None, None, None, 0, 64, 0, 16, 16,
+                            None, None, None) == 0
+    ip = L.IndexParams(H_I=4, d_I=20, m=4, qk_dtype=0, score_dtype=0)   # d_I not a multiple of 16
+    assert lib.csa_index_scores(ctypes.byref(ip), fake, None, fake, fake, None, fake, 1, 1, 8, 8,
+                                fake, None) == 1
+    assert lib.csa_topk(fake, 5, fake, 4, 1, 1, 8, 2, fake, fake, None, 0, None) == 1
+    ap = L.AttnParams(H=4, d=64, n_w=16, scale=0.125, m=4, k=0, dtype=0)
+    assert lib.csa_sparse_attn(ctypes.byref(ap), fake, fake, 8, fake, fake, fake, 64, fake, fake,
+                               1, 1, fake, None, None, 0, None) == 1   # idx given with k = 0
+    assert lib.csa_quantize(1, 2, fake, 4, 24, fake, fake, None) == 1  # d not a multiple of 16
+
+
+def test_workspace_sizes_are_host_only_and_positive():
+    for w in workloads.ALL.values():
+        if w.kind == "csa_prefill":
+            n = L.csa_prefill_workspace_size(runner.prefill_params(w))
+        else:
+            n = L.csa_decode_workspace_size(runner.decode_params(w))
+        assert n > 0
+    # a too-small workspace is an argument error
+    w = workloads.CSA_DECODE_64K
+    p = runner.decode_params(w)
+    x = L.DecodeTensors()
+    assert L.lib().csa_decode(ctypes.byref(p), ctypes.byref(x), 1 << 20, 16, None) == 1
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(L, "_lib", None)
+    monkeypatch.setattr(L, "LIB_PATH", "/nonexistent/libcsa.so")
+    with pytest.raises(L.CsaError):
+        L.lib()

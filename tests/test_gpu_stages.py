@@ -1,0 +1,303 @@
+"""Stage-isolated parity of the CUDA kernels against the CPU oracle.
+
+Every stage gets identical inputs on both sides (drawn by the seeded
+generator, or produced by the oracle for the stage's own inputs), and every
+call goes through the C ABI.  Sizes span several tiles and a ragged tail.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from long_context_sparse_05_b200 import _lib as L
+from long_context_sparse_05_b200 import synth
+from oracle import codecs, csa
+
+from helpers import assert_abs_close, assert_rel_close, f64, topk_band_check
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def _branch(b, n, c, m, seed, dtype, overlap=True, device=DEV):
+    d = {}
+    d["C_a"] = synth.draw("C_a", (b, n, c), seed, device, dtype)
+    d["Z_a"] = synth.draw("Z_a", (b, n, c), seed, device, dtype)
+    d["B_a"] = synth.draw("B_a", (m, c), seed, device, "f32", spread=0.5)
+    if overlap:
+        d["C_b"] = synth.draw("C_b", (b, n, c), seed, device, dtype)
+        d["Z_b"] = synth.draw("Z_b", (b, n, c), seed, device, dtype)
+        d["B_b"] = synth.draw("B_b", (m, c), seed, device, "f32", spread=0.5)
+    return d
+
+
+def _oracle_compress(d, s, m, overlap, E, d_rope, apply_norm=True, eps=1e-6):
+    g = {k: f64(v[s]) if v.dim() == 3 else f64(v) for k, v in d.items()}
+    return csa.compress_range(g["C_a"], g["Z_a"], g["B_a"], g.get("C_b"), g.get("Z_b"), g.get("B_b"),
+                              m, overlap, 0, E, d_rope, 1e4, eps, apply_norm)
+
+
+def _run_compress(d, b, n, c, m, overlap, E, d_rope, in_dt, out_dt, apply_norm=True, E_cap=None,
+                  entry_begin=0):
+    E_cap = E_cap or E
+    if out_dt in ("f32", "bf16"):
+        out = torch.zeros((b, E_cap, c), dtype=torch.float32 if out_dt == "f32" else torch.bfloat16,
+                          device=DEV)
+        sc = None
+    elif out_dt == "fp8":
+        out = torch.zeros((b, E_cap, c), dtype=torch.uint8, device=DEV)
+        sc = torch.zeros((b, E_cap), dtype=torch.float32, device=DEV)
+    else:
+        out = torch.zeros((b, E_cap, c // 2), dtype=torch.uint8, device=DEV)
+        sc = torch.zeros((b, E_cap, c // 16), dtype=torch.uint8, device=DEV)
+    p = L.CompressParams(m=m, overlap=int(overlap), c=c, d_rope=d_rope, rope_theta=1e4, eps=1e-6,
+                         apply_norm=int(apply_norm), in_dtype=L.DTYPE[in_dt],
+                         out_dtype=L.DTYPE[out_dt])
+    L.csa_compress(p, d["C_a"], d["Z_a"], d["B_a"], d.get("C_b"), d.get("Z_b"), d.get("B_b"), b, n,
+                   entry_begin, E - entry_begin, E_cap, out, sc)
+    torch.cuda.synchronize()
+    return out, sc
+
+
+@pytest.mark.parametrize("c,d_rope,seed", [(64, 16, 0), (32, 16, 1)])
+def test_compress_f32_tiny(c, d_rope, seed):
+    b, n, m = 1, 1024, 4
+    d = _branch(b, n, c, m, seed, "f32")
+    out, _ = _run_compress(d, b, n, c, m, True, n // m, d_rope, "f32", "f32")
+    ref = _oracle_compress(d, 0, m, True, n // m, d_rope)
+    assert_rel_close(f64(out[0]), ref, 1e-5, "compress f32")
+
+
+def test_compress_bf16_c4a_ragged_and_partial():
+    b, n, c, m = 2, 520, 512, 4          # 130 entries: not a multiple of any tile
+    E = n // m
+    d = _branch(b, n, c, m, 11, "bf16")
+    out32, _ = _run_compress(d, b, n, c, m, True, E, 64, "bf16", "f32")
+    out16, _ = _run_compress(d, b, n, c, m, True, E, 64, "bf16", "bf16")
+    for s in range(b):
+        ref = _oracle_compress(d, s, m, True, E, 64)
+        assert_rel_close(f64(out32[s]), ref, 1e-5, "compress bf16->f32")
+        assert_rel_close(f64(out16[s]), ref, 2e-2, "compress bf16->bf16")
+        # bf16 output is the round-to-nearest of the float32 result (torch's own cast)
+        assert torch.equal(out16[s], out32[s].to(torch.bfloat16))
+    # updating a tail range leaves the rest of the cache untouched
+    part, _ = _run_compress(d, b, n, c, m, True, E, 64, "bf16", "f32", E_cap=E + 3, entry_begin=100)
+    assert torch.all(part[:, :100] == 0) and torch.all(part[:, E:] == 0)
+    assert torch.equal(part[:, 100:E], out32[:, 100:E])
+
+
+def test_compress_hca_c128a():
+    b, n, c, m = 2, 128 * 5, 512, 128
+    d = _branch(b, n, c, m, 12, "bf16", overlap=False)
+    out, _ = _run_compress(d, b, n, c, m, False, n // m, 64, "bf16", "f32")
+    for s in range(b):
+        assert_rel_close(f64(out[s]), _oracle_compress(d, s, m, False, n // m, 64), 1e-5, "c128a")
+
+
+def test_compress_m1_is_identity():
+    b, n, c = 2, 40, 64
+    d = _branch(b, n, c, 1, 13, "f32", overlap=False)
+    out, _ = _run_compress(d, b, n, c, 1, False, n, 0, "f32", "f32", apply_norm=False)
+    assert torch.equal(out, d["C_a"])
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+def test_compress_index_branch_quantised(fmt):
+    b, n, c, m = 2, 1000, 128, 4
+    E = n // m
+    d = _branch(b, n, c, m, 14, "bf16")
+    codes, sc = _run_compress(d, b, n, c, m, True, E, 64, "bf16", fmt)
+    out32, _ = _run_compress(d, b, n, c, m, True, E, 64, "bf16", "f32")
+    # the fused quantiser equals the stand-alone quantiser applied to the kernel's own float32 rows
+    rows = b * E
+    c2 = torch.empty_like(codes)
+    s2 = torch.empty_like(sc)
+    L.csa_quantize(L.CSA_F32, L.DTYPE[fmt], out32, rows, c, c2, s2)
+    torch.cuda.synchronize()
+    assert torch.equal(c2, codes) and torch.equal(s2, sc)
+    for s in range(b):
+        ref = _oracle_compress(d, s, m, True, E, 64)
+        assert_rel_close(f64(out32[s]), ref, 1e-5, "index branch f32")
+        # against the oracle's own entries: a code may move one step only where the float32 and
+        # float64 values straddle a rounding point
+        if fmt == "fp8":
+            deq = codecs.dequant_fp8_rows(codes[s].cpu().numpy(), sc[s].cpu().numpy())
+            deq_ref = codecs.dequant_fp8_rows(*codecs.quant_fp8_rows(ref.astype(np.float32)))
+        else:
+            deq = codecs.dequant_nvfp4(codes[s].cpu().numpy(), sc[s].cpu().numpy())
+            deq_ref = codecs.dequant_nvfp4(*codecs.quant_nvfp4(ref.astype(np.float32)))
+        step = np.abs(deq - deq_ref)
+        frac = np.mean(step > 0)
+        assert frac < 0.01, frac
+        lim = 0.13 if fmt == "fp8" else 0.5
+        assert np.all(step <= lim * (np.abs(ref) + 1.0)), np.max(step)
+
+
+@pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
+@pytest.mark.parametrize("in_dt", ["bf16", "f32"])
+def test_quantize_bit_exact(fmt, in_dt):
+    rows, d = 777, 128
+    x = synth.draw("q_I", (rows, d), 21, DEV, in_dt)
+    x[5] = 0
+    x[6] *= 1e-3
+    x[7] *= 300
+    cbytes = d if fmt == "fp8" else d // 2
+    codes = torch.empty((rows, cbytes), dtype=torch.uint8, device=DEV)
+    sc = torch.empty((rows,), dtype=torch.float32, device=DEV) if fmt == "fp8" else \
+        torch.empty((rows, d // 16), dtype=torch.uint8, device=DEV)
+    L.csa_quantize(L.DTYPE[in_dt], L.DTYPE[fmt], x, rows, d, codes, sc)
+    torch.cuda.synchronize()
+    xs = x.float().cpu().numpy()
+    c_ref, s_ref = codecs.quant_fp8_rows(xs) if fmt == "fp8" else codecs.quant_nvfp4(xs)
+    np.testing.assert_array_equal(codes.cpu().numpy(), c_ref)
+    np.testing.assert_array_equal(sc.cpu().numpy(), s_ref)
+
+
+def _index_inputs(b, T, E, H, d, fmt, seed):
+    """Quantised q/k produced by the oracle's quantiser, so both sides score identical codes."""
+    rng = np.random.default_rng(seed)
+    q = rng.normal(size=(b, T, H, d)).astype(np.float32)
+    k = rng.normal(size=(b, E, d)).astype(np.float32)
+    w = (rng.uniform(size=(b, T, H)) / 64).astype(np.float32)
+    if fmt == "f32":
+        return dict(q=q, qs=None, k=k, ks=None, w=w, qd=q.astype(np.float64), kd=k.astype(np.float64))
+    if fmt == "fp8":
+        qc, qs = codecs.quant_fp8_rows(q)
+        kc, ks = codecs.quant_fp8_rows(k)
+        return dict(q=qc, qs=qs, k=kc, ks=ks, w=w, qd=codecs.dequant_fp8_rows(qc, qs),
+                    kd=codecs.dequant_fp8_rows(kc, ks))
+    qc, qs = codecs.quant_nvfp4(q)
+    kc, ks = codecs.quant_nvfp4(k)
+    return dict(q=qc, qs=qs, k=kc, ks=ks, w=w, qd=codecs.dequant_nvfp4(qc, qs),
+                kd=codecs.dequant_nvfp4(kc, ks))
+
+
+def _dev(a):
+    return None if a is None else torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+
+
+@pytest.mark.parametrize("fmt,H,d,T,E,m,score", [
+    ("fp8", 64, 128, 1, 1000, 4, "bf16"),     # decode-like, ragged 128-entry tiles
+    ("nvfp4", 64, 128, 1, 1000, 4, "bf16"),
+    ("fp8", 64, 128, 37, 80, 4, "bf16"),      # prefill-like: causal mask across queries
+    ("f32", 4, 32, 50, 64, 4, "f32"),         # tiny fp32 configuration
+])
+def test_index_scores(fmt, H, d, T, E, m, score):
+    b = 2
+    x = _index_inputs(b, T, E, H, d, fmt, 31)
+    if T == 1:
+        qpos = np.full((b, T), m * E - 1, dtype=np.int32)
+        qpos[1, 0] = m * 600 + 2            # second sequence sees only 600 entries
+    else:
+        qpos = np.tile(np.arange(T, dtype=np.int32) * (m * E // T) + 3, (b, 1))
+    scores = torch.empty((b, T, E), dtype=torch.bfloat16 if score == "bf16" else torch.float32,
+                         device=DEV)
+    p = L.IndexParams(H_I=H, d_I=d, m=m, qk_dtype=L.DTYPE[fmt], score_dtype=L.DTYPE[score])
+    L.csa_index_scores(p, _dev(x["q"]), _dev(x["qs"]), _dev(x["w"]), _dev(x["k"]), _dev(x["ks"]),
+                       _dev(qpos), b, T, E, E, scores)
+    torch.cuda.synchronize()
+    g = f64(scores)
+    for s in range(b):
+        exact = csa.index_scores(x["qd"][s], x["w"][s], x["kd"][s], qpos[s], m, "f64")
+        fin = np.isfinite(exact)
+        np.testing.assert_array_equal(np.isfinite(g[s]), fin)
+        assert np.all(np.isneginf(g[s][~fin]))
+        # float32 accumulation then one rounding: within one bf16 ulp (or float32 rel 1e-5)
+        tol = (bf16_ulp_arr(exact[fin]) * 1.01) if score == "bf16" else 1e-5 * (np.abs(exact[fin]) + 1e-3)
+        err = np.abs(g[s][fin] - exact[fin])
+        assert np.all(err <= tol + 1e-7), np.max(err - tol)
+
+
+def bf16_ulp_arr(x):
+    from helpers import bf16_ulp
+    return bf16_ulp(x)
+
+
+@pytest.mark.parametrize("score", ["bf16", "f32"])
+def test_topk_bit_exact(score):
+    b, T, E, m = 2, 6, 3000, 4
+    rng = np.random.default_rng(41)
+    sc = np.round(rng.normal(size=(b, T, E)) * 8) / 8           # heavy ties
+    sc[:, 1] = rng.normal(size=E)
+    sc[:, 2] = 0.0                                               # all tied
+    qpos = np.array([[m * E - 1, m * E - 1, m * E - 1, 4 * 300 + 1, 9, 0]] * b, dtype=np.int32)
+    qpos[1, 4] = 4 * 517 - 1                                     # E(t) = 517 > k
+    for k in (16, 512):
+        tdt = torch.bfloat16 if score == "bf16" else torch.float32
+        st = torch.from_numpy(sc).to(tdt).to(DEV)
+        idx = torch.empty((b, T, k), dtype=torch.int32, device=DEV)
+        cnt = torch.empty((b, T), dtype=torch.int32, device=DEV)
+        L.csa_topk(st, L.DTYPE[score], _dev(qpos), m, b, T, E, k, idx, cnt)
+        torch.cuda.synchronize()
+        stored = f64(st)
+        for s in range(b):
+            ri, rc = csa.topk(stored[s], qpos[s], m, k)
+            np.testing.assert_array_equal(cnt[s].cpu().numpy(), rc)
+            np.testing.assert_array_equal(idx[s].cpu().numpy(), ri)
+
+
+def test_topk_1m_row():
+    E, k, m = 262144, 1024, 4
+    sc = synth.draw("q", (1, 1, E), 42, "cpu", "bf16")
+    st = sc.to(DEV)
+    qpos = torch.full((1, 1), m * E - 1, dtype=torch.int32, device=DEV)
+    idx = torch.empty((1, 1, k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((1, 1), dtype=torch.int32, device=DEV)
+    L.csa_topk(st, L.CSA_BF16, qpos, m, 1, 1, E, k, idx, cnt)
+    torch.cuda.synchronize()
+    ri, rc = csa.topk(f64(sc)[0], np.array([m * E - 1]), m, k)
+    np.testing.assert_array_equal(idx[0].cpu().numpy(), ri)
+
+
+def _attn_case(b, T, H, d, E, n, k, n_w, dtype, dense, seed):
+    rng = np.random.default_rng(seed)
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    q = synth.draw("q", (b, T, H, d), seed, DEV, dtype)
+    kv = synth.draw("C_b", (b, E, d), seed, DEV, dtype)
+    win = synth.draw("C_a", (b, n, d), seed, DEV, dtype)
+    sink = synth.draw("sink", (H,), seed, DEV, "f32")
+    qpos = np.stack([np.sort(rng.integers(0, n, size=T)) for _ in range(b)]).astype(np.int32)
+    qpos[0, -1] = n - 1
+    qpos[0, 0] = 0
+    m = max(1, (n // E))
+    if dense:
+        idx_np = cnt_np = None
+    else:
+        idx_np = np.full((b, T, k), -1, np.int32)
+        cnt_np = np.zeros((b, T), np.int32)
+        for s in range(b):
+            scr = rng.normal(size=(T, E))
+            idx_np[s], cnt_np[s] = csa.topk(scr, qpos[s], m, k)
+    return dict(q=q, kv=kv, win=win, sink=sink, qpos=qpos, idx=idx_np, cnt=cnt_np, m=m, tdt=tdt)
+
+
+@pytest.mark.parametrize("H,d,k,n_w,dtype,dense,T,E,n", [
+    (64, 512, 512, 128, "bf16", False, 1, 1500, 6000),   # decode shape, ragged
+    (64, 512, 512, 128, "bf16", True, 1, 700, 2800),     # HCA-style dense, E(t) up to 700
+    (64, 512, 64, 128, "bf16", False, 9, 300, 1200),     # prefill shape, several queries
+    (4, 64, 16, 16, "f32", False, 40, 256, 1024),        # tiny fp32
+])
+def test_sparse_attention(H, d, k, n_w, dtype, dense, T, E, n):
+    b = 2
+    c = _attn_case(b, T, H, d, E, n, k, n_w, dtype, dense, 51)
+    scale = 1.0 / math.sqrt(d)
+    out = torch.empty((b, T, H, d), dtype=c["tdt"], device=DEV)
+    lse = torch.empty((b, T, H), dtype=torch.float32, device=DEV)
+    p = L.AttnParams(H=H, d=d, n_w=n_w, scale=scale, m=c["m"], k=0 if dense else k,
+                     dtype=L.DTYPE[dtype])
+    wsb = L.csa_sparse_attn_workspace_size(p, b, T, E)
+    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    L.csa_sparse_attn(p, c["q"], c["kv"], E, _dev(c["idx"]), _dev(c["cnt"]), c["win"], n,
+                      _dev(c["qpos"]), c["sink"], b, T, out, lse, ws, wsb)
+    torch.cuda.synchronize()
+    for s in range(b):
+        o, l = csa.sparse_attn(f64(c["q"][s]), f64(c["kv"][s]),
+                               None if dense else c["idx"][s], None if dense else c["cnt"][s],
+                               f64(c["win"][s]), c["qpos"][s], f64(c["sink"]), n_w, scale, m=c["m"])
+        if dtype == "bf16":
+            assert_abs_close(f64(out[s]), o, 2e-2, "attention bf16")
+        else:
+            assert_rel_close(f64(out[s]), o, 1e-5, "attention f32")
+        assert_abs_close(f64(lse[s]), l, 1e-3 * (1 + np.max(np.abs(l))), "lse")
