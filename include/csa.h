@@ -70,6 +70,15 @@ const char* csa_status_string(csa_status s);
 /* Library version as major * 10000 + minor * 100 + patch. */
 int csa_version(void);
 
+/*
+ * Synchronises `stream`, then reads and clears the library's device error
+ * word: CSA_OK, or CSA_ERR_TIMEOUT when a bounded device-side wait of a
+ * tensor-core kernel gave up since the last call (the outputs of that launch
+ * are then NaN, never silently wrong).  The word is one int per device held
+ * by the library for its lifetime.
+ */
+int csa_device_error(cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Stage 1: KV compressor                                                    */
 /* ------------------------------------------------------------------------ */

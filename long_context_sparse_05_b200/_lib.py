@@ -80,6 +80,7 @@ _lib = None
 _SIGS = {
     "csa_status_string": (ctypes.c_char_p, [c_int]),
     "csa_version": (c_int, []),
+    "csa_device_error": (c_int, [c_void_p]),
     "csa_compress": (c_int, [ctypes.POINTER(CompressParams)] + [c_void_p] * 6 +
                      [c_int] * 5 + [c_void_p, c_void_p, c_void_p]),
     "csa_quantize": (c_int, [c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
@@ -139,6 +140,11 @@ def _stream(s):
 def _check(status):
     if status != 0:
         raise CsaError(lib().csa_status_string(status).decode())
+
+
+def csa_device_error(stream=None):
+    """Synchronise and read/clear the device error word (0 = no bounded wait gave up)."""
+    return int(lib().csa_device_error(_stream(stream)))
 
 
 def csa_status_string(status):

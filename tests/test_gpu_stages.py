@@ -120,19 +120,21 @@ def test_compress_index_branch_quantised(fmt):
     for s in range(b):
         ref = _oracle_compress(d, s, m, True, E, 64)
         assert_rel_close(f64(out32[s]), ref, 1e-5, "index branch f32")
-        # against the oracle's own entries: a code may move one step only where the float32 and
-        # float64 values straddle a rounding point
+        # against the oracle's own entries: scales agree to float32 rounding of amax, and a code
+        # may move one step only where the float32 and float64 values straddle a rounding point
+        gc, gs = codes[s].cpu().numpy(), sc[s].cpu().numpy()
         if fmt == "fp8":
-            deq = codecs.dequant_fp8_rows(codes[s].cpu().numpy(), sc[s].cpu().numpy())
-            deq_ref = codecs.dequant_fp8_rows(*codecs.quant_fp8_rows(ref.astype(np.float32)))
+            rc, rs = codecs.quant_fp8_rows(ref.astype(np.float32))
+            np.testing.assert_allclose(gs, rs, rtol=1e-5)
+            deq, deq_ref = codecs.dequant_fp8_rows(gc, gs), codecs.dequant_fp8_rows(rc, rs)
+            step = 2.0 ** -3 * np.abs(deq_ref) + 2.0 ** -9 * rs[:, None]   # one E4M3 step
         else:
-            deq = codecs.dequant_nvfp4(codes[s].cpu().numpy(), sc[s].cpu().numpy())
-            deq_ref = codecs.dequant_nvfp4(*codecs.quant_nvfp4(ref.astype(np.float32)))
-        step = np.abs(deq - deq_ref)
-        frac = np.mean(step > 0)
-        assert frac < 0.01, frac
-        lim = 0.13 if fmt == "fp8" else 0.5
-        assert np.all(step <= lim * (np.abs(ref) + 1.0)), np.max(step)
+            rc, rs = codecs.quant_nvfp4(ref.astype(np.float32))
+            assert np.mean(gs != rs) < 0.01
+            deq, deq_ref = codecs.dequant_nvfp4(gc, gs), codecs.dequant_nvfp4(rc, rs)
+            step = np.repeat(codecs.e4m3_decode(rs), 16, axis=1) * 2.0      # widest E2M1 step
+        assert np.mean(gc != rc) < 0.01, np.mean(gc != rc)
+        assert np.all(np.abs(deq - deq_ref) <= step * 1.001 + 1e-12)
 
 
 @pytest.mark.parametrize("fmt", ["fp8", "nvfp4"])
