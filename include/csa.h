@@ -295,7 +295,10 @@ typedef struct {
 
 csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, void* ws,
                       size_t ws_bytes, cudaStream_t stream);
+/* Device workspace csa_decode needs (bytes); host only. */
 size_t csa_decode_workspace_size(const csa_decode_params* p);
+/* Number of kernel launches one csa_decode call makes with these parameters; host only. */
+int csa_decode_launch_count(const csa_decode_params* p);
 
 /*
  * CSA prefill of b sequences of n tokens; every token t = 0..n-1 is a query.
@@ -334,7 +337,10 @@ typedef struct {
 
 csa_status csa_prefill(const csa_prefill_params* p, const csa_prefill_tensors* x, void* ws,
                        size_t ws_bytes, cudaStream_t stream);
+/* Device workspace csa_prefill needs (bytes); host only. */
 size_t csa_prefill_workspace_size(const csa_prefill_params* p);
+/* Number of kernel launches one csa_prefill call makes with these parameters; host only. */
+int csa_prefill_launch_count(const csa_prefill_params* p);
 
 #ifdef __cplusplus
 }

@@ -98,6 +98,8 @@ _SIGS = {
     "csa_prefill": (c_int, [ctypes.POINTER(PrefillParams), ctypes.POINTER(PrefillTensors),
                             c_void_p, c_size_t, c_void_p]),
     "csa_prefill_workspace_size": (c_size_t, [ctypes.POINTER(PrefillParams)]),
+    "csa_decode_launch_count": (c_int, [ctypes.POINTER(DecodeParams)]),
+    "csa_prefill_launch_count": (c_int, [ctypes.POINTER(PrefillParams)]),
 }
 
 
@@ -220,10 +222,10 @@ def csa_prefill(p, tensors, ws, ws_bytes=None, stream=None):
                              _stream(stream)))
 
 
-def attn_launches(H, d, k, dtype):
-    """Kernels one csa_sparse_attn call launches: the tensor-core path (64 heads x 512, bf16)
-    is a split kernel plus a merge; every other shape is one CUDA-core kernel."""
-    return 2 if (H == 64 and d == 512 and dtype == "bf16" and _TC_ATTN) else 1
+
+def csa_decode_launch_count(p):
+    return int(lib().csa_decode_launch_count(ctypes.byref(p)))
 
 
-_TC_ATTN = False
+def csa_prefill_launch_count(p):
+    return int(lib().csa_prefill_launch_count(ctypes.byref(p)))

@@ -191,6 +191,15 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
 
 }  // namespace
 
+int csa_decode_launch_count(const csa_decode_params* p) {
+  if (!p || p->b <= 0) return 0;
+  int n = 2;                                   // positions, latent compressor
+  if (!p->hca) n += 1 + (p->idx_dtype != CSA_F32 ? 1 : 0) + 1 + 1;   // index compressor,
+                                               // quantiser, indexer, top-k
+  n += attn_launch_count(p->H, p->c, p->hca ? 0 : p->k, p->n_w, p->b, 1, p->E_cap, p->kv_dtype);
+  return n;
+}
+
 size_t csa_decode_workspace_size(const csa_decode_params* p) {
   if (!p) return 0;
   return decode_layout(p, nullptr, 0, nullptr);
@@ -287,6 +296,12 @@ size_t prefill_layout(const csa_prefill_params* p, void* ws, size_t cap, Prefill
 }
 
 }  // namespace
+
+int csa_prefill_launch_count(const csa_prefill_params* p) {
+  if (!p || p->b <= 0) return 0;
+  return 1 + 2 + (p->idx_dtype != CSA_F32 ? 1 : 0) + 1 + 1 +
+         attn_launch_count(p->H, p->c, p->k, p->n_w, p->b, p->n, p->n / p->m, p->kv_dtype);
+}
 
 size_t csa_prefill_workspace_size(const csa_prefill_params* p) {
   if (!p) return 0;

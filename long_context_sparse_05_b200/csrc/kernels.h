@@ -46,6 +46,8 @@ csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st);
 csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t ws_bytes,
                           cudaStream_t st);
 size_t attn_tc_workspace_bytes(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype);
+bool attn_tc_supported(int H, int d, int dtype);
+int attn_launch_count(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype);
 
 // Small helpers.
 csa_status launch_fill_i32(int32_t* p, int count, int value, cudaStream_t st);

@@ -181,14 +181,11 @@ def prefill_flops(w: Workload):
     return idx, attn
 
 
+
 def decode_launches_per_step(w: Workload):
-    """Kernels csa_decode launches per step (position fill, compressor(s), quantiser, indexer,
-    top-k, attention and its merge)."""
-    if w.kind == "hca_decode":
-        return 1 + 1 + L.attn_launches(w.H, w.c, 0, w.dtype)
-    return 1 + 2 + 1 + 1 + 1 + L.attn_launches(w.H, w.c, w.k, w.dtype)
+    """Kernels one csa_decode call launches (reported by the library)."""
+    return L.csa_decode_launch_count(decode_params(w))
 
 
 def prefill_launches(w: Workload):
-    q = 0 if w.idx_dtype == "f32" else 1
-    return 1 + 2 + q + 1 + 1 + L.attn_launches(w.H, w.c, w.k, w.dtype)
+    return L.csa_prefill_launch_count(prefill_params(w))

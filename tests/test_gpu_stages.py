@@ -303,3 +303,39 @@ def test_sparse_attention(H, d, k, n_w, dtype, dense, T, E, n):
         else:
             assert_rel_close(f64(out[s]), o, 1e-5, "attention f32")
         assert_abs_close(f64(lse[s]), l, 1e-3 * (1 + np.max(np.abs(l))), "lse")
+
+
+@pytest.mark.parametrize("tile_of_spike", [1, 2])
+def test_attention_lazy_rescale_path(tile_of_spike):
+    """A row far above the first tile's maximum (in a later tile) forces the running-max
+    update and the rescale of the accumulator; the result must still match the oracle."""
+    b, T, H, d, E, n, k, n_w = 1, 3, 64, 512, 600, 2400, 256, 128
+    c = _attn_case(b, T, H, d, E, n, k, n_w, "bf16", False, 61)
+    qpos = c["qpos"]
+    qpos[0, :] = [n - 1, n - 2, 1500]
+    c["qpos"] = qpos
+    rng = np.random.default_rng(5)
+    for t in range(T):
+        scr = rng.normal(size=(1, E))
+        c["idx"][0, t], c["cnt"][0, t] = [a[0] for a in csa.topk(scr, qpos[0, t:t + 1], c["m"], k)]
+    # plant: the selected entry at list position 128 * tile_of_spike + 5 is 30 x q[head 0] / |q|
+    q0 = c["q"][0, 0, 0].float()
+    pos = 128 * tile_of_spike + 5
+    e = int(c["idx"][0, 0, pos]) if pos < k else None
+    if e is None:
+        u = int(qpos[0, 0]) - n_w + 1 + (pos - k)      # window token at list position pos
+        c["win"][0, u] = (30 * q0 / q0.norm()).to(torch.bfloat16)
+    else:
+        c["kv"][0, e] = (30 * q0 / q0.norm()).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(d)
+    out = torch.empty((b, T, H, d), dtype=torch.bfloat16, device=DEV)
+    p = L.AttnParams(H=H, d=d, n_w=n_w, scale=scale, m=c["m"], k=k, dtype=L.CSA_BF16)
+    wsb = L.csa_sparse_attn_workspace_size(p, b, T, E)
+    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    L.csa_sparse_attn(p, c["q"], c["kv"], E, _dev(c["idx"]), _dev(c["cnt"]), c["win"], n,
+                      _dev(c["qpos"]), c["sink"], b, T, out, None, ws, wsb)
+    torch.cuda.synchronize()
+    o, _ = csa.sparse_attn(f64(c["q"][0]), f64(c["kv"][0]), c["idx"][0], c["cnt"][0],
+                           f64(c["win"][0]), c["qpos"][0], f64(c["sink"]), n_w, scale)
+    assert_abs_close(f64(out[0]), o, 2e-2, "attention with rescale")
+    assert L.csa_device_error() == 0
