@@ -47,56 +47,64 @@ def load_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons; ``window`` keeps the samples taken
+    while the timed region ran (host wall-clock bounds), widened to the nearest samples."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.samples = []   # (host time, sm, max, reasons)
 
     def start(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.th = threading.Thread(target=self._read, daemon=True)
             self.th.start()
+            time.sleep(0.5)
         except OSError:
             self.proc = None
 
     def _read(self):
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 10:
+                continue
+            try:
+                sm, mx = float(f[2]), float(f[3])
+            except ValueError:
+                continue
+            rs = [nm for nm, v in zip(names, f[6:10]) if v.lower() == "active"]
+            self.samples.append((time.time(), sm, mx, rs))
 
-    def stop(self):
+    def stop(self, t0, t1):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not inside and self.samples:
+            # the timed region was shorter than the sampling period: nearest samples on each side
+            before = [x for x in self.samples if x[0] < t0][-1:]
+            after = [x for x in self.samples if x[0] > t1][:1]
+            inside = before + after
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        reasons = sorted({r for x in inside for r in x[3]})
+        return {"sm_mhz": float(np.median([x[1] for x in inside])), "sm_max_mhz": inside[-1][2],
+                "reasons": reasons, "samples": len(inside),
+                "timed_region_s": round(t1 - t0, 4)}
 
 
 def dist_setup(n_gpus):
@@ -143,6 +151,8 @@ def timed_loop(fn, steps, flush_buf, stream):
 def bench_decode(w, args, world, rank, peaks):
     dev = "cuda"
     stream = torch.cuda.current_stream()
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
     inp = synth.make_inputs(w, device=dev)
     st = runner.DecodeState(w, inp)
     st.build_caches()
@@ -155,14 +165,14 @@ def bench_decode(w, args, world, rank, peaks):
         step()
     torch.cuda.synchronize()
 
-    clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
     barrier(world)
     torch.cuda.synchronize()
+    t0 = time.time()
     times = timed_loop(step, args.steps, flush, stream)
     torch.cuda.synchronize()
+    t1 = time.time()
     barrier(world)
-    ck = clocks.stop()
+    ck = clocks.stop(t0, t1)
     ms = max_over_ranks(float(np.mean(times)), world)
     tokens_per_step = w.b * world
     value = tokens_per_step / (ms * 1e-3)
@@ -282,15 +292,17 @@ def bench_prefill(w, args, world, rank, peaks):
     inp = synth.make_inputs(w, device="cuda")
     st = runner.PrefillState(w, inp)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    clocks = ClockSampler(torch.cuda.current_device())
+    clocks.start()
     for _ in range(args.warmup):
         st.run(stream)
     torch.cuda.synchronize()
-    clocks = ClockSampler(torch.cuda.current_device())
-    clocks.start()
     barrier(world)
+    t0 = time.time()
     times = timed_loop(lambda: st.run(stream), args.steps, flush, stream)
+    t1 = time.time()
     barrier(world)
-    ck = clocks.stop()
+    ck = clocks.stop(t0, t1)
     ms = max_over_ranks(float(np.mean(times)), world)
     f_idx, f_attn = runner.prefill_flops(w)
     p_fp8 = 2 * peaks["bf16"]
@@ -420,8 +432,8 @@ def cpu_baseline(w, budget_s=20.0):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default=workloads.CSA_DECODE_64K.name,
                     choices=sorted(workloads.ALL))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
