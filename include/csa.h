@@ -247,6 +247,39 @@ csa_status csa_sparse_attn(const csa_attn_params* p, const void* q, const void* 
 
 size_t csa_sparse_attn_workspace_size(const csa_attn_params* p, int b, int T, int E_cap);
 
+/*
+ * csa_sparse_attn for callers that cannot allocate device memory.  Some
+ * callers may not call cudaMalloc at all: a plugin running inside a host
+ * framework that owns every byte of device memory and hands out no allocator,
+ * or a latency-critical decode loop that must never hit cudaMalloc, which can
+ * synchronise the device and has unbounded latency.  This entry point takes
+ * the same arguments as csa_sparse_attn minus the workspace and needs no
+ * allocation: the split partials live in one fixed scratch array inside the
+ * library (a file-scope device array of CSA_NOALLOC_SCRATCH_BYTES), which
+ * every GPU that loads the library holds until the process exits.  The
+ * method on the pages has no counterpart of this; it only changes where the
+ * scratch lives.
+ *
+ *  - The first call on a device (with that device current) looks up the
+ *    array's device address; make that first call before any stream capture.
+ *  - A problem whose workspace (csa_sparse_attn_workspace_size) exceeds
+ *    CSA_NOALLOC_SCRATCH_BYTES is rejected with CSA_ERR_INVALID_ARG and
+ *    nothing is launched.
+ *  - Every call on a device shares the one array, and the array keeps the
+ *    last call's contents: calls that may overlap on the GPU (different
+ *    streams, or several host threads) race on it and must be serialised by
+ *    the caller.  The kernels write every scratch word before reading it, so
+ *    nothing needs clearing between calls.
+ *  - The call allocates nothing: no cudaMalloc, no cudaFree, no allocating
+ *    library routine.
+ */
+#define CSA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+csa_status csa_sparse_attn_noalloc(const csa_attn_params* p, const void* q, const void* kv_comp,
+                                   int E_cap, const int32_t* idx, const int32_t* count,
+                                   const void* kv_win, int n, const int32_t* q_pos,
+                                   const float* sink, int b, int T, void* out, float* lse,
+                                   cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Fused drivers                                                             */
 /* ------------------------------------------------------------------------ */

@@ -92,6 +92,9 @@ _SIGS = {
                                 c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "csa_sparse_attn_workspace_size": (c_size_t, [ctypes.POINTER(AttnParams), c_int, c_int, c_int]),
+    "csa_sparse_attn_noalloc": (c_int, [ctypes.POINTER(AttnParams), c_void_p, c_void_p, c_int,
+                                        c_void_p, c_void_p, c_void_p, c_int, c_void_p, c_void_p,
+                                        c_int, c_int, c_void_p, c_void_p, c_void_p]),
     "csa_decode": (c_int, [ctypes.POINTER(DecodeParams), ctypes.POINTER(DecodeTensors), c_void_p,
                            c_size_t, c_void_p]),
     "csa_decode_workspace_size": (c_size_t, [ctypes.POINTER(DecodeParams)]),
@@ -189,6 +192,17 @@ def csa_sparse_attn(p, q, kv_comp, E_cap, idx, count, kv_win, n, q_pos, sink, b,
     _check(lib().csa_sparse_attn(ctypes.byref(p), _ptr(q), _ptr(kv_comp), E_cap, _ptr(idx),
                                  _ptr(count), _ptr(kv_win), n, _ptr(q_pos), _ptr(sink), b, T,
                                  _ptr(out), _ptr(lse), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def csa_sparse_attn_noalloc(p, q, kv_comp, E_cap, idx, count, kv_win, n, q_pos, sink, b, T, out,
+                            lse=None, stream=None):
+    """csa_sparse_attn without a workspace: the library's fixed scratch array is used."""
+    _check(lib().csa_sparse_attn_noalloc(ctypes.byref(p), _ptr(q), _ptr(kv_comp), E_cap, _ptr(idx),
+                                         _ptr(count), _ptr(kv_win), n, _ptr(q_pos), _ptr(sink), b,
+                                         T, _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def _fill(struct_cls, names, tensors):

@@ -32,6 +32,7 @@
 #include "tc_common.cuh"
 
 #include <climits>
+#include <mutex>
 
 namespace csa {
 
@@ -499,3 +500,51 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
 }
 
 }  // namespace csa
+
+// ---------------------------------------------------------------------------
+// Allocation-free variant: the split partials live in a fixed device array of
+// this file instead of a caller workspace (see csa_sparse_attn_noalloc in csa.h).
+// ---------------------------------------------------------------------------
+namespace csa {
+namespace {
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[CSA_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address must come from the
+// runtime; it is looked up once per device.
+csa_status noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return CSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return CSA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return CSA_ERR_CUDA;
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return CSA_OK;
+}
+
+}  // namespace
+}  // namespace csa
+
+extern "C" csa_status csa_sparse_attn_noalloc(const csa_attn_params* p, const void* q,
+                                              const void* kv_comp, int E_cap, const int32_t* idx,
+                                              const int32_t* count, const void* kv_win, int n,
+                                              const int32_t* q_pos, const float* sink, int b, int T,
+                                              void* out, float* lse, cudaStream_t stream) {
+  if (!p) return CSA_ERR_INVALID_ARG;
+  if (csa_sparse_attn_workspace_size(p, b, T, E_cap) > CSA_NOALLOC_SCRATCH_BYTES)
+    return CSA_ERR_INVALID_ARG;
+  void* scratch = nullptr;
+  const csa_status st = csa::noalloc_scratch(&scratch);
+  if (st != CSA_OK) return st;
+  return csa_sparse_attn(p, q, kv_comp, E_cap, idx, count, kv_win, n, q_pos, sink, b, T, out, lse,
+                         scratch, CSA_NOALLOC_SCRATCH_BYTES, stream);
+}
