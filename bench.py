@@ -438,10 +438,17 @@ def main():
                     choices=sorted(workloads.ALL))
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--context", type=int, default=0,
+                    help="override the context length (profiling of a smaller case, not a bench line)")
+    ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     w = workloads.ALL[args.workload]
+    if args.context:
+        w = workloads.shrink(w, n=args.context)
+    if args.batch:
+        w = workloads.shrink(w, b=args.batch)
     peaks = load_peaks()
 
     if args.impl == "reference":

@@ -124,6 +124,11 @@ csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, i
   if (m < 1 || b < 0 || T < 0 || E < 0 || k < 1) return CSA_ERR_INVALID_ARG;
   if (b == 0 || T == 0) return CSA_OK;
   if (!scores || !q_pos || !idx || !count) return CSA_ERR_INVALID_ARG;
+  if (k <= 32767) {
+    const csa_status st = launch_topk_search(scores, score_dtype, q_pos, m, b * T, E, k, idx, count,
+                                             stream);
+    if (st != CSA_ERR_UNSUPPORTED) return st;
+  }
   return launch_topk(scores, score_dtype, q_pos, m, b * T, E, k, idx, count, stream);
 }
 

@@ -143,6 +143,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(s_flag + 4);
   uint64_t* bar_o = bar_s + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_o + 1);
+  const __nv_bfloat16** s_rows = reinterpret_cast<const __nv_bfloat16**>(tmem_holder + 2);  // [128]
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -226,8 +227,10 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         gather_rows(sQ, kQBlkBytes, kH, warp, lane,
                     [&](int h) { return qb + (size_t)h * kD; }, p.kv);
       }
-      gather_rows(sKV, kKVBlkBytes, kRows, warp, lane,
-                  [&](int rr) { return row_src(p, Q, qrow, j * kRows + rr); }, p.kv);
+      // source of every row of the tile: one coalesced pass over the index list
+      s_rows[r] = row_src(p, Q, qrow, j * kRows + r);
+      tc::named_bar(3, 128);
+      gather_rows(sKV, kKVBlkBytes, kRows, warp, lane, [&](int rr) { return s_rows[rr]; }, p.kv);
       tc::cp_async_wait_all();
       tc::fence_proxy_async();
       tc::tc_fence_before();
@@ -243,7 +246,8 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       tc::tmem_ld_wait(ra);
       tc::reg_fence(rb);
       const int pos = j * kRows + r;
-      const bool valid = row_src(p, Q, qrow, pos) != nullptr;
+      const bool valid = s_rows[r] != nullptr;
+      (void)pos;
       float lg[64], v[64];
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
@@ -371,8 +375,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         p.part_m[(size_t)item * kH + tid] = s_M[tid];
         p.part_l[(size_t)item * kH + tid] = s_l[tid];
       }
-    }
-    tc::tc_fence_before();
+    }    tc::tc_fence_before();
     tc::named_bar(3, 128);                           // s_M / s_l reads done before the next item
   }
 
@@ -385,32 +388,68 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
 }
 
 // Combines the splits of each (query, head): out = sum_s e^{m_s} O_s / (e^{sink} + sum_s e^{m_s} l_s).
+// CTA per (query, 4 heads); thread t owns dims 4t..4t+3 of the 4 heads (float4 loads).
+constexpr int kMergeHeads = 4;
+constexpr int kMaxSplit = 64;
 __global__ void __launch_bounds__(128) attn_merge_kernel(AttnTc p) {
-  const int qrow = blockIdx.x, h = blockIdx.y;
+  __shared__ float s_m[kMaxSplit][kMergeHeads], s_l[kMaxSplit][kMergeHeads];
+  __shared__ float s_w[kMaxSplit][kMergeHeads];
+  const int qrow = blockIdx.x, h0 = blockIdx.y * kMergeHeads;
   const size_t it0 = (size_t)qrow * p.nsplit;
-  float M = p.sink[h] * kLog2e;
-  for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, p.part_m[(it0 + s) * kH + h]);
-  float den = exp2f(p.sink[h] * kLog2e - M);
-  for (int s = 0; s < p.nsplit; ++s) {
-    const float ms = p.part_m[(it0 + s) * kH + h];
-    if (ms == -INFINITY) continue;
-    den += p.part_l[(it0 + s) * kH + h] * exp2f(ms - M);
+  for (int x = threadIdx.x; x < p.nsplit * kMergeHeads; x += blockDim.x) {
+    const int s = x / kMergeHeads, hh = x % kMergeHeads;
+    s_m[s][hh] = __ldcg(&p.part_m[(it0 + s) * kH + h0 + hh]);
+    s_l[s][hh] = __ldcg(&p.part_l[(it0 + s) * kH + h0 + hh]);
   }
-  const float inv = 1.f / den;
-  for (int d = threadIdx.x; d < kD; d += blockDim.x) {
-    float acc = 0.f;
+  __syncthreads();
+  if (threadIdx.x < kMergeHeads) {
+    const int hh = threadIdx.x;
+    const float sink2 = p.sink[h0 + hh] * kLog2e;
+    float M = sink2;
+    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, s_m[s][hh]);
+    float den = exp2f(sink2 - M);
     for (int s = 0; s < p.nsplit; ++s) {
-      const float ms = p.part_m[(it0 + s) * kH + h];
-      if (ms == -INFINITY) continue;
-      acc = fmaf(p.part_o[((it0 + s) * kH + h) * kD + d], exp2f(ms - M), acc);
+      const float e = s_m[s][hh] == -INFINITY ? 0.f : exp2f(s_m[s][hh] - M);
+      s_w[s][hh] = e;
+      den += s_l[s][hh] * e;
     }
-    p.out[((size_t)qrow * kH + h) * kD + d] = __float2bfloat16_rn(acc * inv);
+    const float inv = 1.f / den;
+    for (int s = 0; s < p.nsplit; ++s) s_w[s][hh] *= inv;
+    if (p.lse) p.lse[(size_t)qrow * kH + h0 + hh] = (M + log2f(den)) * 0.6931471805599453f;
   }
-  if (p.lse && threadIdx.x == 0) p.lse[(size_t)qrow * kH + h] = (M + log2f(den)) * 0.6931471805599453f;
+  __syncthreads();
+  const int d = threadIdx.x * 4;
+  float4 acc[kMergeHeads];
+#pragma unroll
+  for (int hh = 0; hh < kMergeHeads; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < p.nsplit; ++s) {
+    float4 v[kMergeHeads];
+#pragma unroll
+    for (int hh = 0; hh < kMergeHeads; ++hh)
+      v[hh] = s_w[s][hh] != 0.f
+                  ? __ldcg(reinterpret_cast<const float4*>(
+                        &p.part_o[((it0 + s) * kH + h0 + hh) * kD + d]))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int hh = 0; hh < kMergeHeads; ++hh) {
+      const float w = s_w[s][hh];
+      acc[hh].x = fmaf(v[hh].x, w, acc[hh].x); acc[hh].y = fmaf(v[hh].y, w, acc[hh].y);
+      acc[hh].z = fmaf(v[hh].z, w, acc[hh].z); acc[hh].w = fmaf(v[hh].w, w, acc[hh].w);
+    }
+  }
+#pragma unroll
+  for (int hh = 0; hh < kMergeHeads; ++hh) {
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc[hh].x, acc[hh].y);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc[hh].z, acc[hh].w);
+    uint2 u;
+    u.x = *reinterpret_cast<uint32_t*>(&lo);
+    u.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(&p.out[((size_t)qrow * kH + h0 + hh) * kD + d]) = u;
+  }
 }
 
 constexpr size_t kSmemBytes = 1024 + 8 * kKVBlkBytes + 8 * kQBlkBytes + kRows * 128 +
-                              (4 * kH + 4 * kH) * 4 + 16 + 16 + 16;
+                              (4 * kH + 4 * kH) * 4 + 16 + 16 + 16 + kRows * 8;
 
 struct Plan {
   int nsplit, tps;
@@ -481,6 +520,7 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
     const size_t items = (size_t)b * a.T * P.nsplit;
     const size_t need = items * kH * kD * 4 + 2 * items * kH * 4;
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15)) return CSA_ERR_INVALID_ARG;
+    if (P.nsplit > kMaxSplit) return CSA_ERR_UNSUPPORTED;
     p.part_o = reinterpret_cast<float*>(ws);
     p.part_m = p.part_o + items * kH * kD;
     p.part_l = p.part_m + items * kH;
@@ -493,7 +533,7 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
   attn_tc_kernel<<<grid, 160, kSmemBytes, st>>>(p);
   CSA_CHECK_LAUNCH();
   if (P.nsplit > 1) {
-    attn_merge_kernel<<<dim3(b * a.T, kH), 128, 0, st>>>(p);
+    attn_merge_kernel<<<dim3(b * a.T, kH / kMergeHeads), 128, 0, st>>>(p);
     CSA_CHECK_LAUNCH();
   }
   return CSA_OK;

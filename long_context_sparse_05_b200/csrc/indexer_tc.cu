@@ -9,23 +9,27 @@
 // CUDA-core kernel.
 //
 // The score of one (query, entry) pair needs all 64 heads, so the tensor-core
-// product is laid out with entries on M (TMEM lanes) and heads on N (TMEM
-// columns): D[s, (q, j)] = K[s] . Q[q, j], M = 128 entries, N = 64 x QG
-// queries, K = 128 (four MMAs of K = 32).  Each epilogue thread then owns one
-// entry and forms sum_j w[q,j] qs[q,j] ReLU(D[s,(q,j)]) * ks[s] in registers,
-// with no cross-thread reduction (ReLU commutes with the positive scales).
+// product puts entries on M (TMEM lanes) and heads on N (TMEM columns):
+// D[s, (q, j)] = K[s] . Q[q, j], M = 128 entries, N = 64 x QG queries, K = 128
+// (four MMAs of K = 32).  Each epilogue thread owns one entry and forms
+// sum_j (w qs)[q,j] ReLU(D[s,(q,j)]) * ks[s] in registers (ReLU commutes with the
+// positive scales): no cross-thread reduction.
 //
 // Persistent, warp-specialised CTA (192 threads):
-//   warp 0  TMA producer: key tiles [128 x 128 B] through an S-stage ring and
-//           the query group [64 QG x 128 B] once per work unit (2 buffers);
+//   warp 0  TMA producer: per tile the 128 x 128 B key block (128-byte swizzle)
+//           and its 128 fp32 key scales into an S-stage ring; per work unit the
+//           query group (64 QG x 128 B), its head weights and query scales into
+//           one of two buffers;
 //   warp 1  MMA issuer (one thread): 4 x tcgen05.mma kind::f8f6f4 per tile into
-//           one of two TMEM accumulators, commits release the smem stage and
-//           hand the accumulator to the epilogue;
+//           one of NACC TMEM accumulators;
 //   warps 2-5 epilogue: tcgen05.ld of the accumulator, the weighted ReLU sum,
 //           the causal mask, bf16 / fp32 store; tiles no query of the group can
 //           see are written as -inf without any MMA.
+// Every operand the epilogue needs arrives by TMA with its tile, so no thread
+// waits on global memory inside the loop.  A stage is released when the MMAs
+// have read the keys and all four epilogue warps have read the key scales.
 // A work unit is (sequence, query group, chunk of entry tiles); units are dealt
-// round-robin to the persistent CTAs, and every role walks the same sequence.
+// round-robin to the CTAs and their causal extents are computed once, at start.
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -37,105 +41,124 @@ constexpr int kTileE = 128;          // entries per tile (MMA M)
 constexpr int kHeads = 64;           // index heads
 constexpr int kDim = 128;            // index dim (bytes per FP8 row)
 constexpr int kTileBytes = kTileE * kDim;
+constexpr int kMaxLocalUnits = 256;  // units one CTA walks (grid is sized to respect it)
 
 struct IdxTc {
-  const float* w;
-  const float* q_scales;
-  const float* k_scales;
-  const int32_t* q_pos;
   void* scores;
+  const int32_t* q_pos;
   int* err;
   int T, E_cap, E, m;
   int n_qg, tiles, chunk, n_chunks, units;
   int score_f32;
 };
 
-struct Unit {
-  int sb, g, j0, j1, vis_tiles, nq;
+template <int QG>
+struct Layout {
+  static constexpr int N = kHeads * QG;
+  static constexpr int NACC = QG == 1 ? 4 : 2;
+  static constexpr int kQBytes = N * kDim;
+  static constexpr uint32_t kTmemCols = NACC * N <= 32 ? 32 : NACC * N <= 64 ? 64 :
+                                        NACC * N <= 128 ? 128 : NACC * N <= 256 ? 256 : 512;
 };
-
-template <int QG>
-__device__ __forceinline__ Unit decode_unit(const IdxTc& p, int u) {
-  Unit U;
-  const int ch = u % p.n_chunks;
-  const int tmp = u / p.n_chunks;
-  U.g = tmp % p.n_qg;
-  U.sb = tmp / p.n_qg;
-  U.j0 = ch * p.chunk;
-  U.j1 = min(p.tiles, U.j0 + p.chunk);
-  U.nq = min(QG, p.T - U.g * QG);
-  int ev = 0;
-  for (int q = 0; q < U.nq; ++q)
-    ev = max(ev, visible_entries(p.q_pos[(size_t)U.sb * p.T + U.g * QG + q], p.m, p.E));
-  U.vis_tiles = (ev + kTileE - 1) / kTileE;
-  return U;
-}
-
-template <int QG>
-__device__ __forceinline__ int computed_tiles(const Unit& U) {
-  return max(0, min(U.j1, U.vis_tiles) - U.j0);
-}
 
 template <int QG, int S>
 __global__ void __launch_bounds__(192, 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                       IdxTc p) {
-  constexpr int N = kHeads * QG;
-  constexpr int kQBytes = N * kDim;
-  constexpr uint32_t kTmemCols = (2 * N <= 32) ? 32 : (2 * N <= 64 ? 64 : (2 * N <= 128 ? 128 : (2 * N <= 256 ? 256 : 512)));
+                       const __grid_constant__ CUtensorMap tmKS, const __grid_constant__ CUtensorMap tmW,
+                       const __grid_constant__ CUtensorMap tmQS, IdxTc p) {
+  using LY = Layout<QG>;
+  constexpr int N = LY::N;
+  constexpr int NACC = LY::NACC;
+  constexpr int kQBytes = LY::kQBytes;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sA = base;                                   // S x 16 KB
-  uint8_t* sB = sA + S * kTileBytes;                    // 2 x kQBytes
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sB + 2 * kQBytes);
+  uint8_t* sA = base;                                         // S x 16 KB key tiles
+  float* sKS = reinterpret_cast<float*>(sA + S * kTileBytes); // S x 128 key scales
+  uint8_t* sB = reinterpret_cast<uint8_t*>(sKS + S * kTileE); // 2 x kQBytes query groups
+  float* sW = reinterpret_cast<float*>(sB + 2 * kQBytes);     // 2 x N head weights
+  float* sQS = sW + 2 * N;                                    // 2 x N query scales
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sQS + 2 * N);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
   uint64_t* bfull = bars + 2 * S;
   uint64_t* bempty = bfull + 2;
   uint64_t* tfull = bempty + 2;
-  uint64_t* tempty = tfull + 2;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + 2);
-  float* s_wq = reinterpret_cast<float*>(tmem_holder + 4);   // [QG][64]
+  uint64_t* tempty = tfull + NACC;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + NACC);
+  float* s_wq = reinterpret_cast<float*>(tmem_holder + 4);    // [N] w * qs of the current unit
+  int* s_vis = reinterpret_cast<int*>(s_wq + N);              // [kMaxLocalUnits] visible tiles
+  int* s_ev = s_vis + kMaxLocalUnits;                         // [kMaxLocalUnits][QG] visible entries
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bfull[i], 1); tc::mbar_init(&bempty[i], 1);
-      tc::mbar_init(&tfull[i], 1); tc::mbar_init(&tempty[i], 4);
+  // causal extent of every unit this CTA will walk
+  for (int i = threadIdx.x; i * (int)gridDim.x + (int)blockIdx.x < p.units && i < kMaxLocalUnits;
+       i += blockDim.x) {
+    const int u = blockIdx.x + i * gridDim.x;
+    const int tmp = u / p.n_chunks;
+    const int g = tmp % p.n_qg, sb = tmp / p.n_qg;
+    const int nq = min(QG, p.T - g * QG);
+    int evmax = 0;
+    for (int q = 0; q < QG; ++q) {
+      const int ev = q < nq ? visible_entries(p.q_pos[(size_t)sb * p.T + g * QG + q], p.m, p.E) : 0;
+      s_ev[i * QG + q] = ev;
+      evmax = max(evmax, ev);
     }
+    s_vis[i] = (evmax + kTileE - 1) / kTileE;
+  }
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < S; ++i) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], 1 + 4); }
+    for (int i = 0; i < 2; ++i) { tc::mbar_init(&bfull[i], 1); tc::mbar_init(&bempty[i], 1 + 4); }
+    for (int i = 0; i < NACC; ++i) { tc::mbar_init(&tfull[i], 1); tc::mbar_init(&tempty[i], 4); }
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tmK);
     tc::tma_prefetch_desc(&tmQ);
+    tc::tma_prefetch_desc(&tmKS);
   }
-  if (warp == 0) tc::tmem_alloc(tmem_holder, kTmemCols);
+  if (warp == 0) tc::tmem_alloc(tmem_holder, LY::kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
+
+  // per-unit geometry shared by all roles
+  auto unit = [&](int u, int i, int& sb, int& g, int& j0, int& j1, int& nc, int& nq) {
+    const int ch = u % p.n_chunks;
+    const int tmp = u / p.n_chunks;
+    g = tmp % p.n_qg;
+    sb = tmp / p.n_qg;
+    j0 = ch * p.chunk;
+    j1 = min(p.tiles, j0 + p.chunk);
+    nq = min(QG, p.T - g * QG);
+    nc = max(0, min(j1, s_vis[i]) - j0);
+  };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       uint32_t it = 0, ul = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        const Unit U = decode_unit<QG>(p, u);
-        const int nc = computed_tiles<QG>(U);
+      for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
+        int sb, g, j0, j1, nc, nq;
+        unit(u, i, sb, g, j0, j1, nc, nq);
         if (nc == 0) continue;
         const int bb = ul & 1;
         ok = tc::mbar_wait(&bempty[bb], ((ul >> 1) & 1) ^ 1, p.err);
         if (!ok) break;
-        tc::mbar_arrive_expect_tx(&bfull[bb], kQBytes);
-        tc::tma_load_2d(sB + bb * kQBytes, &tmQ, 0, (U.sb * p.T + U.g * QG) * kHeads, &bfull[bb]);
-        for (int j = U.j0; j < U.j0 + nc; ++j, ++it) {
+        const int qrow0 = (sb * p.T + g * QG) * kHeads;
+        tc::mbar_arrive_expect_tx(&bfull[bb], kQBytes + 2 * N * 4);
+        tc::tma_load_2d(sB + bb * kQBytes, &tmQ, 0, qrow0, &bfull[bb]);
+        tc::tma_load_1d(sW + bb * N, &tmW, qrow0, &bfull[bb]);
+        tc::tma_load_1d(sQS + bb * N, &tmQS, qrow0, &bfull[bb]);
+        for (int j = j0; j < j0 + nc; ++j, ++it) {
           const int s = it % S;
           ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
           if (!ok) break;
-          tc::mbar_arrive_expect_tx(&full[s], kTileBytes);
-          tc::tma_load_2d(sA + s * kTileBytes, &tmK, 0, U.sb * p.E_cap + j * kTileE, &full[s]);
+          const int row0 = sb * p.E_cap + j * kTileE;
+          tc::mbar_arrive_expect_tx(&full[s], kTileBytes + kTileE * 4);
+          tc::tma_load_2d(sA + s * kTileBytes, &tmK, 0, row0, &full[s]);
+          tc::tma_load_1d(sKS + s * kTileE, &tmKS, row0, &full[s]);
         }
         ++ul;
       }
@@ -146,9 +169,9 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
       constexpr uint32_t idesc = tc::instr_desc(kTileE, N, 0, 0, 0, 0);   // e4m3 x e4m3 -> f32
       uint32_t it = 0, ul = 0, at = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.units && ok; u += gridDim.x) {
-        const Unit U = decode_unit<QG>(p, u);
-        const int nc = computed_tiles<QG>(U);
+      for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
+        int sb, g, j0, j1, nc, nq;
+        unit(u, i, sb, g, j0, j1, nc, nq);
         if (nc == 0) continue;
         const int bb = ul & 1;
         ok = tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
@@ -156,10 +179,10 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(sB + bb * kQBytes), 16, 1024);
         for (int j = 0; j < nc; ++j, ++it, ++at) {
           const int s = it % S;
-          const int acc = at & 1;
+          const int acc = at % NACC;
           ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err);
           if (!ok) break;
-          ok = tc::mbar_wait(&tempty[acc], ((at >> 1) & 1) ^ 1, p.err);
+          ok = tc::mbar_wait(&tempty[acc], ((at / NACC) & 1) ^ 1, p.err);
           if (!ok) break;
           tc::tc_fence_after();
           const uint64_t adesc = tc::smem_desc_sw128(tc::smem_u32(sA + s * kTileBytes), 16, 1024);
@@ -177,33 +200,36 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     }
   } else {
     // -------------------------------------------------------------- epilogue
-    const int ew = warp - 2;                 // 0..3
     const int lane_base = (warp & 3) * 32;   // TMEM lanes this warp may access
     const int etid = threadIdx.x - 64;       // 0..127
-    uint32_t at = 0;
+    uint32_t it = 0, at = 0, ul = 0;
     bool ok = true;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-      const Unit U = decode_unit<QG>(p, u);
-      tc::named_bar(1, 128);
-      for (int x = etid; x < U.nq * kHeads; x += 128) {
-        const size_t r = ((size_t)U.sb * p.T + U.g * QG) * kHeads + x;
-        s_wq[x] = p.w[r] * p.q_scales[r];
+    for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
+      int sb, g, j0, j1, nc, nq;
+      unit(u, i, sb, g, j0, j1, nc, nq);
+      if (nc > 0) {
+        const int bb = ul & 1;
+        tc::named_bar(1, 128);                         // previous unit's s_wq no longer read
+        ok = ok && tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
+        for (int x = etid; x < N; x += 128) s_wq[x] = sW[bb * N + x] * sQS[bb * N + x];
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bempty[bb]);
+        tc::named_bar(1, 128);
+        ++ul;
       }
-      tc::named_bar(1, 128);
-      int tq[QG], evq[QG];
-#pragma unroll
-      for (int q = 0; q < QG; ++q) {
-        tq[q] = q < U.nq ? U.g * QG + q : 0;
-        evq[q] = q < U.nq ? visible_entries(p.q_pos[(size_t)U.sb * p.T + tq[q]], p.m, p.E) : 0;
-      }
-      for (int j = U.j0; j < U.j1; ++j) {
+      for (int j = j0; j < j1; ++j) {
         const int e = j * kTileE + lane_base + lane;
         float sc[QG];
-        if (j < U.vis_tiles && ok) {
-          const int acc = at & 1;
-          ok = tc::mbar_wait(&tfull[acc], (at >> 1) & 1, p.err);
+        const bool computed = j < j0 + nc;
+        if (computed && ok) {
+          const int s = it % S;
+          const int acc = at % NACC;
+          ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err);   // the stage's key scales landed
+          const float ks = sKS[s * kTileE + lane_base + lane];
+          __syncwarp();
+          if (lane == 0) tc::mbar_arrive(&empty[s]);
+          ok = ok && tc::mbar_wait(&tfull[acc], (at / NACC) & 1, p.err);
           tc::tc_fence_after();
-          const float ks = (e < p.E) ? p.k_scales[(size_t)U.sb * p.E_cap + e] : 0.f;
 #pragma unroll
           for (int q = 0; q < QG; ++q) {
             uint32_t r0[32], r1[32];
@@ -223,6 +249,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
           tc::tc_fence_before();
           __syncwarp();
           if (lane == 0) tc::mbar_arrive(&tempty[acc]);
+          ++it;
           ++at;
         } else {
 #pragma unroll
@@ -231,15 +258,15 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         if (e < p.E) {
 #pragma unroll
           for (int q = 0; q < QG; ++q) {
-            if (q >= U.nq) break;
-            const float v = (e < evq[q] && ok) ? sc[q] : (ok ? -INFINITY : __int_as_float(0x7fc00000));
-            const size_t o = ((size_t)U.sb * p.T + tq[q]) * p.E + e;
+            if (q >= nq) break;
+            const int ev = s_ev[i * QG + q];
+            const float v = !ok ? __int_as_float(0x7fc00000) : (e < ev ? sc[q] : -INFINITY);
+            const size_t o = ((size_t)sb * p.T + g * QG + q) * p.E + e;
             if (p.score_f32) reinterpret_cast<float*>(p.scores)[o] = v;
             else reinterpret_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(v);
           }
         }
       }
-      (void)ew;
     }
   }
 
@@ -247,22 +274,26 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   __syncthreads();
   if (warp == 0) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem_base, kTmemCols);
+    tc::tmem_dealloc(tmem_base, LY::kTmemCols);
   }
 }
 
 template <int QG, int S>
 csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
-  CUtensorMap tmK, tmQ;
-  if (!make_tmap_2d_u8(&tmK, a.k, kDim, (uint64_t)b * a.E_cap, kDim, kTileE)) return CSA_ERR_CUDA;
-  if (!make_tmap_2d_u8(&tmQ, a.q, kDim, (uint64_t)b * a.T * kHeads, kDim, kHeads * QG))
+  using LY = Layout<QG>;
+  CUtensorMap tmK, tmQ, tmKS, tmW, tmQS;
+  const uint64_t qrows = (uint64_t)b * a.T * kHeads;
+  if (!make_tmap_2d_u8(&tmK, a.k, kDim, (uint64_t)b * a.E_cap, kDim, kTileE) ||
+      !make_tmap_2d_u8(&tmQ, a.q, kDim, qrows, kDim, LY::N) ||
+      !make_tmap_1d_f32(&tmKS, a.k_scales, (uint64_t)b * a.E_cap, kTileE) ||
+      !make_tmap_1d_f32(&tmW, a.w, qrows, LY::N) ||
+      !make_tmap_1d_f32(&tmQS, a.q_scales, qrows, LY::N))
     return CSA_ERR_CUDA;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   IdxTc p{};
-  p.w = a.w; p.q_scales = reinterpret_cast<const float*>(a.q_scales);
-  p.k_scales = reinterpret_cast<const float*>(a.k_scales); p.q_pos = a.q_pos; p.scores = a.scores;
+  p.scores = a.scores; p.q_pos = a.q_pos;
   p.err = device_error_word();
   if (!p.err) return CSA_ERR_CUDA;
   p.T = a.T; p.E_cap = a.E_cap; p.E = a.E; p.m = a.m;
@@ -278,14 +309,17 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   if (units > 0x7fffffff) return CSA_ERR_UNSUPPORTED;
   p.units = (int)units;
   p.score_f32 = a.score_dtype == CSA_F32;
-  const size_t smem = 1024 + (size_t)S * kTileBytes + 2 * (size_t)kHeads * QG * kDim +
-                      (2 * S + 8) * 8 + 16 + QG * kHeads * 4;
+  long long grid = units < sms ? units : sms;
+  const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
+  if (grid < min_grid) grid = min_grid;
+  const size_t smem = 1024 + (size_t)S * (kTileBytes + kTileE * 4) + 2 * (size_t)LY::kQBytes +
+                      4 * (size_t)LY::N * 4 + (2 * S + 4 + 2 * LY::NACC) * 8 + 16 +
+                      (size_t)LY::N * 4 + (size_t)kMaxLocalUnits * (1 + QG) * 4;
   auto kern = index_scores_tc_kernel<QG, S>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  const int grid = (int)(units < sms ? units : sms);
-  kern<<<grid, 192, smem, st>>>(tmK, tmQ, p);
+  kern<<<(int)grid, 192, smem, st>>>(tmK, tmQ, tmKS, tmW, tmQS, p);
   CSA_CHECK_LAUNCH();
   return CSA_OK;
 }
@@ -294,8 +328,10 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
 
 csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st) {
   if (a.qk_dtype != CSA_FP8_E4M3 || a.H != kHeads || a.d != kDim) return CSA_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.q) & 15))
-    return CSA_ERR_UNSUPPORTED;
+  if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.q) & 15) ||
+      (reinterpret_cast<uintptr_t>(a.k_scales) & 15) || (reinterpret_cast<uintptr_t>(a.w) & 15) ||
+      (reinterpret_cast<uintptr_t>(a.q_scales) & 15) || (a.E_cap % 4))
+    return CSA_ERR_UNSUPPORTED;   // the TMA copies need 16-byte aligned rows and scale runs
   if (a.T >= 4) return launch_qg<4, 4>(a, b, st);
   return launch_qg<1, 8>(a, b, st);
 }

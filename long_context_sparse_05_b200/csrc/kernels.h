@@ -34,6 +34,8 @@ csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry
                            cudaStream_t st);
 csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
                            void* codes, void* scales, cudaStream_t st);
+csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
+                              int rows, int E, int k, int32_t* idx, int32_t* count, cudaStream_t st);
 csa_status launch_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int rows,
                        int E, int k, int32_t* idx, int32_t* count, cudaStream_t st);
 

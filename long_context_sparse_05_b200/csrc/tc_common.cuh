@@ -85,6 +85,15 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int
         "r"(smem_u32(bar)) : "memory");
 }
 
+// 1-D tiled load (a run of `box` elements) into shared memory.
+__device__ __forceinline__ void tma_load_1d(void* dst, const CUtensorMap* m, int x, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.1d.shared::cluster.global.mbarrier::complete_tx::bytes "
+      "[%0], [%1, {%2}], [%3];"
+      ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------- TMEM
 // Whole warp: allocate `ncols` (power of two >= 32) TMEM columns; the base
 // address is written to *dst (shared memory).
@@ -226,6 +235,8 @@ int* device_error_word();
 // [rows][row_bytes] with a box of [box_rows][box_bytes] and 128-byte swizzle.
 bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
                      uint32_t box_bytes, uint32_t box_rows);
+// 1-D map over `n` float32 values with a box of `box` values (no swizzle).
+bool make_tmap_1d_f32(CUtensorMap* m, const void* base, uint64_t n, uint32_t box);
 // Same for 16-bit elements: [rows][cols] with a box of [box_rows][box_cols].
 bool make_tmap_2d_b16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
                       uint32_t box_cols, uint32_t box_rows);

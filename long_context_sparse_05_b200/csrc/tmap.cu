@@ -60,6 +60,19 @@ bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint6
                 box_rows);
 }
 
+bool make_tmap_1d_f32(CUtensorMap* m, const void* base, uint64_t n, uint32_t box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[1] = {n};
+  cuuint64_t strides[1] = {4};   // unused for rank 1
+  cuuint32_t bx[1] = {box};
+  cuuint32_t es[1] = {1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 1, const_cast<void*>(base), dims, strides, bx,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_2d_b16(CUtensorMap* m, const void* base, uint64_t cols, uint64_t rows,
                       uint32_t box_cols, uint32_t box_rows) {
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, base, cols, rows, cols * 2, box_cols,
