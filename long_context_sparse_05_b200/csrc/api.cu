@@ -198,9 +198,8 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
 
 int csa_decode_launch_count(const csa_decode_params* p) {
   if (!p || p->b <= 0) return 0;
-  int n = 2;                                   // positions, latent compressor
-  if (!p->hca) n += 1 + (p->idx_dtype != CSA_F32 ? 1 : 0) + 1 + 1;   // index compressor,
-                                               // quantiser, indexer, top-k
+  int n = 1;                                   // prologue: compressors, quantiser, positions
+  if (!p->hca) n += 2;                         // indexer, top-k
   n += attn_launch_count(p->H, p->c, p->hca ? 0 : p->k, p->n_w, p->b, 1, p->E_cap, p->kv_dtype);
   return n;
 }
@@ -223,39 +222,59 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
   if (need == 0 || !ws || ws_bytes < csa_decode_workspace_size(p)) return CSA_ERR_INVALID_ARG;
   const int b = p->b;
   const int t = p->L - 1;
-  csa_status st = launch_fill_i32(d.qpos, b, t, stream);
-  if (st) return st;
+  if (!x->C_a || !x->Z_a || !x->B_a || !x->kv_cache || !x->q || !x->kv_win || !x->sink || !x->out)
+    return CSA_ERR_INVALID_ARG;
+  if (!p->hca && (!x->C_b || !x->Z_b || !x->B_b || !x->CI_a || !x->ZI_a || !x->BI_a || !x->CI_b ||
+                  !x->ZI_b || !x->BI_b || !x->kI_cache || !x->q_I || !x->w))
+    return CSA_ERR_INVALID_ARG;
+  if (!p->hca && p->idx_dtype != CSA_F32 && !x->kI_scales) return CSA_ERR_INVALID_ARG;
+  if (p->kv_dtype != CSA_F32 && p->kv_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  if (!p->hca && p->idx_dtype == CSA_F32 && p->kv_dtype != CSA_F32) return CSA_ERR_UNSUPPORTED;
+  if (p->c < 8 || p->c % 8 || p->d_rope < 0 || p->d_rope % 2 || p->d_rope > p->c)
+    return CSA_ERR_INVALID_ARG;
+  if (!p->hca && (p->c_I % 16 || p->d_rope_I < 0 || p->d_rope_I % 2 || p->d_rope_I > p->c_I))
+    return CSA_ERR_INVALID_ARG;
+  if (!aligned16(x->C_a) || !aligned16(x->Z_a) ||
+      (!p->hca && (!aligned16(x->C_b) || !aligned16(x->Z_b) || !aligned16(x->CI_a) ||
+                   !aligned16(x->ZI_a) || !aligned16(x->CI_b) || !aligned16(x->ZI_b))))
+    return CSA_ERR_INVALID_ARG;
 
-  // 1. compress the entry the new token completes (latent, then index key)
-  csa_compress_params cp{p->m, p->hca ? 0 : 1, p->c, p->d_rope, p->rope_theta, p->eps, 1,
-                         p->kv_dtype, p->kv_dtype};
-  st = csa_compress(&cp, x->C_a, x->Z_a, x->B_a, x->C_b, x->Z_b, x->B_b, b, p->L, E - 1, 1,
-                    p->E_cap, x->kv_cache, nullptr, stream);
+  // 1-2. one prologue launch: compress the entry the new token completes (latent and
+  //      index key), quantise the index queries, write the query positions
+  PrologueArgs pa{};
+  pa.main.C_a = x->C_a; pa.main.Z_a = x->Z_a; pa.main.B_a = x->B_a;
+  pa.main.C_b = x->C_b; pa.main.Z_b = x->Z_b; pa.main.B_b = x->B_b;
+  pa.main.n = p->L; pa.main.m = p->m; pa.main.overlap = p->hca ? 0 : 1; pa.main.c = p->c;
+  pa.main.d_rope = p->d_rope; pa.main.apply_norm = 1; pa.main.out_dtype = p->kv_dtype;
+  pa.main.entry_begin = E - 1; pa.main.out_E = p->E_cap; pa.main.theta = p->rope_theta;
+  pa.main.eps = p->eps; pa.main.out = x->kv_cache; pa.main.out_scales = nullptr;
+  pa.nbranch = p->hca ? 1 : 2;
+  pa.b = b; pa.t = t; pa.qpos = d.qpos;
+  const void* qI = x->q_I;
+  const void* qs = nullptr;
+  if (!p->hca) {
+    pa.index = pa.main;
+    pa.index.C_a = x->CI_a; pa.index.Z_a = x->ZI_a; pa.index.B_a = x->BI_a;
+    pa.index.C_b = x->CI_b; pa.index.Z_b = x->ZI_b; pa.index.B_b = x->BI_b;
+    pa.index.c = p->c_I; pa.index.d_rope = p->d_rope_I; pa.index.out_dtype = p->idx_dtype;
+    pa.index.out = x->kI_cache; pa.index.out_scales = x->kI_scales;
+    if (p->idx_dtype != CSA_F32) {
+      pa.q_in = x->q_I; pa.q_rows = b * p->H_I; pa.q_d = p->c_I; pa.q_dtype = p->idx_dtype;
+      pa.q_codes = static_cast<uint8_t*>(d.qI_codes); pa.q_scales = d.qI_scales;
+      qI = d.qI_codes; qs = d.qI_scales;
+    }
+  }
+  csa_status st = launch_decode_prologue(pa, p->kv_dtype, stream);
   if (st) return st;
   const int32_t* idx = nullptr;
   const int32_t* cnt = nullptr;
   if (!p->hca) {
-    csa_compress_params ci{p->m, 1, p->c_I, p->d_rope_I, p->rope_theta, p->eps, 1, p->kv_dtype,
-                           p->idx_dtype};
-    st = csa_compress(&ci, x->CI_a, x->ZI_a, x->BI_a, x->CI_b, x->ZI_b, x->BI_b, b, p->L, E - 1, 1,
-                      p->E_cap, x->kI_cache, x->kI_scales, stream);
-    if (st) return st;
-    // 2. quantise the index queries, score all entries
-    const void* qI = x->q_I;
-    const void* qs = nullptr;
-    if (p->idx_dtype != CSA_F32) {
-      st = csa_quantize(p->kv_dtype, p->idx_dtype, x->q_I, b * p->H_I, p->c_I, d.qI_codes,
-                        d.qI_scales, stream);
-      if (st) return st;
-      qI = d.qI_codes; qs = d.qI_scales;
-    } else if (p->kv_dtype != CSA_F32) {
-      return CSA_ERR_UNSUPPORTED;
-    }
+    // 3. score all entries
     csa_index_params ip{p->H_I, p->c_I, p->m, p->idx_dtype, CSA_BF16};
     st = csa_index_scores(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, 1, p->E_cap, E,
                           d.scores, stream);
     if (st) return st;
-    // 3. top-k
+    // 4. top-k
     int32_t* io = x->idx_out ? x->idx_out : d.idx;
     int32_t* co = x->count_out ? x->count_out : d.count;
     st = csa_topk(d.scores, CSA_BF16, d.qpos, p->m, b, 1, E, p->k, io, co, nullptr, 0, stream);

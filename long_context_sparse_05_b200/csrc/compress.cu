@@ -15,6 +15,9 @@
 #include "common.cuh"
 #include "kernels.h"
 
+#include <algorithm>
+#include <cmath>
+
 namespace csa {
 
 template <typename InT>
@@ -40,18 +43,27 @@ __device__ __forceinline__ void load16(const InT* p, float* dst) {
 
 constexpr int kUnroll = 4;
 
+// Rotation angle p * inv_freq reduced to [-pi, pi] in float64 (Cody-Waite reduction
+// with 2*pi split into a head and a tail), then float32 sin / cos of the reduced angle.
+__device__ __forceinline__ void rope_angle(double ang, float* sn, float* cs) {
+  const double kTwoPiHi = 6.283185307179586;          // 2*pi rounded to float64
+  const double kTwoPiLo = 2.4492935982947064e-16;     // 2*pi - kTwoPiHi
+  const double k = rint(ang * (1.0 / 6.283185307179586));
+  double r = fma(-k, kTwoPiHi, ang);
+  r = fma(-k, kTwoPiLo, r);
+  sincosf((float)r, sn, cs);
+}
+
+// One compressed entry (entry i of sequence s) by the whole CTA; see compress_kernel.
 template <typename InT>
-__global__ void __launch_bounds__(512) compress_kernel(CompressArgs a) {
+__device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int s, float* smem) {
   constexpr int VEC = Vec16<InT>::N;
-  extern __shared__ float smem[];
   const int c = a.c;
   const int cols = c / VEC;
   const int rg = blockDim.x / cols;
   const int tid = threadIdx.x;
   const int cc = tid % cols;
   const int g = tid / cols;
-  const int i = a.entry_begin + blockIdx.x;
-  const int s = blockIdx.y;
   const int m = a.m;
   const int R = a.overlap ? 2 * m : m;
 
@@ -156,13 +168,13 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressArgs a) {
     float x0 = s_x[ch] * inv, x1 = s_x[ch + 1] * inv;
     if (ch >= rope0 && a.d_rope > 0) {
       const int j = (ch - rope0) / 2;
-      const double freq = pow(a.theta, -2.0 * (double)j / (double)a.d_rope);
-      const double ang = (double)((long long)m * i) * freq;
-      double sn, cs;
-      sincos(ang, &sn, &cs);
-      const double y0 = (double)x0 * cs - (double)x1 * sn;
-      const double y1 = (double)x0 * sn + (double)x1 * cs;
-      x0 = (float)y0; x1 = (float)y1;
+      const double freq = j < kMaxRopePairs ? a.inv_freq[j]
+                                            : pow(a.theta, -2.0 * (double)j / (double)a.d_rope);
+      float sn, cs;
+      rope_angle((double)((long long)m * i) * freq, &sn, &cs);
+      const float y0 = x0 * cs - x1 * sn;
+      const float y1 = x0 * sn + x1 * cs;
+      x0 = y0; x1 = y1;
     }
     s_x[ch] = x0; s_x[ch + 1] = x1;
   }
@@ -204,13 +216,18 @@ __global__ void __launch_bounds__(512) compress_kernel(CompressArgs a) {
   }
 }
 
-// One warp per row: FP8 (per-row scale) or NVFP4 (per-16 scale) codes.
+// Layout of the work: one CTA per (entry, sequence); see compress_body.
 template <typename InT>
-__global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int out_dtype,
-                                uint8_t* __restrict__ codes, void* __restrict__ scales) {
+__global__ void __launch_bounds__(512) compress_kernel(CompressArgs a) {
+  extern __shared__ float smem[];
+  compress_body<InT>(a, a.entry_begin + blockIdx.x, blockIdx.y, smem);
+}
+
+// One row of the index-path quantiser by one warp: FP8 (per-row scale) or NVFP4 (per-16 scale).
+template <typename InT>
+__device__ __forceinline__ void quantize_row(const InT* __restrict__ x, int row, int d, int out_dtype,
+                                             uint8_t* __restrict__ codes, void* __restrict__ scales) {
   const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (row >= rows) return;
   const InT* xr = x + (size_t)row * d;
   float am_row = 0.f;
   for (int base = 0; base < d; base += 128) {
@@ -261,8 +278,76 @@ __global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int 
   }
 }
 
-csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry_count,
+template <typename InT>
+__global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int out_dtype,
+                                uint8_t* __restrict__ codes, void* __restrict__ scales) {
+  const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row >= rows) return;
+  quantize_row<InT>(x, row, d, out_dtype, codes, scales);
+}
+
+// Decode prologue in one launch: CTAs [0, b) compress the latent entry of each
+// sequence, [b, 2b) its index-key entry (CSA), the rest quantise the index queries
+// (8 rows per CTA); CTA 0 of that range also writes the query positions.
+template <typename InT>
+__global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
+  extern __shared__ float smem[];
+  const int blk = blockIdx.x;
+  if (blk < a.b * a.nbranch) {
+    const int br = blk / a.b;
+    compress_body<InT>(br == 0 ? a.main : a.index, br == 0 ? a.main.entry_begin : a.index.entry_begin,
+                       blk % a.b, smem);
+    return;
+  }
+  const int qb = blk - a.b * a.nbranch;
+  if (qb == 0 && threadIdx.x < a.b) a.qpos[threadIdx.x] = a.t;
+  const int row = qb * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (row < a.q_rows)
+    quantize_row<InT>(reinterpret_cast<const InT*>(a.q_in), row, a.q_d, a.q_dtype, a.q_codes,
+                      a.q_scales);
+}
+
+void fill_inv_freq(CompressArgs& a) {
+  for (int j = 0; j < kMaxRopePairs; ++j)
+    a.inv_freq[j] = (a.d_rope > 0 && 2 * j < a.d_rope)
+                        ? std::pow(a.theta, -2.0 * (double)j / (double)a.d_rope) : 0.0;
+}
+
+size_t compress_smem_bytes(const CompressArgs& a, int in_dtype, int nt) {
+  const int vec = in_dtype == CSA_F32 ? 4 : 8;
+  const int cols = a.c / vec;
+  return (size_t)(3 * (nt / cols) * a.c + a.c + 32) * sizeof(float);
+}
+
+csa_status launch_decode_prologue(PrologueArgs& a, int in_dtype, cudaStream_t st) {
+  const int nt = 256;
+  const int vec = in_dtype == CSA_F32 ? 4 : 8;
+  fill_inv_freq(a.main);
+  size_t smem = compress_smem_bytes(a.main, in_dtype, nt);
+  if (a.main.c / vec > nt) return CSA_ERR_UNSUPPORTED;
+  if (a.nbranch > 1) {
+    fill_inv_freq(a.index);
+    if (a.index.c / vec > nt) return CSA_ERR_UNSUPPORTED;
+    smem = std::max(smem, compress_smem_bytes(a.index, in_dtype, nt));
+  }
+  if (smem > 200 * 1024) return CSA_ERR_UNSUPPORTED;
+  const int qblocks = std::max(1, (a.q_rows + 7) / 8);
+  const int grid = a.b * a.nbranch + qblocks;
+  if (in_dtype == CSA_F32) {
+    cudaFuncSetAttribute(decode_prologue_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    decode_prologue_kernel<float><<<grid, nt, smem, st>>>(a);
+  } else {
+    cudaFuncSetAttribute(decode_prologue_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    decode_prologue_kernel<__nv_bfloat16><<<grid, nt, smem, st>>>(a);
+  }
+  CSA_CHECK_LAUNCH();
+  return CSA_OK;
+}
+
+csa_status launch_compress(const CompressArgs& a_in, int in_dtype, int b, int entry_count,
                            cudaStream_t st) {
+  CompressArgs a = a_in;
+  fill_inv_freq(a);
   const int vec = in_dtype == CSA_F32 ? 4 : 8;
   const int cols = a.c / vec;
   const int R = a.overlap ? 2 * a.m : a.m;

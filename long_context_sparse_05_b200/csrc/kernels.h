@@ -5,6 +5,8 @@
 
 namespace csa {
 
+constexpr int kMaxRopePairs = 64;   // rotary pairs with a host-built frequency table
+
 struct CompressArgs {
   const void* C_a; const void* Z_a; const float* B_a;
   const void* C_b; const void* Z_b; const float* B_b;
@@ -13,6 +15,14 @@ struct CompressArgs {
   float eps;
   void* out;
   void* out_scales;
+  double inv_freq[kMaxRopePairs];   // theta^(-2j/d_rope) in float64, filled by the launcher
+};
+
+struct PrologueArgs {
+  CompressArgs main, index;        // index used when nbranch == 2
+  int nbranch, b, t;
+  int32_t* qpos;                   // [b] <- t
+  const void* q_in; int q_rows, q_d, q_dtype; uint8_t* q_codes; void* q_scales;
 };
 
 struct IndexArgs {
@@ -32,6 +42,7 @@ struct AttnArgs {
 
 csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry_count,
                            cudaStream_t st);
+csa_status launch_decode_prologue(PrologueArgs& a, int in_dtype, cudaStream_t st);
 csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
                            void* codes, void* scales, cudaStream_t st);
 csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
