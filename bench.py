@@ -227,8 +227,10 @@ def stage_times_decode(w, st, steps, flush, stream):
         res["index_scores"] = np.mean(timed_loop(lambda: L.csa_index_scores(
             ip, codes, qs, x["w"], st.kI_cache, st.kI_scales, qpos, w.b, 1, st.E_cap, E, scores,
             stream), steps, flush, stream))
+        tkb = L.csa_topk_workspace_size(L.CSA_BF16, w.b, 1, E, w.k)
+        tkws = torch.empty((max(tkb, 256),), dtype=torch.uint8, device="cuda")
         res["topk"] = np.mean(timed_loop(lambda: L.csa_topk(
-            scores, L.CSA_BF16, qpos, w.m, w.b, 1, E, w.k, st.idx, st.count, None, 0, stream),
+            scores, L.CSA_BF16, qpos, w.m, w.b, 1, E, w.k, st.idx, st.count, tkws, tkb, stream),
             steps, flush, stream))
         idx, cnt = st.idx, st.count
     else:

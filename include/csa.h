@@ -194,11 +194,14 @@ csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const vo
  * ascending order, padded with -1; count [b][T] holds how many.  The result
  * is exact (a radix select on the stored score bits).
  *   scores  [b][T][E] (CSA_F32 or CSA_BF16)
- *   ws      unused by this build (may be NULL, ws_bytes 0)
+ *   ws      device scratch of csa_topk_workspace_size() bytes: rows longer than
+ *           16384 entries keep a top-k per 16384-entry chunk there first (NULL
+ *           with ws_bytes 0 when the size is 0)
  */
 csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b, int T,
                     int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
                     cudaStream_t stream);
+size_t csa_topk_workspace_size(int score_dtype, int b, int T, int E, int k);
 
 /* ------------------------------------------------------------------------ */
 /* Stage 4: shared-latent MQA over selected entries + window, with sink      */

@@ -88,6 +88,7 @@ _SIGS = {
                          [c_void_p, c_void_p]),
     "csa_topk": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p,
                          c_void_p, c_void_p, c_size_t, c_void_p]),
+    "csa_topk_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
     "csa_sparse_attn": (c_int, [ctypes.POINTER(AttnParams), c_void_p, c_void_p, c_int, c_void_p,
                                 c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -179,6 +180,10 @@ def csa_topk(scores, score_dtype, q_pos, m, b, T, E, k, idx, count, ws=None, ws_
              stream=None):
     _check(lib().csa_topk(_ptr(scores), score_dtype, _ptr(q_pos), m, b, T, E, k, _ptr(idx),
                           _ptr(count), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def csa_topk_workspace_size(score_dtype, b, T, E, k):
+    return int(lib().csa_topk_workspace_size(score_dtype, b, T, E, k))
 
 
 def csa_sparse_attn_workspace_size(p, b, T, E_cap):

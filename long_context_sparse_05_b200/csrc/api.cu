@@ -116,19 +116,23 @@ csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const vo
   return launch_index_scores_simt(a, b, stream);
 }
 
+size_t csa_topk_workspace_size(int score_dtype, int b, int T, int E, int k) {
+  if (b <= 0 || T <= 0 || E <= 0 || k <= 0) return 0;
+  return topk_workspace_bytes(b * T, E, k, score_dtype);
+}
+
 csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b, int T,
                     int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
                     cudaStream_t stream) {
-  (void)ws; (void)ws_bytes;
   if (score_dtype != CSA_F32 && score_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
   if (m < 1 || b < 0 || T < 0 || E < 0 || k < 1) return CSA_ERR_INVALID_ARG;
   if (b == 0 || T == 0) return CSA_OK;
   if (!scores || !q_pos || !idx || !count) return CSA_ERR_INVALID_ARG;
-  if (k <= 32767) {
-    const csa_status st = launch_topk_search(scores, score_dtype, q_pos, m, b * T, E, k, idx, count,
-                                             stream);
-    if (st != CSA_ERR_UNSUPPORTED) return st;
-  }
+  const size_t need = topk_workspace_bytes(b * T, E, k, score_dtype);
+  if (need && (!ws || ws_bytes < need)) return CSA_ERR_INVALID_ARG;
+  const csa_status st = launch_topk_search(scores, score_dtype, q_pos, m, b * T, E, k, idx, count,
+                                           ws, ws_bytes, stream);
+  if (st != CSA_ERR_UNSUPPORTED) return st;
   return launch_topk(scores, score_dtype, q_pos, m, b * T, E, k, idx, count, stream);
 }
 
@@ -168,7 +172,7 @@ namespace {
 
 struct DecodeWs {
   void* qI_codes; void* qI_scales; void* scores; int32_t* idx; int32_t* count; int32_t* qpos;
-  void* attn_ws; size_t attn_ws_bytes;
+  void* attn_ws; size_t attn_ws_bytes; void* topk_ws; size_t topk_ws_bytes;
 };
 
 size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs* o) {
@@ -186,6 +190,8 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
     d.scores = cv.take((size_t)b * E * 2);
     d.idx = static_cast<int32_t*>(cv.take((size_t)b * p->k * 4));
     d.count = static_cast<int32_t*>(cv.take((size_t)b * 4));
+    d.topk_ws_bytes = topk_workspace_bytes(b, E, p->k, CSA_BF16);
+    d.topk_ws = cv.take(d.topk_ws_bytes);
   }
   csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype};
   d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, b, 1, p->E_cap);
@@ -199,7 +205,7 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
 int csa_decode_launch_count(const csa_decode_params* p) {
   if (!p || p->b <= 0) return 0;
   int n = 1;                                   // prologue: compressors, quantiser, positions
-  if (!p->hca) n += 2;                         // indexer, top-k
+  if (!p->hca) n += 1 + (topk_workspace_bytes(p->b, p->L / p->m, p->k, CSA_BF16) ? 2 : 1);
   n += attn_launch_count(p->H, p->c, p->hca ? 0 : p->k, p->n_w, p->b, 1, p->E_cap, p->kv_dtype);
   return n;
 }
@@ -277,7 +283,8 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
     // 4. top-k
     int32_t* io = x->idx_out ? x->idx_out : d.idx;
     int32_t* co = x->count_out ? x->count_out : d.count;
-    st = csa_topk(d.scores, CSA_BF16, d.qpos, p->m, b, 1, E, p->k, io, co, nullptr, 0, stream);
+    st = csa_topk(d.scores, CSA_BF16, d.qpos, p->m, b, 1, E, p->k, io, co, d.topk_ws,
+                  d.topk_ws_bytes, stream);
     if (st) return st;
     idx = io; cnt = co;
   }
@@ -295,7 +302,7 @@ namespace {
 
 struct PrefillWs {
   void* qI_codes; void* qI_scales; void* scores; int32_t* idx; int32_t* count; int32_t* qpos;
-  void* attn_ws; size_t attn_ws_bytes;
+  void* attn_ws; size_t attn_ws_bytes; void* topk_ws; size_t topk_ws_bytes;
 };
 
 size_t prefill_layout(const csa_prefill_params* p, void* ws, size_t cap, PrefillWs* o) {
@@ -312,6 +319,8 @@ size_t prefill_layout(const csa_prefill_params* p, void* ws, size_t cap, Prefill
   d.scores = cv.take(rows * E * (p->score_dtype == CSA_F32 ? 4 : 2));
   d.idx = static_cast<int32_t*>(cv.take(rows * p->k * 4));
   d.count = static_cast<int32_t*>(cv.take(rows * 4));
+  d.topk_ws_bytes = topk_workspace_bytes((int)rows, E, p->k, p->score_dtype);
+  d.topk_ws = cv.take(d.topk_ws_bytes);
   csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype};
   d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, p->b, p->n, E);
   d.attn_ws = cv.take(d.attn_ws_bytes);
@@ -369,7 +378,8 @@ csa_status csa_prefill(const csa_prefill_params* p, const csa_prefill_tensors* x
   if (st) return st;
   int32_t* io = x->idx_out ? x->idx_out : d.idx;
   int32_t* co = x->count_out ? x->count_out : d.count;
-  st = csa_topk(d.scores, p->score_dtype, d.qpos, p->m, b, n, E, p->k, io, co, nullptr, 0, stream);
+  st = csa_topk(d.scores, p->score_dtype, d.qpos, p->m, b, n, E, p->k, io, co, d.topk_ws,
+                d.topk_ws_bytes, stream);
   if (st) return st;
   csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype};
   return csa_sparse_attn(&ap, x->q, x->kv_cache, E, io, co, x->kv_win, n, d.qpos, x->sink, b, n,

@@ -46,7 +46,9 @@ csa_status launch_decode_prologue(PrologueArgs& a, int in_dtype, cudaStream_t st
 csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
                            void* codes, void* scales, cudaStream_t st);
 csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
-                              int rows, int E, int k, int32_t* idx, int32_t* count, cudaStream_t st);
+                              int rows, int E, int k, int32_t* idx, int32_t* count, void* ws,
+                              size_t ws_bytes, cudaStream_t st);
+size_t topk_workspace_bytes(int rows, int E, int k, int score_dtype);
 csa_status launch_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int rows,
                        int E, int k, int32_t* idx, int32_t* count, cudaStream_t st);
 

@@ -247,10 +247,37 @@ def test_topk_1m_row():
     qpos = torch.full((1, 1), m * E - 1, dtype=torch.int32, device=DEV)
     idx = torch.empty((1, 1, k), dtype=torch.int32, device=DEV)
     cnt = torch.empty((1, 1), dtype=torch.int32, device=DEV)
-    L.csa_topk(st, L.CSA_BF16, qpos, m, 1, 1, E, k, idx, cnt)
+    wsb = L.csa_topk_workspace_size(L.CSA_BF16, 1, 1, E, k)
+    assert wsb > 0           # 1M-context rows take the chunked two-pass path
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=DEV)
+    L.csa_topk(st, L.CSA_BF16, qpos, m, 1, 1, E, k, idx, cnt, ws, wsb)
     torch.cuda.synchronize()
     ri, rc = csa.topk(f64(sc)[0], np.array([m * E - 1]), m, k)
     np.testing.assert_array_equal(idx[0].cpu().numpy(), ri)
+
+
+@pytest.mark.parametrize("E,k,ties", [(40000, 1024, False), (40000, 1024, True), (70000, 16, True)])
+def test_topk_chunked_rows_bit_exact(E, k, ties):
+    """Rows longer than one CTA: per-chunk top-k then top-k of the candidates; ties across
+    chunk borders must still go to the lowest entries."""
+    b, T, m = 2, 3, 4
+    rng = np.random.default_rng(E + k)
+    sc = rng.normal(size=(b, T, E))
+    if ties:
+        sc = np.round(sc * 2) / 2
+    qpos = np.array([[m * E - 1, m * 20000 + 1, m * 700 - 1]] * b, dtype=np.int32)
+    st = torch.from_numpy(sc).to(torch.bfloat16).to(DEV)
+    idx = torch.empty((b, T, k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((b, T), dtype=torch.int32, device=DEV)
+    wsb = L.csa_topk_workspace_size(L.CSA_BF16, b, T, E, k)
+    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    L.csa_topk(st, L.CSA_BF16, _dev(qpos), m, b, T, E, k, idx, cnt, ws, wsb)
+    torch.cuda.synchronize()
+    stored = f64(st)
+    for s_ in range(b):
+        ri, rc = csa.topk(stored[s_], qpos[s_], m, k)
+        np.testing.assert_array_equal(cnt[s_].cpu().numpy(), rc)
+        np.testing.assert_array_equal(idx[s_].cpu().numpy(), ri)
 
 
 def _attn_case(b, T, H, d, E, n, k, n_w, dtype, dense, seed):
