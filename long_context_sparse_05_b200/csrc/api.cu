@@ -113,6 +113,8 @@ csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const vo
   a.score_dtype = p->score_dtype; a.E_cap = E_cap; a.E = E; a.scores = scores;
   csa_status st = launch_index_scores_tc(a, b, stream);
   if (st != CSA_ERR_UNSUPPORTED) return st;
+  st = launch_index_scores_fp4_tc(a, b, stream);
+  if (st != CSA_ERR_UNSUPPORTED) return st;
   return launch_index_scores_simt(a, b, stream);
 }
 

@@ -58,6 +58,7 @@ csa_status launch_attn_simt(const AttnArgs& a, int b, int dtype, cudaStream_t st
 
 // Tensor-core (tcgen05) kernels: return CSA_ERR_UNSUPPORTED for shapes they do not cover.
 csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st);
+csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st);
 csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t ws_bytes,
                           cudaStream_t st);
 size_t attn_tc_workspace_bytes(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype);

@@ -235,6 +235,9 @@ int* device_error_word();
 // [rows][row_bytes] with a box of [box_rows][box_bytes] and 128-byte swizzle.
 bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
                      uint32_t box_bytes, uint32_t box_rows);
+// Same with a chosen swizzle (0, 32, 64 or 128 bytes).
+bool make_tmap_2d_u8_swz(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                         uint32_t box_bytes, uint32_t box_rows, int swizzle_bytes);
 // 1-D map over `n` float32 values with a box of `box` values (no swizzle).
 bool make_tmap_1d_f32(CUtensorMap* m, const void* base, uint64_t n, uint32_t box);
 // Same for 16-bit elements: [rows][cols] with a box of [box_rows][box_cols].

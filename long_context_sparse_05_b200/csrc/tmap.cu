@@ -60,6 +60,24 @@ bool make_tmap_2d_u8(CUtensorMap* m, const void* base, uint64_t row_bytes, uint6
                 box_rows);
 }
 
+bool make_tmap_2d_u8_swz(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                         uint32_t box_bytes, uint32_t box_rows, int swizzle_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {row_bytes, rows};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_bytes, box_rows};
+  cuuint32_t es[2] = {1, 1};
+  const CUtensorMapSwizzle sw = swizzle_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                               : swizzle_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                               : swizzle_bytes == 32 ? CU_TENSOR_MAP_SWIZZLE_32B
+                                                     : CU_TENSOR_MAP_SWIZZLE_NONE;
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_1d_f32(CUtensorMap* m, const void* base, uint64_t n, uint32_t box) {
   auto fn = encode_fn();
   if (!fn) return false;

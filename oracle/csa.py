@@ -55,7 +55,7 @@ def compress_pool(C_a, Z_a, B_a, C_b, Z_b, B_b, m, overlap, entries):
     ("内容同样拼接后按权重加和", section "C4A Compressor").
     """
     entries = np.asarray(entries, dtype=np.int64)
-    c = np.asarray(C_a).shape[1]
+    c = C_a.shape[1]
     out = np.empty((len(entries), c), dtype=np.float64)
     for row, i in enumerate(entries):
         wgt = compress_weights(Z_a, B_a, Z_b, B_b, m, overlap, int(i))
@@ -78,7 +78,7 @@ def compress_pool_vec(C_a, Z_a, B_a, C_b, Z_b, B_b, m, overlap, i0, count):
     Used where the oracle needs tens of thousands of entries (decode caches).
     Tested equal to ``compress_pool`` in the pins.
     """
-    c = np.asarray(C_a).shape[1]
+    c = C_a.shape[1]
     sl = slice(m * i0, m * (i0 + count))
     u_a = np.asarray(Z_a[sl], dtype=np.float64).reshape(count, m, c) + np.asarray(B_a, dtype=np.float64)
     k_a = np.asarray(C_a[sl], dtype=np.float64).reshape(count, m, c)
@@ -156,7 +156,7 @@ def compress_range(C_a, Z_a, B_a, C_b, Z_b, B_b, m, overlap, i0, count, d_rope, 
     Entries are independent, so they are processed in chunks of about
     ``chunk_rows`` raw rows only to bound host memory.
     """
-    c = np.asarray(C_a).shape[1]
+    c = C_a.shape[1]
     out = np.empty((count, c), dtype=np.float64)
     step = max(1, chunk_rows // m)
     for j0 in range(i0, i0 + count, step):
@@ -281,7 +281,6 @@ def sparse_attn(q, kv_comp, idx, cnt, kv_win, q_pos, sink, n_w, scale, m=None):
     """
     q = np.asarray(q, dtype=np.float64)
     kv_comp = np.asarray(kv_comp, dtype=np.float64)
-    kv_win = np.asarray(kv_win, dtype=np.float64)
     T = q.shape[0]
     o = np.zeros_like(q)
     lse = np.zeros(q.shape[:2])
@@ -291,7 +290,8 @@ def sparse_attn(q, kv_comp, idx, cnt, kv_win, q_pos, sink, n_w, scale, m=None):
             sel = np.arange(int(visible_entries(t, m)))
         else:
             sel = np.asarray(idx[r, :int(cnt[r])], dtype=np.int64)
-        rows = np.concatenate([kv_comp[sel], kv_win[window_rows(t, n_w)]], axis=0)
+        rows = np.concatenate([kv_comp[sel],
+                               np.asarray(kv_win[window_rows(t, n_w)], dtype=np.float64)], axis=0)
         o[r], lse[r] = attend(q[r], rows, sink, scale)
     return o, lse
 

@@ -68,10 +68,10 @@ def csa_prefill(main, index, q, q_I, w, sink, *, m, d_rope, theta, eps, k, n_w, 
                             index["B_b"], m, True, 0, E, d_rope, theta, eps)
     kI_deq, _ = quantize_rows(kI, idx_dtype)
     rows = np.arange(n) if query_rows is None else np.asarray(query_rows, dtype=np.int64)
-    qI_deq, _ = quantize_rows(np.asarray(q_I)[rows], idx_dtype)
-    scores = csa.index_scores(qI_deq, np.asarray(w)[rows], kI_deq, rows, m, score_dtype)
+    qI_deq, _ = quantize_rows(q_I[rows], idx_dtype)
+    scores = csa.index_scores(qI_deq, w[rows], kI_deq, rows, m, score_dtype)
     idx, cnt = csa.topk(scores, rows, m, k)
-    o, lse = csa.sparse_attn(np.asarray(q)[rows], kv_st, idx, cnt, main["C_a"], rows, sink, n_w, scale)
+    o, lse = csa.sparse_attn(q[rows], kv_st, idx, cnt, main["C_a"], rows, sink, n_w, scale)
     return dict(kv=kv, kv_stored=kv_st, kI=kI, kI_deq=kI_deq, qI_deq=qI_deq, scores=scores,
                 idx=idx, cnt=cnt, out=round_out(o, kv_dtype), out_f64=o, lse=lse, rows=rows)
 
@@ -90,7 +90,7 @@ def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k,
     E = L // m
     t = L - 1
     kI = csa.compress_range(index["C_a"], index["Z_a"], index["B_a"], index["C_b"], index["Z_b"],
-                            index["B_b"], m, True, 0, E, d_rope, theta, eps)
+                            index["B_b"], m, True, 0, E, d_rope, theta, eps, chunk_rows=1 << 16)
     kI_deq, _ = quantize_rows(kI, idx_dtype)
     qI_deq, _ = quantize_rows(np.asarray(q_I)[None], idx_dtype)
     scores = csa.index_scores(qI_deq, np.asarray(w)[None], kI_deq, np.array([t]), m, "bf16")
@@ -99,7 +99,7 @@ def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k,
     kv_sel = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
                                   main["B_b"], m, True, sel, d_rope, theta, eps)
     kv_sel_st = round_out(kv_sel, kv_dtype)
-    rows = np.concatenate([kv_sel_st, np.asarray(main["C_a"])[csa.window_rows(t, n_w)]], axis=0)
+    rows = np.concatenate([kv_sel_st, np.asarray(main["C_a"][csa.window_rows(t, n_w)], dtype=np.float64)], axis=0)
     o, lse = csa.attend(np.asarray(q), rows, sink, scale)
     new_entry = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
                                      main["B_b"], m, True, [E - 1], d_rope, theta, eps)[0]
@@ -118,9 +118,9 @@ def hca_decode_seq(main, q, sink, *, L, m, d_rope, theta, eps, n_w, scale, kv_dt
     E = L // m
     t = L - 1
     kv = csa.compress_range(main["C_a"], main["Z_a"], main["B_a"], None, None, None, m, False,
-                            0, E, d_rope, theta, eps)
+                            0, E, d_rope, theta, eps, chunk_rows=1 << 16)
     kv_st = round_out(kv, kv_dtype)
-    rows = np.concatenate([kv_st, np.asarray(main["C_a"])[csa.window_rows(t, n_w)]], axis=0)
+    rows = np.concatenate([kv_st, np.asarray(main["C_a"][csa.window_rows(t, n_w)], dtype=np.float64)], axis=0)
     o, lse = csa.attend(np.asarray(q), rows, sink, scale)
     return dict(kv=kv, kv_stored=kv_st, new_entry=kv[E - 1], out=round_out(o, kv_dtype),
                 out_f64=o, lse=lse)

@@ -70,3 +70,23 @@ def topk_band_check(gpu_idx, gpu_cnt, exact_scores, ev, k, rel_band=1e-3):
         assert abs(sc[s] - tau) <= band, "entry %d score %r outside the tie band of tau %r" % (
             s, sc[s], tau)
     return len(diff) // 2
+
+
+class LazyRows:
+    """Row access to one sequence of a (large) device tensor, copied to the host in float64 on demand.
+
+    Lets the oracle walk 1M-token inputs without holding them on the host: indexing
+    with a slice or an index array returns a numpy float64 array of those rows.
+    """
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, key):
+        if isinstance(key, np.ndarray):
+            key = torch.from_numpy(np.asarray(key, dtype=np.int64)).to(self.t.device)
+        return self.t[key].to(torch.float64).cpu().numpy()
+
+    def __len__(self):
+        return self.shape[0]
