@@ -123,11 +123,21 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host scalar over the ranks (NCCL ranks reduce on their GPU, gloo on the CPU)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if torch.distributed.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def aggregate(ms_local, tokens_local, world):
+    """Whole-job throughput of independent replicas: all ranks' tokens over the slowest rank's
+    device time.  Returns (ms_per_step, tokens_per_step, tokens_per_second)."""
+    ms = max_over_ranks(ms_local, world)
+    tokens = tokens_local * world
+    return ms, tokens, tokens / (ms * 1e-3)
 
 
 def timed_loop(fn, steps, flush_buf, stream):
@@ -173,9 +183,7 @@ def bench_decode(w, args, world, rank, peaks):
     t1 = time.time()
     barrier(world)
     ck = clocks.stop(t0, t1)
-    ms = max_over_ranks(float(np.mean(times)), world)
-    tokens_per_step = w.b * world
-    value = tokens_per_step / (ms * 1e-3)
+    ms, tokens_per_step, value = aggregate(float(np.mean(times)), w.b, world)
 
     # dominant kernel: the indexer over all E entries (same call the step makes)
     stage = stage_times_decode(w, st, args.steps, flush, stream)
@@ -305,13 +313,12 @@ def bench_prefill(w, args, world, rank, peaks):
     t1 = time.time()
     barrier(world)
     ck = clocks.stop(t0, t1)
-    ms = max_over_ranks(float(np.mean(times)), world)
+    ms, tokens, value = aggregate(float(np.mean(times)), w.b * w.n, world)
     f_idx, f_attn = runner.prefill_flops(w)
     p_fp8 = 2 * peaks["bf16"]
     t_ideal = f_idx / (p_fp8 * 1e12) + f_attn / (peaks["bf16"] * 1e12)
     frac = t_ideal / (ms * 1e-3)
-    tokens = w.b * w.n * world
-    return dict(value=tokens / (ms * 1e-3), ms=ms, tokens_per_step=tokens, clocks=ck, stage={},
+    return dict(value=value, ms=ms, tokens_per_step=tokens, clocks=ck, stage={},
                 roofline={"bound": "tensor", "achieved": round(
                     (f_idx + f_attn) / (ms * 1e-3) / 1e12, 2), "peak": peaks["bf16"],
                     "unit": "TFLOP/s", "frac": round(frac, 4), "traffic": None,

@@ -79,6 +79,14 @@ int csa_version(void);
  */
 int csa_device_error(cudaStream_t stream);
 
+/*
+ * Failure-detection self-test: launches one thread that waits, with a bound of
+ * limit_us microseconds (1 .. 100000), on a barrier nothing ever signals.  The
+ * wait gives up and sets the device error word, so a following
+ * csa_device_error(stream) returns CSA_ERR_TIMEOUT; the context stays usable.
+ */
+csa_status csa_selftest_bounded_wait(int limit_us, cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Stage 1: KV compressor                                                    */
 /* ------------------------------------------------------------------------ */

@@ -81,6 +81,7 @@ _SIGS = {
     "csa_status_string": (ctypes.c_char_p, [c_int]),
     "csa_version": (c_int, []),
     "csa_device_error": (c_int, [c_void_p]),
+    "csa_selftest_bounded_wait": (c_int, [c_int, c_void_p]),
     "csa_compress": (c_int, [ctypes.POINTER(CompressParams)] + [c_void_p] * 6 +
                      [c_int] * 5 + [c_void_p, c_void_p, c_void_p]),
     "csa_quantize": (c_int, [c_int, c_int, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p]),
@@ -151,6 +152,10 @@ def _check(status):
 def csa_device_error(stream=None):
     """Synchronise and read/clear the device error word (0 = no bounded wait gave up)."""
     return int(lib().csa_device_error(_stream(stream)))
+
+
+def csa_selftest_bounded_wait(limit_us, stream=None):
+    _check(lib().csa_selftest_bounded_wait(limit_us, _stream(stream)))
 
 
 def csa_status_string(status):

@@ -94,10 +94,14 @@ csa_status csa_quantize(int in_dtype, int out_dtype, const void* x, int rows, in
   return launch_quantize(in_dtype, out_dtype, x, rows, d, codes, scales, stream);
 }
 
-csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const void* q_scales,
-                            const float* w, const void* k_I, const void* k_scales,
-                            const int32_t* q_pos, int b, int T, int E_cap, int E, void* scores,
-                            cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+
+csa_status index_scores_impl(const csa_index_params* p, const void* q_I, const void* q_scales,
+                             const float* w, const void* k_I, const void* k_scales,
+                             const int32_t* q_pos, int b, int T, int E_cap, int E, void* scores,
+                             cudaStream_t stream, int pdl, int all_visible, int dep_entry) {
   if (!p) return CSA_ERR_INVALID_ARG;
   if (p->H_I < 1 || p->d_I < 16 || p->d_I % 16 || p->m < 1) return CSA_ERR_INVALID_ARG;
   if (p->qk_dtype < CSA_F32 || p->qk_dtype > CSA_NVFP4 || p->qk_dtype == CSA_BF16)
@@ -111,6 +115,7 @@ csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const vo
   a.q = q_I; a.q_scales = q_scales; a.w = w; a.k = k_I; a.k_scales = k_scales; a.q_pos = q_pos;
   a.T = T; a.H = p->H_I; a.d = p->d_I; a.m = p->m; a.qk_dtype = p->qk_dtype;
   a.score_dtype = p->score_dtype; a.E_cap = E_cap; a.E = E; a.scores = scores;
+  a.pdl = pdl; a.all_visible = all_visible; a.dep_entry = dep_entry;
   csa_status st = launch_index_scores_tc(a, b, stream);
   if (st != CSA_ERR_UNSUPPORTED) return st;
   st = launch_index_scores_fp4_tc(a, b, stream);
@@ -118,14 +123,9 @@ csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const vo
   return launch_index_scores_simt(a, b, stream);
 }
 
-size_t csa_topk_workspace_size(int score_dtype, int b, int T, int E, int k) {
-  if (b <= 0 || T <= 0 || E <= 0 || k <= 0) return 0;
-  return topk_workspace_bytes(b * T, E, k, score_dtype);
-}
-
-csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b, int T,
-                    int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
-                    cudaStream_t stream) {
+csa_status topk_impl(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b,
+                     int T, int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                     cudaStream_t stream, bool pdl) {
   if (score_dtype != CSA_F32 && score_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
   if (m < 1 || b < 0 || T < 0 || E < 0 || k < 1) return CSA_ERR_INVALID_ARG;
   if (b == 0 || T == 0) return CSA_OK;
@@ -133,20 +133,16 @@ csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, i
   const size_t need = topk_workspace_bytes(b * T, E, k, score_dtype);
   if (need && (!ws || ws_bytes < need)) return CSA_ERR_INVALID_ARG;
   const csa_status st = launch_topk_search(scores, score_dtype, q_pos, m, b * T, E, k, idx, count,
-                                           ws, ws_bytes, stream);
+                                           ws, ws_bytes, stream, pdl);
   if (st != CSA_ERR_UNSUPPORTED) return st;
   return launch_topk(scores, score_dtype, q_pos, m, b * T, E, k, idx, count, stream);
 }
 
-size_t csa_sparse_attn_workspace_size(const csa_attn_params* p, int b, int T, int E_cap) {
-  if (!p) return 0;
-  return attn_tc_workspace_bytes(p->H, p->d, p->k, p->n_w, b, T, E_cap, p->dtype);
-}
-
-csa_status csa_sparse_attn(const csa_attn_params* p, const void* q, const void* kv_comp, int E_cap,
-                           const int32_t* idx, const int32_t* count, const void* kv_win, int n,
-                           const int32_t* q_pos, const float* sink, int b, int T, void* out,
-                           float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+csa_status sparse_attn_impl(const csa_attn_params* p, const void* q, const void* kv_comp,
+                            int E_cap, const int32_t* idx, const int32_t* count,
+                            const void* kv_win, int n, const int32_t* q_pos, const float* sink,
+                            int b, int T, void* out, float* lse, void* ws, size_t ws_bytes,
+                            cudaStream_t stream, int pdl) {
   if (!p) return CSA_ERR_INVALID_ARG;
   if (p->H < 1 || p->d < 8 || p->d % 8 || p->n_w < 0 || p->m < 1) return CSA_ERR_INVALID_ARG;
   if (p->dtype != CSA_F32 && p->dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
@@ -160,10 +156,47 @@ csa_status csa_sparse_attn(const csa_attn_params* p, const void* q, const void* 
   AttnArgs a{};
   a.q = q; a.kv = kv_comp; a.idx = idx; a.count = count; a.win = kv_win; a.q_pos = q_pos;
   a.sink = sink; a.T = T; a.H = p->H; a.d = p->d; a.n_w = p->n_w; a.m = p->m; a.k = p->k;
-  a.E_cap = E_cap; a.n = n; a.scale = p->scale; a.out = out; a.lse = lse;
+  a.E_cap = E_cap; a.n = n; a.scale = p->scale; a.out = out; a.lse = lse; a.pdl = pdl;
   csa_status st = launch_attn_tc(a, b, p->dtype, ws, ws_bytes, stream);
   if (st != CSA_ERR_UNSUPPORTED) return st;
   return launch_attn_simt(a, b, p->dtype, stream);
+}
+
+}  // namespace
+
+extern "C" {
+
+csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const void* q_scales,
+                            const float* w, const void* k_I, const void* k_scales,
+                            const int32_t* q_pos, int b, int T, int E_cap, int E, void* scores,
+                            cudaStream_t stream) {
+  return index_scores_impl(p, q_I, q_scales, w, k_I, k_scales, q_pos, b, T, E_cap, E, scores,
+                           stream, 0, 0, -1);
+}
+
+size_t csa_topk_workspace_size(int score_dtype, int b, int T, int E, int k) {
+  if (b <= 0 || T <= 0 || E <= 0 || k <= 0) return 0;
+  return topk_workspace_bytes(b * T, E, k, score_dtype);
+}
+
+csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b, int T,
+                    int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                    cudaStream_t stream) {
+  return topk_impl(scores, score_dtype, q_pos, m, b, T, E, k, idx, count, ws, ws_bytes, stream,
+                   false);
+}
+
+size_t csa_sparse_attn_workspace_size(const csa_attn_params* p, int b, int T, int E_cap) {
+  if (!p) return 0;
+  return attn_tc_workspace_bytes(p->H, p->d, p->k, p->n_w, b, T, E_cap, p->dtype);
+}
+
+csa_status csa_sparse_attn(const csa_attn_params* p, const void* q, const void* kv_comp, int E_cap,
+                           const int32_t* idx, const int32_t* count, const void* kv_win, int n,
+                           const int32_t* q_pos, const float* sink, int b, int T, void* out,
+                           float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  return sparse_attn_impl(p, q, kv_comp, E_cap, idx, count, kv_win, n, q_pos, sink, b, T, out, lse,
+                          ws, ws_bytes, stream, 0);
 }
 
 // ---------------------------------------------------------------------------
@@ -278,22 +311,24 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
   const int32_t* cnt = nullptr;
   if (!p->hca) {
     // 3. score all entries
+    // (programmatic dependent launches from here on: each kernel starts while its
+    //  predecessor drains and waits for it only where it reads its outputs)
     csa_index_params ip{p->H_I, p->c_I, p->m, p->idx_dtype, CSA_BF16};
-    st = csa_index_scores(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, 1, p->E_cap, E,
-                          d.scores, stream);
+    st = index_scores_impl(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, 1, p->E_cap,
+                           E, d.scores, stream, 1, 1, E - 1);
     if (st) return st;
     // 4. top-k
     int32_t* io = x->idx_out ? x->idx_out : d.idx;
     int32_t* co = x->count_out ? x->count_out : d.count;
-    st = csa_topk(d.scores, CSA_BF16, d.qpos, p->m, b, 1, E, p->k, io, co, d.topk_ws,
-                  d.topk_ws_bytes, stream);
+    st = topk_impl(d.scores, CSA_BF16, d.qpos, p->m, b, 1, E, p->k, io, co, d.topk_ws,
+                   d.topk_ws_bytes, stream, true);
     if (st) return st;
     idx = io; cnt = co;
   }
   // 4. attention over the selection (or all entries) plus the window
   csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype};
-  return csa_sparse_attn(&ap, x->q, x->kv_cache, p->E_cap, idx, cnt, x->kv_win, p->L, d.qpos,
-                         x->sink, b, 1, x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream);
+  return sparse_attn_impl(&ap, x->q, x->kv_cache, p->E_cap, idx, cnt, x->kv_win, p->L, d.qpos,
+                          x->sink, b, 1, x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream, 1);
 }
 
 // ---------------------------------------------------------------------------
@@ -375,17 +410,17 @@ csa_status csa_prefill(const csa_prefill_params* p, const csa_prefill_tensors* x
     return CSA_ERR_UNSUPPORTED;
   }
   csa_index_params ip{p->H_I, p->c_I, p->m, p->idx_dtype, p->score_dtype};
-  st = csa_index_scores(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, n, E, E, d.scores,
-                        stream);
+  st = index_scores_impl(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, n, E, E,
+                         d.scores, stream, 1, 0, -1);
   if (st) return st;
   int32_t* io = x->idx_out ? x->idx_out : d.idx;
   int32_t* co = x->count_out ? x->count_out : d.count;
-  st = csa_topk(d.scores, p->score_dtype, d.qpos, p->m, b, n, E, p->k, io, co, d.topk_ws,
-                d.topk_ws_bytes, stream);
+  st = topk_impl(d.scores, p->score_dtype, d.qpos, p->m, b, n, E, p->k, io, co, d.topk_ws,
+                 d.topk_ws_bytes, stream, true);
   if (st) return st;
   csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype};
-  return csa_sparse_attn(&ap, x->q, x->kv_cache, E, io, co, x->kv_win, n, d.qpos, x->sink, b, n,
-                         x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream);
+  return sparse_attn_impl(&ap, x->q, x->kv_cache, E, io, co, x->kv_win, n, d.qpos, x->sink, b, n,
+                          x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream, 1);
 }
 
 }  // extern "C"

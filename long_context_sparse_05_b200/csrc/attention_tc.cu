@@ -149,6 +149,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   const int lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
 
+  pdl_launch_dependents();
   if (tid == 0) {
     tc::mbar_init(bar_s, 1);
     tc::mbar_init(bar_o, 1);
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
+  pdl_wait();   // selections, positions and caches come from the preceding kernels
   const uint32_t tmem = *tmem_holder;
   const uint32_t tS = tmem;            // columns [0, 64): S^T
   const uint32_t tO = tmem + 64;       // columns [64, 320): O^T, 4 blocks of 64
@@ -394,6 +396,8 @@ constexpr int kMaxSplit = 64;
 __global__ void __launch_bounds__(128) attn_merge_kernel(AttnTc p) {
   __shared__ float s_m[kMaxSplit][kMergeHeads], s_l[kMaxSplit][kMergeHeads];
   __shared__ float s_w[kMaxSplit][kMergeHeads];
+  pdl_launch_dependents();
+  pdl_wait();
   const int qrow = blockIdx.x, h0 = blockIdx.y * kMergeHeads;
   const size_t it0 = (size_t)qrow * p.nsplit;
   for (int x = threadIdx.x; x < p.nsplit * kMergeHeads; x += blockDim.x) {
@@ -530,12 +534,13 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
     return CSA_ERR_CUDA;
   const long long items = (long long)b * a.T * P.nsplit;
   const int grid = (int)std::min<long long>(items, sms);
-  attn_tc_kernel<<<grid, 160, kSmemBytes, st>>>(p);
-  CSA_CHECK_LAUNCH();
-  if (P.nsplit > 1) {
-    attn_merge_kernel<<<dim3(b * a.T, kH / kMergeHeads), 128, 0, st>>>(p);
-    CSA_CHECK_LAUNCH();
-  }
+  if (csa_launch(attn_tc_kernel, dim3(grid), dim3(160), kSmemBytes, st, a.pdl != 0, p) !=
+      cudaSuccess)
+    return CSA_ERR_CUDA;
+  if (P.nsplit > 1 &&
+      csa_launch(attn_merge_kernel, dim3(b * a.T, kH / kMergeHeads), dim3(128), 0, st, a.pdl != 0,
+                 p) != cudaSuccess)
+    return CSA_ERR_CUDA;
   return CSA_OK;
 }
 

@@ -7,6 +7,8 @@
 #include <cuda_fp4.h>
 #include <stdint.h>
 
+#include <utility>
+
 #include "csa.h"
 
 namespace csa {
@@ -78,6 +80,14 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
+// Programmatic dependent launch: wait until the preceding grid of the stream has
+// completed and its writes are visible (a no-op when the grid was launched
+// without the programmatic attribute), and allow the next grid to launch early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Visible entries of query position t: floor((t+1)/m), clamped to [0, E].
 __device__ __forceinline__ int visible_entries(int t, int m, int E) {
   int e = t < 0 ? 0 : (t + 1) / m;
@@ -85,6 +95,23 @@ __device__ __forceinline__ int visible_entries(int t, int m, int E) {
 }
 
 }  // namespace csa
+
+// Launches `kern` on `st`; with pdl, as a programmatic dependent of the preceding grid.
+template <typename... KArgs, typename... Args>
+inline cudaError_t csa_launch(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, bool pdl, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = pdl ? at : nullptr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 #define CSA_CHECK_LAUNCH()                                  \
   do {                                                      \

@@ -292,6 +292,7 @@ __global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int 
 template <typename InT>
 __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
   extern __shared__ float smem[];
+  pdl_launch_dependents();   // the indexer may start fetching the unchanged key tiles
   const int blk = blockIdx.x;
   if (blk < a.b * a.nbranch) {
     const int br = blk / a.b;

@@ -51,6 +51,8 @@ struct IdxFp4 {
   int T, E_cap, E, m;
   int tiles, chunk, n_chunks, units;
   int score_f32;
+  int all_visible;   // every query sees all E entries: q_pos is not read
+  int dep_tile;      // tiles >= dep_tile hold entries the preceding kernel writes
 };
 
 // Stage layout (bytes): keys | raw scales | rearranged scales.
@@ -140,12 +142,14 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  if (!p.all_visible) pdl_wait();   // the query positions come from the preceding kernel
 
   for (int i = threadIdx.x; i * (int)gridDim.x + (int)blockIdx.x < p.units && i < kMaxLocalUnits;
        i += blockDim.x) {
     const int u = blockIdx.x + i * gridDim.x;
     const int row = u / p.n_chunks;
-    const int ev = visible_entries(p.q_pos[row], p.m, p.E);
+    const int ev = p.all_visible ? p.E : visible_entries(p.q_pos[row], p.m, p.E);
     s_ev[i] = ev;
     s_vis[i] = (ev + kTileE - 1) / kTileE;
   }
@@ -175,6 +179,23 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 
   if (warp == 0) {
     if (lane == 0) {
+      // key tiles the preceding kernel does not write are fetched before waiting on it
+      uint32_t npre = 0;
+      for (int u = blockIdx.x, i = 0; u < p.units && npre == 0; u += gridDim.x, ++i) {
+        int row, j0, j1, nc;
+        unit(u, i, row, j0, j1, nc);
+        if (nc == 0) continue;
+        const int sb = row / p.T;
+        for (int j = j0; j < j0 + nc && (int)npre < S && j < p.dep_tile; ++j, ++npre) {
+          const int row0 = sb * p.E_cap + j * kTileE;
+          uint8_t* st = sStage + npre * kStage;
+          tc::mbar_arrive_expect_tx(&full[npre], kTileBytes + kTileSf);
+          tc::tma_load_2d(st, &tmK, 0, row0, &full[npre]);
+          tc::tma_load_2d(st + kTileBytes, &tmKS, 0, row0 / 2, &full[npre]);
+        }
+        break;
+      }
+      pdl_wait();
       uint32_t it = 0, ul = 0;
       bool ok = true;
       for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
@@ -191,6 +212,7 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         tc::tma_load_1d(qb + kQBytes + kQSf + kPermBytes, &tmW, row * kHeads, &bfull[bb]);
         const int sb = row / p.T;
         for (int j = j0; j < j0 + nc; ++j, ++it) {
+          if (it < npre) continue;                       // fetched before the wait
           const int s = it % S;
           ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
           if (!ok) break;
@@ -360,6 +382,8 @@ csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st
   if (units > 0x7fffffff) return CSA_ERR_UNSUPPORTED;
   p.units = (int)units;
   p.score_f32 = a.score_dtype == CSA_F32;
+  p.all_visible = a.all_visible;
+  p.dep_tile = a.dep_entry < 0 ? 0 : a.dep_entry / kTileE;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
@@ -368,8 +392,9 @@ csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st
   if (cudaFuncSetAttribute(index_scores_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return CSA_ERR_CUDA;
-  index_scores_fp4_kernel<<<(int)grid, 192, smem, st>>>(tmK, tmKS, tmQ, tmQS, tmW, p);
-  CSA_CHECK_LAUNCH();
+  if (csa_launch(index_scores_fp4_kernel, dim3((unsigned)grid), dim3(192), smem, st, a.pdl != 0,
+                 tmK, tmKS, tmQ, tmQS, tmW, p) != cudaSuccess)
+    return CSA_ERR_CUDA;
   return CSA_OK;
 }
 

@@ -50,6 +50,8 @@ struct IdxTc {
   int T, E_cap, E, m;
   int n_qg, tiles, chunk, n_chunks, units;
   int score_f32;
+  int all_visible;   // every query sees all E entries: q_pos is not read
+  int dep_tile;      // tiles >= dep_tile hold entries the preceding kernel writes
 };
 
 template <int QG>
@@ -91,6 +93,8 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  if (!p.all_visible) pdl_wait();   // the query positions come from the preceding kernel
 
   // causal extent of every unit this CTA will walk
   for (int i = threadIdx.x; i * (int)gridDim.x + (int)blockIdx.x < p.units && i < kMaxLocalUnits;
@@ -101,7 +105,8 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     const int nq = min(QG, p.T - g * QG);
     int evmax = 0;
     for (int q = 0; q < QG; ++q) {
-      const int ev = q < nq ? visible_entries(p.q_pos[(size_t)sb * p.T + g * QG + q], p.m, p.E) : 0;
+      const int ev = q >= nq ? 0 : p.all_visible ? p.E
+                   : visible_entries(p.q_pos[(size_t)sb * p.T + g * QG + q], p.m, p.E);
       s_ev[i * QG + q] = ev;
       evmax = max(evmax, ev);
     }
@@ -137,6 +142,22 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
+      // Key tiles the preceding kernel does not write are fetched before waiting on it,
+      // into the first free stages, so that HBM streaming overlaps that kernel.
+      uint32_t npre = 0;
+      for (int u = blockIdx.x, i = 0; u < p.units && npre == 0; u += gridDim.x, ++i) {
+        int sb, g, j0, j1, nc, nq;
+        unit(u, i, sb, g, j0, j1, nc, nq);
+        if (nc == 0) continue;
+        for (int j = j0; j < j0 + nc && (int)npre < S && j < p.dep_tile; ++j, ++npre) {
+          const int row0 = sb * p.E_cap + j * kTileE;
+          tc::mbar_arrive_expect_tx(&full[npre], kTileBytes + kTileE * 4);
+          tc::tma_load_2d(sA + npre * kTileBytes, &tmK, 0, row0, &full[npre]);
+          tc::tma_load_1d(sKS + npre * kTileE, &tmKS, row0, &full[npre]);
+        }
+        break;
+      }
+      pdl_wait();
       uint32_t it = 0, ul = 0;
       bool ok = true;
       for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
@@ -152,6 +173,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         tc::tma_load_1d(sW + bb * N, &tmW, qrow0, &bfull[bb]);
         tc::tma_load_1d(sQS + bb * N, &tmQS, qrow0, &bfull[bb]);
         for (int j = j0; j < j0 + nc; ++j, ++it) {
+          if (it < npre) continue;                       // fetched before the wait
           const int s = it % S;
           ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
           if (!ok) break;
@@ -309,6 +331,8 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   if (units > 0x7fffffff) return CSA_ERR_UNSUPPORTED;
   p.units = (int)units;
   p.score_f32 = a.score_dtype == CSA_F32;
+  p.all_visible = a.all_visible;
+  p.dep_tile = a.dep_entry < 0 ? 0 : a.dep_entry / kTileE;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
@@ -319,8 +343,9 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  kern<<<(int)grid, 192, smem, st>>>(tmK, tmQ, tmKS, tmW, tmQS, p);
-  CSA_CHECK_LAUNCH();
+  if (csa_launch(kern, dim3((unsigned)grid), dim3(192), smem, st, a.pdl != 0, tmK, tmQ, tmKS, tmW,
+                 tmQS, p) != cudaSuccess)
+    return CSA_ERR_CUDA;
   return CSA_OK;
 }
 

@@ -30,6 +30,10 @@ struct IndexArgs {
   const void* k; const void* k_scales; const int32_t* q_pos;
   int T, H, d, m, qk_dtype, score_dtype, E_cap, E;
   void* scores;
+  int pdl;            // launch as a programmatic dependent of the preceding kernel
+  int all_visible;    // every query sees all E entries (decode at t = L-1): q_pos is not read
+  int dep_entry;      // first entry the preceding kernel writes (tiles before it may be
+                      // fetched before waiting on that kernel); -1: all depend
 };
 
 struct AttnArgs {
@@ -38,6 +42,7 @@ struct AttnArgs {
   int T, H, d, n_w, m, k, E_cap, n;
   float scale;
   void* out; float* lse;
+  int pdl;            // launch as a programmatic dependent of the preceding kernel
 };
 
 csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry_count,
@@ -47,7 +52,7 @@ csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows,
                            void* codes, void* scales, cudaStream_t st);
 csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
                               int rows, int E, int k, int32_t* idx, int32_t* count, void* ws,
-                              size_t ws_bytes, cudaStream_t st);
+                              size_t ws_bytes, cudaStream_t st, bool pdl = false);
 size_t topk_workspace_bytes(int rows, int E, int k, int score_dtype);
 csa_status launch_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int rows,
                        int E, int k, int32_t* idx, int32_t* count, cudaStream_t st);

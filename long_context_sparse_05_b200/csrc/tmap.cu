@@ -109,3 +109,26 @@ extern "C" int csa_device_error(cudaStream_t stream) {
   if (cudaMemcpy(p, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return CSA_ERR_CUDA;
   return v;
 }
+
+namespace csa {
+namespace {
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// ever arrives on; the wait gives up after limit_ns and records CSA_ERR_TIMEOUT.
+__global__ void bounded_wait_selftest_kernel(uint64_t limit_ns, int* err) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    tc::mbar_init(&bar, 1);
+    tc::fence_barrier_init();
+    tc::mbar_wait(&bar, 0, err, limit_ns);
+  }
+}
+}  // namespace
+}  // namespace csa
+
+extern "C" csa_status csa_selftest_bounded_wait(int limit_us, cudaStream_t stream) {
+  if (limit_us < 1 || limit_us > 100000) return CSA_ERR_INVALID_ARG;
+  int* err = csa::device_error_word();
+  if (!err) return CSA_ERR_CUDA;
+  csa::bounded_wait_selftest_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000u, err);
+  return cudaGetLastError() == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}

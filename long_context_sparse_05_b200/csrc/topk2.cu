@@ -246,6 +246,8 @@ __global__ void __launch_bounds__(kNT) topk_row_kernel(
     const S* __restrict__ scores, const int32_t* __restrict__ q_pos, int m, int E, int k,
     int32_t* __restrict__ idx, int32_t* __restrict__ count) {
   __shared__ uint32_t s_red[72];
+  pdl_launch_dependents();
+  pdl_wait();
   const int row = blockIdx.x;
   const int ev = visible_entries(q_pos[row], m, E);
   cta_topk<S>(scores + (size_t)row * E, ev, k, nullptr, 0, idx + (size_t)row * k, count + row,
@@ -258,6 +260,8 @@ __global__ void __launch_bounds__(kNT) topk_chunk_kernel(
     const S* __restrict__ scores, const int32_t* __restrict__ q_pos, int m, int E, int k,
     int nchunks, S* __restrict__ cand_scores, int32_t* __restrict__ cand_idx) {
   __shared__ uint32_t s_red[72];
+  pdl_launch_dependents();
+  pdl_wait();
   const int row = blockIdx.x / nchunks, c = blockIdx.x % nchunks;
   const int ev = visible_entries(q_pos[row], m, E);
   const int beg = c * kChunk;
@@ -275,6 +279,8 @@ __global__ void __launch_bounds__(kNT) topk_merge_kernel(
     const int32_t* __restrict__ q_pos, int m, int E, int k, int nchunks,
     int32_t* __restrict__ idx, int32_t* __restrict__ count) {
   __shared__ uint32_t s_red[72];
+  pdl_launch_dependents();
+  pdl_wait();
   const int row = blockIdx.x;
   const int ev = visible_entries(q_pos[row], m, E);
   const size_t slot = (size_t)row * nchunks * k;
@@ -306,20 +312,18 @@ size_t topk_workspace_bytes(int rows, int E, int k, int score_dtype) {
 // pass (needs ws of topk_workspace_bytes), as long as all candidates fit one CTA.
 csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
                               int rows, int E, int k, int32_t* idx, int32_t* count, void* ws,
-                              size_t ws_bytes, cudaStream_t st) {
+                              size_t ws_bytes, cudaStream_t st, bool pdl) {
   if (rows == 0) return CSA_OK;
   if (k > kChunk) return CSA_ERR_UNSUPPORTED;
   const bool bf = score_dtype == CSA_BF16;
   if (E <= kChunk) {
     const int nt = threads_for(E);
-    if (bf)
-      topk_row_kernel<__nv_bfloat16><<<rows, nt, 0, st>>>(
-          reinterpret_cast<const __nv_bfloat16*>(scores), q_pos, m, E, k, idx, count);
-    else
-      topk_row_kernel<float><<<rows, nt, 0, st>>>(reinterpret_cast<const float*>(scores), q_pos,
-                                                  m, E, k, idx, count);
-    CSA_CHECK_LAUNCH();
-    return CSA_OK;
+    const cudaError_t e =
+        bf ? csa_launch(topk_row_kernel<__nv_bfloat16>, dim3(rows), dim3(nt), 0, st, pdl,
+                        reinterpret_cast<const __nv_bfloat16*>(scores), q_pos, m, E, k, idx, count)
+           : csa_launch(topk_row_kernel<float>, dim3(rows), dim3(nt), 0, st, pdl,
+                        reinterpret_cast<const float*>(scores), q_pos, m, E, k, idx, count);
+    return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
   }
   const size_t need = topk_workspace_bytes(rows, E, k, score_dtype);
   if (need == 0) return CSA_ERR_UNSUPPORTED;
@@ -329,23 +333,25 @@ csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t
   int32_t* cand_idx = static_cast<int32_t*>(ws);
   void* cand_sc = cand_idx + ncand;
   const int nt2 = threads_for(nchunks * k);
+  cudaError_t e;
   if (bf) {
-    topk_chunk_kernel<__nv_bfloat16><<<rows * nchunks, kNT, 0, st>>>(
-        reinterpret_cast<const __nv_bfloat16*>(scores), q_pos, m, E, k, nchunks,
-        static_cast<__nv_bfloat16*>(cand_sc), cand_idx);
-    CSA_CHECK_LAUNCH();
-    topk_merge_kernel<__nv_bfloat16><<<rows, nt2, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(cand_sc), cand_idx, q_pos, m, E, k, nchunks, idx, count);
+    e = csa_launch(topk_chunk_kernel<__nv_bfloat16>, dim3(rows * nchunks), dim3(kNT), 0, st, pdl,
+                   reinterpret_cast<const __nv_bfloat16*>(scores), q_pos, m, E, k, nchunks,
+                   static_cast<__nv_bfloat16*>(cand_sc), cand_idx);
+    if (e == cudaSuccess)
+      e = csa_launch(topk_merge_kernel<__nv_bfloat16>, dim3(rows), dim3(nt2), 0, st, pdl,
+                     static_cast<const __nv_bfloat16*>(cand_sc), (const int32_t*)cand_idx, q_pos,
+                     m, E, k, nchunks, idx, count);
   } else {
-    topk_chunk_kernel<float><<<rows * nchunks, kNT, 0, st>>>(
-        reinterpret_cast<const float*>(scores), q_pos, m, E, k, nchunks,
-        static_cast<float*>(cand_sc), cand_idx);
-    CSA_CHECK_LAUNCH();
-    topk_merge_kernel<float><<<rows, nt2, 0, st>>>(static_cast<const float*>(cand_sc), cand_idx,
-                                                   q_pos, m, E, k, nchunks, idx, count);
+    e = csa_launch(topk_chunk_kernel<float>, dim3(rows * nchunks), dim3(kNT), 0, st, pdl,
+                   reinterpret_cast<const float*>(scores), q_pos, m, E, k, nchunks,
+                   static_cast<float*>(cand_sc), cand_idx);
+    if (e == cudaSuccess)
+      e = csa_launch(topk_merge_kernel<float>, dim3(rows), dim3(nt2), 0, st, pdl,
+                     static_cast<const float*>(cand_sc), (const int32_t*)cand_idx, q_pos, m, E, k,
+                     nchunks, idx, count);
   }
-  CSA_CHECK_LAUNCH();
-  return CSA_OK;
+  return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
 }
 
 }  // namespace csa

