@@ -37,6 +37,13 @@
  *  - CSA_NVFP4: two E2M1 codes per byte (element 2j in bits 0-3, 2j+1 in bits
  *    4-7), plus one UE4M3 scale byte per 16 consecutive elements:
  *    value = decode(code) * decode(scale), scale = e4m3(amax(block) / 6).
+ *    Query scales (and csa_quantize output) are row-major [rows][d/16].  Key
+ *    caches (csa_compress output, k_I of the indexer, kI_scales of the fused
+ *    calls) keep their scales TILED, in the order the block-scaled tensor-core
+ *    MMA reads them: a sequence of E_cap entries owns ceil(E_cap/128) tiles of
+ *    128 * d/16 bytes (d a multiple of 64); inside a tile, the scale of block j
+ *    of entry r (0..127) is at byte (j/4)*512 + (r%32)*16 + (r/32)*4 + j%4.
+ *    The buffer is therefore [b][ceil(E_cap/128)*128][d/16] bytes.
  */
 #ifndef CSA_H_
 #define CSA_H_
@@ -114,7 +121,7 @@ csa_status csa_selftest_bounded_wait(int limit_us, cudaStream_t stream);
 typedef struct {
   int m;              /* compression rate (>= 1) */
   int overlap;        /* 1: previous block from the b-branch joins; 0: current block only */
-  int c;              /* channels per entry; multiple of 8 (of 16 for NVFP4 output) */
+  int c;              /* channels per entry; multiple of 8 (of 64 for NVFP4 output) */
   int d_rope;         /* rotary dims at the end of each entry; even, <= c; 0 = none */
   double rope_theta;  /* RoPE base (10000) */
   float eps;          /* RMSNorm epsilon (1e-6) */
@@ -134,8 +141,9 @@ typedef struct {
  *              c bytes (FP8) or c/2 bytes (NVFP4); entry i of sequence s is
  *              written at row s * out_entries_per_seq + i (caches are updated
  *              in place, other rows untouched)
- *   out_scales FP8: float32 [b][out_entries_per_seq]; NVFP4: uint8
- *              [b][out_entries_per_seq][c/16]; NULL for F32/BF16
+ *   out_scales FP8: float32 [b][out_entries_per_seq]; NVFP4: the tiled key-scale
+ *              layout (above), [b][ceil(out_entries_per_seq/128)*128][c/16] bytes,
+ *              c a multiple of 64; NULL for F32/BF16
  */
 csa_status csa_compress(const csa_compress_params* p,
                         const void* C_a, const void* Z_a, const float* B_a,
@@ -179,7 +187,9 @@ typedef struct {
  *   q_I       [b][T][H_I][row]  codes (row as in csa_compress for qk_dtype)
  *   q_scales  FP8: float32 [b][T][H_I]; NVFP4: uint8 [b][T][H_I][d_I/16]; F32: NULL
  *   w         [b][T][H_I] float32 head weights
- *   k_I       [b][E_cap][row] codes;  k_scales like q_scales per entry
+ *   k_I       [b][E_cap][row] codes;  k_scales FP8: float32 [b][E_cap]; NVFP4: the
+ *             tiled key-scale layout, [b][ceil(E_cap/128)*128][d_I/16] bytes (d_I a
+ *             multiple of 64)
  *   q_pos     [b][T] int32 position t of each query
  *   scores    [b][T][E] (score_dtype), E <= E_cap entries scored per query
  */
@@ -325,7 +335,7 @@ typedef struct {
   const float *BI_a, *BI_b;            /* [m][c_I] (CSA) */
   void* kv_cache;                      /* [b][E_cap][c] kv_dtype; entry E-1 written */
   void* kI_cache;                      /* [b][E_cap][row] idx_dtype codes; entry E-1 written */
-  void* kI_scales;                     /* FP8: float32 [b][E_cap]; NVFP4: uint8 [b][E_cap][c_I/16] */
+  void* kI_scales;                     /* FP8: float32 [b][E_cap]; NVFP4: tiled, see above */
   const void* kv_win;                  /* [b][L][c] raw window rows */
   const void* q;                       /* [b][H][c] */
   const void* q_I;                     /* [b][H_I][c_I] unquantised (kv_dtype) */

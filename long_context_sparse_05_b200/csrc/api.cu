@@ -63,7 +63,7 @@ csa_status csa_compress(const csa_compress_params* p, const void* C_a, const voi
     return CSA_ERR_INVALID_ARG;
   if (p->in_dtype != CSA_F32 && p->in_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
   if (p->out_dtype < CSA_F32 || p->out_dtype > CSA_NVFP4) return CSA_ERR_INVALID_ARG;
-  if (p->out_dtype == CSA_NVFP4 && p->c % 16) return CSA_ERR_INVALID_ARG;
+  if (p->out_dtype == CSA_NVFP4 && p->c % 64) return CSA_ERR_INVALID_ARG;   // tiled key scales
   if (p->in_dtype == CSA_F32 && p->c % 4) return CSA_ERR_INVALID_ARG;
   if (b < 0 || n < 0 || entry_begin < 0 || entry_count < 0) return CSA_ERR_INVALID_ARG;
   if ((long long)p->m * (entry_begin + entry_count) > n) return CSA_ERR_INVALID_ARG;
@@ -111,6 +111,7 @@ csa_status index_scores_impl(const csa_index_params* p, const void* q_I, const v
   if (b == 0 || T == 0 || E == 0) return CSA_OK;
   if (!q_I || !w || !k_I || !q_pos || !scores) return CSA_ERR_INVALID_ARG;
   if (p->qk_dtype != CSA_F32 && (!q_scales || !k_scales)) return CSA_ERR_INVALID_ARG;
+  if (p->qk_dtype == CSA_NVFP4 && p->d_I % 64) return CSA_ERR_INVALID_ARG;   // tiled key scales
   IndexArgs a{};
   a.q = q_I; a.q_scales = q_scales; a.w = w; a.k = k_I; a.k_scales = k_scales; a.q_pos = q_pos;
   a.T = T; a.H = p->H_I; a.d = p->d_I; a.m = p->m; a.qk_dtype = p->qk_dtype;
@@ -275,6 +276,7 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
     return CSA_ERR_INVALID_ARG;
   if (!p->hca && (p->c_I % 16 || p->d_rope_I < 0 || p->d_rope_I % 2 || p->d_rope_I > p->c_I))
     return CSA_ERR_INVALID_ARG;
+  if (!p->hca && p->idx_dtype == CSA_NVFP4 && p->c_I % 64) return CSA_ERR_INVALID_ARG;
   if (!aligned16(x->C_a) || !aligned16(x->Z_a) ||
       (!p->hca && (!aligned16(x->C_b) || !aligned16(x->Z_b) || !aligned16(x->CI_a) ||
                    !aligned16(x->ZI_a) || !aligned16(x->CI_b) || !aligned16(x->ZI_b))))

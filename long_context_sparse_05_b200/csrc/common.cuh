@@ -88,6 +88,22 @@ __device__ __forceinline__ void pdl_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// NVFP4 key-scale layout.  A sequence's key scales are stored in tiles of 128
+// entries, each tile in the order the block-scaled tensor-core MMA reads from
+// tensor memory (tcgen05.cp 32x128b, 4x replicated): for every 64-element K
+// block, 512 bytes laid out as [row % 32][row / 32][block % 4].  A sequence of
+// E_cap entries occupies ceil(E_cap / 128) tiles of 128 * c / 16 bytes
+// (c a multiple of 64).
+__host__ __device__ __forceinline__ size_t nvfp4_key_scale_offset(long long e, int blk, int c) {
+  const long long tile = e >> 7;
+  const int r = (int)(e & 127);
+  return (size_t)tile * (size_t)(8 * c) + (size_t)(blk >> 2) * 512 + (size_t)(r & 31) * 16 +
+         (size_t)(r >> 5) * 4 + (size_t)(blk & 3);
+}
+__host__ __device__ __forceinline__ size_t nvfp4_key_scale_seq_bytes(long long E_cap, int c) {
+  return (size_t)((E_cap + 127) >> 7) * (size_t)(8 * c);
+}
+
 // Visible entries of query position t: floor((t+1)/m), clamped to [0, E].
 __device__ __forceinline__ int visible_entries(int t, int m, int E) {
   int e = t < 0 ? 0 : (t + 1) / m;

@@ -198,7 +198,7 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
     if (tid == 0) reinterpret_cast<float*>(a.out_scales)[orow] = scale;
   } else {  // CSA_NVFP4
     uint8_t* o = reinterpret_cast<uint8_t*>(a.out) + orow * (c / 2);
-    uint8_t* so = reinterpret_cast<uint8_t*>(a.out_scales) + orow * (c / 16);
+    uint8_t* so = reinterpret_cast<uint8_t*>(a.out_scales) + (size_t)s * nvfp4_key_scale_seq_bytes(a.out_E, c);
     for (int blk = tid; blk < c / 16; blk += blockDim.x) {
       float am = 0.f;
 #pragma unroll
@@ -211,7 +211,7 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
             ? f32x2_to_e2m1x2(s_x[blk * 16 + e] / sv, s_x[blk * 16 + e + 1] / sv)
             : (uint8_t)0;
       }
-      so[blk] = sc;
+      so[nvfp4_key_scale_offset(i, blk, c)] = sc;
     }
   }
 }

@@ -14,16 +14,29 @@
 // Layout of one MMA (M = 128 entries, N = 64 heads, K = 64 elements): A and B are
 // K-major tiles with 64-byte swizzle (rows of 64 bytes = all 128 elements, two
 // MMAs of 32 bytes each).  Scale factors live in TMEM: for each K block of 64,
-// four columns hold the four UE4M3 scales of rows 0-31, 32-63, 64-95, 96-127
-// (one byte per 16-element block), replicated in all four lane quarters; they are
-// brought there from shared memory by tcgen05.cp 32x128b.warpx4 after the MMA warp
-// has rearranged the raw per-row scales (8 bytes per row) into that order.
+// four columns hold the four UE4M3 scales of rows 0-31, 32-63, 64-95, 96-127,
+// replicated in all four lane quarters, copied there by tcgen05.cp 32x128b.warpx4.
+// The key cache keeps its scales in exactly that order (tiles of 128 entries, see
+// nvfp4_key_scale_offset), so a stage's scales go from HBM to shared memory in
+// one bulk copy and on to TMEM without any rearrangement.  Query scales arrive
+// row-major and are rearranged once per work unit.
 //
-// CTA (192 threads), one query per work unit (decode):
-//   warp 0  TMA producer: per tile the key block (8 KB) and its raw scales (1 KB);
-//           per unit the query block (4 KB), its raw scales and head weights;
-//   warp 1  scale rearrangement (all lanes) and MMA issue (lane 0);
-//   warps 2-5 epilogue: tcgen05.ld, weighted ReLU head sum, causal mask, store.
+// Pipeline granularity: a stage is two tiles (256 entries, 16 KB of codes + 2 KB
+// of scales), so the MMA warp pays one stage wait and one accumulator wait per
+// four MMAs; on sm_100a a thread's first shared-memory access after issuing
+// tcgen05 operations costs a few hundred cycles, so per-stage waits are what the
+// issue rate is made of.
+//
+// CTA (320 threads), one query per work unit (decode):
+//   warp 0  producer: per stage one 2-D TMA box of 256 key rows and one bulk copy
+//           of the stage's scales; per unit the query codes (TMA), its raw scales
+//           and head weights;
+//   warp 1  query-scale rearrangement (all lanes, once per unit) and MMA issue
+//           (lane 0): 4 tcgen05.cp + 4 MMAs per stage into one of NACC
+//           accumulators of 2 x 64 columns;
+//   warps 2-9 epilogue, two warpgroups taking alternate stages (warps w and w+4
+//           share a TMEM lane quarter): tcgen05.ld, weighted ReLU head sum with the
+//           weights read as broadcast 128-bit shared loads, causal mask, store.
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -32,32 +45,41 @@ namespace csa {
 namespace {
 
 constexpr int kTileE = 128;
+constexpr int kTPS = 2;                          // tiles per stage
+constexpr int kStageE = kTileE * kTPS;           // 256 entries
 constexpr int kHeads = 64;
-constexpr int kRowB = 64;                    // bytes per FP4 row (128 elements)
-constexpr int kSfRowB = 8;                   // scale bytes per row
-constexpr int kTileBytes = kTileE * kRowB;   // 8 KB
-constexpr int kTileSf = kTileE * kSfRowB;    // 1 KB raw scales
-constexpr int kQBytes = kHeads * kRowB;      // 4 KB
-constexpr int kQSf = kHeads * kSfRowB;       // 512 B raw scales
-constexpr int kPermBytes = 2 * 512;          // two K blocks in the tcgen05.cp layout
-constexpr int NACC = 4;
-constexpr int S = 12;                        // stages: also keeps one CTA per SM (TMEM)
+constexpr int kDim = 128;                        // elements per row
+constexpr int kRowB = 64;                        // bytes per FP4 row
+constexpr int kSfTileB = 1024;                   // scale bytes of one tile (tiled layout)
+constexpr int kKeyB = kStageE * kRowB;           // 16 KB
+constexpr int kStage = kKeyB + kTPS * kSfTileB;  // 18 KB, a multiple of 1 KB
+constexpr int kQBytes = kHeads * kRowB;          // 4 KB
+constexpr int kQSf = kHeads * 8;                 // 512 B raw query scales
+constexpr int kPermBytes = 2 * 512;              // query scales in the tcgen05.cp layout
+constexpr int NACC = 3;                          // accumulators of kTPS x 64 columns
+constexpr int S = 8;                             // stages
 constexpr int kMaxLocalUnits = 256;
+constexpr int kEpiGroups = 2;
+constexpr int kThreads = 64 + 128 * kEpiGroups;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = kTPS * kHeads;     // 128
+constexpr uint32_t kSfaCol = NACC * kAccCols;    // 384: NACC x (kTPS x 8) key-scale columns
+constexpr uint32_t kSfbCol = kSfaCol + NACC * kTPS * 8;   // 432: 2 x 8 query-scale columns
+static_assert(kSfbCol + 16 <= kTmemCols, "TMEM budget");
+static_assert(kStage % 1024 == 0, "stages must keep the swizzle alignment");
 
 struct IdxFp4 {
   void* scores;
   const int32_t* q_pos;
+  const uint8_t* k_scales;
   int* err;
   int T, E_cap, E, m;
-  int tiles, chunk, n_chunks, units;
+  int tiles, sf_tiles_cap, stages, chunk, n_chunks, units;
   int score_f32;
   int all_visible;   // every query sees all E entries: q_pos is not read
-  int dep_tile;      // tiles >= dep_tile hold entries the preceding kernel writes
+  int dep_stage;     // stages >= dep_stage hold entries the preceding kernel writes
 };
 
-// Stage layout (bytes): keys | raw scales | rearranged scales.
-constexpr int kStage = kTileBytes + kTileSf + kPermBytes;   // 10 KB: keeps 1 KB alignment
-static_assert(kStage % 1024 == 0, "stages must keep the swizzle alignment");
 // Query buffer: codes | raw scales | rearranged scales | weights, padded to 1 KB so
 // that the swizzled code block of either buffer starts on a 1 KB boundary.
 constexpr int kQBuf = ((kQBytes + kQSf + kPermBytes + kHeads * 4) + 1023) / 1024 * 1024;
@@ -101,8 +123,16 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
                : "memory");
 }
 
-// Lane m0 of the warp rearranges the raw scales of `rows` rows (8 bytes each) into the
-// tcgen05.cp order for both K blocks: word (m0, m1) of block kb = raw word (m0 + 32 m1) * 2 + kb.
+// Untiled bulk copy global -> shared; completion counted on `bar` as transaction bytes.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar)) : "memory");
+}
+
+// Lane m0 of the warp rearranges the row-major query scales (8 bytes per row, `rows`
+// rows) into the tcgen05.cp order for both K blocks: word (m0, m1) of block kb =
+// raw word (m0 + 32 m1) * 2 + kb.
 __device__ __forceinline__ void rearrange_scales(const uint8_t* raw, uint8_t* perm, int rows,
                                                  int lane) {
   const uint32_t* rw = reinterpret_cast<const uint32_t*>(raw);
@@ -118,12 +148,11 @@ __device__ __forceinline__ void rearrange_scales(const uint8_t* raw, uint8_t* pe
   }
 }
 
-__global__ void __launch_bounds__(192, 1)
-index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmKS,
-                        const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmQS,
-                        const __grid_constant__ CUtensorMap tmW, IdxFp4 p) {
+__global__ void __launch_bounds__(kThreads, 1)
+index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
+                        const __grid_constant__ CUtensorMap tmQS, const __grid_constant__ CUtensorMap tmW,
+                        IdxFp4 p) {
   constexpr int N = kHeads;
-  constexpr uint32_t kTmemCols = 512;    // 4 x 64 accumulator + 4 x 8 key-scale + 2 x 8 query-scale
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sStage = base;                               // S x kStage
@@ -136,9 +165,8 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   uint64_t* tfull = bempty + 2;
   uint64_t* tempty = tfull + NACC;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + NACC);
-  float* s_w = reinterpret_cast<float*>(tmem_holder + 4);     // [64] weights of the current unit
-  int* s_vis = reinterpret_cast<int*>(s_w + N);               // [kMaxLocalUnits]
-  int* s_ev = s_vis + kMaxLocalUnits;                         // [kMaxLocalUnits]
+  int* s_vis = reinterpret_cast<int*>(tmem_holder + 4);      // [kMaxLocalUnits] visible stages
+  int* s_ev = s_vis + kMaxLocalUnits;                         // [kMaxLocalUnits] visible entries
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -151,56 +179,63 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     const int row = u / p.n_chunks;
     const int ev = p.all_visible ? p.E : visible_entries(p.q_pos[row], p.m, p.E);
     s_ev[i] = ev;
-    s_vis[i] = (ev + kTileE - 1) / kTileE;
+    s_vis[i] = (ev + kStageE - 1) / kStageE;
   }
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S; ++i) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], 1 + 4); }
-    for (int i = 0; i < 2; ++i) { tc::mbar_init(&bfull[i], 1); tc::mbar_init(&bempty[i], 1 + 4); }
+    for (int i = 0; i < S; ++i) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], 1); }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bfull[i], 1);
+      tc::mbar_init(&bempty[i], 1 + 4 * kEpiGroups);
+    }
     for (int i = 0; i < NACC; ++i) { tc::mbar_init(&tfull[i], 1); tc::mbar_init(&tempty[i], 4); }
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tmK);
-    tc::tma_prefetch_desc(&tmKS);
   }
   if (warp == 0) tc::tmem_alloc(tmem_holder, kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
-  const uint32_t t_sfa = tmem_base + NACC * N;          // NACC x 8 columns
-  const uint32_t t_sfb = t_sfa + NACC * 8;              // 2 x 8 columns
 
-  auto unit = [&](int u, int i, int& row, int& j0, int& j1, int& nc) {
+  // stages [js0, js1) of row `row`; the first nc of them are visible and computed
+  auto unit = [&](int u, int i, int& row, int& js0, int& js1, int& nc) {
     row = u / p.n_chunks;
     const int ch = u % p.n_chunks;
-    j0 = ch * p.chunk;
-    j1 = min(p.tiles, j0 + p.chunk);
-    nc = max(0, min(j1, s_vis[i]) - j0);
+    js0 = ch * p.chunk;
+    js1 = min(p.stages, js0 + p.chunk);
+    nc = max(0, min(js1, s_vis[i]) - js0);
   };
 
   if (warp == 0) {
     if (lane == 0) {
-      // key tiles the preceding kernel does not write are fetched before waiting on it
+      // ---------------------------------------------------------------- producer
+      const int sf_seq = p.sf_tiles_cap;
+      auto load_stage = [&](int slot, int row, int js) {
+        const int sb = row / p.T;
+        const int j0 = js * kTPS;                                // first tile of the stage
+        const int nsf = min(kTPS, sf_seq - j0);                  // scale tiles inside the sequence
+        uint8_t* st = sStage + slot * kStage;
+        tc::mbar_arrive_expect_tx(&full[slot], kKeyB + nsf * kSfTileB);
+        tc::tma_load_2d(st, &tmK, 0, sb * p.E_cap + j0 * kTileE, &full[slot]);
+        bulk_load(st + kKeyB, p.k_scales + ((size_t)sb * sf_seq + j0) * kSfTileB,
+                  nsf * kSfTileB, &full[slot]);
+      };
+      // key stages the preceding kernel does not write are fetched before waiting on it
       uint32_t npre = 0;
       for (int u = blockIdx.x, i = 0; u < p.units && npre == 0; u += gridDim.x, ++i) {
-        int row, j0, j1, nc;
-        unit(u, i, row, j0, j1, nc);
+        int row, js0, js1, nc;
+        unit(u, i, row, js0, js1, nc);
         if (nc == 0) continue;
-        const int sb = row / p.T;
-        for (int j = j0; j < j0 + nc && (int)npre < S && j < p.dep_tile; ++j, ++npre) {
-          const int row0 = sb * p.E_cap + j * kTileE;
-          uint8_t* st = sStage + npre * kStage;
-          tc::mbar_arrive_expect_tx(&full[npre], kTileBytes + kTileSf);
-          tc::tma_load_2d(st, &tmK, 0, row0, &full[npre]);
-          tc::tma_load_2d(st + kTileBytes, &tmKS, 0, row0 / 2, &full[npre]);
-        }
+        for (int js = js0; js < js0 + nc && (int)npre < S && js < p.dep_stage; ++js, ++npre)
+          load_stage(npre, row, js);
         break;
       }
       pdl_wait();
       uint32_t it = 0, ul = 0;
       bool ok = true;
       for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
-        int row, j0, j1, nc;
-        unit(u, i, row, j0, j1, nc);
+        int row, js0, js1, nc;
+        unit(u, i, row, js0, js1, nc);
         if (nc == 0) continue;
         const int bb = ul & 1;
         ok = tc::mbar_wait(&bempty[bb], ((ul >> 1) & 1) ^ 1, p.err);
@@ -210,28 +245,24 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         tc::tma_load_2d(qb, &tmQ, 0, row * kHeads, &bfull[bb]);
         tc::tma_load_2d(qb + kQBytes, &tmQS, 0, row * kHeads / 2, &bfull[bb]);
         tc::tma_load_1d(qb + kQBytes + kQSf + kPermBytes, &tmW, row * kHeads, &bfull[bb]);
-        const int sb = row / p.T;
-        for (int j = j0; j < j0 + nc; ++j, ++it) {
+        for (int js = js0; js < js0 + nc; ++js, ++it) {
           if (it < npre) continue;                       // fetched before the wait
           const int s = it % S;
           ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
           if (!ok) break;
-          const int row0 = sb * p.E_cap + j * kTileE;
-          uint8_t* st = sStage + s * kStage;
-          tc::mbar_arrive_expect_tx(&full[s], kTileBytes + kTileSf);
-          tc::tma_load_2d(st, &tmK, 0, row0, &full[s]);
-          tc::tma_load_2d(st + kTileBytes, &tmKS, 0, row0 / 2, &full[s]);
+          load_stage(s, row, js);
         }
         ++ul;
       }
     }
   } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
     constexpr uint32_t idesc = idesc_mxf4(kTileE, N);
-    uint32_t it = 0, ul = 0, at = 0;
+    uint32_t it = 0, ul = 0;
     bool ok = true;
     for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
-      int row, j0, j1, nc;
-      unit(u, i, row, j0, j1, nc);
+      int row, js0, js1, nc;
+      unit(u, i, row, js0, js1, nc);
       if (nc == 0) continue;
       const int bb = ul & 1;
       uint8_t* qb = sQ + bb * kQBuf;
@@ -240,102 +271,118 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       rearrange_scales(qb + kQBytes, qb + kQBytes + kQSf, kHeads, lane);
       tc::fence_proxy_async();
       __syncwarp();
-      const uint32_t sfb = t_sfb + bb * 8;
       if (lane == 0) {
+        const uint32_t sfb = tmem_base + kSfbCol + bb * 8;
         tc::tc_fence_after();
         tmem_cp_32x128b_x4(sfb, smem_desc_cp(tc::smem_u32(qb + kQBytes + kQSf)));
         tmem_cp_32x128b_x4(sfb + 4, smem_desc_cp(tc::smem_u32(qb + kQBytes + kQSf + 512)));
-      }
-      const uint64_t bdesc = smem_desc_sw64(tc::smem_u32(qb), 512);
-      for (int j = 0; j < nc; ++j, ++it, ++at) {
-        const int s = it % S;
-        const int acc = at % NACC;
-        uint8_t* st = sStage + s * kStage;
-        ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err);
-        if (!ok) break;
-        rearrange_scales(st + kTileBytes, st + kTileBytes + kTileSf, kTileE, lane);
-        tc::fence_proxy_async();
-        __syncwarp();
-        if (lane == 0) {
-          ok = tc::mbar_wait(&tempty[acc], ((at / NACC) & 1) ^ 1, p.err);
-          if (ok) {
-            tc::tc_fence_after();
-            const uint32_t sfa = t_sfa + acc * 8;
-            tmem_cp_32x128b_x4(sfa, smem_desc_cp(tc::smem_u32(st + kTileBytes + kTileSf)));
-            tmem_cp_32x128b_x4(sfa + 4, smem_desc_cp(tc::smem_u32(st + kTileBytes + kTileSf + 512)));
-            const uint64_t adesc = smem_desc_sw64(tc::smem_u32(st), 512);
-            const uint32_t d = tmem_base + acc * N;
+        const uint64_t bdesc = smem_desc_sw64(tc::smem_u32(qb), 512);
+        for (int j = 0; j < nc && ok; ++j, ++it) {
+          const int s = it % S;
+          const int acc = it % NACC;
+          uint8_t* st = sStage + s * kStage;
+          // both waits back to back: the first shared-memory access after the previous
+          // stage's tcgen05 operations carries the cost, the second is cheap
+          ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err) &&
+               tc::mbar_wait(&tempty[acc], ((it / NACC) & 1) ^ 1, p.err);
+          if (!ok) break;
+          tc::tc_fence_after();
+          const uint32_t sfa = tmem_base + kSfaCol + acc * (kTPS * 8);
+#pragma unroll
+          for (int t = 0; t < kTPS; ++t) {
+            const uint32_t src = tc::smem_u32(st + kKeyB + t * kSfTileB);
+            tmem_cp_32x128b_x4(sfa + t * 8, smem_desc_cp(src));
+            tmem_cp_32x128b_x4(sfa + t * 8 + 4, smem_desc_cp(src + 512));
+          }
+#pragma unroll
+          for (int t = 0; t < kTPS; ++t) {
+            const uint64_t adesc = smem_desc_sw64(tc::smem_u32(st + t * kTileE * kRowB), 512);
+            const uint32_t d = tmem_base + acc * kAccCols + t * N;
 #pragma unroll
             for (int kb = 0; kb < 2; ++kb)   // K = 64 elements = 32 bytes per MMA
-              mma_mxf4nvf4(d, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa + 4 * kb, sfb + 4 * kb,
-                           kb > 0);
-            tc::mma_commit(&empty[s]);
-            tc::mma_commit(&tfull[acc]);
+              mma_mxf4nvf4(d, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa + t * 8 + 4 * kb,
+                           sfb + 4 * kb, kb > 0);
           }
+          tc::mma_commit(&empty[s]);
+          tc::mma_commit(&tfull[acc]);
         }
-        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        if (!ok) break;
+        if (ok) tc::mma_commit(&bempty[bb]);
       }
-      if (!ok) break;
-      if (lane == 0) tc::mma_commit(&bempty[bb]);
-      __syncwarp();
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      it = __shfl_sync(0xffffffffu, it, 0);
       ++ul;
     }
   } else {
-    const int lane_base = (warp & 3) * 32;
-    const int etid = threadIdx.x - 64;
-    uint32_t it = 0, at = 0, ul = 0;
+    // ------------------------------------------------------------------ epilogue
+    const int grp = (warp - 2) >> 2;         // warpgroup: takes stages with c % 2 == grp
+    const int lane_base = (warp & 3) * 32;   // TMEM lanes this warp may access
+    uint32_t c = 0, ul = 0;                  // computed stages seen, units with work seen
     bool ok = true;
     for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
-      int row, j0, j1, nc;
-      unit(u, i, row, j0, j1, nc);
-      if (nc > 0) {
-        const int bb = ul & 1;
-        tc::named_bar(1, 128);
-        ok = ok && tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
-        const float* wsrc = reinterpret_cast<const float*>(sQ + bb * kQBuf + kQBytes + kQSf + kPermBytes);
-        if (etid < N) s_w[etid] = wsrc[etid];
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(&bempty[bb]);
-        tc::named_bar(1, 128);
-        ++ul;
-      }
+      int row, js0, js1, nc;
+      unit(u, i, row, js0, js1, nc);
+      // head weights of the unit, read (broadcast) from the query buffer, which is
+      // released once this warp is done with the unit
+      const float4* w4p = reinterpret_cast<const float4*>(sQ + (ul & 1) * kQBuf + kQBytes + kQSf +
+                                                          kPermBytes);
+      if (nc > 0) ok = ok && tc::mbar_wait(&bfull[ul & 1], (ul >> 1) & 1, p.err);
       const int ev = s_ev[i];
-      for (int j = j0; j < j1; ++j) {
-        const int e = j * kTileE + lane_base + lane;
-        float sc = -INFINITY;
-        if (j < j0 + nc && ok) {
-          const int s = it % S;
-          const int acc = at % NACC;
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&empty[s]);   // epilogue reads nothing from the stage
-          ok = tc::mbar_wait(&tfull[acc], (at / NACC) & 1, p.err);
-          tc::tc_fence_after();
-          uint32_t r0[32], r1[32];
-          const uint32_t ta = tmem_base + ((uint32_t)lane_base << 16) + acc * N;
-          tc::tmem_ld32(ta, r0);
-          tc::tmem_ld32(ta + 32, r1);
-          tc::tmem_ld_wait(r0);
-          tc::reg_fence(r1);
-          float a0 = 0.f, a1 = 0.f;
+      for (int js = js0; js < js1; ++js) {
+        float sc[kTPS];
 #pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            a0 = fmaf(s_w[h], fmaxf(__uint_as_float(r0[h]), 0.f), a0);
-            a1 = fmaf(s_w[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), a1);
+        for (int t = 0; t < kTPS; ++t) sc[t] = -INFINITY;
+        if (js < js0 + nc) {
+          const uint32_t cc = c++;
+          if ((int)(cc & 1) != grp) continue;           // the other warpgroup's stage
+          if (ok) {
+            const int acc = cc % NACC;
+            ok = tc::mbar_wait(&tfull[acc], (cc / NACC) & 1, p.err);
+            tc::tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < kTPS; ++t) {
+              uint32_t r0[32], r1[32];
+              const uint32_t ta = tmem_base + ((uint32_t)lane_base << 16) + acc * kAccCols + t * N;
+              tc::tmem_ld32(ta, r0);
+              tc::tmem_ld32(ta + 32, r1);
+              tc::tmem_ld_wait(r0);
+              tc::reg_fence(r1);
+              float a[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+              for (int h4 = 0; h4 < 8; ++h4) {
+                const float4 wa = w4p[h4], wb = w4p[8 + h4];
+                a[0] = fmaf(wa.x, fmaxf(__uint_as_float(r0[4 * h4]), 0.f), a[0]);
+                a[1] = fmaf(wa.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), a[1]);
+                a[2] = fmaf(wa.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), a[2]);
+                a[3] = fmaf(wa.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), a[3]);
+                a[0] = fmaf(wb.x, fmaxf(__uint_as_float(r1[4 * h4]), 0.f), a[0]);
+                a[1] = fmaf(wb.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), a[1]);
+                a[2] = fmaf(wb.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), a[2]);
+                a[3] = fmaf(wb.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), a[3]);
+              }
+              sc[t] = (a[0] + a[1]) + (a[2] + a[3]);
+            }
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
           }
-          sc = a0 + a1;
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&tempty[acc]);
-          ++it;
-          ++at;
+        } else if ((js & 1) != grp) {
+          continue;                                     // fills alternate between the groups
         }
-        if (e < p.E) {
-          const float v = !ok ? __int_as_float(0x7fc00000) : (e < ev ? sc : -INFINITY);
-          const size_t o = (size_t)row * p.E + e;
-          if (p.score_f32) reinterpret_cast<float*>(p.scores)[o] = v;
-          else reinterpret_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(v);
+#pragma unroll
+        for (int t = 0; t < kTPS; ++t) {
+          const int e = (js * kTPS + t) * kTileE + lane_base + lane;
+          if (e < p.E) {
+            const float v = !ok ? __int_as_float(0x7fc00000) : (e < ev ? sc[t] : -INFINITY);
+            const size_t o = (size_t)row * p.E + e;
+            if (p.score_f32) reinterpret_cast<float*>(p.scores)[o] = v;
+            else reinterpret_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(v);
+          }
         }
+      }
+      if (nc > 0) {
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bempty[ul & 1]);
+        ++ul;
       }
     }
   }
@@ -351,15 +398,14 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
 }  // namespace
 
 csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st) {
-  if (a.qk_dtype != CSA_NVFP4 || a.H != kHeads || a.d != 128 || a.T != 1) return CSA_ERR_UNSUPPORTED;
+  if (a.qk_dtype != CSA_NVFP4 || a.H != kHeads || a.d != kDim || a.T != 1) return CSA_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.q) & 15) ||
       (reinterpret_cast<uintptr_t>(a.k_scales) & 15) || (reinterpret_cast<uintptr_t>(a.q_scales) & 15) ||
-      (reinterpret_cast<uintptr_t>(a.w) & 15) || (a.E_cap % 4))
+      (reinterpret_cast<uintptr_t>(a.w) & 15))
     return CSA_ERR_UNSUPPORTED;
-  CUtensorMap tmK, tmKS, tmQ, tmQS, tmW;
+  CUtensorMap tmK, tmQ, tmQS, tmW;
   const uint64_t krows = (uint64_t)b * a.E_cap, qrows = (uint64_t)b * a.T * kHeads;
-  if (!make_tmap_2d_u8_swz(&tmK, a.k, kRowB, krows, kRowB, kTileE, 64) ||
-      !make_tmap_2d_u8_swz(&tmKS, a.k_scales, 16, krows / 2, 16, kTileE / 2, 0) ||
+  if (!make_tmap_2d_u8_swz(&tmK, a.k, kRowB, krows, kRowB, kStageE, 64) ||
       !make_tmap_2d_u8_swz(&tmQ, a.q, kRowB, qrows, kRowB, kHeads, 64) ||
       !make_tmap_2d_u8_swz(&tmQS, a.q_scales, 16, qrows / 2, 16, kHeads / 2, 0) ||
       !make_tmap_1d_f32(&tmW, a.w, qrows, kHeads))
@@ -369,31 +415,34 @@ csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   IdxFp4 p{};
   p.scores = a.scores; p.q_pos = a.q_pos;
+  p.k_scales = reinterpret_cast<const uint8_t*>(a.k_scales);
   p.err = device_error_word();
   if (!p.err) return CSA_ERR_CUDA;
   p.T = a.T; p.E_cap = a.E_cap; p.E = a.E; p.m = a.m;
   p.tiles = (a.E + kTileE - 1) / kTileE;
+  p.sf_tiles_cap = (a.E_cap + kTileE - 1) / kTileE;
+  p.stages = (p.tiles + kTPS - 1) / kTPS;
   const long long rows = (long long)b * a.T;
   int nch = (int)((2LL * sms + rows - 1) / rows);
-  nch = max(1, min(nch, p.tiles));
-  p.chunk = (p.tiles + nch - 1) / nch;
-  p.n_chunks = (p.tiles + p.chunk - 1) / p.chunk;
+  nch = max(1, min(nch, p.stages));
+  p.chunk = (p.stages + nch - 1) / nch;
+  p.n_chunks = (p.stages + p.chunk - 1) / p.chunk;
   const long long units = rows * p.n_chunks;
   if (units > 0x7fffffff) return CSA_ERR_UNSUPPORTED;
   p.units = (int)units;
   p.score_f32 = a.score_dtype == CSA_F32;
   p.all_visible = a.all_visible;
-  p.dep_tile = a.dep_entry < 0 ? 0 : a.dep_entry / kTileE;
+  p.dep_stage = a.dep_entry < 0 ? 0 : a.dep_entry / kStageE;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
   const size_t smem = 1024 + (size_t)S * kStage + 2 * (size_t)kQBuf + (2 * S + 4 + 2 * NACC) * 8 +
-                      16 + kHeads * 4 + (size_t)kMaxLocalUnits * 2 * 4;
+                      16 + (size_t)kMaxLocalUnits * 2 * 4;
   if (cudaFuncSetAttribute(index_scores_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return CSA_ERR_CUDA;
-  if (csa_launch(index_scores_fp4_kernel, dim3((unsigned)grid), dim3(192), smem, st, a.pdl != 0,
-                 tmK, tmKS, tmQ, tmQS, tmW, p) != cudaSuccess)
+  if (csa_launch(index_scores_fp4_kernel, dim3((unsigned)grid), dim3(kThreads), smem, st,
+                 a.pdl != 0, tmK, tmQ, tmQS, tmW, p) != cudaSuccess)
     return CSA_ERR_CUDA;
   return CSA_OK;
 }

@@ -12,15 +12,21 @@
 
 namespace csa {
 
+// Element e of row `row`.  NVFP4 scale byte: `soff` = byte offset of the row's
+// block-0 scale for row-major query scales (scale of block j at soff + j), or,
+// with `tiled`, the key-scale layout (sequence base + entry index in `soff`).
 __device__ __forceinline__ float load_code(const void* base, int dtype, size_t row, int d, int e,
-                                           const void* scales, size_t srow) {
+                                           const void* scales, size_t srow, bool tiled = false,
+                                           const uint8_t* seq_scales = nullptr, long long ent = 0) {
   if (dtype == CSA_F32) return reinterpret_cast<const float*>(base)[row * d + e];
   if (dtype == CSA_FP8_E4M3)
     return e4m3_to_f32(reinterpret_cast<const uint8_t*>(base)[row * d + e]) *
            reinterpret_cast<const float*>(scales)[srow];
   const uint8_t byte = reinterpret_cast<const uint8_t*>(base)[row * (d / 2) + e / 2];
   const float v = e2m1_to_f32((e & 1) ? (byte >> 4) : (byte & 0xF));
-  return v * e4m3_to_f32(reinterpret_cast<const uint8_t*>(scales)[srow * (d / 16) + e / 16]);
+  const uint8_t sc = tiled ? seq_scales[nvfp4_key_scale_offset(ent, e / 16, d)]
+                           : reinterpret_cast<const uint8_t*>(scales)[srow * (d / 16) + e / 16];
+  return v * e4m3_to_f32(sc);
 }
 
 __global__ void __launch_bounds__(128) index_scores_simt_kernel(IndexArgs a) {
@@ -43,11 +49,16 @@ __global__ void __launch_bounds__(128) index_scores_simt_kernel(IndexArgs a) {
   float score = -INFINITY;
   if (s < ev) {
     const size_t krow = (size_t)sb * a.E_cap + s;
+    const bool tiled = a.qk_dtype == CSA_NVFP4;
+    const uint8_t* seq_sc = tiled ? reinterpret_cast<const uint8_t*>(a.k_scales) +
+                                        (size_t)sb * nvfp4_key_scale_seq_bytes(a.E_cap, d)
+                                  : nullptr;
     score = 0.f;
     for (int j = 0; j < H; ++j) {
       float dot = 0.f;
       for (int e = 0; e < d; ++e)
-        dot = fmaf(s_q[j * d + e], load_code(a.k, a.qk_dtype, krow, d, e, a.k_scales, krow), dot);
+        dot = fmaf(s_q[j * d + e],
+                   load_code(a.k, a.qk_dtype, krow, d, e, a.k_scales, krow, tiled, seq_sc, s), dot);
       score = fmaf(s_w[j], fmaxf(dot, 0.f), score);
     }
   }

@@ -15,21 +15,29 @@
 // sum_j (w qs)[q,j] ReLU(D[s,(q,j)]) * ks[s] in registers (ReLU commutes with the
 // positive scales): no cross-thread reduction.
 //
-// Persistent, warp-specialised CTA (192 threads):
-//   warp 0  TMA producer: per tile the 128 x 128 B key block (128-byte swizzle)
-//           and its 128 fp32 key scales into an S-stage ring; per work unit the
-//           query group (64 QG x 128 B), its head weights and query scales into
-//           one of two buffers;
-//   warp 1  MMA issuer (one thread): 4 x tcgen05.mma kind::f8f6f4 per tile into
-//           one of NACC TMEM accumulators;
-//   warps 2-5 epilogue: tcgen05.ld of the accumulator, the weighted ReLU sum,
-//           the causal mask, bf16 / fp32 store; tiles no query of the group can
-//           see are written as -inf without any MMA.
-// Every operand the epilogue needs arrives by TMA with its tile, so no thread
+// A pipeline stage holds TPS tiles of 128 entries (two for one query per unit,
+// one for four): on sm_100a a thread's first shared-memory access after issuing
+// tcgen05 operations costs a few hundred cycles, so the MMA warp's two waits per
+// stage are amortised over 4 x TPS MMAs.
+//
+// Persistent, warp-specialised CTA (320 threads):
+//   warp 0  TMA producer: per stage one 2-D box of 128 TPS key rows (128-byte
+//           swizzle) and their fp32 key scales into an S-stage ring; per work unit
+//           the query group (64 QG x 128 B), its head weights and query scales
+//           into one of two buffers;
+//   warp 1  MMA issuer (one thread): 4 TPS x tcgen05.mma kind::f8f6f4 per stage
+//           into one of NACC TMEM accumulators;
+//   warps 2-9 epilogue, two warpgroups taking alternate stages (warps w and w+4
+//           share a TMEM lane quarter), so one group's TMEM loads overlap the
+//           other's arithmetic: tcgen05.ld of the accumulator, the weighted ReLU
+//           sum (weights in registers for one query, 128-bit shared loads for
+//           four), the causal mask, bf16 / fp32 store; stages no query of the
+//           group can see are written as -inf without any MMA.
+// Every operand the epilogue needs arrives by TMA with its stage, so no thread
 // waits on global memory inside the loop.  A stage is released when the MMAs
-// have read the keys and all four epilogue warps have read the key scales.
-// A work unit is (sequence, query group, chunk of entry tiles); units are dealt
-// round-robin to the CTAs and their causal extents are computed once, at start.
+// have read the keys and the four epilogue warps of its group have read the key
+// scales.  A work unit is (sequence, query group, chunk of stages); units are
+// dealt round-robin to the CTAs and their causal extents are computed once.
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -42,43 +50,51 @@ constexpr int kHeads = 64;           // index heads
 constexpr int kDim = 128;            // index dim (bytes per FP8 row)
 constexpr int kTileBytes = kTileE * kDim;
 constexpr int kMaxLocalUnits = 256;  // units one CTA walks (grid is sized to respect it)
+constexpr int kEpiGroups = 2;        // epilogue warpgroups, alternating stages
+constexpr int kThreads = 64 + 128 * kEpiGroups;
 
 struct IdxTc {
   void* scores;
   const int32_t* q_pos;
   int* err;
   int T, E_cap, E, m;
-  int n_qg, tiles, chunk, n_chunks, units;
+  int n_qg, tiles, stages, chunk, n_chunks, units;
   int score_f32;
   int all_visible;   // every query sees all E entries: q_pos is not read
-  int dep_tile;      // tiles >= dep_tile hold entries the preceding kernel writes
+  int dep_stage;     // stages >= dep_stage hold entries the preceding kernel writes
 };
 
 template <int QG>
 struct Layout {
   static constexpr int N = kHeads * QG;
+  static constexpr int TPS = QG == 1 ? 2 : 1;          // tiles per stage
+  static constexpr int kStageE = kTileE * TPS;
   static constexpr int NACC = QG == 1 ? 4 : 2;
+  static constexpr int kAccCols = TPS * N;
+  static constexpr int kStageKeyB = TPS * kTileBytes;
   static constexpr int kQBytes = N * kDim;
-  static constexpr uint32_t kTmemCols = NACC * N <= 32 ? 32 : NACC * N <= 64 ? 64 :
-                                        NACC * N <= 128 ? 128 : NACC * N <= 256 ? 256 : 512;
+  static constexpr uint32_t kTmemCols = 512;
+  static_assert(NACC * kAccCols <= 512, "TMEM budget");
 };
 
 template <int QG, int S>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kThreads, 1)
 index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                        const __grid_constant__ CUtensorMap tmKS, const __grid_constant__ CUtensorMap tmW,
                        const __grid_constant__ CUtensorMap tmQS, IdxTc p) {
   using LY = Layout<QG>;
   constexpr int N = LY::N;
+  constexpr int TPS = LY::TPS;
   constexpr int NACC = LY::NACC;
   constexpr int kQBytes = LY::kQBytes;
+  constexpr int kStageE = LY::kStageE;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint8_t* sA = base;                                         // S x 16 KB key tiles
-  float* sKS = reinterpret_cast<float*>(sA + S * kTileBytes); // S x 128 key scales
-  uint8_t* sB = reinterpret_cast<uint8_t*>(sKS + S * kTileE); // 2 x kQBytes query groups
-  float* sW = reinterpret_cast<float*>(sB + 2 * kQBytes);     // 2 x N head weights
-  float* sQS = sW + 2 * N;                                    // 2 x N query scales
+  uint8_t* sA = base;                                           // S x TPS x 16 KB key tiles
+  float* sKS = reinterpret_cast<float*>(sA + S * LY::kStageKeyB);   // S x kStageE key scales
+  uint8_t* sB = reinterpret_cast<uint8_t*>(sKS + S * kStageE);  // 2 x kQBytes query groups
+  float* sW = reinterpret_cast<float*>(sB + 2 * kQBytes);       // 2 x N head weights
+  float* sQS = sW + 2 * N;                                      // 2 x N query scales
   uint64_t* bars = reinterpret_cast<uint64_t*>(sQS + 2 * N);
   uint64_t* full = bars;
   uint64_t* empty = bars + S;
@@ -87,8 +103,8 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   uint64_t* tfull = bempty + 2;
   uint64_t* tempty = tfull + NACC;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + NACC);
-  float* s_wq = reinterpret_cast<float*>(tmem_holder + 4);    // [N] w * qs of the current unit
-  int* s_vis = reinterpret_cast<int*>(s_wq + N);              // [kMaxLocalUnits] visible tiles
+  float* s_wq = reinterpret_cast<float*>(tmem_holder + 4);    // [kEpiGroups][N] w * qs of the unit
+  int* s_vis = reinterpret_cast<int*>(s_wq + kEpiGroups * N); // [kMaxLocalUnits] visible stages
   int* s_ev = s_vis + kMaxLocalUnits;                         // [kMaxLocalUnits][QG] visible entries
 
   const int warp = threadIdx.x >> 5;
@@ -110,11 +126,14 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
       s_ev[i * QG + q] = ev;
       evmax = max(evmax, ev);
     }
-    s_vis[i] = (evmax + kTileE - 1) / kTileE;
+    s_vis[i] = (evmax + kStageE - 1) / kStageE;
   }
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], 1 + 4); }
-    for (int i = 0; i < 2; ++i) { tc::mbar_init(&bfull[i], 1); tc::mbar_init(&bempty[i], 1 + 4); }
+    for (int i = 0; i < 2; ++i) {
+      tc::mbar_init(&bfull[i], 1);
+      tc::mbar_init(&bempty[i], 1 + 4 * kEpiGroups);
+    }
     for (int i = 0; i < NACC; ++i) { tc::mbar_init(&tfull[i], 1); tc::mbar_init(&tempty[i], 4); }
     tc::fence_barrier_init();
     tc::tma_prefetch_desc(&tmK);
@@ -127,42 +146,44 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   tc::tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
 
-  // per-unit geometry shared by all roles
-  auto unit = [&](int u, int i, int& sb, int& g, int& j0, int& j1, int& nc, int& nq) {
+  // per-unit geometry shared by all roles: stages [js0, js1), the first nc computed
+  auto unit = [&](int u, int i, int& sb, int& g, int& js0, int& js1, int& nc, int& nq) {
     const int ch = u % p.n_chunks;
     const int tmp = u / p.n_chunks;
     g = tmp % p.n_qg;
     sb = tmp / p.n_qg;
-    j0 = ch * p.chunk;
-    j1 = min(p.tiles, j0 + p.chunk);
+    js0 = ch * p.chunk;
+    js1 = min(p.stages, js0 + p.chunk);
     nq = min(QG, p.T - g * QG);
-    nc = max(0, min(j1, s_vis[i]) - j0);
+    nc = max(0, min(js1, s_vis[i]) - js0);
   };
 
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      // Key tiles the preceding kernel does not write are fetched before waiting on it,
-      // into the first free stages, so that HBM streaming overlaps that kernel.
+      auto load_stage = [&](int slot, int sb, int js) {
+        const int row0 = sb * p.E_cap + js * kStageE;
+        tc::mbar_arrive_expect_tx(&full[slot], LY::kStageKeyB + kStageE * 4);
+        tc::tma_load_2d(sA + slot * LY::kStageKeyB, &tmK, 0, row0, &full[slot]);
+        tc::tma_load_1d(sKS + slot * kStageE, &tmKS, row0, &full[slot]);
+      };
+      // Key stages the preceding kernel does not write are fetched before waiting on it,
+      // into the first free slots, so that HBM streaming overlaps that kernel.
       uint32_t npre = 0;
       for (int u = blockIdx.x, i = 0; u < p.units && npre == 0; u += gridDim.x, ++i) {
-        int sb, g, j0, j1, nc, nq;
-        unit(u, i, sb, g, j0, j1, nc, nq);
+        int sb, g, js0, js1, nc, nq;
+        unit(u, i, sb, g, js0, js1, nc, nq);
         if (nc == 0) continue;
-        for (int j = j0; j < j0 + nc && (int)npre < S && j < p.dep_tile; ++j, ++npre) {
-          const int row0 = sb * p.E_cap + j * kTileE;
-          tc::mbar_arrive_expect_tx(&full[npre], kTileBytes + kTileE * 4);
-          tc::tma_load_2d(sA + npre * kTileBytes, &tmK, 0, row0, &full[npre]);
-          tc::tma_load_1d(sKS + npre * kTileE, &tmKS, row0, &full[npre]);
-        }
+        for (int js = js0; js < js0 + nc && (int)npre < S && js < p.dep_stage; ++js, ++npre)
+          load_stage(npre, sb, js);
         break;
       }
       pdl_wait();
       uint32_t it = 0, ul = 0;
       bool ok = true;
       for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
-        int sb, g, j0, j1, nc, nq;
-        unit(u, i, sb, g, j0, j1, nc, nq);
+        int sb, g, js0, js1, nc, nq;
+        unit(u, i, sb, g, js0, js1, nc, nq);
         if (nc == 0) continue;
         const int bb = ul & 1;
         ok = tc::mbar_wait(&bempty[bb], ((ul >> 1) & 1) ^ 1, p.err);
@@ -172,15 +193,12 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         tc::tma_load_2d(sB + bb * kQBytes, &tmQ, 0, qrow0, &bfull[bb]);
         tc::tma_load_1d(sW + bb * N, &tmW, qrow0, &bfull[bb]);
         tc::tma_load_1d(sQS + bb * N, &tmQS, qrow0, &bfull[bb]);
-        for (int j = j0; j < j0 + nc; ++j, ++it) {
+        for (int js = js0; js < js0 + nc; ++js, ++it) {
           if (it < npre) continue;                       // fetched before the wait
           const int s = it % S;
           ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
           if (!ok) break;
-          const int row0 = sb * p.E_cap + j * kTileE;
-          tc::mbar_arrive_expect_tx(&full[s], kTileBytes + kTileE * 4);
-          tc::tma_load_2d(sA + s * kTileBytes, &tmK, 0, row0, &full[s]);
-          tc::tma_load_1d(sKS + s * kTileE, &tmKS, row0, &full[s]);
+          load_stage(s, sb, js);
         }
         ++ul;
       }
@@ -189,29 +207,34 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t idesc = tc::instr_desc(kTileE, N, 0, 0, 0, 0);   // e4m3 x e4m3 -> f32
-      uint32_t it = 0, ul = 0, at = 0;
+      uint32_t it = 0, ul = 0;
       bool ok = true;
       for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
-        int sb, g, j0, j1, nc, nq;
-        unit(u, i, sb, g, j0, j1, nc, nq);
+        int sb, g, js0, js1, nc, nq;
+        unit(u, i, sb, g, js0, js1, nc, nq);
         if (nc == 0) continue;
         const int bb = ul & 1;
         ok = tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
         if (!ok) break;
         const uint64_t bdesc = tc::smem_desc_sw128(tc::smem_u32(sB + bb * kQBytes), 16, 1024);
-        for (int j = 0; j < nc; ++j, ++it, ++at) {
+        for (int j = 0; j < nc; ++j, ++it) {
           const int s = it % S;
-          const int acc = at % NACC;
-          ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err);
-          if (!ok) break;
-          ok = tc::mbar_wait(&tempty[acc], ((at / NACC) & 1) ^ 1, p.err);
+          const int acc = it % NACC;
+          // both waits back to back: the first shared-memory access after the previous
+          // stage's tcgen05 operations carries the cost, the second is cheap
+          ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err) &&
+               tc::mbar_wait(&tempty[acc], ((it / NACC) & 1) ^ 1, p.err);
           if (!ok) break;
           tc::tc_fence_after();
-          const uint64_t adesc = tc::smem_desc_sw128(tc::smem_u32(sA + s * kTileBytes), 16, 1024);
-          const uint32_t d = tmem_base + acc * N;
 #pragma unroll
-          for (int kk = 0; kk < kDim / 32; ++kk)   // K = 32 bytes of E4M3 per MMA
-            tc::mma_f8f6f4(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0);
+          for (int t = 0; t < TPS; ++t) {
+            const uint64_t adesc =
+                tc::smem_desc_sw128(tc::smem_u32(sA + s * LY::kStageKeyB + t * kTileBytes), 16, 1024);
+            const uint32_t d = tmem_base + acc * LY::kAccCols + t * N;
+#pragma unroll
+            for (int kk = 0; kk < kDim / 32; ++kk)   // K = 32 bytes of E4M3 per MMA
+              tc::mma_f8f6f4(d, adesc + 2 * kk, bdesc + 2 * kk, idesc, kk > 0);
+          }
           tc::mma_commit(&empty[s]);
           tc::mma_commit(&tfull[acc]);
         }
@@ -222,70 +245,110 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     }
   } else {
     // -------------------------------------------------------------- epilogue
+    const int ew = warp - 2;                 // 0..7
+    const int grp = ew >> 2;                 // warpgroup: takes stages with c % 2 == grp
     const int lane_base = (warp & 3) * 32;   // TMEM lanes this warp may access
-    const int etid = threadIdx.x - 64;       // 0..127
-    uint32_t it = 0, at = 0, ul = 0;
+    const int gtid = (ew & 3) * 32 + lane;   // 0..127 within the group
+    float* my_wq = s_wq + grp * N;
+    float wq1[QG == 1 ? kHeads : 1];         // one query: its 64 weights live in registers
+    uint32_t c = 0, ul = 0;                  // computed stages seen, units with work seen
     bool ok = true;
     for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
-      int sb, g, j0, j1, nc, nq;
-      unit(u, i, sb, g, j0, j1, nc, nq);
+      int sb, g, js0, js1, nc, nq;
+      unit(u, i, sb, g, js0, js1, nc, nq);
       if (nc > 0) {
         const int bb = ul & 1;
-        tc::named_bar(1, 128);                         // previous unit's s_wq no longer read
+        tc::named_bar(1 + grp, 128);                   // previous unit's my_wq no longer read
         ok = ok && tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
-        for (int x = etid; x < N; x += 128) s_wq[x] = sW[bb * N + x] * sQS[bb * N + x];
+        for (int x = gtid; x < N; x += 128) my_wq[x] = sW[bb * N + x] * sQS[bb * N + x];
         __syncwarp();
         if (lane == 0) tc::mbar_arrive(&bempty[bb]);
-        tc::named_bar(1, 128);
+        tc::named_bar(1 + grp, 128);
+        if constexpr (QG == 1) {
+#pragma unroll
+          for (int h = 0; h < kHeads; h += 4) {
+            const float4 w4 = *reinterpret_cast<const float4*>(my_wq + h);
+            wq1[h] = w4.x; wq1[h + 1] = w4.y; wq1[h + 2] = w4.z; wq1[h + 3] = w4.w;
+          }
+        }
         ++ul;
       }
-      for (int j = j0; j < j1; ++j) {
-        const int e = j * kTileE + lane_base + lane;
-        float sc[QG];
-        const bool computed = j < j0 + nc;
-        if (computed && ok) {
-          const int s = it % S;
-          const int acc = at % NACC;
-          ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err);   // the stage's key scales landed
-          const float ks = sKS[s * kTileE + lane_base + lane];
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&empty[s]);
-          ok = ok && tc::mbar_wait(&tfull[acc], (at / NACC) & 1, p.err);
-          tc::tc_fence_after();
+      for (int js = js0; js < js1; ++js) {
+        float sc[TPS][QG];
 #pragma unroll
-          for (int q = 0; q < QG; ++q) {
-            uint32_t r0[32], r1[32];
-            const uint32_t ta = tmem_base + ((uint32_t)lane_base << 16) + acc * N + q * kHeads;
-            tc::tmem_ld32(ta, r0);
-            tc::tmem_ld32(ta + 32, r1);
-            tc::tmem_ld_wait(r0);
-            tc::reg_fence(r1);
-            float a0 = 0.f, a1 = 0.f;
+        for (int t = 0; t < TPS; ++t)
 #pragma unroll
-            for (int h = 0; h < 32; ++h) {
-              a0 = fmaf(s_wq[q * kHeads + h], fmaxf(__uint_as_float(r0[h]), 0.f), a0);
-              a1 = fmaf(s_wq[q * kHeads + 32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), a1);
+          for (int q = 0; q < QG; ++q) sc[t][q] = -INFINITY;
+        if (js < js0 + nc) {
+          const uint32_t cc = c++;
+          if ((int)(cc & 1) != grp) continue;           // the other warpgroup's stage
+          if (ok) {
+            const int s = cc % S;
+            const int acc = cc % NACC;
+            ok = tc::mbar_wait(&full[s], (cc / S) & 1, p.err);   // the stage's key scales landed
+            float ks[TPS];
+#pragma unroll
+            for (int t = 0; t < TPS; ++t) ks[t] = sKS[s * kStageE + t * kTileE + lane_base + lane];
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&empty[s]);
+            ok = ok && tc::mbar_wait(&tfull[acc], (cc / NACC) & 1, p.err);
+            tc::tc_fence_after();
+#pragma unroll
+            for (int t = 0; t < TPS; ++t) {
+#pragma unroll
+              for (int q = 0; q < QG; ++q) {
+                uint32_t r0[32], r1[32];
+                const uint32_t ta = tmem_base + ((uint32_t)lane_base << 16) + acc * LY::kAccCols +
+                                    t * N + q * kHeads;
+                tc::tmem_ld32(ta, r0);
+                tc::tmem_ld32(ta + 32, r1);
+                tc::tmem_ld_wait(r0);
+                tc::reg_fence(r1);
+                float a[4] = {0.f, 0.f, 0.f, 0.f};
+                if constexpr (QG == 1) {
+#pragma unroll
+                  for (int h = 0; h < 32; ++h) {
+                    a[h & 3] = fmaf(wq1[h], fmaxf(__uint_as_float(r0[h]), 0.f), a[h & 3]);
+                    a[h & 3] = fmaf(wq1[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), a[h & 3]);
+                  }
+                } else {
+                  const float4* w4p = reinterpret_cast<const float4*>(my_wq + q * kHeads);
+#pragma unroll
+                  for (int h4 = 0; h4 < 8; ++h4) {
+                    const float4 wa = w4p[h4], wb = w4p[8 + h4];
+                    a[0] = fmaf(wa.x, fmaxf(__uint_as_float(r0[4 * h4]), 0.f), a[0]);
+                    a[1] = fmaf(wa.y, fmaxf(__uint_as_float(r0[4 * h4 + 1]), 0.f), a[1]);
+                    a[2] = fmaf(wa.z, fmaxf(__uint_as_float(r0[4 * h4 + 2]), 0.f), a[2]);
+                    a[3] = fmaf(wa.w, fmaxf(__uint_as_float(r0[4 * h4 + 3]), 0.f), a[3]);
+                    a[0] = fmaf(wb.x, fmaxf(__uint_as_float(r1[4 * h4]), 0.f), a[0]);
+                    a[1] = fmaf(wb.y, fmaxf(__uint_as_float(r1[4 * h4 + 1]), 0.f), a[1]);
+                    a[2] = fmaf(wb.z, fmaxf(__uint_as_float(r1[4 * h4 + 2]), 0.f), a[2]);
+                    a[3] = fmaf(wb.w, fmaxf(__uint_as_float(r1[4 * h4 + 3]), 0.f), a[3]);
+                  }
+                }
+                sc[t][q] = ((a[0] + a[1]) + (a[2] + a[3])) * ks[t];
+              }
             }
-            sc[q] = (a0 + a1) * ks;
+            tc::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&tempty[acc]);
           }
-          tc::tc_fence_before();
-          __syncwarp();
-          if (lane == 0) tc::mbar_arrive(&tempty[acc]);
-          ++it;
-          ++at;
-        } else {
-#pragma unroll
-          for (int q = 0; q < QG; ++q) sc[q] = -INFINITY;
+        } else if ((js & 1) != grp) {
+          continue;                                     // fills alternate between the groups
         }
-        if (e < p.E) {
 #pragma unroll
-          for (int q = 0; q < QG; ++q) {
-            if (q >= nq) break;
-            const int ev = s_ev[i * QG + q];
-            const float v = !ok ? __int_as_float(0x7fc00000) : (e < ev ? sc[q] : -INFINITY);
-            const size_t o = ((size_t)sb * p.T + g * QG + q) * p.E + e;
-            if (p.score_f32) reinterpret_cast<float*>(p.scores)[o] = v;
-            else reinterpret_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(v);
+        for (int t = 0; t < TPS; ++t) {
+          const int e = (js * TPS + t) * kTileE + lane_base + lane;
+          if (e < p.E) {
+#pragma unroll
+            for (int q = 0; q < QG; ++q) {
+              if (q >= nq) break;
+              const int ev = s_ev[i * QG + q];
+              const float v = !ok ? __int_as_float(0x7fc00000) : (e < ev ? sc[t][q] : -INFINITY);
+              const size_t o = ((size_t)sb * p.T + g * QG + q) * p.E + e;
+              if (p.score_f32) reinterpret_cast<float*>(p.scores)[o] = v;
+              else reinterpret_cast<__nv_bfloat16*>(p.scores)[o] = __float2bfloat16_rn(v);
+            }
           }
         }
       }
@@ -305,9 +368,9 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   using LY = Layout<QG>;
   CUtensorMap tmK, tmQ, tmKS, tmW, tmQS;
   const uint64_t qrows = (uint64_t)b * a.T * kHeads;
-  if (!make_tmap_2d_u8(&tmK, a.k, kDim, (uint64_t)b * a.E_cap, kDim, kTileE) ||
+  if (!make_tmap_2d_u8(&tmK, a.k, kDim, (uint64_t)b * a.E_cap, kDim, LY::kStageE) ||
       !make_tmap_2d_u8(&tmQ, a.q, kDim, qrows, kDim, LY::N) ||
-      !make_tmap_1d_f32(&tmKS, a.k_scales, (uint64_t)b * a.E_cap, kTileE) ||
+      !make_tmap_1d_f32(&tmKS, a.k_scales, (uint64_t)b * a.E_cap, LY::kStageE) ||
       !make_tmap_1d_f32(&tmW, a.w, qrows, LY::N) ||
       !make_tmap_1d_f32(&tmQS, a.q_scales, qrows, LY::N))
     return CSA_ERR_CUDA;
@@ -321,30 +384,31 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   p.T = a.T; p.E_cap = a.E_cap; p.E = a.E; p.m = a.m;
   p.n_qg = (a.T + QG - 1) / QG;
   p.tiles = (a.E + kTileE - 1) / kTileE;
+  p.stages = (p.tiles + LY::TPS - 1) / LY::TPS;
   const long long groups = (long long)b * p.n_qg;
-  // split each query group's tiles into chunks so that there are at least ~2 units per SM
+  // split each query group's stages into chunks so that there are at least ~2 units per SM
   int nch = (int)((2LL * sms + groups - 1) / groups);
-  nch = max(1, min(nch, p.tiles));
-  p.chunk = (p.tiles + nch - 1) / nch;
-  p.n_chunks = (p.tiles + p.chunk - 1) / p.chunk;
+  nch = max(1, min(nch, p.stages));
+  p.chunk = (p.stages + nch - 1) / nch;
+  p.n_chunks = (p.stages + p.chunk - 1) / p.chunk;
   const long long units = groups * p.n_chunks;
   if (units > 0x7fffffff) return CSA_ERR_UNSUPPORTED;
   p.units = (int)units;
   p.score_f32 = a.score_dtype == CSA_F32;
   p.all_visible = a.all_visible;
-  p.dep_tile = a.dep_entry < 0 ? 0 : a.dep_entry / kTileE;
+  p.dep_stage = a.dep_entry < 0 ? 0 : a.dep_entry / LY::kStageE;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
-  const size_t smem = 1024 + (size_t)S * (kTileBytes + kTileE * 4) + 2 * (size_t)LY::kQBytes +
+  const size_t smem = 1024 + (size_t)S * (LY::kStageKeyB + LY::kStageE * 4) + 2 * (size_t)LY::kQBytes +
                       4 * (size_t)LY::N * 4 + (2 * S + 4 + 2 * LY::NACC) * 8 + 16 +
-                      (size_t)LY::N * 4 + (size_t)kMaxLocalUnits * (1 + QG) * 4;
+                      kEpiGroups * (size_t)LY::N * 4 + (size_t)kMaxLocalUnits * (1 + QG) * 4;
   auto kern = index_scores_tc_kernel<QG, S>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)
     return CSA_ERR_CUDA;
-  if (csa_launch(kern, dim3((unsigned)grid), dim3(192), smem, st, a.pdl != 0, tmK, tmQ, tmKS, tmW,
-                 tmQS, p) != cudaSuccess)
+  if (csa_launch(kern, dim3((unsigned)grid), dim3(kThreads), smem, st, a.pdl != 0, tmK, tmQ, tmKS,
+                 tmW, tmQS, p) != cudaSuccess)
     return CSA_ERR_CUDA;
   return CSA_OK;
 }
@@ -358,7 +422,7 @@ csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st) {
       (reinterpret_cast<uintptr_t>(a.q_scales) & 15) || (a.E_cap % 4))
     return CSA_ERR_UNSUPPORTED;   // the TMA copies need 16-byte aligned rows and scale runs
   if (a.T >= 4) return launch_qg<4, 4>(a, b, st);
-  return launch_qg<1, 8>(a, b, st);
+  return launch_qg<1, 5>(a, b, st);
 }
 
 }  // namespace csa

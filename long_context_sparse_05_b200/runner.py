@@ -27,7 +27,9 @@ def alloc_index_cache(b, E_cap, c_I, idx_dtype, device):
     if idx_dtype == "fp8":
         scales = torch.empty((b, E_cap), dtype=torch.float32, device=device)
     else:
-        scales = torch.empty((b, E_cap, c_I // 16), dtype=torch.uint8, device=device)
+        # tiled NVFP4 key-scale layout: whole tiles of 128 entries per sequence
+        e_pad = (E_cap + 127) // 128 * 128
+        scales = torch.empty((b, e_pad, c_I // 16), dtype=torch.uint8, device=device)
     return codes, scales
 
 

@@ -72,6 +72,43 @@ def topk_band_check(gpu_idx, gpu_cnt, exact_scores, ev, k, rel_band=1e-3):
     return len(diff) // 2
 
 
+def nvfp4_key_scale_index(E_cap, c):
+    """Flat byte index, inside one sequence's tiled NVFP4 key-scale area, of (entry, block).
+
+    Tiles of 128 entries; inside a tile, for each 64-element K block, 512 bytes
+    ordered [entry % 32][(entry % 128) // 32][block % 4] (the order the block-scaled
+    tensor-core MMA reads).  Returns an int array [E_cap][c // 16].
+    """
+    e = np.arange(E_cap)[:, None]
+    blk = np.arange(c // 16)[None, :]
+    r = e % 128
+    return (e // 128) * (8 * c) + (blk // 4) * 512 + (r % 32) * 16 + (r // 32) * 4 + blk % 4
+
+
+def nvfp4_scales_to_tiled(rows, E_cap=None):
+    """Row-major key scales [..., E, c/16] -> the tiled key-scale layout [..., E_pad, c/16]."""
+    rows = np.asarray(rows)
+    E, nb = rows.shape[-2], rows.shape[-1]
+    E_cap = E_cap or E
+    e_pad = (E_cap + 127) // 128 * 128
+    idx = nvfp4_key_scale_index(E, nb * 16)
+    lead = rows.shape[:-2]
+    out = np.zeros(lead + (e_pad * nb,), dtype=rows.dtype)
+    flat = rows.reshape(lead + (E * nb,))
+    out[..., idx.reshape(-1)] = flat
+    return out.reshape(lead + (e_pad, nb))
+
+
+def nvfp4_scales_from_tiled(tiled, E):
+    """Inverse of nvfp4_scales_to_tiled: the first E entries in row-major order."""
+    tiled = np.asarray(tiled)
+    nb = tiled.shape[-1]
+    lead = tiled.shape[:-2]
+    flat = tiled.reshape(lead + (-1,))
+    idx = nvfp4_key_scale_index(E, nb * 16)
+    return flat[..., idx.reshape(-1)].reshape(lead + (E, nb))
+
+
 class LazyRows:
     """Row access to one sequence of a (large) device tensor, copied to the host in float64 on demand.
 

@@ -15,7 +15,8 @@ from long_context_sparse_05_b200 import _lib as L
 from long_context_sparse_05_b200 import synth
 from oracle import codecs, csa
 
-from helpers import assert_abs_close, assert_rel_close, f64, topk_band_check
+from helpers import (assert_abs_close, assert_rel_close, f64, nvfp4_scales_from_tiled,
+                     nvfp4_scales_to_tiled, topk_band_check)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -51,7 +52,7 @@ def _run_compress(d, b, n, c, m, overlap, E, d_rope, in_dt, out_dt, apply_norm=T
         sc = torch.zeros((b, E_cap), dtype=torch.float32, device=DEV)
     else:
         out = torch.zeros((b, E_cap, c // 2), dtype=torch.uint8, device=DEV)
-        sc = torch.zeros((b, E_cap, c // 16), dtype=torch.uint8, device=DEV)
+        sc = torch.zeros((b, (E_cap + 127) // 128 * 128, c // 16), dtype=torch.uint8, device=DEV)
     p = L.CompressParams(m=m, overlap=int(overlap), c=c, d_rope=d_rope, rope_theta=1e4, eps=1e-6,
                          apply_norm=int(apply_norm), in_dtype=L.DTYPE[in_dt],
                          out_dtype=L.DTYPE[out_dt])
@@ -113,10 +114,13 @@ def test_compress_index_branch_quantised(fmt):
     # the fused quantiser equals the stand-alone quantiser applied to the kernel's own float32 rows
     rows = b * E
     c2 = torch.empty_like(codes)
-    s2 = torch.empty_like(sc)
+    s2 = torch.empty((rows,), dtype=torch.float32, device=DEV) if fmt == "fp8" else \
+        torch.empty((rows, c // 16), dtype=torch.uint8, device=DEV)
     L.csa_quantize(L.CSA_F32, L.DTYPE[fmt], out32, rows, c, c2, s2)
     torch.cuda.synchronize()
-    assert torch.equal(c2, codes) and torch.equal(s2, sc)
+    if fmt == "nvfp4":   # the cache keeps its scales in the tiled layout; the quantiser row-major
+        sc = torch.from_numpy(nvfp4_scales_from_tiled(sc.cpu().numpy(), E)).to(DEV)
+    assert torch.equal(c2, codes) and torch.equal(s2.reshape(sc.shape), sc)
     for s in range(b):
         ref = _oracle_compress(d, s, m, True, E, 64)
         assert_rel_close(f64(out32[s]), ref, 1e-5, "index branch f32")
@@ -172,8 +176,9 @@ def _index_inputs(b, T, E, H, d, fmt, seed):
                     kd=codecs.dequant_fp8_rows(kc, ks))
     qc, qs = codecs.quant_nvfp4(q)
     kc, ks = codecs.quant_nvfp4(k)
-    return dict(q=qc, qs=qs, k=kc, ks=ks, w=w, qd=codecs.dequant_nvfp4(qc, qs),
-                kd=codecs.dequant_nvfp4(kc, ks))
+    # the library reads key scales in its tiled layout (query scales stay row-major)
+    return dict(q=qc, qs=qs, k=kc, ks=nvfp4_scales_to_tiled(ks), w=w,
+                qd=codecs.dequant_nvfp4(qc, qs), kd=codecs.dequant_nvfp4(kc, ks))
 
 
 def _dev(a):
