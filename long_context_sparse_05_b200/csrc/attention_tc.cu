@@ -19,10 +19,13 @@
 // The running max is updated lazily (only when a tile's max exceeds it by 2^8),
 // which rescales the O^T accumulator in TMEM.
 //
-// Work item = (query, split of its tiles).  With one split the CTA writes the
-// normalised output (the sink joins the denominator); with several, it writes
-// an unnormalised fp32 partial (O, running max, running sum) and
-// attn_merge_kernel combines the splits with the sink (log-sum-exp merge).
+// Work item = (query, split of its rows).  With one split the CTA writes the
+// normalised output (the sink joins the denominator).  With several (decode), the
+// splits of one query form a thread-block cluster: each CTA writes an
+// unnormalised fp32 partial (O, running max, running sum) to the workspace,
+// the cluster synchronises (barrier.cluster, release / acquire), and then every
+// CTA of the cluster merges one slice of the 512 output dims over all splits
+// with the sink (log-sum-exp merge), so no second kernel runs.
 //
 // CTA: warps 0-3 gather, read TMEM and run the softmax (warp w owns TMEM lanes
 // 32w..32w+31); warp 4 lane 0 issues every MMA.  Ordering uses two named
@@ -52,7 +55,10 @@ struct AttnTc {
   __nv_bfloat16* out; float* lse;
   float* part_o; float* part_m; float* part_l;
   int* err;
-  int T, n_w, m, k, E_cap, n, rows_total, nsplit, tps, dense;
+  int T, n_w, m, k, E_cap, n, rows_total, nsplit, rps, dense;
+  int cluster;   // nsplit > 1: 1 = the splits of a query are one cluster and merge through
+                 // distributed shared memory; 0 = partials go to the workspace and
+                 // attn_merge_kernel combines them
   float scale_log2;
 };
 
@@ -128,6 +134,211 @@ __device__ __forceinline__ void xpose_reduce64(float (&v)[64], int lane) {
   xpose_step<kMax, 1, 2>(v, lane);
 }
 
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(tc::smem_u32(local)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_dsmem4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
+  return v;
+}
+
+constexpr int kMaxSplit = 16;         // splits of one query merged inside one cluster
+constexpr int kMaxSplitGlobal = 32;   // splits of one query merged through the workspace
+
+// Cluster merge layout (inside the KV / query tile area, free once PV is done):
+//   [0, 64 KB)           this split's unnormalised O, bf16 [512 dims][64 heads], the 16-byte
+//                        chunk c of dim d's row stored at chunk c ^ (d & 7)
+//   [64 KB, 144 KB)      received slices: split j's rows of this CTA's dims at slot j
+//   [144 KB, 152 KB)     received running maxima and sums: [split][2][64] fp32
+constexpr int kCmRecvO = 64 * 1024;
+constexpr int kCmRecvML = 144 * 1024;
+__device__ __forceinline__ int cm_chunk(int d, int chunk) { return chunk ^ (d & 7); }
+
+// Bulk copy of `bytes` from this CTA's shared memory to a peer's (cluster address), counted
+// as transaction bytes on the peer's mbarrier.
+__device__ __forceinline__ void bulk_to_peer(uint32_t dst_cluster, const void* src, uint32_t bytes,
+                                             uint32_t bar_cluster) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst_cluster), "r"(tc::smem_u32(src)), "r"(bytes), "r"(bar_cluster) : "memory");
+}
+
+// Dims of the output slice merged by cluster rank `rank`.
+__device__ __forceinline__ void cm_slice(int ns, int rank, int& d0, int& d1) {
+  const int dps = ((kD + ns - 1) / ns + 7) & ~7;
+  d0 = min(kD, rank * dps);
+  d1 = min(kD, d0 + dps);
+}
+
+// Merge of the splits of query `qrow` for output dims [d0, d1) (a multiple of 4 wide):
+// out = sum_s e^{m_s} O_s / (e^{sink} + sum_s e^{m_s} l_s); every thread of the CTA joins.
+// The partials are [split][dim][head] fp32; the slice of every split, and all running
+// maxima and sums, are staged into shared memory with one batch of cp.async copies
+// (one memory round trip), then combined there.
+__device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool write_lse,
+                            uint8_t* stage /* >= nsplit * (d1 - d0) * 256 bytes */,
+                            float* s_ml /* [2][cap][kH] */, float* s_mw /* [cap][kH] */,
+                            int cap, const void* dummy) {
+  const int tid = threadIdx.x;
+  const int ns = p.nsplit;
+  const int dsl = d1 - d0;
+  const size_t it0 = (size_t)qrow * ns;
+  // running maxima and sums: ns x 64 floats each, contiguous over the splits
+  for (int c = tid; c < 2 * ns * 16; c += blockDim.x) {
+    const int which = c / (ns * 16), cc = c % (ns * 16);
+    const float* src = (which == 0 ? p.part_m : p.part_l) + it0 * kH + cc * 4;
+    tc::cp_async16(s_ml + which * cap * kH + cc * 4, src, 16);
+  }
+  // the slice of every split: dsl x 64 floats, contiguous within a split
+  const int cps = dsl * 16;                       // 16-byte chunks per split
+  for (int c = tid; c < ns * cps; c += blockDim.x) {
+    const int sp = c / cps, cc = c % cps;
+    const float* src = p.part_o + ((it0 + sp) * kD + d0) * kH + cc * 4;
+    tc::cp_async16(stage + ((size_t)sp * dsl * kH + cc * 4) * 4, dsl > 0 ? (const void*)src : dummy,
+                   dsl > 0 ? 16 : 0);
+  }
+  tc::cp_async_wait_all();
+  __syncthreads();
+  if (tid < kH) {
+    const int h = tid;
+    const float sink2 = p.sink[h] * kLog2e;
+    float M = sink2;
+    for (int sp = 0; sp < ns; ++sp) M = fmaxf(M, s_ml[sp * kH + h]);
+    float den = exp2f(sink2 - M);
+    for (int sp = 0; sp < ns; ++sp) {
+      const float ms = s_ml[sp * kH + h];
+      const float e = ms == -INFINITY ? 0.f : exp2f(ms - M);
+      s_mw[sp * kH + h] = e;
+      den += s_ml[cap * kH + sp * kH + h] * e;
+    }
+    const float inv = 1.f / den;
+    for (int sp = 0; sp < ns; ++sp) s_mw[sp * kH + h] *= inv;
+    if (write_lse && p.lse) p.lse[(size_t)qrow * kH + h] = (M + log2f(den)) * 0.6931471805599453f;
+  }
+  __syncthreads();
+  const float* st = reinterpret_cast<const float*>(stage);
+  const int nd4 = dsl >> 2;
+  for (int x = tid; x < kH * nd4; x += blockDim.x) {
+    const int h = x % kH;                         // consecutive threads: consecutive heads
+    const int dd = 4 * (x / kH);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sp = 0; sp < ns; ++sp) {
+      const float w = s_mw[sp * kH + h];
+      const float* src = st + ((size_t)sp * dsl + dd) * kH + h;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) acc[u] = fmaf(src[u * kH], w, acc[u]);
+    }
+    __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
+    __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
+    uint2 u2;
+    u2.x = *reinterpret_cast<uint32_t*>(&lo);
+    u2.y = *reinterpret_cast<uint32_t*>(&hi);
+    *reinterpret_cast<uint2*>(&p.out[((size_t)qrow * kH + h) * kD + d0 + dd]) = u2;
+  }
+}
+
+// Cluster merge of query `qrow` (every thread of the CTA joins).  Each split pushes the
+// rows of its O that another rank merges, plus its running max and sum, into that rank's
+// shared memory with bulk copies; then rank r combines output dims [d0, d1) locally:
+// out = sum_j e^{m_j} O_j / (e^{sink} + sum_j e^{m_j} l_j).
+__device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int rank, uint8_t* area,
+                                              const float* s_M, const float* s_l, float* s_mw,
+                                              uint64_t* bar_r, bool ok) {
+  const int tid = threadIdx.x;
+  const int ns = p.nsplit;
+  int d0, d1;
+  cm_slice(ns, rank, d0, d1);
+  const int dsl = d1 - d0;
+  const int dps = ((kD + ns - 1) / ns + 7) & ~7;
+  if (tid == 0) {
+    // what this CTA receives: every split's slice of its dims and its max and sum
+    tc::mbar_arrive_expect_tx(bar_r, (uint32_t)(ns * (dsl * kH * 2 + 2 * kH * 4)));
+    for (int r = 0; r < ns; ++r) {
+      int r0, r1;
+      cm_slice(ns, r, r0, r1);
+      const uint32_t bar = dsmem_addr(bar_r, r);
+      uint8_t* slot = area + kCmRecvO + (size_t)rank * dps * kH * 2;
+      uint8_t* ml = area + kCmRecvML + (size_t)rank * 2 * kH * 4;
+      if (r1 > r0)
+        bulk_to_peer(dsmem_addr(slot, r), area + (size_t)r0 * kH * 2, (uint32_t)((r1 - r0) * kH * 2), bar);
+      bulk_to_peer(dsmem_addr(ml, r), s_M, kH * 4, bar);
+      bulk_to_peer(dsmem_addr(ml + kH * 4, r), s_l, kH * 4, bar);
+    }
+  }
+  const bool got = tc::mbar_wait(bar_r, 0, p.err);
+  const float* rml = reinterpret_cast<const float*>(area + kCmRecvML);
+  if (tid < kH) {
+    const int h = tid;
+    const float sink2 = p.sink[h] * kLog2e;
+    float M = sink2;
+    for (int j = 0; j < ns; ++j) M = fmaxf(M, rml[j * 2 * kH + h]);
+    float den = exp2f(sink2 - M);
+    for (int j = 0; j < ns; ++j) {
+      const float mj = rml[j * 2 * kH + h];
+      const float e = mj == -INFINITY ? 0.f : exp2f(mj - M);
+      s_mw[j * kH + h] = e;
+      den += rml[j * 2 * kH + kH + h] * e;
+    }
+    const float inv = 1.f / den;
+    for (int j = 0; j < ns; ++j) s_mw[j * kH + h] *= inv;
+    if (rank == 0 && p.lse) p.lse[(size_t)qrow * kH + h] = (M + log2f(den)) * 0.6931471805599453f;
+  }
+  __syncthreads();
+  // thread = (head, pair of dims); consecutive threads: consecutive dim pairs of one head
+  const int npair = dsl >> 1;
+  const __nv_bfloat16* recv = reinterpret_cast<const __nv_bfloat16*>(area + kCmRecvO);
+  for (int x = tid; x < kH * npair; x += blockDim.x) {
+    const int h = x / npair, dd = 2 * (x - h * npair);
+    const int c = h >> 3, e = h & 7;
+    float a0 = 0.f, a1 = 0.f;
+    for (int j = 0; j < ns; ++j) {
+      const __nv_bfloat16* slot = recv + (size_t)j * dps * kH;
+      const float w = s_mw[j * kH + h];
+      const int da = d0 + dd, db = da + 1;
+      a0 = fmaf(__bfloat162float(slot[dd * kH + cm_chunk(da, c) * 8 + e]), w, a0);
+      a1 = fmaf(__bfloat162float(slot[(dd + 1) * kH + cm_chunk(db, c) * 8 + e]), w, a1);
+    }
+    if (!ok || !got) a0 = a1 = __int_as_float(0x7fc00000);
+    *reinterpret_cast<__nv_bfloat162*>(&p.out[((size_t)qrow * kH + h) * kD + d0 + dd]) =
+        __floats2bfloat162_rn(a0, a1);
+  }
+}
+
+// Workspace merge (dense decode with more splits than a cluster holds): CTA per
+// (query, slice of 16 dims).
+constexpr int kMergeDims = 16;
+__global__ void __launch_bounds__(128) attn_merge_kernel(AttnTc p) {
+  extern __shared__ __align__(16) float mm_smem[];
+  float* s_ml = mm_smem;                                  // [2][kMaxSplitGlobal][kH]
+  float* s_mw = s_ml + 2 * kMaxSplitGlobal * kH;          // [kMaxSplitGlobal][kH]
+  uint8_t* stage = reinterpret_cast<uint8_t*>(s_mw + kMaxSplitGlobal * kH);
+  pdl_launch_dependents();
+  pdl_wait();
+  const int qrow = blockIdx.x;
+  const int d0 = blockIdx.y * kMergeDims;
+  merge_slice(p, qrow, d0, min(kD, d0 + kMergeDims), blockIdx.y == 0, stage, s_ml, s_mw,
+              kMaxSplitGlobal, p.q);
+}
+
 __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -142,8 +353,11 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   int* s_flag = reinterpret_cast<int*>(s_l + kH);
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(s_flag + 4);
   uint64_t* bar_o = bar_s + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_o + 1);
+  uint64_t* bar_r = bar_o + 1;                  // cluster merge: received slices
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_r + 1);
   const __nv_bfloat16** s_rows = reinterpret_cast<const __nv_bfloat16**>(tmem_holder + 2);  // [128]
+  float* s_mw = reinterpret_cast<float*>(                    // [kMaxSplit][kH] merge weights
+      (reinterpret_cast<uintptr_t>(s_rows + kRows) + 15) & ~(uintptr_t)15);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -153,13 +367,21 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   if (tid == 0) {
     tc::mbar_init(bar_s, 1);
     tc::mbar_init(bar_o, 1);
+    tc::mbar_init(bar_r, 1);
     tc::fence_barrier_init();
   }
   if (warp == 0) tc::tmem_alloc(tmem_holder, 512);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  pdl_wait();   // selections, positions and caches come from the preceding kernels
+  // the first item's query heads are an input of this call: fetch them before waiting
+  // on the preceding kernels (selections, positions and caches come from those)
+  const bool q_pre = (int)blockIdx.x < p.rows_total * p.nsplit && warp < 4;
+  if (q_pre) {
+    const __nv_bfloat16* qb = p.q + (size_t)(blockIdx.x / p.nsplit) * kH * kD;
+    gather_rows(sQ, kQBlkBytes, kH, warp, lane, [&](int h) { return qb + (size_t)h * kD; }, p.q);
+  }
+  pdl_wait();
   const uint32_t tmem = *tmem_holder;
   const uint32_t tS = tmem;            // columns [0, 64): S^T
   const uint32_t tO = tmem + 64;       // columns [64, 320): O^T, 4 blocks of 64
@@ -172,9 +394,11 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
     const int qrow = item / p.nsplit;
     const int split = item % p.nsplit;
     const QInfo Q = query_info(p, qrow);
-    const int ntiles = (Q.nrows + kRows - 1) / kRows;
-    const int jb = split * p.tps;
-    const int je = min(jb + p.tps, ntiles);
+    // rows [rb, re) of the query's list, in sub-tiles of up to 128 rows
+    const int rb = split * p.rps;
+    const int re = min(rb + p.rps, Q.nrows);
+    const int jb = 0;
+    const int je = re > rb ? (re - rb + kRows - 1) / kRows : 0;
 
     if (warp == 4) {
       // ---------------------------------------------------------------- MMA issuer
@@ -211,8 +435,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         }
         __syncwarp();
       }
-      continue;
-    }
+    } else {
 
     // ------------------------------------------------------------------ warps 0-3
     const int r = warp * 32 + lane;                  // this thread's TMEM lane / tile row
@@ -224,13 +447,16 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         ++no;
         tc::tc_fence_after();
       }
-      if (j == jb) {
+      if (j == jb && !(q_pre && item == (int)blockIdx.x)) {
         const __nv_bfloat16* qb = p.q + (size_t)qrow * kH * kD;
         gather_rows(sQ, kQBlkBytes, kH, warp, lane,
                     [&](int h) { return qb + (size_t)h * kD; }, p.kv);
       }
       // source of every row of the tile: one coalesced pass over the index list
-      s_rows[r] = row_src(p, Q, qrow, j * kRows + r);
+      {
+        const int pos = rb + j * kRows + r;
+        s_rows[r] = pos < re ? row_src(p, Q, qrow, pos) : nullptr;
+      }
       tc::named_bar(3, 128);
       gather_rows(sKV, kKVBlkBytes, kRows, warp, lane, [&](int rr) { return s_rows[rr]; }, p.kv);
       tc::cp_async_wait_all();
@@ -247,9 +473,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       tc::tmem_ld32(tS + lane_addr + 32, rb);
       tc::tmem_ld_wait(ra);
       tc::reg_fence(rb);
-      const int pos = j * kRows + r;
       const bool valid = s_rows[r] != nullptr;
-      (void)pos;
       float lg[64], v[64];
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
@@ -325,13 +549,18 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
     }
 
     if (je <= jb) {
-      // empty split: nothing to add
-      if (p.nsplit > 1 && tid < kH) {
+      // empty split: nothing to add.  Cluster mode: its running max stays -inf (weight 0)
+      // and its O is zeroed so that the merge's 0 * O stays 0.
+      if (p.nsplit > 1 && !p.cluster && tid < kH) {
         p.part_m[(size_t)item * kH + tid] = -INFINITY;
         p.part_l[(size_t)item * kH + tid] = 0.f;
       }
-      continue;
-    }
+      if (p.nsplit > 1 && p.cluster) {
+        uint4* z = reinterpret_cast<uint4*>(sKV);
+        for (int x = tid; x < kD * kH * 2 / 16; x += 128) z[x] = make_uint4(0u, 0u, 0u, 0u);
+        tc::fence_proxy_async();
+      }
+    } else {
     ok = ok && tc::mbar_wait(bar_o, no & 1, p.err);
     ++no;
     tc::tc_fence_after();
@@ -359,7 +588,8 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         const float den = s_l[tid] + exp2f(sk[tid] * kLog2e - s_M[tid]);
         p.lse[(size_t)qrow * kH + tid] = (s_M[tid] + log2f(den)) * 0.6931471805599453f;
       }
-    } else {
+    } else if (p.cluster) {
+      // unnormalised O into shared memory (bf16) for the cluster merge (KV tile area, free now)
       for (int mb = 0; mb < 4; ++mb) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -368,17 +598,58 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
           tc::tmem_ld_wait(o);
           const int d = mb * 128 + r;
 #pragma unroll
-          for (int h = 0; h < 32; ++h)
-            p.part_o[((size_t)item * kH + half * 32 + h) * kD + d] =
-                ok ? __uint_as_float(o[h]) : __int_as_float(0x7fc00000);
+          for (int c4 = 0; c4 < 4; ++c4) {    // 8 heads = one 16-byte chunk
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * c4 + 2 * e]),
+                                                              __uint_as_float(o[8 * c4 + 2 * e + 1]));
+              w4[e] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(sKV + (size_t)d * kH * 2 + cm_chunk(d, half * 4 + c4) * 16) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+      }
+      tc::fence_proxy_async();   // the bulk copies read these rows through the async proxy
+    } else {
+      for (int mb = 0; mb < 4; ++mb) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
+          tc::tmem_ld_wait(o);
+          const int d = mb * 128 + r;
+          float4* dst = reinterpret_cast<float4*>(&p.part_o[((size_t)item * kD + d) * kH + half * 32]);
+#pragma unroll
+          for (int h4 = 0; h4 < 8; ++h4) {
+            float4 v = make_float4(__uint_as_float(o[4 * h4]), __uint_as_float(o[4 * h4 + 1]),
+                                   __uint_as_float(o[4 * h4 + 2]), __uint_as_float(o[4 * h4 + 3]));
+            if (!ok) v = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                     __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+            dst[h4] = v;
+          }
         }
       }
       if (tid < kH) {
         p.part_m[(size_t)item * kH + tid] = s_M[tid];
         p.part_l[(size_t)item * kH + tid] = s_l[tid];
       }
-    }    tc::tc_fence_before();
+    }
+    }
+    tc::tc_fence_before();
     tc::named_bar(3, 128);                           // s_M / s_l reads done before the next item
+    }   // warps 0-3
+
+    if (p.nsplit > 1 && p.cluster) {
+      // every split of this query has its O, max and sum in shared memory: merge one
+      // slice of the dims, then keep this CTA's shared memory alive until all peers
+      // have read it
+      if (tid < kH) tc::fence_proxy_async();   // s_M / s_l are read by bulk copies too
+      cluster_sync_all();
+      cluster_merge(p, qrow, (int)cluster_rank(), sKV, s_M, s_l, s_mw, bar_r, ok);
+      cluster_sync_all();
+    }
   }
 
   tc::tc_fence_before();
@@ -389,97 +660,80 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   }
 }
 
-// Combines the splits of each (query, head): out = sum_s e^{m_s} O_s / (e^{sink} + sum_s e^{m_s} l_s).
-// CTA per (query, 4 heads); thread t owns dims 4t..4t+3 of the 4 heads (float4 loads).
-constexpr int kMergeHeads = 4;
-constexpr int kMaxSplit = 64;
-__global__ void __launch_bounds__(128) attn_merge_kernel(AttnTc p) {
-  __shared__ float s_m[kMaxSplit][kMergeHeads], s_l[kMaxSplit][kMergeHeads];
-  __shared__ float s_w[kMaxSplit][kMergeHeads];
-  pdl_launch_dependents();
-  pdl_wait();
-  const int qrow = blockIdx.x, h0 = blockIdx.y * kMergeHeads;
-  const size_t it0 = (size_t)qrow * p.nsplit;
-  for (int x = threadIdx.x; x < p.nsplit * kMergeHeads; x += blockDim.x) {
-    const int s = x / kMergeHeads, hh = x % kMergeHeads;
-    s_m[s][hh] = __ldcg(&p.part_m[(it0 + s) * kH + h0 + hh]);
-    s_l[s][hh] = __ldcg(&p.part_l[(it0 + s) * kH + h0 + hh]);
-  }
-  __syncthreads();
-  if (threadIdx.x < kMergeHeads) {
-    const int hh = threadIdx.x;
-    const float sink2 = p.sink[h0 + hh] * kLog2e;
-    float M = sink2;
-    for (int s = 0; s < p.nsplit; ++s) M = fmaxf(M, s_m[s][hh]);
-    float den = exp2f(sink2 - M);
-    for (int s = 0; s < p.nsplit; ++s) {
-      const float e = s_m[s][hh] == -INFINITY ? 0.f : exp2f(s_m[s][hh] - M);
-      s_w[s][hh] = e;
-      den += s_l[s][hh] * e;
-    }
-    const float inv = 1.f / den;
-    for (int s = 0; s < p.nsplit; ++s) s_w[s][hh] *= inv;
-    if (p.lse) p.lse[(size_t)qrow * kH + h0 + hh] = (M + log2f(den)) * 0.6931471805599453f;
-  }
-  __syncthreads();
-  const int d = threadIdx.x * 4;
-  float4 acc[kMergeHeads];
-#pragma unroll
-  for (int hh = 0; hh < kMergeHeads; ++hh) acc[hh] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < p.nsplit; ++s) {
-    float4 v[kMergeHeads];
-#pragma unroll
-    for (int hh = 0; hh < kMergeHeads; ++hh)
-      v[hh] = s_w[s][hh] != 0.f
-                  ? __ldcg(reinterpret_cast<const float4*>(
-                        &p.part_o[((it0 + s) * kH + h0 + hh) * kD + d]))
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int hh = 0; hh < kMergeHeads; ++hh) {
-      const float w = s_w[s][hh];
-      acc[hh].x = fmaf(v[hh].x, w, acc[hh].x); acc[hh].y = fmaf(v[hh].y, w, acc[hh].y);
-      acc[hh].z = fmaf(v[hh].z, w, acc[hh].z); acc[hh].w = fmaf(v[hh].w, w, acc[hh].w);
-    }
-  }
-#pragma unroll
-  for (int hh = 0; hh < kMergeHeads; ++hh) {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(acc[hh].x, acc[hh].y);
-    __nv_bfloat162 hi = __floats2bfloat162_rn(acc[hh].z, acc[hh].w);
-    uint2 u;
-    u.x = *reinterpret_cast<uint32_t*>(&lo);
-    u.y = *reinterpret_cast<uint32_t*>(&hi);
-    *reinterpret_cast<uint2*>(&p.out[((size_t)qrow * kH + h0 + hh) * kD + d]) = u;
-  }
-}
-
 constexpr size_t kSmemBytes = 1024 + 8 * kKVBlkBytes + 8 * kQBlkBytes + kRows * 128 +
-                              (4 * kH + 4 * kH) * 4 + 16 + 16 + 16 + kRows * 8;
+                              (4 * kH + 4 * kH) * 4 + 16 + 16 + 16 + kRows * 8 +
+                              16 + 16 + kMaxSplit * kH * 4;
 
 struct Plan {
-  int nsplit, tps;
+  int nsplit, rps;   // splits per query and rows per split
+  int cluster;       // merge inside a cluster (else through the workspace)
 };
-
-Plan plan(int H, int d, int k, int n_w, int b, int T, int E_cap, bool dense, int sms) {
-  Plan P{1, 1};
-  const long long rows_max = (long long)(dense ? E_cap : k) + n_w;
-  const int tmax = (int)((rows_max + kRows - 1) / kRows);
-  P.tps = tmax;
-  if (T == 1) {
-    // decode: split each query's tiles so the grid covers the SMs about twice
-    long long want = (2LL * sms + b - 1) / b;
-    int ns = (int)std::min<long long>(std::max<long long>(1, want), tmax);
-    P.tps = (tmax + ns - 1) / ns;
-    P.nsplit = (tmax + P.tps - 1) / P.tps;
-  }
-  (void)H; (void)d;
-  return P;
-}
 
 int sm_count() {
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   return sms;
+}
+
+// How many clusters of `cs` attention CTAs the device can hold at once (cached per device).
+int max_active_clusters(int cs) {
+  static int cache[64][kMaxSplit + 1] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || cs < 1 || cs > kMaxSplit) return 0;
+  if (cache[dev][cs]) return cache[dev][cs] - 1;
+  int n = 0;
+  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kSmemBytes) == cudaSuccess &&
+      (cs <= 8 || cudaFuncSetAttribute(attn_tc_kernel,
+                                       cudaFuncAttributeNonPortableClusterSizeAllowed, 1) ==
+                      cudaSuccess)) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs);
+    cfg.blockDim = dim3(160);
+    cfg.dynamicSmemBytes = kSmemBytes;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = 1;
+    if (cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg) != cudaSuccess) n = 0;
+  }
+  cudaGetLastError();   // a refused query leaves no error behind
+  cache[dev][cs] = n + 1;
+  return n;
+}
+
+// Decode (one query per sequence) splits each query's rows over several CTAs, at
+// most one CTA per SM over the whole grid and at least 16 rows per split.
+//  - selected entries (CSA): the splits of a query form one cluster, as large as lets
+//    all b clusters be resident at once (at most kMaxSplit); merged in the cluster;
+//  - dense (HCA, thousands of rows per query): up to kMaxSplitGlobal splits, merged
+//    through the workspace by attn_merge_kernel.
+// Prefill: one split per query.
+Plan plan(int k, int n_w, int b, int T, int E_cap, bool dense, int sms) {
+  const long long rows_max = (long long)(dense ? E_cap : k) + n_w;
+  Plan P{1, (int)std::min<long long>(rows_max, INT_MAX), 0};
+  if (T == 1 && b > 0) {
+    const int cap = dense ? kMaxSplitGlobal : kMaxSplit;
+    int ns = std::max(1, std::min(cap, sms / b));
+    ns = (int)std::min<long long>(ns, std::max<long long>(1, rows_max / 16));
+    if (!dense)
+      while (ns > 1 && max_active_clusters(ns) < b) --ns;
+    long long rps = (rows_max + ns - 1) / ns;
+    rps = (rps + 15) / 16 * 16;
+    P.rps = (int)rps;
+    P.nsplit = (int)((rows_max + rps - 1) / rps);
+    P.cluster = !dense && P.nsplit > 1;
+  }
+  return P;
+}
+
+size_t merge_smem_bytes() {
+  return (size_t)3 * kMaxSplitGlobal * kH * 4 + (size_t)kMaxSplitGlobal * kMergeDims * kH * 4;
 }
 
 }  // namespace
@@ -490,14 +744,14 @@ bool attn_tc_supported(int H, int d, int dtype) {
 
 int attn_launch_count(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype) {
   if (!attn_tc_supported(H, d, dtype)) return 1;
-  const Plan P = plan(H, d, k, n_w, b, T, E_cap, k <= 0, sm_count());
-  return P.nsplit > 1 ? 2 : 1;
+  const Plan P = plan(k, n_w, b, T, E_cap, k <= 0, sm_count());
+  return P.nsplit > 1 && !P.cluster ? 2 : 1;
 }
 
 size_t attn_tc_workspace_bytes(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype) {
   if (!attn_tc_supported(H, d, dtype) || b <= 0 || T <= 0) return 0;
-  const Plan P = plan(H, d, k, n_w, b, T, E_cap, k <= 0, sm_count());
-  if (P.nsplit <= 1) return 0;
+  const Plan P = plan(k, n_w, b, T, E_cap, k <= 0, sm_count());
+  if (P.nsplit <= 1 || P.cluster) return 0;
   const size_t items = (size_t)b * T * P.nsplit;
   return items * kH * kD * 4 + 2 * items * kH * 4 + 256;
 }
@@ -507,7 +761,7 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
   if (!attn_tc_supported(a.H, a.d, dtype)) return CSA_ERR_UNSUPPORTED;
   const bool dense = a.idx == nullptr;
   const int sms = sm_count();
-  const Plan P = plan(a.H, a.d, dense ? 0 : a.k, a.n_w, b, a.T, a.E_cap, dense, sms);
+  const Plan P = plan(dense ? 0 : a.k, a.n_w, b, a.T, a.E_cap, dense, sms);
   AttnTc p{};
   p.q = reinterpret_cast<const __nv_bfloat16*>(a.q);
   p.kv = reinterpret_cast<const __nv_bfloat16*>(a.kv ? a.kv : a.win);
@@ -518,13 +772,14 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
   p.err = device_error_word();
   if (!p.err) return CSA_ERR_CUDA;
   p.T = a.T; p.n_w = a.n_w; p.m = a.m; p.k = a.k; p.E_cap = a.kv ? a.E_cap : 0; p.n = a.n;
-  p.rows_total = b * a.T; p.nsplit = P.nsplit; p.tps = P.tps; p.dense = dense ? 1 : 0;
+  p.rows_total = b * a.T; p.nsplit = P.nsplit; p.rps = P.rps; p.dense = dense ? 1 : 0;
+  p.cluster = P.cluster;
   p.scale_log2 = a.scale * kLog2e;
-  if (P.nsplit > 1) {
+  if (P.nsplit > 1 && !P.cluster) {
     const size_t items = (size_t)b * a.T * P.nsplit;
     const size_t need = items * kH * kD * 4 + 2 * items * kH * 4;
     if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15)) return CSA_ERR_INVALID_ARG;
-    if (P.nsplit > kMaxSplit) return CSA_ERR_UNSUPPORTED;
+    if (P.nsplit > kMaxSplitGlobal) return CSA_ERR_UNSUPPORTED;
     p.part_o = reinterpret_cast<float*>(ws);
     p.part_m = p.part_o + items * kH * kD;
     p.part_l = p.part_m + items * kH;
@@ -533,14 +788,43 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
                            (int)kSmemBytes) != cudaSuccess)
     return CSA_ERR_CUDA;
   const long long items = (long long)b * a.T * P.nsplit;
-  const int grid = (int)std::min<long long>(items, sms);
-  if (csa_launch(attn_tc_kernel, dim3(grid), dim3(160), kSmemBytes, st, a.pdl != 0, p) !=
-      cudaSuccess)
+  if (!P.cluster) {
+    const int grid = (int)std::min<long long>(items, sms);
+    if (csa_launch(attn_tc_kernel, dim3(grid), dim3(160), kSmemBytes, st, a.pdl != 0, p) !=
+        cudaSuccess)
+      return CSA_ERR_CUDA;
+    if (P.nsplit > 1) {
+      const size_t msm = merge_smem_bytes();
+      if (cudaFuncSetAttribute(attn_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)msm) != cudaSuccess)
+        return CSA_ERR_CUDA;
+      if (csa_launch(attn_merge_kernel, dim3(b * a.T, kD / kMergeDims), dim3(128), msm, st,
+                     a.pdl != 0, p) != cudaSuccess)
+        return CSA_ERR_CUDA;
+    }
+    return CSA_OK;
+  }
+  // one CTA per (query, split); the splits of a query form one cluster
+  if (items > 0x7fffffff) return CSA_ERR_UNSUPPORTED;
+  if (P.nsplit > 8 &&
+      cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) !=
+          cudaSuccess)
     return CSA_ERR_CUDA;
-  if (P.nsplit > 1 &&
-      csa_launch(attn_merge_kernel, dim3(b * a.T, kH / kMergeHeads), dim3(128), 0, st, a.pdl != 0,
-                 p) != cudaSuccess)
-    return CSA_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)items);
+  cfg.blockDim = dim3(160);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = (unsigned)P.nsplit;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = a.pdl ? 2 : 1;
+  if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, p) != cudaSuccess) return CSA_ERR_CUDA;
   return CSA_OK;
 }
 
