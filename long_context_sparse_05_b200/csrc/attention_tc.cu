@@ -262,33 +262,32 @@ __device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool writ
 // out = sum_j e^{m_j} O_j / (e^{sink} + sum_j e^{m_j} l_j).
 __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int rank, uint8_t* area,
                                               const float* s_M, const float* s_l, float* s_mw,
-                                              uint64_t* bar_r, bool ok) {
+                                              const float* s_sink2, uint64_t* bar_r, bool ok) {
   const int tid = threadIdx.x;
   const int ns = p.nsplit;
   int d0, d1;
   cm_slice(ns, rank, d0, d1);
   const int dsl = d1 - d0;
   const int dps = ((kD + ns - 1) / ns + 7) & ~7;
-  if (tid == 0) {
-    // what this CTA receives: every split's slice of its dims and its max and sum
-    tc::mbar_arrive_expect_tx(bar_r, (uint32_t)(ns * (dsl * kH * 2 + 2 * kH * 4)));
-    for (int r = 0; r < ns; ++r) {
-      int r0, r1;
-      cm_slice(ns, r, r0, r1);
-      const uint32_t bar = dsmem_addr(bar_r, r);
-      uint8_t* slot = area + kCmRecvO + (size_t)rank * dps * kH * 2;
-      uint8_t* ml = area + kCmRecvML + (size_t)rank * 2 * kH * 4;
-      if (r1 > r0)
-        bulk_to_peer(dsmem_addr(slot, r), area + (size_t)r0 * kH * 2, (uint32_t)((r1 - r0) * kH * 2), bar);
-      bulk_to_peer(dsmem_addr(ml, r), s_M, kH * 4, bar);
-      bulk_to_peer(dsmem_addr(ml + kH * 4, r), s_l, kH * 4, bar);
-    }
+  // what this CTA receives: every split's slice of its dims and its max and sum
+  if (tid == 0) tc::mbar_arrive_expect_tx(bar_r, (uint32_t)(ns * (dsl * kH * 2 + 2 * kH * 4)));
+  if (tid < ns) {   // thread r sends to rank r
+    const int r = tid;
+    int r0, r1;
+    cm_slice(ns, r, r0, r1);
+    const uint32_t bar = dsmem_addr(bar_r, r);
+    uint8_t* slot = area + kCmRecvO + (size_t)rank * dps * kH * 2;
+    uint8_t* ml = area + kCmRecvML + (size_t)rank * 2 * kH * 4;
+    if (r1 > r0)
+      bulk_to_peer(dsmem_addr(slot, r), area + (size_t)r0 * kH * 2, (uint32_t)((r1 - r0) * kH * 2), bar);
+    bulk_to_peer(dsmem_addr(ml, r), s_M, kH * 4, bar);
+    bulk_to_peer(dsmem_addr(ml + kH * 4, r), s_l, kH * 4, bar);
   }
   const bool got = tc::mbar_wait(bar_r, 0, p.err);
   const float* rml = reinterpret_cast<const float*>(area + kCmRecvML);
   if (tid < kH) {
     const int h = tid;
-    const float sink2 = p.sink[h] * kLog2e;
+    const float sink2 = s_sink2[h];
     float M = sink2;
     for (int j = 0; j < ns; ++j) M = fmaxf(M, rml[j * 2 * kH + h]);
     float den = exp2f(sink2 - M);
@@ -303,23 +302,32 @@ __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int ran
     if (rank == 0 && p.lse) p.lse[(size_t)qrow * kH + h] = (M + log2f(den)) * 0.6931471805599453f;
   }
   __syncthreads();
-  // thread = (head, pair of dims); consecutive threads: consecutive dim pairs of one head
-  const int npair = dsl >> 1;
+  // thread = (chunk of 8 heads, dim); consecutive threads: consecutive dims, so each
+  // split is one conflict-free 16-byte shared load per thread and each head's output
+  // run is a coalesced store
   const __nv_bfloat16* recv = reinterpret_cast<const __nv_bfloat16*>(area + kCmRecvO);
-  for (int x = tid; x < kH * npair; x += blockDim.x) {
-    const int h = x / npair, dd = 2 * (x - h * npair);
-    const int c = h >> 3, e = h & 7;
-    float a0 = 0.f, a1 = 0.f;
+  for (int x = tid; x < dsl * 8; x += blockDim.x) {
+    const int c = x / dsl, dd = x - c * dsl;
+    const int d = d0 + dd;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < ns; ++j) {
-      const __nv_bfloat16* slot = recv + (size_t)j * dps * kH;
-      const float w = s_mw[j * kH + h];
-      const int da = d0 + dd, db = da + 1;
-      a0 = fmaf(__bfloat162float(slot[dd * kH + cm_chunk(da, c) * 8 + e]), w, a0);
-      a1 = fmaf(__bfloat162float(slot[(dd + 1) * kH + cm_chunk(db, c) * 8 + e]), w, a1);
+      const uint4 v = *reinterpret_cast<const uint4*>(recv + ((size_t)j * dps + dd) * kH +
+                                                      cm_chunk(d, c) * 8);
+      const float4 wa = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c);
+      const float4 wb = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c + 4);
+      const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&u[e]);
+        acc[2 * e] = fmaf(__low2float(b2), w[2 * e], acc[2 * e]);
+        acc[2 * e + 1] = fmaf(__high2float(b2), w[2 * e + 1], acc[2 * e + 1]);
+      }
     }
-    if (!ok || !got) a0 = a1 = __int_as_float(0x7fc00000);
-    *reinterpret_cast<__nv_bfloat162*>(&p.out[((size_t)qrow * kH + h) * kD + d0 + dd]) =
-        __floats2bfloat162_rn(a0, a1);
+    __nv_bfloat16* o = p.out + ((size_t)qrow * kH + 8 * c) * kD + d;
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      o[(size_t)e * kD] = __float2bfloat16_rn((ok && got) ? acc[e] : __int_as_float(0x7fc00000));
   }
 }
 
@@ -358,12 +366,14 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   const __nv_bfloat16** s_rows = reinterpret_cast<const __nv_bfloat16**>(tmem_holder + 2);  // [128]
   float* s_mw = reinterpret_cast<float*>(                    // [kMaxSplit][kH] merge weights
       (reinterpret_cast<uintptr_t>(s_rows + kRows) + 15) & ~(uintptr_t)15);
+  float* s_sink2 = s_mw + kMaxSplit * kH;                   // [kH] sink logits, log2 units
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
 
   pdl_launch_dependents();
+  if (tid < kH) s_sink2[tid] = p.sink[tid] * kLog2e;   // an input: read before the wait
   if (tid == 0) {
     tc::mbar_init(bar_s, 1);
     tc::mbar_init(bar_o, 1);
@@ -647,7 +657,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       // have read it
       if (tid < kH) tc::fence_proxy_async();   // s_M / s_l are read by bulk copies too
       cluster_sync_all();
-      cluster_merge(p, qrow, (int)cluster_rank(), sKV, s_M, s_l, s_mw, bar_r, ok);
+      cluster_merge(p, qrow, (int)cluster_rank(), sKV, s_M, s_l, s_mw, s_sink2, bar_r, ok);
       cluster_sync_all();
     }
   }
@@ -662,7 +672,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
 
 constexpr size_t kSmemBytes = 1024 + 8 * kKVBlkBytes + 8 * kQBlkBytes + kRows * 128 +
                               (4 * kH + 4 * kH) * 4 + 16 + 16 + 16 + kRows * 8 +
-                              16 + 16 + kMaxSplit * kH * 4;
+                              16 + 16 + kMaxSplit * kH * 4 + kH * 4;
 
 struct Plan {
   int nsplit, rps;   // splits per query and rows per split

@@ -53,29 +53,28 @@ template <> struct Keys<float> {
   }
 };
 
-// Block-wide sums of NV unsigned values (every thread gets them).  s_red holds
-// 32 x NV words plus NV result words.
+// Block-wide sums of NV unsigned values (every thread gets them), with one barrier:
+// each warp writes its partial sums into one of two buffers (alternating per call, so
+// a fast warp's next call cannot overwrite a buffer still being read), and every
+// thread adds up the warps' partials itself.  s_red holds 2 x 64 words (NV <= 2).
 template <int NV>
-__device__ __forceinline__ void block_sums(uint32_t (&v)[NV], uint32_t* s_red) {
+__device__ __forceinline__ void block_sums(uint32_t (&v)[NV], uint32_t* s_red, uint32_t& parity) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  static_assert(NV <= 2, "two 64-word buffers");
+  uint32_t* buf = s_red + parity * 64;
+  parity ^= 1u;
 #pragma unroll
   for (int i = 0; i < NV; ++i) {
     const uint32_t w = __reduce_add_sync(0xffffffffu, v[i]);
-    if (lane == 0) s_red[wid * NV + i] = w;
-  }
-  __syncthreads();
-  if (wid == 0) {
-#pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      const uint32_t x = lane < nw ? s_red[lane * NV + i] : 0u;
-      const uint32_t t = __reduce_add_sync(0xffffffffu, x);
-      if (lane == 0) s_red[32 * NV + i] = t;
-    }
+    if (lane == 0) buf[wid * NV + i] = w;
   }
   __syncthreads();
 #pragma unroll
-  for (int i = 0; i < NV; ++i) v[i] = s_red[32 * NV + i];
-  __syncthreads();   // s_red is reused by the next call
+  for (int i = 0; i < NV; ++i) v[i] = 0u;
+  for (int w = 0; w < nw; ++w) {
+#pragma unroll
+    for (int i = 0; i < NV; ++i) v[i] += buf[w * NV + i];
+  }
 }
 
 // Top-k of one row (or chunk) of `n` entries held by the CTA.
@@ -92,6 +91,7 @@ __device__ __forceinline__ void cta_topk(const S* __restrict__ src, int n, int k
   using Bits = typename K::Bits;
   const int tid = threadIdx.x;
   const int NT = blockDim.x;
+  uint32_t parity = 0;                           // block_sums buffer selector
   if (n <= k) {                                  // everything is kept
     for (int j = tid; j < k; j += NT) {
       const bool v = j < n;
@@ -171,7 +171,7 @@ __device__ __forceinline__ void cta_topk(const S* __restrict__ src, int n, int k
       c[0] += (key[e] >= sp[0] ? 1u : 0u) | (key[e] >= sp[1] ? 0x10000u : 0u);
       c[1] += key[e] >= sp[2] ? 1u : 0u;
     }
-    block_sums<2>(c, s_red);
+    block_sums<2>(c, s_red, parity);
     const uint32_t c0 = c[0] & 0xffffu, c1 = c[0] >> 16, c2 = c[1];
     uint32_t nlo = lo, nhi = hi;
     if (c2 >= (uint32_t)k) { nlo = sp[2]; }
@@ -192,7 +192,7 @@ __device__ __forceinline__ void cta_topk(const S* __restrict__ src, int n, int k
   }
   const uint32_t n_gt = __popc(gt_mask), n_eq = __popc(eq_mask);
   uint32_t tot[1] = {n_gt};
-  block_sums<1>(tot, s_red);
+  block_sums<1>(tot, s_red, parity);
   const int need = k - (int)tot[0];              // equal keys to take, lowest entries first
 
   // exclusive block scan of (gt | eq << 16)
@@ -204,19 +204,20 @@ __device__ __forceinline__ void cta_topk(const S* __restrict__ src, int n, int k
     const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
     if (lane >= o) x += y;
   }
-  if (lane == 31) s_red[wid] = x;
+  uint32_t* sc = s_red + 128;                   // apart from block_sums' buffers
+  if (lane == 31) sc[wid] = x;
   __syncthreads();
   if (wid == 0) {
-    uint32_t w = lane < nw ? s_red[lane] : 0u;
+    uint32_t w = lane < nw ? sc[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
       if (lane >= o) w += y;
     }
-    if (lane < nw) s_red[lane] = w;
+    if (lane < nw) sc[lane] = w;
   }
   __syncthreads();
-  const uint32_t excl = (wid > 0 ? s_red[wid - 1] : 0u) + x - packed;
+  const uint32_t excl = (wid > 0 ? sc[wid - 1] : 0u) + x - packed;
   const int gt_before = (int)(excl & 0xffffu);
   const int eq_before = (int)(excl >> 16);
   const int take_eq = min(max(need - eq_before, 0), (int)n_eq);
@@ -245,7 +246,7 @@ template <typename S>
 __global__ void __launch_bounds__(kNT) topk_row_kernel(
     const S* __restrict__ scores, const int32_t* __restrict__ q_pos, int m, int E, int k,
     int32_t* __restrict__ idx, int32_t* __restrict__ count) {
-  __shared__ uint32_t s_red[72];
+  __shared__ uint32_t s_red[128 + 32];
   pdl_launch_dependents();
   pdl_wait();
   const int row = blockIdx.x;
@@ -259,7 +260,7 @@ template <typename S>
 __global__ void __launch_bounds__(kNT) topk_chunk_kernel(
     const S* __restrict__ scores, const int32_t* __restrict__ q_pos, int m, int E, int k,
     int nchunks, S* __restrict__ cand_scores, int32_t* __restrict__ cand_idx) {
-  __shared__ uint32_t s_red[72];
+  __shared__ uint32_t s_red[128 + 32];
   pdl_launch_dependents();
   pdl_wait();
   const int row = blockIdx.x / nchunks, c = blockIdx.x % nchunks;
@@ -278,7 +279,7 @@ __global__ void __launch_bounds__(kNT) topk_merge_kernel(
     const S* __restrict__ cand_scores, const int32_t* __restrict__ cand_idx,
     const int32_t* __restrict__ q_pos, int m, int E, int k, int nchunks,
     int32_t* __restrict__ idx, int32_t* __restrict__ count) {
-  __shared__ uint32_t s_red[72];
+  __shared__ uint32_t s_red[128 + 32];
   pdl_launch_dependents();
   pdl_wait();
   const int row = blockIdx.x;
