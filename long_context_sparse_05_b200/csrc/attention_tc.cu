@@ -56,9 +56,10 @@ struct AttnTc {
   float* part_o; float* part_m; float* part_l;
   int* err;
   int T, n_w, m, k, E_cap, n, rows_total, nsplit, rps, dense;
-  int cluster;   // nsplit > 1: 1 = the splits of a query are one cluster and merge through
-                 // distributed shared memory; 0 = partials go to the workspace and
-                 // attn_merge_kernel combines them
+  int cluster;   // nsplit > 1: 1 = the splits of a query are one cluster and merge inside
+                 // the kernel; 0 = fp32 partials go to the workspace and attn_merge_kernel
+                 // combines them
+  uint8_t* part_bf;   // cluster mode: per item, bf16 O [512][64] (swizzled rows), max, sum
   float scale_log2;
 };
 
@@ -144,42 +145,36 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   return r;
 }
 
-__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(tc::smem_u32(local)), "r"(rank));
-  return r;
-}
-__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float4 ld_dsmem4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr) : "memory");
-  return v;
-}
-
 constexpr int kMaxSplit = 16;         // splits of one query merged inside one cluster
 constexpr int kMaxSplitGlobal = 32;   // splits of one query merged through the workspace
 
-// Cluster merge layout (inside the KV / query tile area, free once PV is done):
-//   [0, 64 KB)           this split's unnormalised O, bf16 [512 dims][64 heads], the 16-byte
-//                        chunk c of dim d's row stored at chunk c ^ (d & 7)
-//   [64 KB, 144 KB)      received slices: split j's rows of this CTA's dims at slot j
+// Cluster merge.  Each split stores its unnormalised O (bf16 [512 dims][64 heads], the
+// 16-byte chunk c of dim d's row at chunk c ^ (d & 7)), its running max and sum to the
+// workspace with bulk stores; after a cluster barrier every rank bulk-loads, from every
+// split, the rows of the dims it merges.  Shared memory (KV / query tile area, free
+// once PV is done):
+//   [0, 64 KB)           this split's O, staged for the bulk store
+//   [64 KB, 144 KB)      received slices: split j's rows of this rank's dims at slot j
 //   [144 KB, 152 KB)     received running maxima and sums: [split][2][64] fp32
 constexpr int kCmRecvO = 64 * 1024;
 constexpr int kCmRecvML = 144 * 1024;
+constexpr size_t kPartB = (size_t)kD * kH * 2 + 2 * kH * 4;   // one split's record
 __device__ __forceinline__ int cm_chunk(int d, int chunk) { return chunk ^ (d & 7); }
 
-// Bulk copy of `bytes` from this CTA's shared memory to a peer's (cluster address), counted
-// as transaction bytes on the peer's mbarrier.
-__device__ __forceinline__ void bulk_to_peer(uint32_t dst_cluster, const void* src, uint32_t bytes,
-                                             uint32_t bar_cluster) {
+__device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+               ::"l"(gdst), "r"(tc::smem_u32(ssrc)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_store_commit_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_load_g(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-      ::"r"(dst_cluster), "r"(tc::smem_u32(src)), "r"(bytes), "r"(bar_cluster) : "memory");
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(tc::smem_u32(sdst)), "l"(gsrc), "r"(bytes), "r"(tc::smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // Dims of the output slice merged by cluster rank `rank`.
@@ -260,68 +255,96 @@ __device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool writ
 // rows of its O that another rank merges, plus its running max and sum, into that rank's
 // shared memory with bulk copies; then rank r combines output dims [d0, d1) locally:
 // out = sum_j e^{m_j} O_j / (e^{sink} + sum_j e^{m_j} l_j).
-__device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int rank, uint8_t* area,
-                                              const float* s_M, const float* s_l, float* s_mw,
-                                              const float* s_sink2, uint64_t* bar_r, bool ok) {
+__device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int item, int rank,
+                                              uint8_t* area, const float* s_M, const float* s_l,
+                                              float* s_mw, const float* s_sink2, uint64_t* bar_r,
+                                              bool ok) {
   const int tid = threadIdx.x;
   const int ns = p.nsplit;
   int d0, d1;
   cm_slice(ns, rank, d0, d1);
   const int dsl = d1 - d0;
   const int dps = ((kD + ns - 1) / ns + 7) & ~7;
-  // what this CTA receives: every split's slice of its dims and its max and sum
-  if (tid == 0) tc::mbar_arrive_expect_tx(bar_r, (uint32_t)(ns * (dsl * kH * 2 + 2 * kH * 4)));
-  if (tid < ns) {   // thread r sends to rank r
-    const int r = tid;
-    int r0, r1;
-    cm_slice(ns, r, r0, r1);
-    const uint32_t bar = dsmem_addr(bar_r, r);
-    uint8_t* slot = area + kCmRecvO + (size_t)rank * dps * kH * 2;
-    uint8_t* ml = area + kCmRecvML + (size_t)rank * 2 * kH * 4;
-    if (r1 > r0)
-      bulk_to_peer(dsmem_addr(slot, r), area + (size_t)r0 * kH * 2, (uint32_t)((r1 - r0) * kH * 2), bar);
-    bulk_to_peer(dsmem_addr(ml, r), s_M, kH * 4, bar);
-    bulk_to_peer(dsmem_addr(ml + kH * 4, r), s_l, kH * 4, bar);
+  // this split's record to the workspace (the rows were fenced for the async proxy)
+  if (tid == 0) {
+    uint8_t* rec = p.part_bf + (size_t)item * kPartB;
+    bulk_store(rec, area, kD * kH * 2);
+    bulk_store(rec + kD * kH * 2, s_M, kH * 4);
+    bulk_store(rec + kD * kH * 2 + kH * 4, s_l, kH * 4);
+    bulk_store_commit_wait();
+    fence_proxy_async_global();
+  }
+  cluster_sync_all();   // every split's record is in the workspace
+  if (tid == 0) {
+    fence_proxy_async_global();
+    tc::mbar_arrive_expect_tx(bar_r, (uint32_t)(ns * (dsl * kH * 2 + 2 * kH * 4)));
+    const size_t it0 = (size_t)qrow * ns;
+    for (int j = 0; j < ns; ++j) {
+      const uint8_t* rec = p.part_bf + (it0 + j) * kPartB;
+      if (dsl > 0)
+        bulk_load_g(area + kCmRecvO + (size_t)j * dps * kH * 2, rec + (size_t)d0 * kH * 2,
+                    (uint32_t)(dsl * kH * 2), bar_r);
+      bulk_load_g(area + kCmRecvML + (size_t)j * 2 * kH * 4, rec + kD * kH * 2, 2 * kH * 4, bar_r);
+    }
   }
   const bool got = tc::mbar_wait(bar_r, 0, p.err);
   const float* rml = reinterpret_cast<const float*>(area + kCmRecvML);
   if (tid < kH) {
+    // all maxima and sums of this head first (independent loads), then the weights
     const int h = tid;
+    float mj[kMaxSplit], lj[kMaxSplit];
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j) {
+      mj[j] = j < ns ? rml[j * 2 * kH + h] : -INFINITY;
+      lj[j] = j < ns ? rml[j * 2 * kH + kH + h] : 0.f;
+    }
     const float sink2 = s_sink2[h];
     float M = sink2;
-    for (int j = 0; j < ns; ++j) M = fmaxf(M, rml[j * 2 * kH + h]);
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j) M = fmaxf(M, mj[j]);
     float den = exp2f(sink2 - M);
-    for (int j = 0; j < ns; ++j) {
-      const float mj = rml[j * 2 * kH + h];
-      const float e = mj == -INFINITY ? 0.f : exp2f(mj - M);
-      s_mw[j * kH + h] = e;
-      den += rml[j * 2 * kH + kH + h] * e;
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j) {
+      mj[j] = mj[j] == -INFINITY ? 0.f : exp2f(mj[j] - M);
+      den = fmaf(lj[j], mj[j], den);
     }
     const float inv = 1.f / den;
-    for (int j = 0; j < ns; ++j) s_mw[j * kH + h] *= inv;
+#pragma unroll
+    for (int j = 0; j < kMaxSplit; ++j)
+      if (j < ns) s_mw[j * kH + h] = mj[j] * inv;
     if (rank == 0 && p.lse) p.lse[(size_t)qrow * kH + h] = (M + log2f(den)) * 0.6931471805599453f;
   }
   __syncthreads();
   // thread = (chunk of 8 heads, dim); consecutive threads: consecutive dims, so each
   // split is one conflict-free 16-byte shared load per thread and each head's output
-  // run is a coalesced store
+  // run is a coalesced store.  Four splits' loads are in flight at a time.
   const __nv_bfloat16* recv = reinterpret_cast<const __nv_bfloat16*>(area + kCmRecvO);
   for (int x = tid; x < dsl * 8; x += blockDim.x) {
     const int c = x / dsl, dd = x - c * dsl;
     const int d = d0 + dd;
+    const int off = dd * kH + cm_chunk(d, c) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j < ns; ++j) {
-      const uint4 v = *reinterpret_cast<const uint4*>(recv + ((size_t)j * dps + dd) * kH +
-                                                      cm_chunk(d, c) * 8);
-      const float4 wa = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c);
-      const float4 wb = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c + 4);
-      const float w[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
-      const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+    for (int j0 = 0; j0 < ns; j0 += 4) {
+      uint4 v[4];
+      float4 wa[4], wb[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&u[e]);
-        acc[2 * e] = fmaf(__low2float(b2), w[2 * e], acc[2 * e]);
-        acc[2 * e + 1] = fmaf(__high2float(b2), w[2 * e + 1], acc[2 * e + 1]);
+      for (int u = 0; u < 4; ++u) {
+        const int j = min(j0 + u, ns - 1);
+        v[u] = *reinterpret_cast<const uint4*>(recv + (size_t)j * dps * kH + off);
+        wa[u] = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c);
+        wb[u] = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c + 4);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (j0 + u >= ns) break;
+        const float w[8] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w, wb[u].x, wb[u].y, wb[u].z, wb[u].w};
+        const uint32_t q[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&q[e]);
+          acc[2 * e] = fmaf(__low2float(b2), w[2 * e], acc[2 * e]);
+          acc[2 * e + 1] = fmaf(__high2float(b2), w[2 * e + 1], acc[2 * e + 1]);
+        }
       }
     }
     __nv_bfloat16* o = p.out + ((size_t)qrow * kH + 8 * c) * kD + d;
@@ -655,10 +678,9 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       // every split of this query has its O, max and sum in shared memory: merge one
       // slice of the dims, then keep this CTA's shared memory alive until all peers
       // have read it
-      if (tid < kH) tc::fence_proxy_async();   // s_M / s_l are read by bulk copies too
-      cluster_sync_all();
-      cluster_merge(p, qrow, (int)cluster_rank(), sKV, s_M, s_l, s_mw, s_sink2, bar_r, ok);
-      cluster_sync_all();
+      if (tid < kH) tc::fence_proxy_async();   // s_M / s_l are read by the bulk stores too
+      __syncthreads();
+      cluster_merge(p, qrow, item, (int)cluster_rank(), sKV, s_M, s_l, s_mw, s_sink2, bar_r, ok);
     }
   }
 
@@ -761,8 +783,9 @@ int attn_launch_count(int H, int d, int k, int n_w, int b, int T, int E_cap, int
 size_t attn_tc_workspace_bytes(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype) {
   if (!attn_tc_supported(H, d, dtype) || b <= 0 || T <= 0) return 0;
   const Plan P = plan(k, n_w, b, T, E_cap, k <= 0, sm_count());
-  if (P.nsplit <= 1 || P.cluster) return 0;
+  if (P.nsplit <= 1) return 0;
   const size_t items = (size_t)b * T * P.nsplit;
+  if (P.cluster) return items * kPartB + 256;
   return items * kH * kD * 4 + 2 * items * kH * 4 + 256;
 }
 
@@ -785,6 +808,12 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
   p.rows_total = b * a.T; p.nsplit = P.nsplit; p.rps = P.rps; p.dense = dense ? 1 : 0;
   p.cluster = P.cluster;
   p.scale_log2 = a.scale * kLog2e;
+  if (P.nsplit > 1 && P.cluster) {
+    const size_t items = (size_t)b * a.T * P.nsplit;
+    if (!ws || ws_bytes < items * kPartB || (reinterpret_cast<uintptr_t>(ws) & 15))
+      return CSA_ERR_INVALID_ARG;
+    p.part_bf = static_cast<uint8_t*>(ws);
+  }
   if (P.nsplit > 1 && !P.cluster) {
     const size_t items = (size_t)b * a.T * P.nsplit;
     const size_t need = items * kH * kD * 4 + 2 * items * kH * 4;

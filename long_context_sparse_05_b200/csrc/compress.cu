@@ -308,6 +308,189 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
                       a.q_scales);
 }
 
+// One entry of a long non-overlapped block (c128a: m = 128 rows) split over the CTAs of
+// a cluster: rank r pools rows [r m / CS, (r + 1) m / CS) of the block into per-channel
+// partial (max, sum, weighted sum), the ranks exchange them through distributed shared
+// memory, and rank r finishes channels [r c / CS, (r + 1) c / CS): combine, RMSNorm (the
+// sum of squares is exchanged once more), RoPE, store.  F32 / BF16 outputs only.
+__device__ __forceinline__ uint32_t cs_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cs_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+__device__ __forceinline__ float cs_ld(const float* local, uint32_t rank) {
+  uint32_t la = static_cast<uint32_t>(__cvta_generic_to_shared(local)), ra;
+  float v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(la), "r"(rank));
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+
+template <typename InT>
+__global__ void __launch_bounds__(256) compress_split_kernel(CompressArgs a, int32_t* qpos, int nq,
+                                                             int t) {
+  extern __shared__ float smem[];
+  constexpr int VEC = Vec16<InT>::N;
+  const int c = a.c;
+  const int cols = c / VEC;
+  const int rg = blockDim.x / cols;
+  const int tid = threadIdx.x;
+  const int cc = tid % cols, g = tid / cols;
+  const int m = a.m;
+  const int CS = gridDim.x;
+  const int rank = (int)cs_rank();
+  const int s = blockIdx.y;
+  const int i = a.entry_begin;
+  const int rpr = m / CS;
+  pdl_launch_dependents();
+  pdl_wait();
+  if (qpos && blockIdx.x == 0 && blockIdx.y == 0)
+    for (int x = tid; x < nq; x += blockDim.x) qpos[x] = t;   // query positions of the step
+
+  const InT* Ca = reinterpret_cast<const InT*>(a.C_a) + (size_t)s * a.n * c;
+  const InT* Za = reinterpret_cast<const InT*>(a.Z_a) + (size_t)s * a.n * c;
+  float mx[VEC], sum[VEC], acc[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) { mx[v] = -INFINITY; sum[v] = 0.f; acc[v] = 0.f; }
+  if (g < rg) {
+    for (int q0 = g; q0 < rpr; q0 += rg * kUnroll) {
+      float zv[kUnroll][VEC], cv[kUnroll][VEC], bv[kUnroll][VEC];
+      bool live[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int q = q0 + u * rg;
+        live[u] = q < rpr;
+        if (live[u]) {
+          const int r = rank * rpr + q;             // row inside the block
+          const size_t row = (size_t)m * i + r;
+          load16<InT>(Za + row * c + cc * VEC, zv[u]);
+          load16<InT>(Ca + row * c + cc * VEC, cv[u]);
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) bv[u][v] = __ldg(a.B_a + (size_t)r * c + cc * VEC + v);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        if (!live[u]) continue;
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          const float x = zv[u][v] + bv[u][v];
+          if (x > mx[v]) {
+            const float sc = expf(mx[v] - x);
+            sum[v] = sum[v] * sc + 1.f;
+            acc[v] = acc[v] * sc + cv[u][v];
+            mx[v] = x;
+          } else {
+            const float e = expf(x - mx[v]);
+            sum[v] += e;
+            acc[v] = fmaf(e, cv[u][v], acc[v]);
+          }
+        }
+      }
+    }
+  }
+  // this CTA's partial over its rows: merge the row groups
+  float* s_mx = smem;                 // [rg][c], row group 0 ends up holding the CTA partial
+  float* s_sum = s_mx + rg * c;
+  float* s_acc = s_sum + rg * c;
+  float* s_x = s_acc + rg * c;        // [c]
+  float* s_red = s_x + c;             // [32]
+  float* s_ss = s_red + 32;           // [1] this rank's sum of squares
+  if (g < rg) {
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) {
+      s_mx[g * c + cc * VEC + v] = mx[v];
+      s_sum[g * c + cc * VEC + v] = sum[v];
+      s_acc[g * c + cc * VEC + v] = acc[v];
+    }
+  }
+  __syncthreads();
+  for (int ch = tid; ch < c; ch += blockDim.x) {
+    float M = -INFINITY;
+    for (int q = 0; q < rg; ++q) M = fmaxf(M, s_mx[q * c + ch]);
+    float S = 0.f, A = 0.f;
+    for (int q = 0; q < rg; ++q) {
+      const float mq = s_mx[q * c + ch];
+      if (mq == -INFINITY) continue;
+      const float e = expf(mq - M);
+      S = fmaf(s_sum[q * c + ch], e, S);
+      A = fmaf(s_acc[q * c + ch], e, A);
+    }
+    s_sum[ch] = S;                 // row group 0 slots: the partial of this CTA
+    s_acc[ch] = A;
+    s_mx[ch] = M;
+  }
+  cs_sync();   // every rank's partial is in its shared memory
+  // channels of this rank: combine the ranks' partials
+  const int cpr = c / CS;
+  const int ch0 = rank * cpr;
+  float ss = 0.f;
+  for (int k = tid; k < cpr; k += blockDim.x) {
+    const int ch = ch0 + k;
+    float Mr[16], Sr[16], Ar[16];
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      if (r < CS) {
+        Mr[r] = cs_ld(s_mx + ch, r); Sr[r] = cs_ld(s_sum + ch, r); Ar[r] = cs_ld(s_acc + ch, r);
+        M = fmaxf(M, Mr[r]);
+      }
+    }
+    float S = 0.f, A = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      if (r < CS && Mr[r] != -INFINITY) {
+        const float e = expf(Mr[r] - M);
+        S = fmaf(Sr[r], e, S);
+        A = fmaf(Ar[r], e, A);
+      }
+    }
+    const float x = A / S;
+    s_x[ch] = x;
+    ss = fmaf(x, x, ss);
+  }
+  float inv = 1.f;
+  if (a.apply_norm) {
+    const float part = block_sum(ss, s_red);
+    if (tid == 0) s_ss[0] = part;
+    cs_sync();   // every rank's sum of squares is published
+    float tot = 0.f;
+    for (int r = 0; r < CS; ++r) tot += cs_ld(s_ss, r);
+    inv = 1.f / sqrtf(tot / (float)c + a.eps);
+  } else {
+    __syncthreads();
+  }
+  // RMSNorm + RoPE on this rank's channels (pairs stay inside a rank: cpr is even)
+  const int rope0 = c - a.d_rope;
+  const size_t orow = (size_t)s * a.out_E + i;
+  for (int pj = tid; pj < cpr / 2; pj += blockDim.x) {
+    const int ch = ch0 + 2 * pj;
+    float x0 = s_x[ch] * inv, x1 = s_x[ch + 1] * inv;
+    if (ch >= rope0 && a.d_rope > 0) {
+      const int j = (ch - rope0) / 2;
+      const double freq = j < kMaxRopePairs ? a.inv_freq[j]
+                                            : pow(a.theta, -2.0 * (double)j / (double)a.d_rope);
+      float sn, cs;
+      rope_angle((double)((long long)m * i) * freq, &sn, &cs);
+      const float y0 = x0 * cs - x1 * sn;
+      const float y1 = x0 * sn + x1 * cs;
+      x0 = y0; x1 = y1;
+    }
+    if (a.out_dtype == CSA_F32) {
+      float* o = reinterpret_cast<float*>(a.out) + orow * c;
+      o[ch] = x0; o[ch + 1] = x1;
+    } else {
+      __nv_bfloat16* o = reinterpret_cast<__nv_bfloat16*>(a.out) + orow * c;
+      *reinterpret_cast<__nv_bfloat162*>(o + ch) = __floats2bfloat162_rn(x0, x1);
+    }
+  }
+  cs_sync();   // peers are done reading this CTA's shared memory
+}
+
 void fill_inv_freq(CompressArgs& a) {
   for (int j = 0; j < kMaxRopePairs; ++j)
     a.inv_freq[j] = (a.d_rope > 0 && 2 * j < a.d_rope)
@@ -320,7 +503,51 @@ size_t compress_smem_bytes(const CompressArgs& a, int in_dtype, int nt) {
   return (size_t)(3 * (nt / cols) * a.c + a.c + 32) * sizeof(float);
 }
 
+// Split launch for one long non-overlapped block per sequence (c128a decode).
+csa_status launch_compress_split(CompressArgs& a, int in_dtype, int b, int32_t* qpos, int t,
+                                 cudaStream_t st, bool pdl) {
+  constexpr int CS = 8;
+  const int nt = 256;
+  const int vec = in_dtype == CSA_F32 ? 4 : 8;
+  const int cols = a.c / vec;
+  if (cols > nt || a.m % CS || a.c % (2 * CS) || a.overlap) return CSA_ERR_UNSUPPORTED;
+  if (a.out_dtype != CSA_F32 && a.out_dtype != CSA_BF16) return CSA_ERR_UNSUPPORTED;
+  if ((a.c - a.d_rope) % 2) return CSA_ERR_UNSUPPORTED;
+  fill_inv_freq(a);
+  const int rg = nt / cols;
+  const size_t smem = (size_t)(3 * rg * a.c + a.c + 32 + 4) * sizeof(float);
+  if (smem > 200 * 1024) return CSA_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(CS, b);
+  cfg.blockDim = dim3(nt);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = CS;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl ? 2 : 1;
+  cudaError_t e;
+  if (in_dtype == CSA_F32) {
+    cudaFuncSetAttribute(compress_split_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaLaunchKernelEx(&cfg, compress_split_kernel<float>, a, qpos, b, t);
+  } else {
+    cudaFuncSetAttribute(compress_split_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaLaunchKernelEx(&cfg, compress_split_kernel<__nv_bfloat16>, a, qpos, b, t);
+  }
+  return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+}
+
 csa_status launch_decode_prologue(PrologueArgs& a, int in_dtype, cudaStream_t st) {
+  if (a.nbranch == 1 && a.q_rows == 0 && !a.main.overlap && a.main.m >= 64) {
+    // c128a: the block's rows over a cluster (the query positions come from the caller)
+    const csa_status r = launch_compress_split(a.main, in_dtype, a.b, a.qpos, a.t, st, false);
+    if (r != CSA_ERR_UNSUPPORTED) return r;
+  }
   const int nt = 256;
   const int vec = in_dtype == CSA_F32 ? 4 : 8;
   fill_inv_freq(a.main);
