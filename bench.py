@@ -171,6 +171,17 @@ def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
 # decode
 # ---------------------------------------------------------------------------
 
+# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu captures
+# under profiles/ (ncu_full_csa_decode_64k_fp8_b4.md: the FP8 indexer at batch 4;
+# ncu_full_index_scores_fp4_ctx256k_b2.md: the NVFP4 indexer at 256K context, batch 2),
+# scaled to the bench's launch by the entries processed (the traffic is linear in them).
+# A kernel changed after its capture has no entry here (traffic is then reported as null).
+PROFILED_TRAFFIC = {
+    ("csa_decode_64k_fp8", "index_scores"): 8717056 * (16 * 16384) / (4 * 16384),
+    ("csa_decode_1m_nvfp4", "index_scores"): 9477632 * (4 * 262144) / (2 * 65536),
+}
+
+
 def bench_decode(w, args, world, rank, peaks):
     dev = "cuda"
     stream = torch.cuda.current_stream()
@@ -215,7 +226,7 @@ def bench_decode(w, args, world, rank, peaks):
     return dict(value=value, ms=ms, tokens_per_step=tokens_per_step, clocks=ck, stage=stage,
                 roofline={"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
                           "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                          "traffic": None, "kernel": dom,
+                          "traffic": PROFILED_TRAFFIC.get((w.name, dom)), "kernel": dom,
                           "algorithmic_bytes_per_launch": dom_bytes},
                 step_roofline={"algorithmic_bytes": step_bytes,
                                "achieved_gbs": round(step_bytes / (ms * 1e-3) / 1e9, 1),

@@ -48,6 +48,9 @@ constexpr int kKVBlkBytes = kRows * 128;   // one column block of the KV tile: 1
 constexpr int kQBlkBytes = kH * 128;       // one column block of q: 8 KB
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleThresh = 8.0f;     // log2 units
+constexpr int kSW = 8;                     // gather / softmax warps (two per TMEM lane quarter)
+constexpr int kThreadsA = 32 * kSW + 32;   // plus the MMA warp
+constexpr int kST = 32 * kSW;              // softmax threads
 
 struct AttnTc {
   const __nv_bfloat16* q; const __nv_bfloat16* kv; const int32_t* idx; const int32_t* count;
@@ -92,11 +95,11 @@ __device__ __forceinline__ const __nv_bfloat16* row_src(const AttnTc& p, const Q
 }
 
 // Copy `nrows_blk` rows of 512 bf16 into the swizzled column-block layout.
-// Warp w of the 4 gather warps copies rows w, w+4, ...; two 16-byte chunks per lane per row.
+// Warp w of the kSW gather warps copies rows w, w + kSW, ...; two 16-byte chunks per lane per row.
 template <typename SrcFn>
 __device__ __forceinline__ void gather_rows(uint8_t* dst, int blk_bytes, int nrows_blk, int gw,
                                             int lane, SrcFn src_of, const void* dummy) {
-  for (int r = gw; r < nrows_blk; r += 4) {
+  for (int r = gw; r < nrows_blk; r += kSW) {
     const __nv_bfloat16* src = src_of(r);
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -112,8 +115,8 @@ __device__ __forceinline__ void gather_rows(uint8_t* dst, int blk_bytes, int nro
 // One halving step of the transpose-reduction: lanes with bit `OFF` set keep the
 // upper half of their HALF live values, the others the lower half, and each
 // combines what it keeps with what its partner sends.
-template <bool kMax, int OFF, int HALF>
-__device__ __forceinline__ void xpose_step(float (&v)[64], int lane) {
+template <bool kMax, int OFF, int HALF, int N>
+__device__ __forceinline__ void xpose_step(float (&v)[N], int lane) {
   const bool hi = (lane & OFF) != 0;
 #pragma unroll
   for (int i = 0; i < HALF; ++i) {
@@ -124,15 +127,15 @@ __device__ __forceinline__ void xpose_step(float (&v)[64], int lane) {
   }
 }
 
-// Transpose-reduction of 64 values over the 32 lanes of a warp (62 shuffles):
-// afterwards lane L holds the reduction of heads 2L (v[0]) and 2L+1 (v[1]).
+// Transpose-reduction of 32 values over the 32 lanes of a warp (31 shuffles):
+// afterwards lane L holds the reduction of value L over the warp (v[0]).
 template <bool kMax>
-__device__ __forceinline__ void xpose_reduce64(float (&v)[64], int lane) {
-  xpose_step<kMax, 16, 32>(v, lane);
-  xpose_step<kMax, 8, 16>(v, lane);
-  xpose_step<kMax, 4, 8>(v, lane);
-  xpose_step<kMax, 2, 4>(v, lane);
-  xpose_step<kMax, 1, 2>(v, lane);
+__device__ __forceinline__ void xpose_reduce32(float (&v)[32], int lane) {
+  xpose_step<kMax, 16, 16>(v, lane);
+  xpose_step<kMax, 8, 8>(v, lane);
+  xpose_step<kMax, 4, 4>(v, lane);
+  xpose_step<kMax, 2, 2>(v, lane);
+  xpose_step<kMax, 1, 1>(v, lane);
 }
 
 __device__ __forceinline__ void cluster_sync_all() {
@@ -290,52 +293,47 @@ __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int ite
   const bool got = tc::mbar_wait(bar_r, 0, p.err);
   const float* rml = reinterpret_cast<const float*>(area + kCmRecvML);
   if (tid < kH) {
-    // all maxima and sums of this head first (independent loads), then the weights
+    // maxima first (independent loads, four at a time), then the weights
     const int h = tid;
-    float mj[kMaxSplit], lj[kMaxSplit];
-#pragma unroll
-    for (int j = 0; j < kMaxSplit; ++j) {
-      mj[j] = j < ns ? rml[j * 2 * kH + h] : -INFINITY;
-      lj[j] = j < ns ? rml[j * 2 * kH + kH + h] : 0.f;
-    }
     const float sink2 = s_sink2[h];
     float M = sink2;
-#pragma unroll
-    for (int j = 0; j < kMaxSplit; ++j) M = fmaxf(M, mj[j]);
+#pragma unroll 4
+    for (int j = 0; j < ns; ++j) M = fmaxf(M, rml[j * 2 * kH + h]);
     float den = exp2f(sink2 - M);
-#pragma unroll
-    for (int j = 0; j < kMaxSplit; ++j) {
-      mj[j] = mj[j] == -INFINITY ? 0.f : exp2f(mj[j] - M);
-      den = fmaf(lj[j], mj[j], den);
+#pragma unroll 4
+    for (int j = 0; j < ns; ++j) {
+      const float mj = rml[j * 2 * kH + h];
+      const float e = mj == -INFINITY ? 0.f : exp2f(mj - M);
+      s_mw[j * kH + h] = e;
+      den = fmaf(rml[j * 2 * kH + kH + h], e, den);
     }
     const float inv = 1.f / den;
-#pragma unroll
-    for (int j = 0; j < kMaxSplit; ++j)
-      if (j < ns) s_mw[j * kH + h] = mj[j] * inv;
+#pragma unroll 4
+    for (int j = 0; j < ns; ++j) s_mw[j * kH + h] *= inv;
     if (rank == 0 && p.lse) p.lse[(size_t)qrow * kH + h] = (M + log2f(den)) * 0.6931471805599453f;
   }
   __syncthreads();
   // thread = (chunk of 8 heads, dim); consecutive threads: consecutive dims, so each
   // split is one conflict-free 16-byte shared load per thread and each head's output
-  // run is a coalesced store.  Four splits' loads are in flight at a time.
+  // run is a coalesced store.  Two splits' loads are in flight at a time.
   const __nv_bfloat16* recv = reinterpret_cast<const __nv_bfloat16*>(area + kCmRecvO);
   for (int x = tid; x < dsl * 8; x += blockDim.x) {
     const int c = x / dsl, dd = x - c * dsl;
     const int d = d0 + dd;
     const int off = dd * kH + cm_chunk(d, c) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j0 = 0; j0 < ns; j0 += 4) {
-      uint4 v[4];
-      float4 wa[4], wb[4];
+    for (int j0 = 0; j0 < ns; j0 += 2) {
+      uint4 v[2];
+      float4 wa[2], wb[2];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 2; ++u) {
         const int j = min(j0 + u, ns - 1);
         v[u] = *reinterpret_cast<const uint4*>(recv + (size_t)j * dps * kH + off);
         wa[u] = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c);
         wb[u] = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c + 4);
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 2; ++u) {
         if (j0 + u >= ns) break;
         const float w[8] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w, wb[u].x, wb[u].y, wb[u].z, wb[u].w};
         const uint32_t q[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
@@ -370,7 +368,7 @@ __global__ void __launch_bounds__(128) attn_merge_kernel(AttnTc p) {
               kMaxSplitGlobal, p.q);
 }
 
-__global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
+__global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint8_t* sKV = base;                          // 8 x 16 KB
@@ -409,7 +407,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
   tc::tc_fence_after();
   // the first item's query heads are an input of this call: fetch them before waiting
   // on the preceding kernels (selections, positions and caches come from those)
-  const bool q_pre = (int)blockIdx.x < p.rows_total * p.nsplit && warp < 4;
+  const bool q_pre = (int)blockIdx.x < p.rows_total * p.nsplit && warp < kSW;
   if (q_pre) {
     const __nv_bfloat16* qb = p.q + (size_t)(blockIdx.x / p.nsplit) * kH * kD;
     gather_rows(sQ, kQBlkBytes, kH, warp, lane, [&](int h) { return qb + (size_t)h * kD; }, p.q);
@@ -433,12 +431,12 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
     const int jb = 0;
     const int je = re > rb ? (re - rb + kRows - 1) / kRows : 0;
 
-    if (warp == 4) {
+    if (warp == kSW) {
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t idS = tc::instr_desc(128, kH, 1, 1, 0, 0);   // bf16 K-major x K-major
       constexpr uint32_t idO = tc::instr_desc(128, kH, 1, 1, 1, 1);   // bf16 MN-major x MN-major
       for (int j = jb; j < je; ++j) {
-        tc::named_bar(1, 160);                       // tile (and q) in shared memory
+        tc::named_bar(1, kThreadsA);                 // tile (and q) in shared memory
         if (lane == 0) {
           tc::tc_fence_after();
           for (int kb = 0; kb < 8; ++kb) {
@@ -452,7 +450,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
           tc::mma_commit(bar_s);
         }
         __syncwarp();
-        tc::named_bar(2, 160);                       // P^T in shared memory, O rescaled
+        tc::named_bar(2, kThreadsA);                 // P^T in shared memory, O rescaled
         if (lane == 0) {
           tc::tc_fence_after();
           for (int mb = 0; mb < 4; ++mb) {
@@ -470,9 +468,12 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       }
     } else {
 
-    // ------------------------------------------------------------------ warps 0-3
-    const int r = warp * 32 + lane;                  // this thread's TMEM lane / tile row
-    const uint32_t lane_addr = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------ softmax warps 0..kSW-1
+    // warps w and w + 4 share TMEM lane quarter w % 4 (tile rows); w / 4 picks the
+    // 32 heads (S columns) and the two 128-dim O blocks this thread handles
+    const int qd = warp & 3, hf = warp >> 2;
+    const int r = qd * 32 + lane;                    // this thread's TMEM lane / tile row
+    const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
     if (tid < kH) { s_M[tid] = -INFINITY; s_l[tid] = 0.f; }
     for (int j = jb; j < je; ++j) {
       if (j > jb) {                                  // previous PV done: KV, P and O are free
@@ -486,40 +487,36 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
                     [&](int h) { return qb + (size_t)h * kD; }, p.kv);
       }
       // source of every row of the tile: one coalesced pass over the index list
-      {
+      if (hf == 0) {
         const int pos = rb + j * kRows + r;
         s_rows[r] = pos < re ? row_src(p, Q, qrow, pos) : nullptr;
       }
-      tc::named_bar(3, 128);
+      tc::named_bar(3, kST);
       gather_rows(sKV, kKVBlkBytes, kRows, warp, lane, [&](int rr) { return s_rows[rr]; }, p.kv);
       tc::cp_async_wait_all();
       tc::fence_proxy_async();
       tc::tc_fence_before();
-      tc::named_bar(1, 160);
+      tc::named_bar(1, kThreadsA);
 
-      // logits of row r for all heads
+      // logits of row r for this thread's 32 heads
       ok = ok && tc::mbar_wait(bar_s, ns & 1, p.err);
       ++ns;
       tc::tc_fence_after();
-      uint32_t ra[32], rb[32];
-      tc::tmem_ld32(tS + lane_addr, ra);
-      tc::tmem_ld32(tS + lane_addr + 32, rb);
-      tc::tmem_ld_wait(ra);
-      tc::reg_fence(rb);
+      uint32_t lgb[32];                              // logits (float bits), log2 units
+      tc::tmem_ld32(tS + lane_addr + 32 * hf, lgb);
+      tc::tmem_ld_wait(lgb);
       const bool valid = s_rows[r] != nullptr;
-      float lg[64], v[64];
+      float v[32];
 #pragma unroll
       for (int h = 0; h < 32; ++h) {
-        lg[h] = valid ? __uint_as_float(ra[h]) * p.scale_log2 : -INFINITY;
-        lg[h + 32] = valid ? __uint_as_float(rb[h]) * p.scale_log2 : -INFINITY;
+        const float l = valid ? __uint_as_float(lgb[h]) * p.scale_log2 : -INFINITY;
+        lgb[h] = __float_as_uint(l);
+        v[h] = l;
       }
-#pragma unroll
-      for (int h = 0; h < 64; ++h) v[h] = lg[h];
-      xpose_reduce64<true>(v, lane);
+      xpose_reduce32<true>(v, lane);
       if (tid == 0) s_flag[0] = 0;   // every read of the previous tile's flag is behind two barriers
-      s_red[warp * kH + 2 * lane] = v[0];
-      s_red[warp * kH + 2 * lane + 1] = v[1];
-      tc::named_bar(3, 128);
+      s_red[qd * kH + 32 * hf + lane] = v[0];
+      tc::named_bar(3, kST);
       if (tid < kH) {
         const float tm = fmaxf(fmaxf(s_red[tid], s_red[kH + tid]), fmaxf(s_red[2 * kH + tid], s_red[3 * kH + tid]));
         const float Mr = s_M[tid];
@@ -532,10 +529,10 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         s_M[tid] = Mu;
         if (resc) atomicOr(&s_flag[0], 1);
       }
-      tc::named_bar(3, 128);
+      tc::named_bar(3, kST);
       if (s_flag[0] && j > jb) {
-        // rescale the O^T accumulator: column h of every block times alpha[h]
-        for (int mb = 0; mb < 4; ++mb) {
+        // rescale the O^T accumulator: column h of this thread's two blocks times alpha[h]
+        for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
 #pragma unroll
           for (int half = 0; half < 2; ++half) {
             uint32_t o[32];
@@ -550,15 +547,17 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         }
         tc::tmem_st_wait();
       }
-      // probabilities: bf16 into P^T (row r = one swizzled 128-byte line), then their sums
+      // probabilities: bf16 into P^T (row r = one swizzled 128-byte line, this thread's
+      // four 16-byte chunks), then their sums
 #pragma unroll
-      for (int cblk = 0; cblk < 8; ++cblk) {
+      for (int cb = 0; cb < 4; ++cb) {
+        const int cblk = 4 * hf + cb;
         uint32_t w4[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int h0 = cblk * 8 + 2 * e;
-          const float p0 = exp2f(lg[h0] - s_Mu[h0]);
-          const float p1 = exp2f(lg[h0 + 1] - s_Mu[h0 + 1]);
+          const int h0 = cb * 8 + 2 * e;              // within this thread's 32 heads
+          const float p0 = exp2f(__uint_as_float(lgb[h0]) - s_Mu[32 * hf + h0]);
+          const float p1 = exp2f(__uint_as_float(lgb[h0 + 1]) - s_Mu[32 * hf + h0 + 1]);
           const __nv_bfloat162 pr = __floats2bfloat162_rn(p0, p1);
           w4[e] = *reinterpret_cast<const uint32_t*>(&pr);
           v[h0] = __low2float(pr);
@@ -567,18 +566,17 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
         *reinterpret_cast<uint4*>(sP + r * 128 + ((cblk ^ (r & 7)) << 4)) =
             make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
-      xpose_reduce64<false>(v, lane);
-      tc::named_bar(3, 128);                         // everyone has read s_red (max pass)
-      s_red[warp * kH + 2 * lane] = v[0];
-      s_red[warp * kH + 2 * lane + 1] = v[1];
-      tc::named_bar(3, 128);
+      xpose_reduce32<false>(v, lane);
+      tc::named_bar(3, kST);                         // everyone has read s_red (max pass)
+      s_red[qd * kH + 32 * hf + lane] = v[0];
+      tc::named_bar(3, kST);
       if (tid < kH) {
         const float ts = s_red[tid] + s_red[kH + tid] + s_red[2 * kH + tid] + s_red[3 * kH + tid];
         s_l[tid] = (j == jb ? 0.f : s_l[tid] * s_alpha[tid]) + ts;
       }
       tc::fence_proxy_async();
       tc::tc_fence_before();
-      tc::named_bar(2, 160);
+      tc::named_bar(2, kThreadsA);
     }
 
     if (je <= jb) {
@@ -590,18 +588,18 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       }
       if (p.nsplit > 1 && p.cluster) {
         uint4* z = reinterpret_cast<uint4*>(sKV);
-        for (int x = tid; x < kD * kH * 2 / 16; x += 128) z[x] = make_uint4(0u, 0u, 0u, 0u);
+        for (int x = tid; x < kD * kH * 2 / 16; x += kST) z[x] = make_uint4(0u, 0u, 0u, 0u);
         tc::fence_proxy_async();
       }
     } else {
     ok = ok && tc::mbar_wait(bar_o, no & 1, p.err);
     ++no;
     tc::tc_fence_after();
-    tc::named_bar(3, 128);                           // s_l / s_M final
-    // finalise: thread owns dims d = 128 mb + r of every head
+    tc::named_bar(3, kST);                           // s_l / s_M final
+    // finalise: thread owns dims d = 128 mb + r of every head, mb in {2 hf, 2 hf + 1}
     if (p.nsplit == 1) {
       const float* sk = p.sink;
-      for (int mb = 0; mb < 4; ++mb) {
+      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t o[32];
@@ -623,7 +621,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       }
     } else if (p.cluster) {
       // unnormalised O into shared memory (bf16) for the cluster merge (KV tile area, free now)
-      for (int mb = 0; mb < 4; ++mb) {
+      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t o[32];
@@ -646,7 +644,7 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
       }
       tc::fence_proxy_async();   // the bulk copies read these rows through the async proxy
     } else {
-      for (int mb = 0; mb < 4; ++mb) {
+      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
           uint32_t o[32];
@@ -671,8 +669,8 @@ __global__ void __launch_bounds__(160, 1) attn_tc_kernel(AttnTc p) {
     }
     }
     tc::tc_fence_before();
-    tc::named_bar(3, 128);                           // s_M / s_l reads done before the next item
-    }   // warps 0-3
+    tc::named_bar(3, kST);                           // s_M / s_l reads done before the next item
+    }   // softmax warps
 
     if (p.nsplit > 1 && p.cluster) {
       // every split of this query has its O, max and sum in shared memory: merge one
@@ -723,7 +721,7 @@ int max_active_clusters(int cs) {
                       cudaSuccess)) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs);
-    cfg.blockDim = dim3(160);
+    cfg.blockDim = dim3(kThreadsA);
     cfg.dynamicSmemBytes = kSmemBytes;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -829,7 +827,7 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
   const long long items = (long long)b * a.T * P.nsplit;
   if (!P.cluster) {
     const int grid = (int)std::min<long long>(items, sms);
-    if (csa_launch(attn_tc_kernel, dim3(grid), dim3(160), kSmemBytes, st, a.pdl != 0, p) !=
+    if (csa_launch(attn_tc_kernel, dim3(grid), dim3(kThreadsA), kSmemBytes, st, a.pdl != 0, p) !=
         cudaSuccess)
       return CSA_ERR_CUDA;
     if (P.nsplit > 1) {
@@ -851,7 +849,7 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
     return CSA_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)items);
-  cfg.blockDim = dim3(160);
+  cfg.blockDim = dim3(kThreadsA);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
   cudaLaunchAttribute at[2];
