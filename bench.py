@@ -171,15 +171,21 @@ def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
 # decode
 # ---------------------------------------------------------------------------
 
-# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu captures
-# under profiles/ (ncu_full_csa_decode_64k_fp8_b4.md: the FP8 indexer at batch 4;
-# ncu_full_index_scores_fp4_ctx256k_b2.md: the NVFP4 indexer at 256K context, batch 2),
-# scaled to the bench's launch by the entries processed (the traffic is linear in them).
-# A kernel changed after its capture has no entry here (traffic is then reported as null).
-PROFILED_TRAFFIC = {
-    ("csa_decode_64k_fp8", "index_scores"): 8717056 * (16 * 16384) / (4 * 16384),
-    ("csa_decode_1m_nvfp4", "index_scores"): 9477632 * (4 * 262144) / (2 * 65536),
+# DRAM bytes (read + write) per processed key entry of the dominant kernel, from the ncu
+# captures under profiles/ (ncu_full_csa_decode_64k_fp8_b4.md: the FP8 indexer at batch 4,
+# 16384 entries per sequence; ncu_full_index_scores_fp4_ctx256k_b2.md: the NVFP4 indexer at
+# 256K context, batch 2, 65536 entries per sequence). The traffic is linear in the entries, so
+# one launch's figure is this times b * E of the launch timed. A kernel changed after its
+# capture has no entry here (traffic is then reported as null).
+PROFILED_TRAFFIC_PER_ENTRY = {
+    ("index_scores", "fp8"): 8717056 / (4 * 16384),
+    ("index_scores", "nvfp4"): 9477632 / (2 * 65536),
 }
+
+
+def profiled_traffic(w, kernel):
+    per = PROFILED_TRAFFIC_PER_ENTRY.get((kernel, w.idx_dtype))
+    return None if per is None else round(per * w.b * w.E)
 
 
 def bench_decode(w, args, world, rank, peaks):
@@ -226,7 +232,7 @@ def bench_decode(w, args, world, rank, peaks):
     return dict(value=value, ms=ms, tokens_per_step=tokens_per_step, clocks=ck, stage=stage,
                 roofline={"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
                           "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                          "traffic": PROFILED_TRAFFIC.get((w.name, dom)), "kernel": dom,
+                          "traffic": profiled_traffic(w, dom), "kernel": dom,
                           "algorithmic_bytes_per_launch": dom_bytes},
                 step_roofline={"algorithmic_bytes": step_bytes,
                                "achieved_gbs": round(step_bytes / (ms * 1e-3) / 1e9, 1),
@@ -279,34 +285,45 @@ def stage_times_decode(w, st, steps, flush, stream):
 
 
 def e2e_decode(w, st, steps, flush, stream):
-    """Same step through the public API with host inputs: H2D of the step's new inputs from pinned
-    memory (q, q_I, w and the raw rows of the completing block), decode, D2H of the output."""
+    """Same step through the public API with host inputs: every step copies its new
+    inputs (q, q_I, w and the m raw rows of the completing block of every C / Z
+    tensor) from one pinned host buffer to one device staging buffer (a single H2D
+    copy), places the raw rows into the sequence tensors with device-to-device
+    copies, runs the decode call on the staged q / q_I / w, and reads the output back
+    (one D2H copy)."""
     x = st.x
     t = w.n - 1
     r0 = t - (w.m - 1)
     names = ["C_a", "Z_a", "C_b", "Z_b", "CI_a", "ZI_a", "CI_b", "ZI_b"]
     names = [n for n in names if n in x]
-    host = {n: x[n][:, r0:t + 1].contiguous().cpu().pin_memory() for n in names}
-    hq = x["q"].cpu().pin_memory()
-    hqI = x["q_I"].cpu().pin_memory() if "q_I" in x else None
-    hw = x["w"].cpu().pin_memory() if "w" in x else None
+    parts = [("q", x["q"])]
+    if "q_I" in x:
+        parts += [("q_I", x["q_I"]), ("w", x["w"])]
+    parts += [(n, x[n][:, r0:t + 1]) for n in names]
+    # one staging layout shared by host and device: each part 256-byte aligned
+    offs, off = {}, 0
+    for n, v in parts:
+        offs[n] = off
+        off += (v.numel() * v.element_size() + 255) // 256 * 256
+    hstage = torch.empty(off, dtype=torch.uint8).pin_memory()
+    dstage = torch.empty(off, dtype=torch.uint8, device="cuda")
+
+    def view(buf, n, v):
+        nb = v.numel() * v.element_size()
+        return buf[offs[n]:offs[n] + nb].view(v.dtype).view(v.shape)
+
+    for n, v in parts:
+        view(hstage, n, v).copy_(v.contiguous().cpu())
+    dviews = {n: view(dstage, n, v) for n, v in parts}
     hout = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
-    dq = torch.empty_like(x["q"])
-    dqI = torch.empty_like(x["q_I"]) if hqI is not None else None
-    dw = torch.empty_like(x["w"]) if hw is not None else None
-    h2d = sum(v.numel() * v.element_size() for v in host.values()) + hq.numel() * hq.element_size()
-    if hqI is not None:
-        h2d += hqI.numel() * hqI.element_size() + hw.numel() * hw.element_size()
+    h2d = sum(v.numel() * v.element_size() for _, v in parts)
     d2h = hout.numel() * hout.element_size()
 
     def one():
-        for n, h in host.items():
-            x[n][:, r0:t + 1].copy_(h, non_blocking=True)
-        dq.copy_(hq, non_blocking=True)
-        if hqI is not None:
-            dqI.copy_(hqI, non_blocking=True)
-            dw.copy_(hw, non_blocking=True)
-        st.step(stream, q=dq, q_I=dqI, w_=dw)
+        dstage.copy_(hstage, non_blocking=True)
+        for n in names:
+            x[n][:, r0:t + 1].copy_(dviews[n])
+        st.step(stream, q=dviews["q"], q_I=dviews.get("q_I"), w_=dviews.get("w"))
         hout.copy_(st.out, non_blocking=True)
 
     for _ in range(3):
@@ -314,7 +331,8 @@ def e2e_decode(w, st, steps, flush, stream):
     times = timed_loop(one, steps, flush, stream)
     ms = float(np.mean(times))
     return {"value": w.b / (ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4)}
+            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
+            "copies_per_step": {"h2d": 1, "d2d": len(names), "d2h": 1}}
 
 
 # ---------------------------------------------------------------------------
