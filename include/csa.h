@@ -210,11 +210,15 @@ csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const vo
  * min(E, floor((t+1)/m)); equal scores go to the lower s; if E(t) <= k all
  * visible entries are kept.  idx [b][T][k] lists the kept entries in
  * ascending order, padded with -1; count [b][T] holds how many.  The result
- * is exact (a radix select on the stored score bits).
+ * is exact (a search over the stored score bits; scores must not be NaN).
+ * Few long rows are each spread over a thread-block cluster of up to 16 CTAs
+ * (up to 16 x 16384 entries a row); only rows beyond what a cluster holds
+ * need scratch.
  *   scores  [b][T][E] (CSA_F32 or CSA_BF16)
- *   ws      device scratch of csa_topk_workspace_size() bytes: rows longer than
- *           16384 entries keep a top-k per 16384-entry chunk there first (NULL
- *           with ws_bytes 0 when the size is 0)
+ *   ws      device scratch of csa_topk_workspace_size() bytes: rows too long for
+ *           one cluster keep a top-k per 16384-entry chunk there first (NULL
+ *           with ws_bytes 0 when the size is 0).  The size depends on the
+ *           current device (its SM count) as well as on the shape.
  */
 csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, int m, int b, int T,
                     int E, int k, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,

@@ -18,12 +18,21 @@
 // One packed block scan (keys above tau in the low 16 bits, keys equal to tau in
 // the high 16) writes the selection in ascending entry order.
 //
-// Rows longer than one CTA holds (512 threads x 32) are cut into chunks: every
-// chunk keeps its own top-k (the global top-k is contained in the union, and
-// since chunks are contiguous index ranges the lowest-index rule for ties
-// carries over), and a second pass selects the top-k of the candidates.
+// Few long rows (decode: one query per sequence) spread each row over a thread-block
+// cluster of 2..16 CTAs, each holding a contiguous slice.  Every count of the search
+// is then a cluster sum: each CTA publishes its block total in shared memory, one
+// cluster barrier makes the totals visible, and every warp reads the cluster's totals
+// through distributed shared memory (double-buffered, so one barrier per round).  The
+// final counts of keys above / equal to tau give each CTA its exclusive prefix over
+// the lower ranks, so the selection still comes out in ascending entry order.
+//
+// Rows longer than a cluster holds (16 x 16384) are cut into chunks: every chunk
+// keeps its own top-k (the global top-k is contained in the union, and since chunks
+// are contiguous index ranges the lowest-index rule for ties carries over), and a
+// second pass selects the top-k of the candidates.
 #include "common.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace csa {
 
@@ -32,6 +41,7 @@ namespace {
 constexpr int kEPT = 32;            // entries per thread
 constexpr int kNT = 512;            // threads of the largest CTA
 constexpr int kChunk = kNT * kEPT;  // entries one CTA holds
+constexpr int kMaxClusterRanks = 16;
 
 template <typename S> struct Keys;
 template <> struct Keys<__nv_bfloat16> {
@@ -294,30 +304,420 @@ __global__ void __launch_bounds__(kNT) topk_merge_kernel(
               count + row, nullptr, s_red);
 }
 
+// ---- cluster path -----------------------------------------------------------
+
+__device__ __forceinline__ uint32_t cl_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cl_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cl_arrive() {
+  asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cl_wait() {
+  asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cl_map(const void* local, uint32_t rank) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;"
+               : "=r"(ra) : "r"(tc::smem_u32(local)), "r"(rank));
+  return ra;
+}
+// 16-byte store into another CTA's shared memory, counted on that CTA's mbarrier.
+__device__ __forceinline__ void st_async16(uint32_t raddr, uint4 v, uint32_t rbar) {
+  asm volatile(
+      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
+      ::"r"(raddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w), "r"(rbar) : "memory");
+}
+
+constexpr int kMsgWords = 8;   // one message: 8 words (16 bucket counts of 16 bits)
+
+// Cluster exchange number `ex`: warp 0 of every CTA pushes its message (held by every
+// lane of warp 0) into row `rank` of receive slot (ex & 1) of every CTA of the
+// cluster; every thread then waits, bounded, for its own slot to hold all cs rows.
+// Slot reuse is safe: a CTA sends exchange ex + 2 only after it received exchange
+// ex + 1 from every CTA, and a CTA sends exchange ex + 1 only after a block barrier
+// that follows all of its reads of exchange ex.
+__device__ __forceinline__ bool cl_push(const uint4 (&msg)[2], uint32_t* s_slot, uint64_t* s_bar,
+                                        int ex, uint32_t cs, uint32_t rank, int* err) {
+  const int slot = ex & 1;
+  uint32_t* row = s_slot + (slot * kMaxClusterRanks + rank) * kMsgWords;
+  uint64_t* bar = s_bar + slot;
+  if (threadIdx.x == 0) tc::mbar_arrive_expect_tx(bar, cs * kMsgWords * 4);
+  if (threadIdx.x < cs) {
+    const uint32_t rrow = cl_map(row, threadIdx.x), rbar = cl_map(bar, threadIdx.x);
+    st_async16(rrow, msg[0], rbar);
+    st_async16(rrow + 16, msg[1], rbar);
+  }
+  return tc::mbar_wait(bar, (ex >> 1) & 1, err);
+}
+// Lane l < cs of the calling warp gets row l of receive slot (ex & 1); other lanes zeros.
+__device__ __forceinline__ void cl_row(const uint32_t* s_slot, int ex, uint32_t cs, uint4 (&r)[2]) {
+  const uint32_t lane = threadIdx.x & 31;
+  if (lane < cs) {
+    const uint4* p = reinterpret_cast<const uint4*>(
+        s_slot + ((ex & 1) * kMaxClusterRanks + lane) * kMsgWords);
+    r[0] = p[0];
+    r[1] = p[1];
+  } else {
+    r[0] = r[1] = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// One row over a cluster: CTA `rank` holds entries [rank * per, rank * per + per) of
+// the row's `ev` visible entries, EPT consecutive entries per thread.  The search
+// keeps the invariant of the single-CTA search (at least k keys >= lo, fewer than k
+// keys > hi) but splits [lo, hi] into 16 power-of-two buckets per round: bucket
+// b(key) = min((key - lo) >> s, 15) with 16 << s covering the range, so a round
+// leaves a range of at most 2^s keys and ends on the exact k-th key when s = 0.
+template <typename S, int EPT>
+__global__ void __launch_bounds__(kNT) topk_cluster_kernel(
+    const S* __restrict__ scores, const int32_t* __restrict__ q_pos, int m, int E, int k, int per,
+    int32_t* __restrict__ idx, int32_t* __restrict__ count, int* err) {
+  using K = Keys<S>;
+  using Bits = typename K::Bits;
+  static_assert(EPT % 8 == 0, "keys are counted in groups of 8");
+  __shared__ __align__(16) uint32_t s_part[kNT / 32][kMsgWords];   // warp partial sums
+  __shared__ __align__(16) uint32_t s_slot[2 * kMaxClusterRanks * kMsgWords];
+  __shared__ __align__(8) uint64_t s_bar[2];
+  __shared__ uint32_t s_sc[32];
+  const uint32_t cs = cl_size(), rank = cl_rank();
+  const int tid = threadIdx.x, NT = blockDim.x;
+  const int lane = tid & 31, wid = tid >> 5, nw = NT >> 5;
+  if (tid == 0) {
+    tc::mbar_init(&s_bar[0], 1);
+    tc::mbar_init(&s_bar[1], 1);
+    tc::fence_barrier_init();
+  }
+  cl_arrive();                                   // barriers initialised before any push
+  pdl_launch_dependents();
+  pdl_wait();
+  const int row = blockIdx.x / cs;
+  const int base = (int)rank * per;
+  const Bits* bits = reinterpret_cast<const Bits*>(scores + (size_t)row * E + base);
+  const int nl = max(0, min(E - base, per));     // entries of this slice in the row
+  const int j0 = tid * EPT;
+
+  // keys first (independent of the query position), then the visible count
+  uint32_t key[EPT];
+  const bool vec = ((reinterpret_cast<uintptr_t>(bits + j0) & 15) == 0) && j0 + EPT <= nl;
+  if (vec) {
+    constexpr int kPer = 16 / sizeof(Bits);
+#pragma unroll
+    for (int v = 0; v < EPT / kPer; ++v) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(bits + j0) + v);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if constexpr (sizeof(Bits) == 2) {
+          key[v * kPer + 2 * i] = w[i] & 0xffffu;
+          key[v * kPer + 2 * i + 1] = w[i] >> 16;
+        } else {
+          key[v * kPer + i] = w[i];
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) key[e] = j0 + e < nl ? bits[j0 + e] : 0u;
+  }
+  const int ev = visible_entries(q_pos[row], m, E);
+  const int n = max(0, min(ev - base, per));     // this CTA's visible entries
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) key[e] = j0 + e < n ? K::key(key[e]) : 0u;   // past n: key 0
+
+  int32_t* out = idx + (size_t)row * k;
+  if (ev <= k) {                                 // everything visible is kept
+    for (int j = (int)rank * NT + tid; j < k; j += (int)cs * NT) out[j] = j < ev ? j : -1;
+    if (rank == 0 && tid == 0) count[row] = ev;
+    cl_wait();
+    return;
+  }
+
+  int ex = 0;
+  uint4 msg[2], r[2];
+  // cluster-wide [min, max] of the valid keys
+  {
+    uint32_t kmin = 0xffffffffu, kmax = 0;
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) {
+      const bool v = j0 + e < n;
+      kmin = v ? min(kmin, key[e]) : kmin;
+      kmax = v ? max(kmax, key[e]) : kmax;
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) { s_part[wid][0] = kmin; s_part[wid][1] = kmax; }
+    __syncthreads();
+    if (wid == 0) {
+      const uint32_t a = lane < nw ? s_part[lane][0] : 0xffffffffu;
+      const uint32_t b = lane < nw ? s_part[lane][1] : 0u;
+      msg[0] = make_uint4(__reduce_min_sync(0xffffffffu, a), __reduce_max_sync(0xffffffffu, b), 0u, 0u);
+      msg[1] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    cl_wait();                                   // every CTA's barriers are initialised
+    cl_push(msg, s_slot, s_bar, ex, cs, rank, err);
+    cl_row(s_slot, ex, cs, r);
+    ++ex;
+    const bool in = (uint32_t)lane < cs;
+    kmin = __reduce_min_sync(0xffffffffu, in ? r[0].x : 0xffffffffu);
+    kmax = __reduce_max_sync(0xffffffffu, in ? r[0].y : 0u);
+    kmin = min(kmin, kmax);                      // (only a failed exchange leaves kmin > kmax)
+    msg[0].x = kmin;                             // lo / hi below
+    msg[0].y = kmax;
+  }
+  uint32_t lo = msg[0].x, hi = msg[0].y;
+  int rounds = 0;
+  while (lo < hi && rounds < 8) {                // 8 rounds resolve any 32-bit range
+    ++rounds;
+    const int p = 32 - __clz(hi - lo);           // 2^p > hi - lo
+    const int sh = max(p - 4, 0);
+    // bucket counts: 4-bit fields per group of 8 keys, widened to bytes, then to 16 bits
+    uint32_t ev_lo = 0, od_lo = 0, ev_hi = 0, od_hi = 0;   // byte fields: even / odd buckets
+#pragma unroll
+    for (int g = 0; g < EPT / 8; ++g) {
+      uint32_t a_lo = 0, a_hi = 0;               // buckets 0-7 / 8-15, 4 bits each
+#pragma unroll
+      for (int e = g * 8; e < g * 8 + 8; ++e) {
+        const uint32_t kk = key[e];
+        const uint32_t b = min((kk - lo) >> sh, 15u);
+        const uint32_t t = 1u << ((b & 7u) << 2);
+        const bool v = kk >= lo;
+        a_lo += (v && b < 8u) ? t : 0u;
+        a_hi += (v && b >= 8u) ? t : 0u;
+      }
+      ev_lo += a_lo & 0x0f0f0f0fu;
+      od_lo += (a_lo >> 4) & 0x0f0f0f0fu;
+      ev_hi += a_hi & 0x0f0f0f0fu;
+      od_hi += (a_hi >> 4) & 0x0f0f0f0fu;
+    }
+    // word j holds buckets 2j (low half) and 2j + 1 (high half)
+    uint32_t wv[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      wv[j] = __byte_perm(ev_lo, od_lo, 0x4440u | j | (j << 8) | 0x0) & 0x00ff00ffu;
+      wv[4 + j] = __byte_perm(ev_hi, od_hi, 0x4440u | j | (j << 8)) & 0x00ff00ffu;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wv[j] = __reduce_add_sync(0xffffffffu, wv[j]);
+    if (lane == 0) {
+      *reinterpret_cast<uint4*>(&s_part[wid][0]) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      *reinterpret_cast<uint4*>(&s_part[wid][4]) = make_uint4(wv[4], wv[5], wv[6], wv[7]);
+    }
+    __syncthreads();
+    if (wid == 0) {
+      uint4 a = make_uint4(0u, 0u, 0u, 0u), b = a;
+      for (int w = 0; w < nw; ++w) {
+        const uint4 x = *reinterpret_cast<const uint4*>(&s_part[w][0]);
+        const uint4 y = *reinterpret_cast<const uint4*>(&s_part[w][4]);
+        a.x += x.x; a.y += x.y; a.z += x.z; a.w += x.w;
+        b.x += y.x; b.y += y.y; b.z += y.z; b.w += y.w;
+      }
+      msg[0] = a;
+      msg[1] = b;
+    }
+    cl_push(msg, s_slot, s_bar, ex, cs, rank, err);
+    cl_row(s_slot, ex, cs, r);
+    ++ex;
+    // cluster totals per bucket (16 bits per CTA, summed in 32 bits), then the highest
+    // bucket whose suffix count reaches k
+    const uint32_t rw[8] = {r[0].x, r[0].y, r[0].z, r[0].w, r[1].x, r[1].y, r[1].z, r[1].w};
+    uint32_t suffix = 0;
+    int sel = 0;
+    bool found = false;
+#pragma unroll
+    for (int b = 15; b >= 0; --b) {
+      const uint32_t h = (b & 1) ? (rw[b >> 1] >> 16) : (rw[b >> 1] & 0xffffu);
+      suffix += __reduce_add_sync(0xffffffffu, h);
+      if (!found && suffix >= (uint32_t)k) { sel = b; found = true; }
+    }
+    const uint64_t top = (uint64_t)lo + ((uint64_t)(sel + 1) << sh) - 1;
+    lo = lo + ((uint32_t)sel << sh);
+    hi = (uint32_t)min((uint64_t)hi, top);
+  }
+  const uint32_t tau = lo;
+
+  uint32_t gt_mask = 0, eq_mask = 0;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const bool v = j0 + e < n;
+    gt_mask |= (v && key[e] > tau ? 1u : 0u) << e;
+    eq_mask |= (v && key[e] == tau ? 1u : 0u) << e;
+  }
+  const uint32_t n_gt = __popc(gt_mask), n_eq = __popc(eq_mask);
+  const uint32_t packed = n_gt | (n_eq << 16);
+  // inclusive warp scan of (gt | eq << 16); warp totals to s_sc
+  uint32_t x = packed;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_sc[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t w = lane < nw ? s_sc[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    const uint32_t cta = __shfl_sync(0xffffffffu, w, 31);   // this CTA's (gt | eq << 16)
+    msg[0] = make_uint4(cta, 0u, 0u, 0u);
+    msg[1] = make_uint4(0u, 0u, 0u, 0u);
+    if (lane < nw) s_sc[lane] = w;
+  }
+  cl_push(msg, s_slot, s_bar, ex, cs, rank, err);
+  cl_row(s_slot, ex, cs, r);
+  int need, G, Q;                                // k - keys above tau; lower ranks' gt / eq
+  {
+    const bool lower = (uint32_t)lane < rank;
+    need = k - (int)__reduce_add_sync(0xffffffffu, r[0].x & 0xffffu);
+    G = (int)__reduce_add_sync(0xffffffffu, lower ? (r[0].x & 0xffffu) : 0u);
+    Q = (int)__reduce_add_sync(0xffffffffu, lower ? (r[0].x >> 16) : 0u);
+  }
+  cl_arrive();                                   // no CTA leaves before all pushes landed
+
+  const uint32_t excl = (wid > 0 ? s_sc[wid - 1] : 0u) + x - packed;
+  const int gt_before = G + (int)(excl & 0xffffu);
+  const int eq_before = Q + (int)(excl >> 16);
+  const int take_eq = min(max(need - eq_before, 0), (int)n_eq);
+  uint32_t eq_take = 0, rest = eq_mask;
+  for (int i = 0; i < take_eq; ++i) {
+    const uint32_t low = rest & (0u - rest);
+    eq_take |= low;
+    rest ^= low;
+  }
+  uint32_t sel = gt_mask | eq_take;
+  int pos = gt_before + min(eq_before, need);
+  while (sel) {
+    const int e = __ffs(sel) - 1;
+    sel &= sel - 1;
+    if (pos >= 0 && pos < k) out[pos] = base + j0 + e;
+    ++pos;
+  }
+  if (rank == 0 && tid == 0) count[row] = k;
+  cl_wait();
+}
+
 int threads_for(int n) {
   const int nt = (n + kEPT - 1) / kEPT;
   return nt <= 128 ? 128 : (nt <= 256 ? 256 : 512);
 }
 
+constexpr int kMaxCluster = 16;
+constexpr int kMinPerCta = 2048;   // below this a CTA's rounds cost less than a cluster barrier
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess) return sms;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <typename S, int EPT>
+cudaError_t prep_cluster_kernel(int cs) {
+  if (cs > 8)
+    return cudaFuncSetAttribute(topk_cluster_kernel<S, EPT>,
+                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  return cudaSuccess;
+}
+
+// Whether one cluster of `cs` CTAs of `nt` threads fits the device (cached per device).
+bool cluster_fits(int cs, int nt, bool bf, int ept) {
+  static int cache[16][2][2][kMaxCluster + 1][5] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return false;
+  const int ti = nt <= 32 ? 0 : nt <= 64 ? 1 : nt <= 128 ? 2 : nt <= 256 ? 3 : 4;
+  int& c = cache[dev][bf][ept == 32][cs][ti];
+  if (c) return c > 1;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs);
+  cfg.blockDim = dim3(nt);
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cs;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int n = 0;
+  cudaError_t e;
+  if (bf) {
+    e = ept == 32 ? prep_cluster_kernel<__nv_bfloat16, 32>(cs) : prep_cluster_kernel<__nv_bfloat16, 8>(cs);
+    if (e == cudaSuccess)
+      e = ept == 32 ? cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<__nv_bfloat16, 32>, &cfg)
+                    : cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<__nv_bfloat16, 8>, &cfg);
+  } else {
+    e = ept == 32 ? prep_cluster_kernel<float, 32>(cs) : prep_cluster_kernel<float, 8>(cs);
+    if (e == cudaSuccess)
+      e = ept == 32 ? cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<float, 32>, &cfg)
+                    : cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<float, 8>, &cfg);
+  }
+  if (e != cudaSuccess) { cudaGetLastError(); n = 0; }
+  c = n > 0 ? 2 : 1;
+  return n > 0;
+}
+
+enum TopkMode { kRow, kCluster, kChunked, kNone };
+struct TopkPlan {
+  TopkMode mode;
+  int cs, ept, per, nt;   // cluster path: CTAs per row, entries per thread / per CTA, threads
+};
+
+// Rows of up to kChunk entries with enough rows to fill the device: one CTA each.
+// Fewer, longer rows: a cluster per row, as many CTAs as the device has SMs for (at
+// least ceil(E / kChunk), at most 16, at least kMinPerCta entries each).  Rows beyond
+// a 16-CTA cluster: chunk pass + candidate pass, if the candidates fit one CTA.
+TopkPlan topk_plan(int rows, int E, int k, bool bf) {
+  TopkPlan p{kNone, 1, kEPT, kChunk, kNT};
+  if (k > kChunk) return p;
+  const int sms = sm_count();
+  int need = 1;
+  while (need * kChunk < E) need *= 2;            // CTAs a row needs at the least
+  int cs = 1;
+  while (cs * 2 <= kMaxCluster && (long long)rows * cs * 2 <= sms && (long long)E >= (long long)cs * 2 * kMinPerCta)
+    cs *= 2;
+  cs = max(cs, need);
+  while (cs > 1 && cs <= kMaxCluster) {
+    const int per0 = (E + cs - 1) / cs;
+    const int ept = per0 <= 4096 ? 8 : kEPT;
+    const int per = (per0 + 32 * ept - 1) / (32 * ept) * (32 * ept);
+    const int nt = per / ept;
+    if (cluster_fits(cs, nt, bf, ept)) return TopkPlan{kCluster, cs, ept, per, nt};
+    if (cs / 2 < need) break;
+    cs /= 2;
+  }
+  if (E <= kChunk) { p.mode = kRow; return p; }
+  const int nchunks = (E + kChunk - 1) / kChunk;
+  if ((size_t)nchunks * k <= (size_t)kChunk) p.mode = kChunked;
+  return p;
+}
+
 }  // namespace
 
 size_t topk_workspace_bytes(int rows, int E, int k, int score_dtype) {
-  if (E <= kChunk || k > kChunk) return 0;
+  const bool bf = score_dtype == CSA_BF16;
+  if (topk_plan(rows, E, k, bf).mode != kChunked) return 0;
   const int nchunks = (E + kChunk - 1) / kChunk;
-  if ((size_t)nchunks * k > (size_t)kChunk) return 0;   // candidates must fit one CTA
-  const size_t es = score_dtype == CSA_BF16 ? 2 : 4;
+  const size_t es = bf ? 2 : 4;
   return (size_t)rows * nchunks * k * (es + 4) + 256;
 }
 
-// Rows of up to kChunk entries: one CTA each.  Longer rows: chunk pass + candidate
-// pass (needs ws of topk_workspace_bytes), as long as all candidates fit one CTA.
 csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
                               int rows, int E, int k, int32_t* idx, int32_t* count, void* ws,
                               size_t ws_bytes, cudaStream_t st, bool pdl) {
   if (rows == 0) return CSA_OK;
-  if (k > kChunk) return CSA_ERR_UNSUPPORTED;
   const bool bf = score_dtype == CSA_BF16;
-  if (E <= kChunk) {
+  const TopkPlan pl = topk_plan(rows, E, k, bf);
+  if (pl.mode == kNone) return CSA_ERR_UNSUPPORTED;
+  if (pl.mode == kRow) {
     const int nt = threads_for(E);
     const cudaError_t e =
         bf ? csa_launch(topk_row_kernel<__nv_bfloat16>, dim3(rows), dim3(nt), 0, st, pdl,
@@ -326,8 +726,39 @@ csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t
                         reinterpret_cast<const float*>(scores), q_pos, m, E, k, idx, count);
     return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
   }
+  if (pl.mode == kCluster) {
+    int* err = device_error_word();
+    if (!err) return CSA_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows * pl.cs);
+    cfg.blockDim = dim3(pl.nt);
+    cfg.stream = st;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = pl.cs;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl ? 2 : 1;
+    cudaError_t e;
+    if (bf) {
+      const auto* sc = reinterpret_cast<const __nv_bfloat16*>(scores);
+      e = pl.ept == 32 ? cudaLaunchKernelEx(&cfg, topk_cluster_kernel<__nv_bfloat16, 32>, sc, q_pos, m,
+                                            E, k, pl.per, idx, count, err)
+                       : cudaLaunchKernelEx(&cfg, topk_cluster_kernel<__nv_bfloat16, 8>, sc, q_pos, m,
+                                            E, k, pl.per, idx, count, err);
+    } else {
+      const auto* sc = reinterpret_cast<const float*>(scores);
+      e = pl.ept == 32 ? cudaLaunchKernelEx(&cfg, topk_cluster_kernel<float, 32>, sc, q_pos, m, E, k,
+                                            pl.per, idx, count, err)
+                       : cudaLaunchKernelEx(&cfg, topk_cluster_kernel<float, 8>, sc, q_pos, m, E, k,
+                                            pl.per, idx, count, err);
+    }
+    return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA;
+  }
   const size_t need = topk_workspace_bytes(rows, E, k, score_dtype);
-  if (need == 0) return CSA_ERR_UNSUPPORTED;
   if (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 15)) return CSA_ERR_UNSUPPORTED;
   const int nchunks = (E + kChunk - 1) / kChunk;
   const size_t ncand = (size_t)rows * nchunks * k;

@@ -253,8 +253,7 @@ def test_topk_1m_row():
     idx = torch.empty((1, 1, k), dtype=torch.int32, device=DEV)
     cnt = torch.empty((1, 1), dtype=torch.int32, device=DEV)
     wsb = L.csa_topk_workspace_size(L.CSA_BF16, 1, 1, E, k)
-    assert wsb > 0           # 1M-context rows take the chunked two-pass path
-    ws = torch.empty((wsb,), dtype=torch.uint8, device=DEV)
+    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
     L.csa_topk(st, L.CSA_BF16, qpos, m, 1, 1, E, k, idx, cnt, ws, wsb)
     torch.cuda.synchronize()
     ri, rc = csa.topk(f64(sc)[0], np.array([m * E - 1]), m, k)
@@ -277,6 +276,57 @@ def test_topk_chunked_rows_bit_exact(E, k, ties):
     wsb = L.csa_topk_workspace_size(L.CSA_BF16, b, T, E, k)
     ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
     L.csa_topk(st, L.CSA_BF16, _dev(qpos), m, b, T, E, k, idx, cnt, ws, wsb)
+    torch.cuda.synchronize()
+    stored = f64(st)
+    for s_ in range(b):
+        ri, rc = csa.topk(stored[s_], qpos[s_], m, k)
+        np.testing.assert_array_equal(cnt[s_].cpu().numpy(), rc)
+        np.testing.assert_array_equal(idx[s_].cpu().numpy(), ri)
+
+
+@pytest.mark.parametrize("score", ["bf16", "f32"])
+@pytest.mark.parametrize("E,k,b", [(16384, 512, 16), (262144, 1024, 4), (9000, 512, 3)])
+def test_topk_cluster_rows_bit_exact(score, E, k, b):
+    """Few long rows, each spread over a cluster of CTAs: ties across the CTAs' slice
+    borders go to the lowest entries, and short visible prefixes leave whole CTAs empty."""
+    m = 4
+    rng = np.random.default_rng(E + k + b)
+    sc = rng.normal(size=(b, 1, E))
+    sc[1::2] = np.round(sc[1::2] * 2) / 2                       # heavy ties on odd rows
+    sc[-1, 0, : E // 2] = 0.0                                    # a tied plateau
+    qpos = np.full((b, 1), m * E - 1, dtype=np.int32)
+    qpos[1, 0] = m * (k + 5) - 1                                 # E(t) = k + 5
+    qpos[2 % b, 0] = m * (E // 3) + 2                            # ragged prefix
+    if b > 3:
+        qpos[3, 0] = m * (k - 7)                                 # E(t) < k: all kept
+    tdt = torch.bfloat16 if score == "bf16" else torch.float32
+    st = torch.from_numpy(sc).to(tdt).to(DEV)
+    idx = torch.empty((b, 1, k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((b, 1), dtype=torch.int32, device=DEV)
+    wsb = L.csa_topk_workspace_size(L.DTYPE[score], b, 1, E, k)
+    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    L.csa_topk(st, L.DTYPE[score], _dev(qpos), m, b, 1, E, k, idx, cnt, ws, wsb)
+    torch.cuda.synchronize()
+    stored = f64(st)
+    for s_ in range(b):
+        ri, rc = csa.topk(stored[s_], qpos[s_], m, k)
+        np.testing.assert_array_equal(cnt[s_].cpu().numpy(), rc)
+        np.testing.assert_array_equal(idx[s_].cpu().numpy(), ri)
+
+
+def test_topk_rows_beyond_a_cluster():
+    """Rows longer than 16 x 16384 entries take the chunk pass + candidate pass."""
+    E, k, m, b = 300000, 512, 4, 2
+    rng = np.random.default_rng(7)
+    sc = np.round(rng.normal(size=(b, 1, E)) * 4) / 4
+    qpos = np.array([[m * E - 1], [m * 280001 + 3]], dtype=np.int32)
+    st = torch.from_numpy(sc).to(torch.bfloat16).to(DEV)
+    idx = torch.empty((b, 1, k), dtype=torch.int32, device=DEV)
+    cnt = torch.empty((b, 1), dtype=torch.int32, device=DEV)
+    wsb = L.csa_topk_workspace_size(L.CSA_BF16, b, 1, E, k)
+    assert wsb > 0
+    ws = torch.empty((wsb,), dtype=torch.uint8, device=DEV)
+    L.csa_topk(st, L.CSA_BF16, _dev(qpos), m, b, 1, E, k, idx, cnt, ws, wsb)
     torch.cuda.synchronize()
     stored = f64(st)
     for s_ in range(b):
