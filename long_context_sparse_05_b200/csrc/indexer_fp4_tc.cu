@@ -19,24 +19,34 @@
 // The key cache keeps its scales in exactly that order (tiles of 128 entries, see
 // nvfp4_key_scale_offset), so a stage's scales go from HBM to shared memory in
 // one bulk copy and on to TMEM without any rearrangement.  Query scales arrive
-// row-major and are rearranged once per work unit.
+// row-major and are rearranged once per work unit (tcgen05.cp by the MMA warp).
+// Key scales are written into TMEM by the epilogue warps (tcgen05.st, each warp its
+// lane quarter) rather than by tcgen05.cp: on sm_100a the MMA thread's shared-memory
+// accesses after tcgen05 operations wait for the tensor pipe, so every copy in
+// the MMA thread's stream lengthens each stage, while the epilogue warps have room.
 //
 // Pipeline granularity: a stage is two tiles (256 entries, 16 KB of codes + 2 KB
-// of scales), so the MMA warp pays one stage wait and one accumulator wait per
-// four MMAs; on sm_100a a thread's first shared-memory access after issuing
-// tcgen05 operations costs a few hundred cycles, so per-stage waits are what the
-// issue rate is made of.
+// of scales), so the MMA warp pays one round of barrier waits per four MMAs.
 //
-// CTA (320 threads), one query per work unit (decode):
+// CTA (480 threads), one query per work unit (decode):
 //   warp 0  producer: per stage one 2-D TMA box of 256 key rows and one bulk copy
 //           of the stage's scales; per unit the query codes (TMA), its raw scales
 //           and head weights;
 //   warp 1  query-scale rearrangement (all lanes, once per unit) and MMA issue
-//           (lane 0): 4 tcgen05.cp + 4 MMAs per stage into one of NACC
-//           accumulators of 2 x 64 columns;
-//   warps 2-9 epilogue, two warpgroups taking alternate stages (warps w and w+4
-//           share a TMEM lane quarter): tcgen05.ld, weighted ReLU head sum with the
-//           weights read as broadcast 128-bit shared loads, causal mask, store.
+//           (lane 0): 4 MMAs per stage into one of NACC accumulators of 2 x 64
+//           columns, each with its own 16 key-scale columns.  Per stage it touches
+//           no shared memory: on sm_100a a warp's shared-memory access after its own
+//           tcgen05 operations waits for the tensor pipe, so the stage barriers are
+//           polled by warp 14, which hands each ready stage over at a named barrier
+//           (a barrier reduction also carries a failed wait);
+//   warps 2-13 epilogue, three warpgroups, group g taking the stages s with
+//           s % 3 == g, i.e. accumulator g (one consumer per accumulator barrier):
+//           tcgen05.ld, weighted ReLU head sum with the weights read as broadcast
+//           128-bit shared loads, causal mask, store; then the key scales of the
+//           group's next stage (three ahead, same accumulator) into its scale
+//           columns.  tempty[a] thus means "accumulator a is free and holds the
+//           scales of its next stage"; its phase k belongs to stage a + 3k, and the
+//           scales of stages 0-2 are written up front.
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -59,8 +69,10 @@ constexpr int kPermBytes = 2 * 512;              // query scales in the tcgen05.
 constexpr int NACC = 3;                          // accumulators of kTPS x 64 columns
 constexpr int S = 8;                             // stages
 constexpr int kMaxLocalUnits = 256;
-constexpr int kEpiGroups = 2;
-constexpr int kThreads = 64 + 128 * kEpiGroups;
+constexpr int kEpiGroups = 3;                    // one epilogue warpgroup per accumulator
+constexpr int kThreads = 96 + 128 * kEpiGroups;   // producer, MMA, 12 epilogue, waiter
+constexpr int kWaitWarp = kThreads / 32 - 1;       // warp 14
+static_assert(NACC == kEpiGroups, "each accumulator has its own epilogue warpgroup");
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kAccCols = kTPS * kHeads;     // 128
 constexpr uint32_t kSfaCol = NACC * kAccCols;    // 384: NACC x (kTPS x 8) key-scale columns
@@ -121,6 +133,26 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d, uint64_t a, uint64_t b,
 __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
   asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
                : "memory");
+}
+
+// 16 consecutive 32-bit TMEM columns of this warp's lane quarter from registers.
+// Named-barrier rendezvous of `n` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool bar_red_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r) : "r"(v ? 1u : 0u), "r"(id), "r"(n) : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+        "r"(r[14]), "r"(r[15]) : "memory");
 }
 
 // Untiled bulk copy global -> shared; completion counted on `bar` as transaction bytes.
@@ -260,64 +292,106 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     constexpr uint32_t idesc = idesc_mxf4(kTileE, N);
     uint32_t it = 0, ul = 0;
     bool ok = true;
-    for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
+    // every stage of every unit goes through the rendezvous with the waiter warp, also
+    // after a failure (then nothing is issued), so that neither warp is left waiting
+    for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
       int row, js0, js1, nc;
       unit(u, i, row, js0, js1, nc);
       if (nc == 0) continue;
       const int bb = ul & 1;
       uint8_t* qb = sQ + bb * kQBuf;
-      ok = tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
-      if (!ok) break;
-      rearrange_scales(qb + kQBytes, qb + kQBytes + kQSf, kHeads, lane);
-      tc::fence_proxy_async();
+      if (ok) ok = tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
+      if (ok) {
+        rearrange_scales(qb + kQBytes, qb + kQBytes + kQSf, kHeads, lane);
+        tc::fence_proxy_async();
+      }
       __syncwarp();
-      if (lane == 0) {
-        const uint32_t sfb = tmem_base + kSfbCol + bb * 8;
+      const uint32_t sfb = tmem_base + kSfbCol + bb * 8;
+      if (ok && lane == 0) {
         tc::tc_fence_after();
         tmem_cp_32x128b_x4(sfb, smem_desc_cp(tc::smem_u32(qb + kQBytes + kQSf)));
         tmem_cp_32x128b_x4(sfb + 4, smem_desc_cp(tc::smem_u32(qb + kQBytes + kQSf + 512)));
-        const uint64_t bdesc = smem_desc_sw64(tc::smem_u32(qb), 512);
-        for (int j = 0; j < nc && ok; ++j, ++it) {
-          const int s = it % S;
-          const int acc = it % NACC;
-          uint8_t* st = sStage + s * kStage;
-          // both waits back to back: the first shared-memory access after the previous
-          // stage's tcgen05 operations carries the cost, the second is cheap
-          ok = tc::mbar_wait(&full[s], (it / S) & 1, p.err) &&
-               tc::mbar_wait(&tempty[acc], ((it / NACC) & 1) ^ 1, p.err);
-          if (!ok) break;
-          tc::tc_fence_after();
-          const uint32_t sfa = tmem_base + kSfaCol + acc * (kTPS * 8);
-#pragma unroll
-          for (int t = 0; t < kTPS; ++t) {
-            const uint32_t src = tc::smem_u32(st + kKeyB + t * kSfTileB);
-            tmem_cp_32x128b_x4(sfa + t * 8, smem_desc_cp(src));
-            tmem_cp_32x128b_x4(sfa + t * 8 + 4, smem_desc_cp(src + 512));
-          }
-#pragma unroll
-          for (int t = 0; t < kTPS; ++t) {
-            const uint64_t adesc = smem_desc_sw64(tc::smem_u32(st + t * kTileE * kRowB), 512);
-            const uint32_t d = tmem_base + acc * kAccCols + t * N;
-#pragma unroll
-            for (int kb = 0; kb < 2; ++kb)   // K = 64 elements = 32 bytes per MMA
-              mma_mxf4nvf4(d, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa + t * 8 + 4 * kb,
-                           sfb + 4 * kb, kb > 0);
-          }
-          tc::mma_commit(&empty[s]);
-          tc::mma_commit(&tfull[acc]);
-        }
-        if (ok) tc::mma_commit(&bempty[bb]);
       }
-      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-      it = __shfl_sync(0xffffffffu, it, 0);
+      const uint64_t bdesc = smem_desc_sw64(tc::smem_u32(qb), 512);
+      for (int j = 0; j < nc; ++j, ++it) {
+        // the waiter has seen this stage's accumulator free (with its key scales) and
+        // its key codes landed (bar.red is warp-aligned: the warp reconverges first)
+        __syncwarp();
+        const bool failed = bar_red_or(1, 64, false);
+        ok = ok && !failed;
+        if (!ok || lane != 0) continue;
+        tc::tc_fence_after();
+        const int s = it % S;
+        const int acc = it % NACC;
+        uint8_t* st = sStage + s * kStage;
+        const uint32_t sfa = tmem_base + kSfaCol + acc * (kTPS * 8);
+#pragma unroll
+        for (int t = 0; t < kTPS; ++t) {
+          const uint64_t adesc = smem_desc_sw64(tc::smem_u32(st + t * kTileE * kRowB), 512);
+          const uint32_t d = tmem_base + acc * kAccCols + t * N;
+#pragma unroll
+          for (int kb = 0; kb < 2; ++kb)   // K = 64 elements = 32 bytes per MMA
+            mma_mxf4nvf4(d, adesc + 2 * kb, bdesc + 2 * kb, idesc, sfa + t * 8 + 4 * kb,
+                         sfb + 4 * kb, kb > 0);
+        }
+        tc::mma_commit(&empty[s]);
+        tc::mma_commit(&tfull[acc]);
+      }
+      if (ok && lane == 0) tc::mma_commit(&bempty[bb]);
       ++ul;
+    }
+  } else if (warp == kWaitWarp) {
+    // ------------------------------------------------------------------ stage waiter
+    uint32_t it = 0;
+    bool ok = true;
+    for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
+      int row, js0, js1, nc;
+      unit(u, i, row, js0, js1, nc);
+      for (int j = 0; j < nc; ++j, ++it) {
+        // accumulator free with this stage's key scales in place (phase it / NACC),
+        // and the stage's key codes landed
+        if (ok && lane == 0)
+          ok = tc::mbar_wait(&tempty[it % NACC], (it / NACC) & 1, p.err) &&
+               tc::mbar_wait(&full[it % S], (it / S) & 1, p.err);
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        bar_red_or(1, 64, !ok);
+      }
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    const int grp = (warp - 2) >> 2;         // warpgroup: takes stages with c % 2 == grp
+    const int grp = (warp - 2) >> 2;         // warpgroup: takes stages with c % 3 == grp
     const int lane_base = (warp & 3) * 32;   // TMEM lanes this warp may access
     uint32_t c = 0, ul = 0;                  // computed stages seen, units with work seen
     bool ok = true;
+    uint32_t total_c = 0;                    // stages this CTA computes
+    for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
+      int row, js0, js1, nc;
+      unit(u, i, row, js0, js1, nc);
+      total_c += nc;
+    }
+    // key scales of stage x into the scale columns of accumulator x % NACC (this
+    // warp's lane quarter; the four warps of the group write the same values, the
+    // layout tcgen05.cp 32x128b.warpx4 would produce)
+    auto write_sfa = [&](uint32_t x) -> bool {
+      const int s = x % S;
+      if (!tc::mbar_wait(&full[s], (x / S) & 1, p.err)) return false;
+      const uint8_t* src = sStage + s * kStage + kKeyB + lane * 16;
+      uint32_t v[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {            // q = tile * 2 + K block: 512-byte blocks
+        const uint4 w = *reinterpret_cast<const uint4*>(src + q * 512);
+        v[4 * q] = w.x; v[4 * q + 1] = w.y; v[4 * q + 2] = w.z; v[4 * q + 3] = w.w;
+      }
+      tmem_st16(tmem_base + ((uint32_t)lane_base << 16) + kSfaCol + (x % NACC) * (kTPS * 8), v);
+      tc::tmem_st_wait();
+      return true;
+    };
+    for (uint32_t x = grp; x < (uint32_t)NACC; x += kEpiGroups) {   // phase 0 of tempty[x]
+      if (ok && x < total_c) ok = write_sfa(x);
+      tc::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) tc::mbar_arrive(&tempty[x]);
+    }
     for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
       int row, js0, js1, nc;
       unit(u, i, row, js0, js1, nc);
@@ -333,7 +407,7 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         for (int t = 0; t < kTPS; ++t) sc[t] = -INFINITY;
         if (js < js0 + nc) {
           const uint32_t cc = c++;
-          if ((int)(cc & 1) != grp) continue;           // the other warpgroup's stage
+          if ((int)(cc % kEpiGroups) != grp) continue;  // another warpgroup's stage
           if (ok) {
             const int acc = cc % NACC;
             ok = tc::mbar_wait(&tfull[acc], (cc / NACC) & 1, p.err);
@@ -361,12 +435,13 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
               }
               sc[t] = (a[0] + a[1]) + (a[2] + a[3]);
             }
+            if (ok && cc + NACC < total_c) ok = write_sfa(cc + NACC);
             tc::tc_fence_before();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&tempty[acc]);
           }
-        } else if ((js & 1) != grp) {
-          continue;                                     // fills alternate between the groups
+        } else if (js % kEpiGroups != grp) {
+          continue;                                     // fills rotate over the groups
         }
 #pragma unroll
         for (int t = 0; t < kTPS; ++t) {
