@@ -179,7 +179,7 @@ def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
 # capture has no entry here (traffic is then reported as null).
 PROFILED_TRAFFIC_PER_ENTRY = {
     ("index_scores", "fp8"): 8717056 / (4 * 16384),
-    ("index_scores", "nvfp4"): 9477632 / (2 * 65536),
+    ("index_scores", "nvfp4"): 9491712 / (2 * 65536),
 }
 
 
