@@ -14,23 +14,24 @@
 //   * the MN-major A operand of O^T[d, h] += V^T[d, r] P^T[r, h] (M=4x128 dims, N=64, K=128 rows)
 // so every row is read from memory once.  S^T lands in TMEM with rows on lanes:
 // the per-head max and sum over rows are warp transpose-reductions (62 shuffles
-// for 64 heads) plus a 4-warp combine in shared memory.  P^T is written to
+// for 64 heads) plus a combine in shared memory.  P^T is written to
 // shared memory MN-major (row r's 64 heads are one swizzled 128-byte line).
 // The running max is updated lazily (only when a tile's max exceeds it by 2^8),
 // which rescales the O^T accumulator in TMEM.
 //
 // Work item = (query, split of its rows).  With one split the CTA writes the
-// normalised output (the sink joins the denominator).  With several (decode), the
-// splits of one query form a thread-block cluster: each CTA writes an
-// unnormalised fp32 partial (O, running max, running sum) to the workspace,
-// the cluster synchronises (barrier.cluster, release / acquire), and then every
-// CTA of the cluster merges one slice of the 512 output dims over all splits
-// with the sink (log-sum-exp merge), so no second kernel runs.
+// normalised output (the sink joins the denominator).  With several (CSA decode),
+// the splits of one query form a thread-block cluster: each CTA bulk-stores an
+// unnormalised bf16 record (O, running max, running sum) to the workspace, the
+// cluster synchronises (barrier.cluster, release / acquire), and then every CTA
+// bulk-loads one slice of the 512 output dims from every split and merges it with
+// the sink (log-sum-exp merge), so no second kernel runs.  Dense decode (HCA, tens
+// of splits) writes fp32 partials and a small merge kernel combines them.
 //
-// CTA: warps 0-3 gather, read TMEM and run the softmax (warp w owns TMEM lanes
-// 32w..32w+31); warp 4 lane 0 issues every MMA.  Ordering uses two named
-// barriers (tile ready, P ready) and two mbarriers signalled by tcgen05.commit
-// (S ready, O ready).
+// CTA (288 threads): warps 0-7 gather, read TMEM and run the softmax, two warps per
+// TMEM lane quarter (warp w owns lanes 32 (w % 4).., 32 heads each); warp 8 lane 0
+// issues every MMA.  Ordering uses named barriers (tile ready, P ready) and
+// mbarriers signalled by tcgen05.commit (S ready, O ready).
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -254,10 +255,10 @@ __device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool writ
   }
 }
 
-// Cluster merge of query `qrow` (every thread of the CTA joins).  Each split pushes the
-// rows of its O that another rank merges, plus its running max and sum, into that rank's
-// shared memory with bulk copies; then rank r combines output dims [d0, d1) locally:
-// out = sum_j e^{m_j} O_j / (e^{sink} + sum_j e^{m_j} l_j).
+// Cluster merge of query `qrow` (every thread of the CTA joins).  Each split bulk-stores
+// its record to the workspace; after the cluster barrier rank r bulk-loads, from every
+// split, the rows of output dims [d0, d1) and the running maxima and sums, and combines
+// them: out = sum_j e^{m_j} O_j / (e^{sink} + sum_j e^{m_j} l_j).
 __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int item, int rank,
                                               uint8_t* area, const float* s_M, const float* s_l,
                                               float* s_mw, const float* s_sink2, uint64_t* bar_r,
