@@ -421,6 +421,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   const int items = p.rows_total * p.nsplit;
   uint32_t ns = 0, no = 0;             // commits waited on bar_s / bar_o
   bool ok = true;
+  bool q_ready = false;                // softmax warps: this item's query heads are on their way
 
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
     const int qrow = item / p.nsplit;
@@ -475,6 +476,8 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
     const int qd = warp & 3, hf = warp >> 2;
     const int r = qd * 32 + lane;                    // this thread's TMEM lane / tile row
     const uint32_t lane_addr = (uint32_t)(qd * 32) << 16;
+    const bool have_q = (q_pre && item == (int)blockIdx.x) || q_ready;
+    q_ready = false;
     if (tid < kH) { s_M[tid] = -INFINITY; s_l[tid] = 0.f; }
     for (int j = jb; j < je; ++j) {
       if (j > jb) {                                  // previous PV done: KV, P and O are free
@@ -482,7 +485,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         ++no;
         tc::tc_fence_after();
       }
-      if (j == jb && !(q_pre && item == (int)blockIdx.x)) {
+      if (j == jb && !have_q) {
         const __nv_bfloat16* qb = p.q + (size_t)qrow * kH * kD;
         gather_rows(sQ, kQBlkBytes, kH, warp, lane,
                     [&](int h) { return qb + (size_t)h * kD; }, p.kv);
@@ -503,6 +506,14 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       ok = ok && tc::mbar_wait(bar_s, ns & 1, p.err);
       ++ns;
       tc::tc_fence_after();
+      if (j == je - 1 && p.nsplit == 1 && item + (int)gridDim.x < items) {
+        // the last S^T of this item is done with the query heads: fetch the next
+        // item's now, behind this tile's softmax, PV and the output (one split per
+        // query only: with several, the cluster merge uses this shared memory)
+        const __nv_bfloat16* qn = p.q + (size_t)(item + (int)gridDim.x) * kH * kD;
+        gather_rows(sQ, kQBlkBytes, kH, warp, lane, [&](int h) { return qn + (size_t)h * kD; }, p.q);
+        q_ready = true;
+      }
       uint32_t lgb[32];                              // logits (float bits), log2 units
       tc::tmem_ld32(tS + lane_addr + 32 * hf, lgb);
       tc::tmem_ld_wait(lgb);
@@ -599,7 +610,15 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
     tc::named_bar(3, kST);                           // s_l / s_M final
     // finalise: thread owns dims d = 128 mb + r of every head, mb in {2 hf, 2 hf + 1}
     if (p.nsplit == 1) {
-      const float* sk = p.sink;
+      // one reciprocal denominator per head (the sink joins it), kept where the
+      // per-tile rescale factors were
+      float* s_inv = s_alpha;
+      if (tid < kH) {
+        const float den = s_l[tid] + exp2f(s_sink2[tid] - s_M[tid]);
+        s_inv[tid] = 1.f / den;
+        if (p.lse) p.lse[(size_t)qrow * kH + tid] = (s_M[tid] + log2f(den)) * 0.6931471805599453f;
+      }
+      tc::named_bar(3, kST);
       for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
@@ -610,15 +629,10 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
 #pragma unroll
           for (int h = 0; h < 32; ++h) {
             const int hh = half * 32 + h;
-            const float den = s_l[hh] + exp2f(sk[hh] * kLog2e - s_M[hh]);
-            const float val = ok ? __uint_as_float(o[h]) / den : __int_as_float(0x7fc00000);
+            const float val = ok ? __uint_as_float(o[h]) * s_inv[hh] : __int_as_float(0x7fc00000);
             p.out[((size_t)qrow * kH + hh) * kD + d] = __float2bfloat16_rn(val);
           }
         }
-      }
-      if (p.lse && tid < kH) {
-        const float den = s_l[tid] + exp2f(sk[tid] * kLog2e - s_M[tid]);
-        p.lse[(size_t)qrow * kH + tid] = (s_M[tid] + log2f(den)) * 0.6931471805599453f;
       }
     } else if (p.cluster) {
       // unnormalised O into shared memory (bf16) for the cluster merge (KV tile area, free now)
