@@ -188,6 +188,8 @@ def _dev(a):
 @pytest.mark.parametrize("fmt,H,d,T,E,m,score", [
     ("fp8", 64, 128, 1, 1000, 4, "bf16"),     # decode-like, ragged 128-entry tiles
     ("nvfp4", 64, 128, 1, 1000, 4, "bf16"),
+    ("fp8", 64, 128, 1, 40000, 4, "bf16"),    # long rows: CTAs that take two work units
+    ("nvfp4", 64, 128, 1, 40000, 4, "bf16"),
     ("fp8", 64, 128, 37, 80, 4, "bf16"),      # prefill-like: causal mask across queries
     ("f32", 4, 32, 50, 64, 4, "f32"),         # tiny fp32 configuration
 ])
@@ -205,6 +207,7 @@ def test_index_scores(fmt, H, d, T, E, m, score):
     L.csa_index_scores(p, _dev(x["q"]), _dev(x["qs"]), _dev(x["w"]), _dev(x["k"]), _dev(x["ks"]),
                        _dev(qpos), b, T, E, E, scores)
     torch.cuda.synchronize()
+    assert L.csa_device_error() == 0      # no bounded wait gave up
     g = f64(scores)
     for s in range(b):
         exact = csa.index_scores(x["qd"][s], x["w"][s], x["kd"][s], qpos[s], m, "f64")
