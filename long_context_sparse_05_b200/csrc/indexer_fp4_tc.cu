@@ -15,7 +15,7 @@
 // K-major tiles with 64-byte swizzle (rows of 64 bytes = all 128 elements, two
 // MMAs of 32 bytes each).  Scale factors live in TMEM: for each K block of 64,
 // four columns hold the four UE4M3 scales of rows 0-31, 32-63, 64-95, 96-127,
-// replicated in all four lane quarters, copied there by tcgen05.cp 32x128b.warpx4.
+// replicated in all four lane quarters (the layout tcgen05.cp 32x128b.warpx4 makes).
 // The key cache keeps its scales in exactly that order (tiles of 128 entries, see
 // nvfp4_key_scale_offset), so a stage's scales go from HBM to shared memory in
 // one bulk copy and on to TMEM without any rearrangement.  Query scales arrive
