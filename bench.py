@@ -108,12 +108,16 @@ class ClockSampler:
 
 
 def dist_setup(n_gpus):
+    """One process per GPU: the rank's device is made current before the process group
+    exists, so that NCCL binds to it (its barriers and reductions run there)."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
     if world > 1:
         import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
     return world, rank, local
 
 
@@ -519,7 +523,6 @@ def main():
         return
 
     world, rank, local = dist_setup(args.gpus)
-    torch.cuda.set_device(local)
     L.lib()
     if w.kind == "csa_prefill":
         r = bench_prefill(w, args, world, rank, peaks)
