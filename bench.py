@@ -232,7 +232,7 @@ def bench_decode(w, args, world, rank, peaks):
     achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
     step_bytes = runner.decode_bytes_per_step(w)
 
-    e2e = e2e_decode(w, st, args.steps, flush, stream)
+    e2e = e2e_decode(w, st, args.steps, flush, stream, world)
     return dict(value=value, ms=ms, tokens_per_step=tokens_per_step, clocks=ck, stage=stage,
                 roofline={"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
                           "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
@@ -288,7 +288,7 @@ def stage_times_decode(w, st, steps, flush, stream):
     return {k: float(v) for k, v in res.items()}
 
 
-def e2e_decode(w, st, steps, flush, stream):
+def e2e_decode(w, st, steps, flush, stream, world=1):
     """Same step through the public API with host inputs: every step copies its new
     inputs (q, q_I, w and the m raw rows of the completing block of every C / Z
     tensor) from one pinned host buffer to one device staging buffer (a single H2D
@@ -332,9 +332,11 @@ def e2e_decode(w, st, steps, flush, stream):
 
     for _ in range(3):
         one()
+    torch.cuda.synchronize()
+    barrier(world)
     times = timed_loop(one, steps, flush, stream)
-    ms = float(np.mean(times))
-    return {"value": w.b / (ms * 1e-3), "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
+    ms, _, value = aggregate(float(np.mean(times)), w.b, world)   # whole job, slowest rank
+    return {"value": value, "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
             "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
             "copies_per_step": {"h2d": 1, "d2d": len(names), "d2h": 1}}
 
