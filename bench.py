@@ -294,7 +294,8 @@ def e2e_decode(w, st, steps, flush, stream, world=1):
     tensor) from one pinned host buffer to one device staging buffer (a single H2D
     copy), places the raw rows into the sequence tensors with device-to-device
     copies, runs the decode call on the staged q / q_I / w, and reads the output back
-    (one D2H copy)."""
+    (one D2H copy).  Whole-job throughput: all ranks' tokens over the slowest rank's
+    time."""
     x = st.x
     t = w.n - 1
     r0 = t - (w.m - 1)
