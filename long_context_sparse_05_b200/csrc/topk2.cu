@@ -19,12 +19,14 @@
 // the high 16) writes the selection in ascending entry order.
 //
 // Few long rows (decode: one query per sequence) spread each row over a thread-block
-// cluster of 2..16 CTAs, each holding a contiguous slice.  Every count of the search
-// is then a cluster sum: each CTA publishes its block total in shared memory, one
-// cluster barrier makes the totals visible, and every warp reads the cluster's totals
-// through distributed shared memory (double-buffered, so one barrier per round).  The
-// final counts of keys above / equal to tau give each CTA its exclusive prefix over
-// the lower ranks, so the selection still comes out in ascending entry order.
+// cluster of 2..16 CTAs, each holding a contiguous slice.  The search there splits
+// the candidate range into 16 power-of-two buckets per round (about 3 rounds for a
+// bf16 row), and every count is a cluster sum: warp 0 of each CTA pushes its 16
+// bucket counts into every CTA's shared memory with st.async, counted on the
+// receiver's mbarrier, so a round costs one one-way message instead of a cluster
+// barrier plus remote reads.  The final counts of keys above / equal to tau give
+// each CTA its exclusive prefix over the lower ranks, so the selection still comes
+// out in ascending entry order.
 //
 // Rows longer than a cluster holds (16 x 16384) are cut into chunks: every chunk
 // keeps its own top-k (the global top-k is contained in the union, and since chunks
@@ -41,12 +43,11 @@ namespace {
 constexpr int kEPT = 32;            // entries per thread
 constexpr int kNT = 512;            // threads of the largest CTA
 constexpr int kChunk = kNT * kEPT;  // entries one CTA holds
-constexpr int kMaxClusterRanks = 16;
+constexpr int kMaxClusterRanks = 16;       // CTAs of the largest (non-portable) cluster
 
 template <typename S> struct Keys;
 template <> struct Keys<__nv_bfloat16> {
   using Bits = uint16_t;
-  static constexpr uint32_t kMax = 0xffffu;
   static constexpr Bits kSentinel = 0xffffu;   // pattern whose key is 0: below every score
   __device__ static __forceinline__ uint32_t key(uint32_t u) {
     if ((u & 0x7fffu) == 0) u = 0;   // -0 ties with +0
@@ -55,7 +56,6 @@ template <> struct Keys<__nv_bfloat16> {
 };
 template <> struct Keys<float> {
   using Bits = uint32_t;
-  static constexpr uint32_t kMax = 0xffffffffu;
   static constexpr Bits kSentinel = 0xffffffffu;
   __device__ static __forceinline__ uint32_t key(uint32_t u) {
     if ((u & 0x7fffffffu) == 0) u = 0;
@@ -611,7 +611,6 @@ int threads_for(int n) {
   return nt <= 128 ? 128 : (nt <= 256 ? 256 : 512);
 }
 
-constexpr int kMaxCluster = 16;
 constexpr int kMinPerCta = 2048;   // below this a CTA's rounds cost less than a cluster barrier
 
 int sm_count() {
@@ -631,7 +630,7 @@ cudaError_t prep_cluster_kernel(int cs) {
 
 // Whether one cluster of `cs` CTAs of `nt` threads fits the device (cached per device).
 bool cluster_fits(int cs, int nt, bool bf, int ept) {
-  static int cache[16][2][2][kMaxCluster + 1][5] = {};
+  static int cache[16][2][2][kMaxClusterRanks + 1][5] = {};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16) return false;
   const int ti = nt <= 32 ? 0 : nt <= 64 ? 1 : nt <= 128 ? 2 : nt <= 256 ? 3 : 4;
@@ -682,10 +681,10 @@ TopkPlan topk_plan(int rows, int E, int k, bool bf) {
   int need = 1;
   while (need * kChunk < E) need *= 2;            // CTAs a row needs at the least
   int cs = 1;
-  while (cs * 2 <= kMaxCluster && (long long)rows * cs * 2 <= sms && (long long)E >= (long long)cs * 2 * kMinPerCta)
+  while (cs * 2 <= kMaxClusterRanks && (long long)rows * cs * 2 <= sms && (long long)E >= (long long)cs * 2 * kMinPerCta)
     cs *= 2;
   cs = max(cs, need);
-  while (cs > 1 && cs <= kMaxCluster) {
+  while (cs > 1 && cs <= kMaxClusterRanks) {
     const int per0 = (E + cs - 1) / cs;
     const int ept = per0 <= 4096 ? 8 : kEPT;
     const int per = (per0 + 32 * ept - 1) / (32 * ept) * (32 * ept);
