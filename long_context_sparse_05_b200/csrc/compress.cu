@@ -12,6 +12,8 @@
 // through shared memory.  Every raw row is read exactly once per entry; the
 // overlap of c4a reads C_b/Z_b for the previous block and C_a/Z_a for the
 // current one, which are different tensors, so no row is read twice overall.
+// The HCA decode step's one entry per sequence (128 rows) is too little work for
+// one CTA to finish quickly: compress_split_kernel spreads it over an 8-CTA cluster.
 #include "common.cuh"
 #include "kernels.h"
 
