@@ -1,0 +1,42 @@
+"""Host-side helpers of bench.py that need no GPU: the DRAM traffic scaled from the
+committed small-case captures, and the roofline denominators."""
+
+import os
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from long_context_sparse_05_b200 import workloads  # noqa: E402
+
+
+def test_profiled_traffic_is_linear_in_the_entries_of_the_launch():
+    for w in (workloads.CSA_DECODE_64K, workloads.CSA_DECODE_1M):
+        full = bench.profiled_traffic(w, "index_scores")
+        per = bench.PROFILED_TRAFFIC_PER_ENTRY[("index_scores", w.idx_dtype)]
+        assert full == round(per * w.b * w.E)
+        # a shape override (as --batch / --context give) scales the figure, not reuses it
+        half = workloads.shrink(w, b=w.b // 2)
+        assert abs(bench.profiled_traffic(half, "index_scores") - full / 2) <= 1
+        short = workloads.shrink(w, n=w.n // 4)
+        assert abs(bench.profiled_traffic(short, "index_scores") - full / 4) <= 1
+
+
+def test_profiled_traffic_per_entry_is_close_to_the_algorithmic_bytes():
+    # key bytes per entry: FP8 128 codes + one fp32 scale, NVFP4 64 packed codes + 8 scales;
+    # the captures add the query side and rounding, a few percent at most
+    assert 132.0 <= bench.PROFILED_TRAFFIC_PER_ENTRY[("index_scores", "fp8")] <= 132.0 * 1.05
+    assert 72.0 <= bench.PROFILED_TRAFFIC_PER_ENTRY[("index_scores", "nvfp4")] <= 72.0 * 1.05
+
+
+def test_no_traffic_without_a_capture():
+    assert bench.profiled_traffic(workloads.HCA_DECODE_1M, "sparse_attn") is None
+
+
+def test_peaks_name_their_source():
+    p = bench.load_peaks()
+    assert p["src"] in ("measured", "fallback")
+    assert p["hbm"] > 1000 and p["bf16"] > 100
+    if os.path.exists(os.path.join(ROOT, "MEASURED_PEAKS.json")):
+        assert p["src"] == "measured"
