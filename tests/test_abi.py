@@ -102,6 +102,18 @@ def test_invalid_arguments_rejected_on_host():
     assert lib.csa_sparse_attn(ctypes.byref(ap), fake, fake, 8, fake, fake, fake, 64, fake, fake,
                                1, 1, fake, None, None, 0, None) == 1   # idx given with k = 0
     assert lib.csa_quantize(1, 2, fake, 4, 24, fake, fake, None) == 1  # d not a multiple of 16
+    # NVFP4 index keys keep their scales in 64-element K blocks: widths must be multiples of 64
+    p4 = L.CompressParams(m=4, overlap=1, c=32, d_rope=16, rope_theta=1e4, eps=1e-6,
+                          apply_norm=1, in_dtype=1, out_dtype=L.CSA_NVFP4)
+    assert lib.csa_compress(ctypes.byref(p4), fake, fake, fake, fake, fake, fake, 1, 64, 0, 16,
+                            16, fake, fake, None) == 1
+    ip4 = L.IndexParams(H_I=4, d_I=32, m=4, qk_dtype=L.CSA_NVFP4, score_dtype=L.CSA_BF16)
+    assert lib.csa_index_scores(ctypes.byref(ip4), fake, fake, fake, fake, fake, fake, 1, 1, 8, 8,
+                                fake, None) == 1
+    dp = runner.decode_params(workloads.CSA_DECODE_1M)
+    dp.c_I = 96                                        # the only defect: every pointer is set
+    x = L.DecodeTensors(**{n: fake for n, _ in L.DecodeTensors._fields_})
+    assert L.lib().csa_decode(ctypes.byref(dp), ctypes.byref(x), 1 << 20, 1 << 30, None) == 1
 
 
 def test_workspace_sizes_are_host_only_and_positive():
