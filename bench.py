@@ -470,6 +470,15 @@ def oracle_prefill_rate(w, budget_s=20.0):
 
 
 def host_threads():
+    """Threads the oracle's heavy parts run on: its matrix products go through numpy's
+    BLAS thread pool (the element-wise parts run on one thread)."""
+    try:
+        import threadpoolctl
+        n = [d["num_threads"] for d in threadpoolctl.threadpool_info() if d.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:
+        pass
     try:
         return len(os.sched_getaffinity(0))
     except AttributeError:
