@@ -441,14 +441,15 @@ def oracle_decode_rate(w, budget_s=20.0):
         return csa.attend(g["q"][0], rows, g["sink"], w.scale)
 
     step()
-    n, t0 = 0, time.perf_counter()
+    n, t0, c0 = 0, time.perf_counter(), time.process_time()
     while True:
         step()
         n += 1
         el = time.perf_counter() - t0
         if el > budget_s or n >= w.b:
             break
-    return n / el, "%d decode step(s) of one sequence (context %d), caches prebuilt" % (n, w.n)
+    par = (time.process_time() - c0) / el
+    return n / el, "%d decode step(s) of one sequence (context %d), caches prebuilt" % (n, w.n), par
 
 
 def oracle_prefill_rate(w, budget_s=20.0):
@@ -460,25 +461,17 @@ def oracle_prefill_rate(w, budget_s=20.0):
                  B_b=g["BI_b"])
     rng = np.random.default_rng(0)
     rows = np.sort(rng.choice(w.n, size=min(w.n, 64), replace=False))
-    t0 = time.perf_counter()
+    t0, c0 = time.perf_counter(), time.process_time()
     pipeline.csa_prefill(main, index, g["q"], g["q_I"], g["w"], g["sink"], m=w.m, d_rope=w.d_rope,
                          theta=w.theta, eps=w.eps, k=w.k, n_w=w.n_w, scale=w.scale,
                          kv_dtype=w.dtype, idx_dtype=w.idx_dtype, score_dtype=w.score_dtype,
                          query_rows=rows)
     el = time.perf_counter() - t0
-    return len(rows) / el, "%d of %d query rows (whole compressor included)" % (len(rows), w.n)
+    par = (time.process_time() - c0) / el
+    return len(rows) / el, "%d of %d query rows (whole compressor included)" % (len(rows), w.n), par
 
 
 def host_threads():
-    """Threads the oracle's heavy parts run on: its matrix products go through numpy's
-    BLAS thread pool (the element-wise parts run on one thread)."""
-    try:
-        import threadpoolctl
-        n = [d["num_threads"] for d in threadpoolctl.threadpool_info() if d.get("user_api") == "blas"]
-        if n:
-            return max(n)
-    except Exception:
-        pass
     try:
         return len(os.sched_getaffinity(0))
     except AttributeError:
@@ -486,12 +479,16 @@ def host_threads():
 
 
 def cpu_baseline(w, budget_s=20.0):
+    """The oracle timed on this host.  `cores` is the number of threads it kept busy on
+    average over the timed run (process CPU time / wall time, at least 1): numpy spreads
+    its large contractions over its BLAS threads and runs element-wise work on one."""
     if w.kind == "csa_prefill":
-        v, sample = oracle_prefill_rate(w, budget_s)
+        v, sample, par = oracle_prefill_rate(w, budget_s)
     else:
-        v, sample = oracle_decode_rate(w, budget_s)
-    return {"value": round(v, 3), "unit": "tok/s", "cores": host_threads(), "kind": "oracle",
-            "sample": sample}
+        v, sample, par = oracle_decode_rate(w, budget_s)
+    sample += "; process CPU time / wall time %.1f on a host of %d threads" % (par, host_threads())
+    return {"value": round(v, 3), "unit": "tok/s", "cores": max(1, int(round(par))),
+            "kind": "oracle", "sample": sample}
 
 
 # ---------------------------------------------------------------------------
