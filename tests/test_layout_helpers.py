@@ -2,7 +2,12 @@
 documents for the key cache and the index-key scales), checked against an explicit
 construction of that layout and for being a bijection."""
 
+import os
+import shutil
+import subprocess
+
 import numpy as np
+import pytest
 
 from helpers import nvfp4_key_scale_index, nvfp4_scales_from_tiled, nvfp4_scales_to_tiled
 
@@ -46,3 +51,34 @@ def test_round_trip_with_batch_dims_and_ragged_length():
     tiled = nvfp4_scales_to_tiled(rows, E_cap=1100)
     assert tiled.shape == (3, 1152, 8)
     np.testing.assert_array_equal(nvfp4_scales_from_tiled(tiled, 1000), rows)
+
+
+def test_kernel_layout_function_matches_the_helpers(tmp_path):
+    """The kernels' own offset function (host-callable, in the CUDA sources) against the
+    helper, on a host-only program built with nvcc: no GPU is touched."""
+    nvcc = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
+    if not os.path.exists(nvcc):
+        pytest.skip("nvcc not available")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "layout.cu"
+    src.write_text(
+        '#include <cstdio>\n#include "common.cuh"\n'
+        "int main() {\n"
+        "  const int cs[2] = {64, 128};\n"
+        "  for (int ci = 0; ci < 2; ++ci)\n"
+        "    for (long long e = 0; e < 300; ++e)\n"
+        "      for (int blk = 0; blk < cs[ci] / 16; ++blk)\n"
+        '        std::printf("%zu\\n", csa::nvfp4_key_scale_offset(e, blk, cs[ci]));\n'
+        '  std::printf("%zu %zu\\n", csa::nvfp4_key_scale_seq_bytes(300, 64),\n'
+        "              csa::nvfp4_key_scale_seq_bytes(256, 128));\n"
+        "  return 0;\n}\n")
+    exe = tmp_path / "layout"
+    subprocess.run([nvcc, "-std=c++17", "-I", os.path.join(root, "include"),
+                    "-I", os.path.join(root, "long_context_sparse_05_b200", "csrc"),
+                    str(src), "-o", str(exe)], check=True, capture_output=True, timeout=300)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True,
+                         timeout=60).stdout.split("\n")
+    got = np.array([int(v) for v in out[:-2]])
+    want = np.concatenate([nvfp4_key_scale_index(300, c).reshape(-1) for c in (64, 128)])
+    np.testing.assert_array_equal(got, want)
+    assert out[-2].split() == [str(3 * 128 * 4), str(2 * 128 * 8)]   # ceil(E/128) tiles of 8c bytes
