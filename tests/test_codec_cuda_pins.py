@@ -1,7 +1,8 @@
-"""The oracle's FP8 (E4M3) and FP4 (E2M1) codecs against CUDA's own conversion
-routines (`cuda_fp8.h`, `cuda_fp4.h`, host-callable), called from a host-only
-program built with nvcc: every code value decoded, and encodings of random values,
-every tie between neighbouring codes, and out-of-range values.  No GPU is used."""
+"""The oracle's FP8 (E4M3) and FP4 (E2M1) codecs and its bf16 rounding against CUDA's
+own conversion routines (`cuda_fp8.h`, `cuda_fp4.h`, `cuda_bf16.h`, host-callable),
+called from a host-only program built with nvcc: every code value decoded, and
+encodings of random values, every tie between neighbouring codes, and out-of-range
+values.  No GPU is used."""
 
 import os
 import shutil
@@ -17,6 +18,7 @@ PROGRAM = r"""
 #include <cstdint>
 #include <vector>
 #include <cuda_fp16.h>
+#include <cuda_bf16.h>
 #include <cuda_fp8.h>
 #include <cuda_fp4.h>
 int main(int argc, char** argv) {
@@ -41,6 +43,10 @@ int main(int argc, char** argv) {
   for (float xi : x) {
     const uint8_t c = __nv_cvt_float_to_fp4(xi, __NV_E2M1, cudaRoundNearest);
     std::fwrite(&c, 1, 1, o);
+  }
+  for (float xi : x) {
+    const unsigned short b = __bfloat16_as_ushort(__float2bfloat16_rn(xi));
+    std::fwrite(&b, 2, 1, o);
   }
   std::fclose(o);
   return 0;
@@ -72,6 +78,11 @@ def cuda_codecs(tmp_path_factory):
         _neighbour_ties(e4m3_vals), _neighbour_ties(e2m1_vals),
         [0.0, -0.0, 500.0, -500.0, 1e30, -1e30, 6.5, -6.5, 100.0],
     ]).astype(np.float32)
+    # float32 values at, just below and just above a bf16 rounding tie, all exponents
+    hi = rng.integers(0, 1 << 16, 3000, dtype=np.uint32) << 16
+    hi = hi[((hi >> 23) & 0xFF) != 0xFF]                       # finite only
+    ties = np.concatenate([hi | 0x8000, hi | 0x7FFF, hi | 0x8001]).view(np.float32)
+    x = np.concatenate([x, ties, np.float32([3.3895e38, 3.4e38, -3.4e38, 1e-40, -1e-40])])
     (d / "x.bin").write_bytes(x.tobytes())
     subprocess.run([str(exe), str(d / "x.bin"), str(d / "out.bin")], check=True, timeout=60)
     raw = (d / "out.bin").read_bytes()
@@ -79,7 +90,8 @@ def cuda_codecs(tmp_path_factory):
     dec4 = np.frombuffer(raw[1024:1088], dtype=np.float32)
     enc8 = np.frombuffer(raw[1088:1088 + x.size], dtype=np.uint8)
     enc4 = np.frombuffer(raw[1088 + x.size:1088 + 2 * x.size], dtype=np.uint8)
-    return dict(x=x, dec8=dec8, dec4=dec4, enc8=enc8, enc4=enc4)
+    bf = np.frombuffer(raw[1088 + 2 * x.size:1088 + 4 * x.size], dtype=np.uint16)
+    return dict(x=x, dec8=dec8, dec4=dec4, enc8=enc8, enc4=enc4, bf16=bf)
 
 
 def test_e4m3_decode_every_code(cuda_codecs):
@@ -103,3 +115,9 @@ def test_e4m3_encode_round_to_nearest_even_and_saturation(cuda_codecs):
 def test_e2m1_encode_round_to_nearest_even_and_saturation(cuda_codecs):
     ours = codecs.e2m1_encode(cuda_codecs["x"])
     np.testing.assert_array_equal(ours, cuda_codecs["enc4"])
+
+
+def test_bf16_round_to_nearest_even(cuda_codecs):
+    x = cuda_codecs["x"]
+    ours = codecs.bf16_bits(codecs.round_to_bf16(x.astype(np.float64)))
+    np.testing.assert_array_equal(ours, cuda_codecs["bf16"])
