@@ -20,7 +20,12 @@
  *
  * Conventions for every call:
  *  - Pointers named as tensors are DEVICE pointers, allocated and owned by the
- *    caller; the library allocates nothing and keeps no state between calls.
+ *    caller; no call allocates device memory.  The library keeps a little state
+ *    of its own for the life of the process: one device error word per device
+ *    (csa_device_error), cached device properties (SM count, which cluster
+ *    sizes fit) and the driver's tensor-map entry point, and the fixed scratch
+ *    array of csa_sparse_attn_noalloc.  Nothing of one call's data is kept for
+ *    the next.
  *  - Every call is asynchronous on the caller's stream; results are ready when
  *    the stream reaches them.  No call synchronises the device.
  *  - Layouts are row-major, batch outermost, last dimension contiguous.  Base
@@ -192,6 +197,11 @@ typedef struct {
  *             multiple of 64)
  *   q_pos     [b][T] int32 position t of each query
  *   scores    [b][T][E] (score_dtype), E <= E_cap entries scored per query
+ *
+ * The tensor-core shapes (H_I = 64, d_I = 128, FP8 or NVFP4) read their operands
+ * with TMA: every pointer must be 16-byte aligned and, for FP8, E_cap a multiple
+ * of 4 (whole 16-byte runs of key scales).  Otherwise the call returns
+ * CSA_ERR_INVALID_ARG; it never falls back to a slower kernel for these shapes.
  */
 csa_status csa_index_scores(const csa_index_params* p, const void* q_I, const void* q_scales,
                             const float* w, const void* k_I, const void* k_scales,
@@ -286,7 +296,9 @@ size_t csa_sparse_attn_workspace_size(const csa_attn_params* p, int b, int T, in
  * scratch lives.
  *
  *  - The first call on a device (with that device current) looks up the
- *    array's device address; make that first call before any stream capture.
+ *    array's device address and keeps it for the process; make that first call
+ *    before any stream capture.  The address is not looked up again, so do not
+ *    use this entry point on a device after cudaDeviceReset there.
  *  - A problem whose workspace (csa_sparse_attn_workspace_size) exceeds
  *    CSA_NOALLOC_SCRATCH_BYTES is rejected with CSA_ERR_INVALID_ARG and
  *    nothing is launched.

@@ -477,7 +477,7 @@ csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st
   if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.q) & 15) ||
       (reinterpret_cast<uintptr_t>(a.k_scales) & 15) || (reinterpret_cast<uintptr_t>(a.q_scales) & 15) ||
       (reinterpret_cast<uintptr_t>(a.w) & 15))
-    return CSA_ERR_UNSUPPORTED;
+    return CSA_ERR_INVALID_ARG;   // the TMA copies need 16-byte aligned rows and scale runs
   CUtensorMap tmK, tmQ, tmQS, tmW;
   const uint64_t krows = (uint64_t)b * a.E_cap, qrows = (uint64_t)b * a.T * kHeads;
   if (!make_tmap_2d_u8_swz(&tmK, a.k, kRowB, krows, kRowB, kStageE, 64) ||

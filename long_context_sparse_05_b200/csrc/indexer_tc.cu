@@ -420,7 +420,7 @@ csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st) {
   if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.q) & 15) ||
       (reinterpret_cast<uintptr_t>(a.k_scales) & 15) || (reinterpret_cast<uintptr_t>(a.w) & 15) ||
       (reinterpret_cast<uintptr_t>(a.q_scales) & 15) || (a.E_cap % 4))
-    return CSA_ERR_UNSUPPORTED;   // the TMA copies need 16-byte aligned rows and scale runs
+    return CSA_ERR_INVALID_ARG;   // the TMA copies need 16-byte aligned rows and scale runs
   if (a.T >= 4) return launch_qg<4, 4>(a, b, st);
   return launch_qg<1, 5>(a, b, st);
 }

@@ -71,7 +71,9 @@ class DecodeState:
         self.x = inputs
         self.device = device
         self.E = w.E
-        self.E_cap = w.E
+        # the FP8 tensor-core indexer reads key scales in whole 16-byte runs: rows of a
+        # multiple of 4 entries
+        self.E_cap = w.E if w.kind == "hca_decode" else (w.E + 3) // 4 * 4
         self.p = decode_params(w, self.E_cap)
         dt = _TDT[w.dtype]
         self.kv_cache = torch.zeros((w.b, self.E_cap, w.c), dtype=dt, device=device)

@@ -42,6 +42,14 @@ def test_binding_covers_every_declared_symbol():
     assert set(declared_functions()) <= set(L._SIGS), set(declared_functions()) - set(L._SIGS)
 
 
+def test_noalloc_scratch_size_matches_header():
+    """The binding's copy of the fixed scratch size is the header's (the tests rely on it)."""
+    m = re.search(r"#define\s+CSA_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)",
+                  open(HEADER).read())
+    assert m, "CSA_NOALLOC_SCRATCH_BYTES not found"
+    assert L.NOALLOC_SCRATCH_BYTES == int(m.group(1)) << int(m.group(2))
+
+
 def test_struct_layouts_match_c():
     structs = {"csa_compress_params": L.CompressParams, "csa_index_params": L.IndexParams,
                "csa_attn_params": L.AttnParams, "csa_decode_params": L.DecodeParams,
@@ -110,6 +118,15 @@ def test_invalid_arguments_rejected_on_host():
     ip4 = L.IndexParams(H_I=4, d_I=32, m=4, qk_dtype=L.CSA_NVFP4, score_dtype=L.CSA_BF16)
     assert lib.csa_index_scores(ctypes.byref(ip4), fake, fake, fake, fake, fake, fake, 1, 1, 8, 8,
                                 fake, None) == 1
+    # the tensor-core indexer shapes (64 heads x 128 dims) need 16-byte aligned operands and
+    # FP8 key-scale rows that are whole 16-byte runs: rejected, never run on a slower kernel
+    for fmt in (L.CSA_FP8_E4M3, L.CSA_NVFP4):
+        ipt = L.IndexParams(H_I=64, d_I=128, m=4, qk_dtype=fmt, score_dtype=L.CSA_BF16)
+        assert lib.csa_index_scores(ctypes.byref(ipt), fake, fake, fake, fake + 8, fake, fake, 1,
+                                    1, 1024, 1024, fake, None) == 1
+    ipt = L.IndexParams(H_I=64, d_I=128, m=4, qk_dtype=L.CSA_FP8_E4M3, score_dtype=L.CSA_BF16)
+    assert lib.csa_index_scores(ctypes.byref(ipt), fake, fake, fake, fake, fake, fake, 1, 1, 1026,
+                                1026, fake, None) == 1
     dp = runner.decode_params(workloads.CSA_DECODE_1M)
     dp.c_I = 96                                        # the only defect: every pointer is set
     x = L.DecodeTensors(**{n: fake for n, _ in L.DecodeTensors._fields_})
