@@ -2,14 +2,24 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
-Default workload: CSA decode at 64K context (16 sequences, FP8 indexer,
+Headline workload: CSA decode at 64K context (16 sequences, FP8 indexer,
 top-k 512, window 128, 64 heads x 512).  A step is one fused decode step for
 the whole batch (compress the entry the new token completes, quantise the
 index query, score every entry, select top-k, attend over selection + window)
 with inputs resident in HBM.  L2 is flushed (a 256 MiB write) before every
-timed step, outside the step's CUDA events.  Multi-GPU runs are independent
-replicas (the path has no exchange step): value = all ranks' tokens / max
-over ranks of the device time.
+timed step, outside the step's CUDA events.  The K-step timed region (each
+bracketed by a barrier and a device synchronise) is repeated until the whole
+run spans at least a second, so the clock sampler sees the GPU under load; the
+line reports the repeat count and the median repeat.  Multi-GPU runs are
+independent replicas (the path has no exchange step): value = all ranks'
+tokens / max over ranks of the device time.
+
+Without --workload the same run also measures, as sub-records under "sub",
+the other parts of the metric: CSA decode at 1M context (NVFP4 indexer), HCA
+decode at 1M context and CSA prefill at 32K (FP8 indexer), each with its own
+roofline, per-kernel fractions, clocks and oracle baseline.  The FP8 dense
+tensor-core peak of the prefill roofline is measured in the same run (a plain
+torch._scaled_mm at 8192^3, best of 10).
 
 Prints one JSON line (rank 0).  ``--impl reference`` times the CPU oracle on
 this host's cores on a bounded sample of the same workload instead.
@@ -171,16 +181,36 @@ def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
     return [a.elapsed_time(b) for a, b in evs]
 
 
-# ---------------------------------------------------------------------------
-# decode
-# ---------------------------------------------------------------------------
+def timed_region(fn, steps, flush, stream, world, min_span_s, max_repeats=4000):
+    """The K-step timed loop, each run bracketed by a barrier and a synchronise, repeated until
+    the runs span ``min_span_s`` of wall time.  One calibration run fixes the repeat count
+    (its wall time is maxed over the ranks, so every rank repeats equally often).
+    Returns (mean ms per step of each repeat, host time at start, at end)."""
+    barrier(world)
+    torch.cuda.synchronize()
+    c0 = time.time()
+    timed_loop(fn, steps, flush, stream)
+    c1 = time.time()
+    one = max_over_ranks(c1 - c0, world)
+    reps = int(min(max_repeats, max(1, math.ceil(min_span_s / max(one, 1e-6)))))
+    out = []
+    t0 = time.time()
+    for r in range(reps):
+        barrier(world)
+        torch.cuda.synchronize()
+        times = timed_loop(fn, steps, flush, stream, nvtx="timed_steps" if r == 0 else None)
+        out.append(float(np.mean(times)))
+        barrier(world)
+    t1 = time.time()
+    return out, t0, t1
 
-# DRAM bytes (read + write) per processed key entry of the dominant kernel, from the ncu
-# captures under profiles/ (ncu_full_csa_decode_64k_fp8_b4.md: the FP8 indexer at batch 4,
-# 16384 entries per sequence; ncu_full_index_scores_fp4_ctx256k_b2.md: the NVFP4 indexer at
-# 256K context, batch 2, 65536 entries per sequence). The traffic is linear in the entries, so
-# one launch's figure is this times b * E of the launch timed. A kernel changed after its
-# capture has no entry here (traffic is then reported as null).
+
+# DRAM bytes (read + write) per processed key entry of a kernel, from the ncu captures under
+# profiles/ (ncu_full_csa_decode_64k_fp8_b4.md: the FP8 indexer at batch 4, 16384 entries per
+# sequence; ncu_full_index_scores_fp4_ctx256k_b2.md: the NVFP4 indexer at 256K context, batch
+# 2, 65536 entries per sequence).  The traffic is linear in the entries, so one launch's figure
+# is this times b * E of the launch timed.  A kernel changed after its capture has no entry
+# here (its traffic is then reported as null).
 PROFILED_TRAFFIC_PER_ENTRY = {
     ("index_scores", "fp8"): 8717056 / (4 * 16384),
     ("index_scores", "nvfp4"): 9491712 / (2 * 65536),
@@ -192,7 +222,35 @@ def profiled_traffic(w, kernel):
     return None if per is None else round(per * w.b * w.E)
 
 
-def bench_decode(w, args, world, rank, peaks):
+def kernel_record(us, amount, peak, unit="GB/s", bound="hbm"):
+    """Achieved rate of one kernel (algorithmic bytes or FLOPs per launch / its event time)."""
+    scale = 1e9 if unit == "GB/s" else 1e12
+    rate = amount / (us * 1e-6) / scale
+    return {"us": round(us, 2), "bound": bound, "work": int(amount), "achieved": round(rate, 1),
+            "unit": unit, "peak": peak, "frac": round(rate / peak, 4)}
+
+
+def decode_stage_bytes(w):
+    """Algorithmic bytes of each decode stage call, every input read and output written once
+    (b sequences).  compress: the raw C and Z rows of the completing block (and of the previous
+    block for c4a) plus the entry; quantize: q_I in, codes and scales out; index_scores: every
+    key row with its scale, the query codes, scales and weights, the scores out; topk: the
+    scores in, the selection out; sparse_attn: the selected and window rows, q in, out."""
+    eb = 2 if w.dtype == "bf16" else 4
+    rows_in = (4 if w.overlap else 2) * w.m
+    d = {"compress": w.b * (rows_in * w.c * eb + w.c * eb)}
+    if w.kind != "hca_decode":
+        krow = {"fp8": w.c_I + 4, "nvfp4": w.c_I // 2 + w.c_I // 16, "f32": 4 * w.c_I}[w.idx_dtype]
+        d["quantize"] = w.b * w.H_I * (w.c_I * eb + krow)
+        d["index_scores"] = w.b * w.E * krow + w.b * w.H_I * (krow + 4) + w.b * w.E * 2
+        d["topk"] = w.b * w.E * 2 + w.b * (w.k + 1) * 4
+        d["sparse_attn"] = w.b * ((w.k + w.n_w) * w.c * eb + 2 * w.H * w.c * eb + w.k * 4)
+    else:
+        d["sparse_attn"] = w.b * ((w.E + w.n_w) * w.c * eb + 2 * w.H * w.c * eb)
+    return d
+
+
+def bench_decode(w, args, world, rank, peaks, min_span_s):
     dev = "cuda"
     stream = torch.cuda.current_stream()
     clocks = ClockSampler(torch.cuda.current_device())
@@ -209,43 +267,36 @@ def bench_decode(w, args, world, rank, peaks):
         step()
     torch.cuda.synchronize()
 
-    barrier(world)
-    torch.cuda.synchronize()
-    t0 = time.time()
-    times = timed_loop(step, args.steps, flush, stream, nvtx="timed_steps")
-    torch.cuda.synchronize()
-    t1 = time.time()
-    barrier(world)
+    reps, t0, t1 = timed_region(step, args.steps, flush, stream, world, min_span_s)
     ck = clocks.stop(t0, t1)
-    ms, tokens_per_step, value = aggregate(float(np.mean(times)), w.b, world)
+    ck["repeats"] = len(reps)
+    ms, tokens_per_step, value = aggregate(float(np.median(reps)), w.b, world)
 
-    # dominant kernel: the indexer over all E entries (same call the step makes)
+    # every stage call of the step timed alone; the longest one is the roofline kernel
     stage = stage_times_decode(w, st, args.steps, flush, stream)
-    idx_bytes = w.b * w.E * {"fp8": w.c_I + 4, "nvfp4": w.c_I // 2 + w.c_I // 16}.get(
-        w.idx_dtype, w.c * 2)
-    dom = "index_scores" if w.kind != "hca_decode" else "sparse_attn"
-    if w.kind == "hca_decode":
-        dom_bytes = w.b * (w.E + w.n_w) * w.c * 2 + 2 * w.b * w.H * w.c * 2
-    else:
-        dom_bytes = idx_bytes + w.b * w.H_I * (w.c_I + 4 + 4)
-    dom_ms = stage[dom]
-    achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+    sbytes = decode_stage_bytes(w)
+    kernels = {k: kernel_record(stage[k] * 1e3, sbytes[k], peaks["hbm"]) for k in stage}
+    dom = max(kernels, key=lambda k: kernels[k]["us"])
+    roof = dict(kernels[dom])
+    roof.pop("us")
+    roof["kernel"] = dom
+    roof["traffic"] = profiled_traffic(w, dom)
     step_bytes = runner.decode_bytes_per_step(w)
 
     e2e = e2e_decode(w, st, args.steps, flush, stream, world)
+    del st, inp, flush
+    torch.cuda.empty_cache()
     return dict(value=value, ms=ms, tokens_per_step=tokens_per_step, clocks=ck, stage=stage,
-                roofline={"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm"],
-                          "unit": "GB/s", "frac": round(achieved / peaks["hbm"], 4),
-                          "traffic": profiled_traffic(w, dom), "kernel": dom,
-                          "algorithmic_bytes_per_launch": dom_bytes},
+                roofline=roof, kernels=kernels,
                 step_roofline={"algorithmic_bytes": step_bytes,
                                "achieved_gbs": round(step_bytes / (ms * 1e-3) / 1e9, 1),
                                "frac": round(step_bytes / (ms * 1e-3) / 1e9 / peaks["hbm"], 4)},
-                e2e=e2e, launches=runner.decode_launches_per_step(w) * args.steps)
+                e2e=e2e, launches=runner.decode_launches_per_step(w) * args.steps * len(reps),
+                repeats=len(reps))
 
 
 def stage_times_decode(w, st, steps, flush, stream):
-    """Mean µs of each stage call of the decode step, each timed alone with events."""
+    """Mean ms of each stage call of the decode step, each timed alone with events."""
     x = st.x
     E = w.E
     t = w.n - 1
@@ -346,7 +397,79 @@ def e2e_decode(w, st, steps, flush, stream, world=1):
 # prefill
 # ---------------------------------------------------------------------------
 
-def bench_prefill(w, args, world, rank, peaks):
+def measure_tc_peaks(peaks):
+    """Dense FP8 tensor-core peak of this GPU, measured here: torch._scaled_mm (a plain library
+    GEMM) of two 8192 x 8192 E4M3 matrices into bf16, best of 10 after warm-up, 2 N^3 FLOPs.
+    Falls back to twice the bf16 peak (the nominal ratio) when the call is not available."""
+    n = 8192
+    try:
+        a = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn)
+        b = torch.randn(n, n, device="cuda").to(torch.float8_e4m3fn).t()
+        one = torch.ones((), device="cuda")
+        f = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)  # noqa: E731
+        for _ in range(5):
+            f()
+        torch.cuda.synchronize()
+        best = float("inf")
+        for _ in range(10):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            f()
+            e1.record()
+            torch.cuda.synchronize()
+            best = min(best, e0.elapsed_time(e1))
+        fp8 = 2.0 * n ** 3 / (best * 1e-3) / 1e12
+        del a, b
+        torch.cuda.empty_cache()
+        return {"fp8_tflops": round(fp8, 1), "fp8_src": "measured: torch._scaled_mm e4m3 8192^3, best of 10"}
+    except Exception as e:   # noqa: BLE001
+        return {"fp8_tflops": 2.0 * peaks["bf16"],
+                "fp8_src": "2 x bf16 (nominal ratio): _scaled_mm unavailable (%s)" % type(e).__name__}
+
+
+def stage_times_prefill(w, st, steps, flush, stream):
+    """Mean ms of each stage call of the prefill, each timed alone with events."""
+    x = st.x
+    E = w.E
+    res = {}
+    cp = runner.compress_params(w, "main")
+    ci = runner.compress_params(w, "index")
+    res["compress"] = np.mean(timed_loop(lambda: (
+        L.csa_compress(cp, x["C_a"], x["Z_a"], x["B_a"], x["C_b"], x["Z_b"], x["B_b"], w.b, w.n, 0,
+                       E, E, st.kv_cache, None, stream),
+        L.csa_compress(ci, x["CI_a"], x["ZI_a"], x["BI_a"], x["CI_b"], x["ZI_b"], x["BI_b"], w.b,
+                       w.n, 0, E, E, st.kI_cache, st.kI_scales, stream)), steps, flush, stream,
+        warm=2))
+    rows = w.b * w.n
+    codes = torch.empty((rows * w.H_I, runner.row_bytes(w.idx_dtype, w.c_I)), dtype=torch.uint8,
+                        device="cuda")
+    qs = torch.empty((rows * w.H_I,), dtype=torch.float32, device="cuda")
+    res["quantize"] = np.mean(timed_loop(lambda: L.csa_quantize(
+        L.DTYPE[w.dtype], L.DTYPE[w.idx_dtype], x["q_I"], rows * w.H_I, w.c_I, codes, qs, stream),
+        steps, flush, stream, warm=2))
+    qpos = torch.arange(w.n, dtype=torch.int32, device="cuda").repeat(w.b, 1).contiguous()
+    scores = torch.empty((w.b, w.n, E), dtype=torch.bfloat16, device="cuda")
+    ip = L.IndexParams(H_I=w.H_I, d_I=w.c_I, m=w.m, qk_dtype=L.DTYPE[w.idx_dtype],
+                       score_dtype=L.CSA_BF16)
+    res["index_scores"] = np.mean(timed_loop(lambda: L.csa_index_scores(
+        ip, codes, qs, x["w"], st.kI_cache, st.kI_scales, qpos, w.b, w.n, E, E, scores, stream),
+        steps, flush, stream, warm=2))
+    tkb = L.csa_topk_workspace_size(L.CSA_BF16, w.b, w.n, E, w.k)
+    tkws = torch.empty((max(tkb, 256),), dtype=torch.uint8, device="cuda")
+    res["topk"] = np.mean(timed_loop(lambda: L.csa_topk(
+        scores, L.CSA_BF16, qpos, w.m, w.b, w.n, E, w.k, st.idx, st.count, tkws, tkb, stream),
+        steps, flush, stream, warm=2))
+    del scores
+    ap = L.AttnParams(H=w.H, d=w.c, n_w=w.n_w, scale=w.scale, m=w.m, k=w.k, dtype=L.DTYPE[w.dtype])
+    wsb = L.csa_sparse_attn_workspace_size(ap, w.b, w.n, E)
+    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device="cuda")
+    res["sparse_attn"] = np.mean(timed_loop(lambda: L.csa_sparse_attn(
+        ap, x["q"], st.kv_cache, E, st.idx, st.count, x["C_a"], w.n, qpos, x["sink"], w.b, w.n,
+        st.out, None, ws, wsb, stream), steps, flush, stream, warm=2))
+    return {k: float(v) for k, v in res.items()}
+
+
+def bench_prefill(w, args, world, rank, peaks, min_span_s):
     stream = torch.cuda.current_stream()
     inp = synth.make_inputs(w, device="cuda")
     st = runner.PrefillState(w, inp)
@@ -356,29 +479,68 @@ def bench_prefill(w, args, world, rank, peaks):
     for _ in range(args.warmup):
         st.run(stream)
     torch.cuda.synchronize()
-    barrier(world)
-    t0 = time.time()
-    times = timed_loop(lambda: st.run(stream), args.steps, flush, stream, nvtx="timed_steps")
-    t1 = time.time()
-    barrier(world)
+    reps, t0, t1 = timed_region(lambda: st.run(stream), args.steps, flush, stream, world,
+                                min_span_s)
     ck = clocks.stop(t0, t1)
-    ms, tokens, value = aggregate(float(np.mean(times)), w.b * w.n, world)
+    ck["repeats"] = len(reps)
+    ms, tokens, value = aggregate(float(np.median(reps)), w.b * w.n, world)
     f_idx, f_attn = runner.prefill_flops(w)
-    p_fp8 = 2 * peaks["bf16"]
-    t_ideal = f_idx / (p_fp8 * 1e12) + f_attn / (peaks["bf16"] * 1e12)
-    frac = t_ideal / (ms * 1e-3)
-    return dict(value=value, ms=ms, tokens_per_step=tokens, clocks=ck, stage={},
-                roofline={"bound": "tensor", "achieved": round(
-                    (f_idx + f_attn) / (ms * 1e-3) / 1e12, 2), "peak": peaks["bf16"],
-                    "unit": "TFLOP/s", "frac": round(frac, 4), "traffic": None,
-                    "kernel": "whole prefill (dtype-weighted)",
-                    "flops_index_fp8": f_idx, "flops_attn_bf16": f_attn},
-                e2e=None, launches=runner.prefill_launches(w) * args.steps)
+    p_fp8, p_bf16 = peaks["fp8"], peaks["bf16"]
+    # dtype-weighted: FP8 FLOPs count at the bf16 / FP8 peak ratio, so that achieved / peak is
+    # the ideal time at each dtype's peak over the measured time
+    t_ideal = f_idx / (p_fp8 * 1e12) + f_attn / (p_bf16 * 1e12)
+    weighted = (f_idx * p_bf16 / p_fp8 + f_attn) / (ms * 1e-3) / 1e12
+    stage = stage_times_prefill(w, st, max(2, min(args.steps, 5)), flush, stream)
+    eb = 2 if w.dtype == "bf16" else 4
+    E = w.E
+    cbytes = w.b * (4 * w.n * (w.c + w.c_I) * eb + E * w.c * eb + E * (w.c_I + 4))
+    qbytes = w.b * w.n * w.H_I * (w.c_I * eb + w.c_I + 4)
+    tbytes = w.b * w.n * (E * 2 + (w.k + 1) * 4)
+    kernels = {
+        "compress": kernel_record(stage["compress"] * 1e3, cbytes, peaks["hbm"]),
+        "quantize": kernel_record(stage["quantize"] * 1e3, qbytes, peaks["hbm"]),
+        "index_scores": kernel_record(stage["index_scores"] * 1e3, f_idx, p_fp8, "TFLOP/s",
+                                      "tensor"),
+        "topk": kernel_record(stage["topk"] * 1e3, tbytes, peaks["hbm"]),
+        "sparse_attn": kernel_record(stage["sparse_attn"] * 1e3, f_attn, p_bf16, "TFLOP/s",
+                                     "tensor"),
+    }
+    del st, inp, flush
+    torch.cuda.empty_cache()
+    return dict(value=value, ms=ms, tokens_per_step=tokens, clocks=ck, stage=stage,
+                roofline={"bound": "tensor", "achieved": round(weighted, 1), "peak": p_bf16,
+                          "unit": "TFLOP/s", "frac": round(t_ideal / (ms * 1e-3), 4),
+                          "traffic": None,
+                          "kernel": "index_scores + sparse_attn (dtype-weighted, whole prefill)",
+                          "achieved_raw_tflops": round((f_idx + f_attn) / (ms * 1e-3) / 1e12, 1),
+                          "flops_index_fp8": f_idx, "flops_attn_bf16": f_attn,
+                          "peak_fp8": p_fp8, "frac_vs_sustained_bf16":
+                          round((f_idx / (p_fp8 * peaks["bf16_sus"] / p_bf16) +
+                                 f_attn / peaks["bf16_sus"]) / 1e12 / (ms * 1e-3), 4)},
+                kernels=kernels, e2e=None,
+                launches=runner.prefill_launches(w) * args.steps * len(reps), repeats=len(reps))
 
 
 # ---------------------------------------------------------------------------
 # reference arm / cpu baseline: the CPU oracle on a bounded sample
 # ---------------------------------------------------------------------------
+
+class HostRows:
+    """Row access to one sequence of a host tensor, converted to float64 only for the rows
+    indexed (so the oracle can walk 1M-token inputs without a float64 copy of them)."""
+
+    def __init__(self, t):
+        self.t = t
+        self.shape = tuple(t.shape)
+
+    def __getitem__(self, key):
+        if isinstance(key, np.ndarray):
+            key = torch.from_numpy(np.asarray(key, dtype=np.int64))
+        return self.t[key].double().numpy()
+
+    def __len__(self):
+        return self.shape[0]
+
 
 def oracle_decode_rate(w, budget_s=20.0):
     """tok/s of the oracle's decode step on this host's cores, on sampled sequences.
@@ -387,29 +549,31 @@ def oracle_decode_rate(w, budget_s=20.0):
     timed step compresses the new entry, quantises q_I, scores every entry,
     selects top-k and attends over the selection and the window.
     """
-    from oracle import codecs, csa, pipeline
+    from oracle import csa, pipeline
 
     inp = synth.make_inputs(workloads.shrink(w, b=1), device="cpu")
-    g = {k: (v[0] if v.dim() >= 3 else v).double().numpy() for k, v in inp.items()}
+    g = {k: (HostRows(v[0]) if v.dim() >= 3 else v.double().numpy()) for k, v in inp.items()}
     t = w.n - 1
     E = w.E
     main = dict(C_a=g["C_a"], Z_a=g["Z_a"], B_a=g["B_a"], C_b=g.get("C_b"), Z_b=g.get("Z_b"),
                 B_b=g.get("B_b"))
     hca = w.kind == "hca_decode"
+    q = g["q"][0]
     if not hca:
         index = dict(C_a=g["CI_a"], Z_a=g["ZI_a"], B_a=g["BI_a"], C_b=g["CI_b"], Z_b=g["ZI_b"],
                      B_b=g["BI_b"])
+        qI, wI = g["q_I"][0], g["w"][0]
         kI = csa.compress_range(index["C_a"], index["Z_a"], index["B_a"], index["C_b"],
                                 index["Z_b"], index["B_b"], w.m, True, 0, E - 1, w.d_rope_I,
-                                w.theta, w.eps, chunk_rows=1 << 14)
+                                w.theta, w.eps, chunk_rows=1 << 16)
         kI_deq, _ = pipeline.quantize_rows(kI, w.idx_dtype)
         # the latent cache is state: only the rows a step can gather are filled in
         nk = csa.compress_entries(index["C_a"], index["Z_a"], index["B_a"], index["C_b"],
                                   index["Z_b"], index["B_b"], w.m, True, [E - 1], w.d_rope_I,
                                   w.theta, w.eps)
-        qd, _ = pipeline.quantize_rows(g["q_I"][0][None], w.idx_dtype)
+        qd, _ = pipeline.quantize_rows(qI[None], w.idx_dtype)
         kd = np.concatenate([kI_deq, pipeline.quantize_rows(nk, w.idx_dtype)[0]])
-        sc = csa.index_scores(qd, g["w"][0][None], kd, np.array([t]), w.m, "bf16")
+        sc = csa.index_scores(qd, wI[None], kd, np.array([t]), w.m, "bf16")
         sel0 = csa.topk(sc, np.array([t]), w.m, w.k)[0][0]
         sel0 = sel0[(sel0 >= 0) & (sel0 < E - 1)]
         kv_cache = np.zeros((E - 1, w.c))
@@ -419,26 +583,27 @@ def oracle_decode_rate(w, budget_s=20.0):
     else:
         kv_cache = csa.compress_range(main["C_a"], main["Z_a"], main["B_a"], None, None, None,
                                       w.m, False, 0, E - 1, w.d_rope, w.theta, w.eps,
-                                      chunk_rows=1 << 14)
+                                      chunk_rows=1 << 16)
+    win = g["C_a"][csa.window_rows(t, w.n_w)]
 
     def step():
         new = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
                                    main["B_b"], w.m, not hca, [E - 1], w.d_rope, w.theta, w.eps)
         kv = np.concatenate([kv_cache, pipeline.round_out(new, w.dtype)])
         if hca:
-            rows = np.concatenate([kv, g["C_a"][csa.window_rows(t, w.n_w)]])
+            rows = np.concatenate([kv, win])
         else:
             nk = csa.compress_entries(index["C_a"], index["Z_a"], index["B_a"], index["C_b"],
                                       index["Z_b"], index["B_b"], w.m, True, [E - 1], w.d_rope_I,
                                       w.theta, w.eps)
             nkd, _ = pipeline.quantize_rows(nk, w.idx_dtype)
             kd = np.concatenate([kI_deq, nkd])
-            qd, _ = pipeline.quantize_rows(g["q_I"][0][None], w.idx_dtype)
-            sc = csa.index_scores(qd, g["w"][0][None], kd, np.array([t]), w.m, "bf16")
+            qd, _ = pipeline.quantize_rows(qI[None], w.idx_dtype)
+            sc = csa.index_scores(qd, wI[None], kd, np.array([t]), w.m, "bf16")
             idx, cnt = csa.topk(sc, np.array([t]), w.m, w.k)
             sel = idx[0, :cnt[0]]
-            rows = np.concatenate([kv[sel], g["C_a"][csa.window_rows(t, w.n_w)]])
-        return csa.attend(g["q"][0], rows, g["sink"], w.scale)
+            rows = np.concatenate([kv[sel], win])
+        return csa.attend(q, rows, g["sink"], w.scale)
 
     step()
     n, t0, c0 = 0, time.perf_counter(), time.process_time()
@@ -493,22 +658,53 @@ def cpu_baseline(w, budget_s=20.0):
 
 # ---------------------------------------------------------------------------
 
+SUB_WORKLOADS = (workloads.CSA_DECODE_1M, workloads.HCA_DECODE_1M, workloads.CSA_PREFILL_32K)
+
+
+def run_workload(w, args, world, rank, peaks, min_span_s, cpu_budget_s):
+    """One workload's record: throughput, rooflines, per-kernel fractions, clocks, e2e and (rank
+    0 of a single-GPU run) the oracle's rate on this host."""
+    if w.kind == "csa_prefill":
+        r = bench_prefill(w, args, world, rank, peaks, min_span_s)
+    else:
+        r = bench_decode(w, args, world, rank, peaks, min_span_s)
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_baseline(w, cpu_budget_s)
+    rec = {"value": round(r["value"], 2), "unit": "tok/s", "ms_per_step": round(r["ms"], 5),
+           "steps": args.steps, "repeats": r["repeats"],
+           "dtype": w.dtype + ("+" + w.idx_dtype if w.c_I else ""),
+           "config": {"workload": w.name, "batch_per_gpu": w.b, "context": w.n, "m": w.m,
+                      "top_k": w.k, "window": w.n_w, "heads": w.H, "latent": w.c,
+                      "index_heads": w.H_I, "index_dim": w.c_I, "parallelism":
+                      "replicas%d" % world, "l2": "flushed (256 MiB write) before each step"},
+           "roofline": r["roofline"], "kernels": r["kernels"], "cpu_baseline": cb,
+           "e2e": r["e2e"], "gpu_launches": r["launches"], "clocks": r["clocks"],
+           "stage_us": {k: round(v * 1e3, 2) for k, v in r["stage"].items()}}
+    if "step_roofline" in r:
+        rec["step_roofline"] = r["step_roofline"]
+    return rec
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=500)
-    ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=workloads.CSA_DECODE_64K.name,
-                    choices=sorted(workloads.ALL))
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None, choices=sorted(workloads.ALL),
+                    help="run only this workload (default: the 64K CSA decode headline plus "
+                         "the 1M CSA / HCA decode and 32K prefill sub-records)")
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--min-span", type=float, default=1.0,
+                    help="seconds the repeated timed region of the headline spans at least")
     ap.add_argument("--context", type=int, default=0,
                     help="override the context length (profiling of a smaller case, not a bench line)")
     ap.add_argument("--batch", type=int, default=0, help="override the batch (profiling only)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    w = workloads.ALL[args.workload]
+    w = workloads.ALL[args.workload or workloads.CSA_DECODE_64K.name]
     if args.context:
         w = workloads.shrink(w, n=args.context)
     if args.batch:
@@ -533,29 +729,24 @@ def main():
 
     world, rank, local = dist_setup(args.gpus)
     L.lib()
-    if w.kind == "csa_prefill":
-        r = bench_prefill(w, args, world, rank, peaks)
-    else:
-        r = bench_decode(w, args, world, rank, peaks)
-    cb = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cb = cpu_baseline(w)
+    peaks.update(measure_tc_peaks(peaks))
+    peaks["fp8"] = peaks["fp8_tflops"]
+    head = run_workload(w, args, world, rank, peaks, args.min_span, 20.0)
+    subs = {}
+    if args.workload is None and not args.context and not args.batch:
+        for w2 in SUB_WORKLOADS:
+            subs[w2.name] = run_workload(w2, args, world, rank, peaks, 0.5, 10.0)
     if rank == 0:
-        line = {"metric": METRIC, "value": round(r["value"], 2), "unit": "tok/s",
-                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": round(r["ms"], 5), "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": w.dtype + ("+" + w.idx_dtype if w.c_I else ""),
-                "data": "synthetic",
-                "config": {"workload": w.name, "batch_per_gpu": w.b, "context": w.n, "m": w.m,
-                           "top_k": w.k, "window": w.n_w, "heads": w.H, "latent": w.c,
-                           "index_heads": w.H_I, "index_dim": w.c_I, "parallelism":
-                           "replicas%d" % world, "l2": "flushed (256 MiB write) before each step"},
-                "roofline": r["roofline"], "cpu_baseline": cb, "e2e": r["e2e"],
-                "gpu_launches": r["launches"], "clocks": r["clocks"],
-                "stage_us": {k: round(v * 1e3, 2) for k, v in r["stage"].items()},
-                "peaks": peaks["src"]}
-        if "step_roofline" in r:
-            line["step_roofline"] = r["step_roofline"]
+        line = {"metric": METRIC, "value": head["value"], "unit": "tok/s", "n_gpus": world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": head["dtype"], "data": "synthetic"}
+        line.update({k: v for k, v in head.items() if k not in line})
+        line["peaks"] = {"src": peaks["src"], "hbm_gbs": peaks["hbm"], "bf16_tflops": peaks["bf16"],
+                         "bf16_tflops_sustained": peaks["bf16_sus"],
+                         "fp8_tflops": peaks["fp8"], "fp8_src": peaks["fp8_src"]}
+        if subs:
+            line["sub"] = subs
         print(json.dumps(line))
     if world > 1:
         torch.distributed.destroy_process_group()
