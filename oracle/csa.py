@@ -234,6 +234,44 @@ def topk(scores, q_pos, m, k):
     return idx, cnt
 
 
+def pool_topk(q_I, w, k_I, pool, pool_cnt, q_pos, m, k, out_dtype="bf16"):
+    """Hierarchical sparse indexer: re-score only a candidate pool, keep the k best of it.
+
+    "DeepSeek Technical Reports", section CSA2 (Hierarchical Sparse Indexer): a
+    full indexer scans the whole context for a larger candidate pool; a later
+    Reindex layer scores again with its own query, but searches that pool only.
+    For query r: the candidates are pool[r, :pool_cnt[r]] that are visible to
+    its position (s < E(t)); each is scored exactly as ``index_scores`` scores it
+    (rounded once to ``out_dtype``); the k highest are kept, equal scores going to
+    the lower entry, and returned ascending by entry, -1 padded, with a count.
+    q_I [T][H_I][d_I], w [T][H_I], k_I [E][d_I] (dequantised float64), pool
+    [T][P] int entry ids, pool_cnt [T].
+    """
+    q_I = np.asarray(q_I, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    k_I = np.asarray(k_I, dtype=np.float64)
+    T = q_I.shape[0]
+    idx = np.full((T, k), -1, dtype=np.int32)
+    cnt = np.zeros(T, dtype=np.int32)
+    for r in range(T):
+        ev = int(visible_entries(q_pos[r], m))
+        cand = np.asarray(pool[r, :int(pool_cnt[r])], dtype=np.int64)
+        cand = cand[(cand >= 0) & (cand < min(ev, k_I.shape[0]))]
+        if len(cand) == 0:
+            continue
+        dots = k_I[cand] @ q_I[r].T                          # [P][H_I]
+        sc = np.maximum(dots, 0.0) @ w[r]                    # [P]
+        if out_dtype == "bf16":
+            sc = codecs.round_to_bf16(sc)
+        elif out_dtype == "f32":
+            sc = sc.astype(np.float32).astype(np.float64)
+        order = np.lexsort((cand, -sc))                      # score desc, entry asc
+        keep = np.sort(cand[order[:min(k, len(cand))]])
+        idx[r, :len(keep)] = keep
+        cnt[r] = len(keep)
+    return idx, cnt
+
+
 # ---------------------------------------------------------------------------
 # (4) Shared-latent MQA with sliding window and sink
 # ---------------------------------------------------------------------------

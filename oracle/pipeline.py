@@ -77,7 +77,7 @@ def csa_prefill(main, index, q, q_I, w, sink, *, m, d_rope, theta, eps, k, n_w, 
 
 
 def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k, n_w, scale,
-                   kv_dtype, idx_dtype):
+                   kv_dtype, idx_dtype, mode="full", idx_in=None, pool=None):
     """One CSA decode step of one sequence with L tokens of context.
 
     The new token is t = L - 1; it completes block E - 1 (E = L / m), so the
@@ -86,6 +86,15 @@ def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k,
     earlier entries of the caches are the compressor's outputs for their own
     blocks (the state the decode step reads), computed here the same way.
     q [H][d]; q_I [H_I][d_I]; w [H_I].
+
+    ``mode`` follows the operating modes of "DeepSeek Technical Reports",
+    section CSA2 (cross-layer KV and index reuse):
+      "full"    the indexer scores all E entries (the default above);
+      "reuse"   no scoring: the selection ``idx_in`` (entry ids, -1 padded) of an
+                earlier layer is attended with this layer's q;
+      "reindex" hierarchical indexer: only the entries of ``pool`` (entry ids,
+                -1 padded) are scored with this layer's q_I, and k kept
+                (``csa.pool_topk``).
     """
     E = L // m
     t = L - 1
@@ -94,7 +103,20 @@ def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k,
     kI_deq, _ = quantize_rows(kI, idx_dtype)
     qI_deq, _ = quantize_rows(np.asarray(q_I)[None], idx_dtype)
     scores = csa.index_scores(qI_deq, np.asarray(w)[None], kI_deq, np.array([t]), m, "bf16")
-    idx, cnt = csa.topk(scores, np.array([t]), m, k)
+    if mode == "full":
+        idx, cnt = csa.topk(scores, np.array([t]), m, k)
+    elif mode == "reuse":
+        sel_in = np.asarray(idx_in).reshape(-1)
+        idx = np.full((1, k), -1, dtype=np.int32)
+        n_in = int(np.sum(sel_in >= 0))
+        idx[0, :n_in] = sel_in[:n_in]
+        cnt = np.array([n_in], dtype=np.int32)
+    elif mode == "reindex":
+        pl = np.asarray(pool).reshape(1, -1)
+        idx, cnt = csa.pool_topk(qI_deq, np.asarray(w)[None], kI_deq, pl,
+                                 np.array([int(np.sum(pl >= 0))]), np.array([t]), m, k)
+    else:
+        raise ValueError(mode)
     sel = idx[0, :cnt[0]].astype(np.int64)
     kv_sel = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
                                   main["B_b"], m, True, sel, d_rope, theta, eps)
