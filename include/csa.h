@@ -235,6 +235,32 @@ csa_status csa_topk(const void* scores, int score_dtype, const int32_t* q_pos, i
                     cudaStream_t stream);
 size_t csa_topk_workspace_size(int score_dtype, int b, int T, int E, int k);
 
+/*
+ * Hierarchical sparse indexer ("DeepSeek Technical Reports", section CSA2,
+ * Hierarchical Sparse Indexer): a Reindex layer scores, with its own index
+ * query, only a candidate pool that an earlier full indexer produced (for
+ * instance a top-P with P > k of the first layer), and keeps the k best of it.
+ * For query row r: the candidates are pool[r][j], j < pool_count[r], that are
+ * visible to q_pos[r] (entry < min(E, floor((t+1)/m))); each is scored exactly
+ * as csa_index_scores scores it (BF16 scores); the k highest are kept, equal
+ * scores going to the lower entry.  idx [b][T][k] lists the kept entries in
+ * the pool's order, -1 padded; count [b][T] holds how many.
+ *   pool        [b][T][P] int32 entry ids, ascending, -1 padded (a csa_topk
+ *               output row is such a pool); idx is then ascending too
+ *   pool_count  [b][T] int32 valid pool entries of each row
+ *   q_I, q_scales, w, k_I, k_scales, q_pos, E_cap, E: as in csa_index_scores
+ *   ws          device scratch of csa_pool_topk_workspace_size() bytes: each row's
+ *               pool is gathered into a key set of its own (the tensor-core
+ *               indexer then scores it as a sequence of P entries)
+ */
+size_t csa_pool_topk_workspace_size(const csa_index_params* p, int b, int T, int P, int k);
+csa_status csa_pool_topk(const csa_index_params* p, const void* q_I, const void* q_scales,
+                         const float* w, const void* k_I, const void* k_scales,
+                         const int32_t* q_pos, int b, int T, int E_cap, int E,
+                         const int32_t* pool, const int32_t* pool_count, int P, int k,
+                         int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                         cudaStream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Stage 4: shared-latent MQA over selected entries + window, with sink      */
 /* ------------------------------------------------------------------------ */
@@ -330,6 +356,19 @@ csa_status csa_sparse_attn_noalloc(const csa_attn_params* p, const void* q, cons
  * place.  CSA then quantises q_I, scores all E entries, selects k and attends
  * over them plus the window; HCA attends over all E entries plus the window.
  */
+/*
+ * Operating modes of a CSA decode layer ("DeepSeek Technical Reports", section
+ * CSA2: cross-layer KV and index reuse):
+ *   CSA_MODE_FULL     the indexer scores all E entries and top-k selects k;
+ *   CSA_MODE_REUSE    no scoring: the selection of an earlier layer (idx_in,
+ *                     count_in) is attended with this layer's q;
+ *   CSA_MODE_REINDEX  the hierarchical indexer: only the candidate pool (pool,
+ *                     pool_count, P entries a row) is scored with this layer's
+ *                     q_I, and its k best are attended (csa_pool_topk).
+ * The step compresses the new entry of both caches in every mode.
+ */
+typedef enum { CSA_MODE_FULL = 0, CSA_MODE_REUSE = 1, CSA_MODE_REINDEX = 2 } csa_decode_mode;
+
 typedef struct {
   int b, L, m, c, H;       /* sequences, context, compression rate, latent dim, heads */
   int c_I, H_I;            /* index-key dim and indexer heads (CSA only) */
@@ -342,6 +381,8 @@ typedef struct {
   int idx_dtype;           /* CSA_FP8_E4M3, CSA_NVFP4 or CSA_F32 (CSA only) */
   int hca;                 /* 1: HCA (no indexer, no previous block, dense attention) */
   int E_cap;               /* entries each cache row-block holds (>= L/m) */
+  int mode;                /* csa_decode_mode (CSA only; HCA takes CSA_MODE_FULL) */
+  int P;                   /* CSA_MODE_REINDEX: pool row length */
 } csa_decode_params;
 
 typedef struct {
@@ -359,8 +400,13 @@ typedef struct {
   const float* sink;                   /* [H] */
   void* out;                           /* [b][H][c] kv_dtype */
   float* lse;                          /* [b][H] or NULL */
-  int32_t* idx_out;                    /* [b][k] selected entries or NULL (CSA) */
+  int32_t* idx_out;                    /* [b][k] selected entries or NULL (CSA; not written
+                                          in CSA_MODE_REUSE) */
   int32_t* count_out;                  /* [b] or NULL (CSA) */
+  const int32_t* idx_in;               /* CSA_MODE_REUSE: [b][k] entries to attend, -1 padded */
+  const int32_t* count_in;             /* CSA_MODE_REUSE: [b] */
+  const int32_t* pool;                 /* CSA_MODE_REINDEX: [b][P] candidate entries */
+  const int32_t* pool_count;           /* CSA_MODE_REINDEX: [b] */
 } csa_decode_tensors;
 
 csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, void* ws,

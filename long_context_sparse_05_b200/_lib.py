@@ -46,12 +46,16 @@ class DecodeParams(ctypes.Structure):
                 ("c_I", c_int), ("H_I", c_int), ("d_rope", c_int), ("d_rope_I", c_int),
                 ("rope_theta", c_double), ("eps", c_float), ("k", c_int), ("n_w", c_int),
                 ("scale", c_float), ("kv_dtype", c_int), ("idx_dtype", c_int), ("hca", c_int),
-                ("E_cap", c_int)]
+                ("E_cap", c_int), ("mode", c_int), ("P", c_int)]
+
+
+CSA_MODE_FULL, CSA_MODE_REUSE, CSA_MODE_REINDEX = 0, 1, 2
 
 
 _DECODE_TENSORS = ["C_a", "Z_a", "C_b", "Z_b", "B_a", "B_b", "CI_a", "ZI_a", "CI_b", "ZI_b",
                    "BI_a", "BI_b", "kv_cache", "kI_cache", "kI_scales", "kv_win", "q", "q_I", "w",
-                   "sink", "out", "lse", "idx_out", "count_out"]
+                   "sink", "out", "lse", "idx_out", "count_out", "idx_in", "count_in", "pool",
+                   "pool_count"]
 
 
 class DecodeTensors(ctypes.Structure):
@@ -90,6 +94,11 @@ _SIGS = {
     "csa_topk": (c_int, [c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p,
                          c_void_p, c_void_p, c_size_t, c_void_p]),
     "csa_topk_workspace_size": (c_size_t, [c_int, c_int, c_int, c_int, c_int]),
+    "csa_pool_topk": (c_int, [ctypes.POINTER(IndexParams)] + [c_void_p] * 6 + [c_int] * 4 +
+                      [c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p, c_void_p, c_size_t,
+                       c_void_p]),
+    "csa_pool_topk_workspace_size": (c_size_t, [ctypes.POINTER(IndexParams), c_int, c_int, c_int,
+                                                c_int]),
     "csa_sparse_attn": (c_int, [ctypes.POINTER(AttnParams), c_void_p, c_void_p, c_int, c_void_p,
                                 c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -189,6 +198,20 @@ def csa_topk(scores, score_dtype, q_pos, m, b, T, E, k, idx, count, ws=None, ws_
 
 def csa_topk_workspace_size(score_dtype, b, T, E, k):
     return int(lib().csa_topk_workspace_size(score_dtype, b, T, E, k))
+
+
+def csa_pool_topk_workspace_size(p, b, T, P, k):
+    return int(lib().csa_pool_topk_workspace_size(ctypes.byref(p), b, T, P, k))
+
+
+def csa_pool_topk(p, q_I, q_scales, w, k_I, k_scales, q_pos, b, T, E_cap, E, pool, pool_count,
+                  P, k, idx, count, ws, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    _check(lib().csa_pool_topk(ctypes.byref(p), _ptr(q_I), _ptr(q_scales), _ptr(w), _ptr(k_I),
+                               _ptr(k_scales), _ptr(q_pos), b, T, E_cap, E, _ptr(pool),
+                               _ptr(pool_count), P, k, _ptr(idx), _ptr(count), _ptr(ws), ws_bytes,
+                               _stream(stream)))
 
 
 def csa_sparse_attn_workspace_size(p, b, T, E_cap):

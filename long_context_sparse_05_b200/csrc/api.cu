@@ -201,6 +201,87 @@ csa_status csa_sparse_attn(const csa_attn_params* p, const void* q, const void* 
 }
 
 // ---------------------------------------------------------------------------
+// hierarchical indexer: top-k within a candidate pool
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct PoolWs {
+  void* gather; void* scores; void* topk_ws; size_t topk_ws_bytes; int32_t* gpos;
+};
+
+size_t pool_layout(int fmt, int d, int rows, int P, int k, void* ws, size_t cap, PoolWs* o) {
+  Carve cv(ws, cap);
+  PoolWs d_{};
+  size_t o_pos = 0;
+  const size_t gb = pool_gather_bytes(fmt, rows, P, d, nullptr, nullptr, &o_pos);
+  d_.gather = cv.take(gb);
+  if (d_.gather) d_.gpos = reinterpret_cast<int32_t*>(static_cast<char*>(d_.gather) + o_pos);
+  d_.scores = cv.take((size_t)rows * P * 2);
+  d_.topk_ws_bytes = topk_workspace_bytes(rows, P, k, CSA_BF16);
+  d_.topk_ws = cv.take(d_.topk_ws_bytes);
+  if (o) *o = d_;
+  return cv.ok ? align256(cv.used) : 0;
+}
+
+csa_status pool_topk_impl(const csa_index_params* p, const void* q_I, const void* q_scales,
+                          const float* w, const void* k_I, const void* k_scales,
+                          const int32_t* q_pos, int b, int T, int E_cap, int E,
+                          const int32_t* pool, const int32_t* pool_count, int P, int k,
+                          int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                          cudaStream_t stream, bool pdl) {
+  if (!p) return CSA_ERR_INVALID_ARG;
+  if (p->H_I < 1 || p->d_I < 16 || p->d_I % 16 || p->m < 1) return CSA_ERR_INVALID_ARG;
+  if (p->qk_dtype != CSA_F32 && p->qk_dtype != CSA_FP8_E4M3 && p->qk_dtype != CSA_NVFP4)
+    return CSA_ERR_INVALID_ARG;
+  if (p->qk_dtype == CSA_NVFP4 && p->d_I % 64) return CSA_ERR_INVALID_ARG;
+  if (b < 0 || T < 0 || E < 0 || E > E_cap || P < 1 || k < 1) return CSA_ERR_INVALID_ARG;
+  if (b == 0 || T == 0) return CSA_OK;
+  if (!q_I || !w || !k_I || !q_pos || !pool || !pool_count || !idx || !count)
+    return CSA_ERR_INVALID_ARG;
+  if (p->qk_dtype != CSA_F32 && (!q_scales || !k_scales)) return CSA_ERR_INVALID_ARG;
+  if (!aligned16(k_I)) return CSA_ERR_INVALID_ARG;
+  const int rows = b * T;
+  PoolWs d{};
+  if (pool_layout(p->qk_dtype, p->d_I, rows, P, k, ws, ws_bytes, &d) == 0 || !ws ||
+      ws_bytes < pool_layout(p->qk_dtype, p->d_I, rows, P, k, nullptr, 0, nullptr))
+    return CSA_ERR_INVALID_ARG;
+  csa_status st = launch_pool_gather(p->qk_dtype, pool, pool_count, q_pos, k_I, k_scales, rows, T,
+                                     P, E_cap, E, p->m, p->d_I, d.gather, stream, pdl);
+  if (st) return st;
+  size_t o_sc = 0;
+  pool_gather_bytes(p->qk_dtype, rows, P, p->d_I, &o_sc, nullptr, nullptr);
+  const int P_cap = (P + 255) / 256 * 256;
+  csa_index_params ip = *p;
+  ip.score_dtype = CSA_BF16;
+  st = index_scores_impl(&ip, q_I, q_scales, w, d.gather,
+                         p->qk_dtype == CSA_F32 ? nullptr : static_cast<char*>(d.gather) + o_sc,
+                         d.gpos, rows, 1, P_cap, P, d.scores, stream, 1, 0, -1);
+  if (st) return st;
+  st = topk_impl(d.scores, CSA_BF16, d.gpos, p->m, rows, 1, P, k, idx, count, d.topk_ws,
+                 d.topk_ws_bytes, stream, true);
+  if (st) return st;
+  return launch_pool_map(d.gather, p->qk_dtype, rows, P, p->d_I, k, idx, count, stream, true);
+}
+
+}  // namespace
+
+size_t csa_pool_topk_workspace_size(const csa_index_params* p, int b, int T, int P, int k) {
+  if (!p || b <= 0 || T <= 0 || P <= 0 || k <= 0) return 0;
+  return pool_layout(p->qk_dtype, p->d_I, b * T, P, k, nullptr, 0, nullptr);
+}
+
+csa_status csa_pool_topk(const csa_index_params* p, const void* q_I, const void* q_scales,
+                         const float* w, const void* k_I, const void* k_scales,
+                         const int32_t* q_pos, int b, int T, int E_cap, int E,
+                         const int32_t* pool, const int32_t* pool_count, int P, int k,
+                         int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+  return pool_topk_impl(p, q_I, q_scales, w, k_I, k_scales, q_pos, b, T, E_cap, E, pool,
+                        pool_count, P, k, idx, count, ws, ws_bytes, stream, false);
+}
+
+// ---------------------------------------------------------------------------
 // decode
 // ---------------------------------------------------------------------------
 
@@ -209,6 +290,7 @@ namespace {
 struct DecodeWs {
   void* qI_codes; void* qI_scales; void* scores; int32_t* idx; int32_t* count; int32_t* qpos;
   void* attn_ws; size_t attn_ws_bytes; void* topk_ws; size_t topk_ws_bytes;
+  void* pool_ws; size_t pool_ws_bytes;
 };
 
 size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs* o) {
@@ -223,11 +305,16 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
       d.qI_scales = cv.take(p->idx_dtype == CSA_FP8_E4M3 ? (size_t)b * p->H_I * 4
                                                           : (size_t)b * p->H_I * (p->c_I / 16));
     }
-    d.scores = cv.take((size_t)b * E * 2);
     d.idx = static_cast<int32_t*>(cv.take((size_t)b * p->k * 4));
     d.count = static_cast<int32_t*>(cv.take((size_t)b * 4));
-    d.topk_ws_bytes = topk_workspace_bytes(b, E, p->k, CSA_BF16);
-    d.topk_ws = cv.take(d.topk_ws_bytes);
+    if (p->mode == CSA_MODE_FULL) {
+      d.scores = cv.take((size_t)b * E * 2);
+      d.topk_ws_bytes = topk_workspace_bytes(b, E, p->k, CSA_BF16);
+      d.topk_ws = cv.take(d.topk_ws_bytes);
+    } else if (p->mode == CSA_MODE_REINDEX) {
+      d.pool_ws_bytes = pool_layout(p->idx_dtype, p->c_I, b, p->P, p->k, nullptr, 0, nullptr);
+      d.pool_ws = cv.take(d.pool_ws_bytes);
+    }
   }
   csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype};
   d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, b, 1, p->E_cap);
@@ -241,7 +328,10 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
 int csa_decode_launch_count(const csa_decode_params* p) {
   if (!p || p->b <= 0) return 0;
   int n = 1;                                   // prologue: compressors, quantiser, positions
-  if (!p->hca) n += 1 + (topk_workspace_bytes(p->b, p->L / p->m, p->k, CSA_BF16) ? 2 : 1);
+  if (!p->hca && p->mode == CSA_MODE_FULL)
+    n += 1 + (topk_workspace_bytes(p->b, p->L / p->m, p->k, CSA_BF16) ? 2 : 1);
+  if (!p->hca && p->mode == CSA_MODE_REINDEX)  // gather, indexer, top-k, map
+    n += 3 + (topk_workspace_bytes(p->b, p->P, p->k, CSA_BF16) ? 2 : 1);
   n += attn_launch_count(p->H, p->c, p->hca ? 0 : p->k, p->n_w, p->b, 1, p->E_cap, p->kv_dtype);
   return n;
 }
@@ -258,7 +348,13 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
   const int E = p->L / p->m;
   if (E > p->E_cap) return CSA_ERR_INVALID_ARG;
   if (!p->hca && (p->k < 1 || p->c_I < 16 || p->H_I < 1)) return CSA_ERR_INVALID_ARG;
+  if (p->mode != CSA_MODE_FULL && p->mode != CSA_MODE_REUSE && p->mode != CSA_MODE_REINDEX)
+    return CSA_ERR_INVALID_ARG;
+  if (p->hca && p->mode != CSA_MODE_FULL) return CSA_ERR_INVALID_ARG;
+  if (p->mode == CSA_MODE_REINDEX && p->P < 1) return CSA_ERR_INVALID_ARG;
   if (p->b == 0) return CSA_OK;
+  if (p->mode == CSA_MODE_REUSE && (!x->idx_in || !x->count_in)) return CSA_ERR_INVALID_ARG;
+  if (p->mode == CSA_MODE_REINDEX && (!x->pool || !x->pool_count)) return CSA_ERR_INVALID_ARG;
   DecodeWs d{};
   const size_t need = decode_layout(p, ws, ws_bytes, &d);
   if (need == 0 || !ws || ws_bytes < csa_decode_workspace_size(p)) return CSA_ERR_INVALID_ARG;
@@ -311,7 +407,20 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
   if (st) return st;
   const int32_t* idx = nullptr;
   const int32_t* cnt = nullptr;
-  if (!p->hca) {
+  if (!p->hca && p->mode == CSA_MODE_REUSE) {
+    // CSA2 Reuse mode: an earlier layer's selection, no scoring
+    idx = x->idx_in; cnt = x->count_in;
+  } else if (!p->hca && p->mode == CSA_MODE_REINDEX) {
+    // CSA2 Reindex mode with the hierarchical indexer: score the candidate pool only
+    int32_t* io = x->idx_out ? x->idx_out : d.idx;
+    int32_t* co = x->count_out ? x->count_out : d.count;
+    csa_index_params ip{p->H_I, p->c_I, p->m, p->idx_dtype, CSA_BF16};
+    st = pool_topk_impl(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, 1, p->E_cap, E,
+                        x->pool, x->pool_count, p->P, p->k, io, co, d.pool_ws, d.pool_ws_bytes,
+                        stream, true);
+    if (st) return st;
+    idx = io; cnt = co;
+  } else if (!p->hca) {
     // 3. score all entries
     // (programmatic dependent launches from here on: each kernel starts while its
     //  predecessor drains and waits for it only where it reads its outputs)

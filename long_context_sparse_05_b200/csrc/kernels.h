@@ -70,6 +70,18 @@ size_t attn_tc_workspace_bytes(int H, int d, int k, int n_w, int b, int T, int E
 bool attn_tc_supported(int H, int d, int dtype);
 int attn_launch_count(int H, int d, int k, int n_w, int b, int T, int E_cap, int dtype);
 
+// Hierarchical indexer: the candidate pool of every query row gathered into a key set of
+// its own (workspace of pool_gather_bytes()), and top-k positions mapped back to entries.
+int pool_row_bytes(int fmt, int d);
+size_t pool_gather_bytes(int fmt, int rows, int P, int d, size_t* off_scales, size_t* off_pool,
+                         size_t* off_pos);
+csa_status launch_pool_gather(int fmt, const int32_t* pool, const int32_t* pool_count,
+                              const int32_t* q_pos, const void* k, const void* k_scales, int rows,
+                              int T, int P, int E_cap, int E, int m, int d, void* ws,
+                              cudaStream_t st, bool pdl);
+csa_status launch_pool_map(const void* ws, int fmt, int rows, int P, int d, int k, int32_t* idx,
+                           const int32_t* count, cudaStream_t st, bool pdl);
+
 // Small helpers.
 csa_status launch_fill_i32(int32_t* p, int count, int value, cudaStream_t st);
 csa_status launch_iota_positions(int32_t* p, int b, int n, cudaStream_t st);

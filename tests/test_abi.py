@@ -131,6 +131,26 @@ def test_invalid_arguments_rejected_on_host():
     dp.c_I = 96                                        # the only defect: every pointer is set
     x = L.DecodeTensors(**{n: fake for n, _ in L.DecodeTensors._fields_})
     assert L.lib().csa_decode(ctypes.byref(dp), ctypes.byref(x), 1 << 20, 1 << 30, None) == 1
+    # CSA2 modes: an unknown mode, Reuse without a selection, Reindex without a pool or with
+    # an empty one, and any mode but Full for HCA
+    for mode, P, drop, hca in ((7, 0, None, 0), (L.CSA_MODE_REUSE, 0, "idx_in", 0),
+                               (L.CSA_MODE_REINDEX, 2048, "pool_count", 0),
+                               (L.CSA_MODE_REINDEX, 0, None, 0), (L.CSA_MODE_REUSE, 0, None, 1)):
+        dp = runner.decode_params(workloads.CSA_DECODE_1M)
+        dp.mode, dp.P, dp.hca = mode, P, hca
+        x = L.DecodeTensors(**{n: fake for n, _ in L.DecodeTensors._fields_})
+        if drop:
+            setattr(x, drop, None)
+        assert L.lib().csa_decode(ctypes.byref(dp), ctypes.byref(x), 1 << 20, 1 << 34, None) == 1
+    # the pool top-k: a pool of length 0, a missing pool count, too small a workspace
+    ip = L.IndexParams(H_I=64, d_I=128, m=4, qk_dtype=L.CSA_FP8_E4M3, score_dtype=L.CSA_BF16)
+    args = [fake] * 6 + [1, 1, 4096, 4096, fake, fake, 1024, 64, fake, fake, fake, 1 << 30, None]
+    bad = list(args); bad[12] = 0
+    assert lib.csa_pool_topk(ctypes.byref(ip), *bad) == 1
+    bad = list(args); bad[11] = None
+    assert lib.csa_pool_topk(ctypes.byref(ip), *bad) == 1
+    bad = list(args); bad[17] = 16
+    assert lib.csa_pool_topk(ctypes.byref(ip), *bad) == 1
 
 
 def test_workspace_sizes_are_host_only_and_positive():
