@@ -21,12 +21,15 @@
 //
 // Work item = (query, split of its rows).  With one split the CTA writes the
 // normalised output (the sink joins the denominator).  With several (CSA decode),
-// the splits of one query form a thread-block cluster: each CTA bulk-stores an
-// unnormalised bf16 record (O, running max, running sum) to the workspace, the
-// cluster synchronises (barrier.cluster, release / acquire), and then every CTA
-// bulk-loads one slice of the 512 output dims from every split and merges it with
-// the sink (log-sum-exp merge), so no second kernel runs.  Dense decode (HCA, tens
-// of splits) writes fp32 partials and a small merge kernel combines them.
+// the splits of one query form a thread-block cluster.  As soon as its last softmax is
+// done, every split pushes its running max and sum per head to every rank (st.async
+// into distributed shared memory, counted on the receiver's mbarrier), so while its PV
+// still runs each rank forms the same log-sum-exp weights e^(M_j - M) / (e^sink +
+// sum_i l_i e^(M_i - M)).  Each split then stages its O scaled by its own weight, as
+// bf16, bulk-stores it to the workspace, the cluster synchronises (barrier.cluster,
+// release / acquire), and every CTA bulk-loads one slice of the 512 output dims from
+// every split and adds them, so no second kernel runs.  Dense decode (HCA, tens of
+// splits) writes fp32 partials and a small merge kernel combines them.
 //
 // CTA (288 threads): warps 0-7 gather, read TMEM and run the softmax, two warps per
 // TMEM lane quarter (warp w owns lanes 32 (w % 4).., 32 heads each); warp 8 lane 0
@@ -52,6 +55,7 @@ constexpr float kRescaleThresh = 8.0f;     // log2 units
 constexpr int kSW = 8;                     // gather / softmax warps (two per TMEM lane quarter)
 constexpr int kThreadsA = 32 * kSW + 32;   // plus the MMA warp
 constexpr int kST = 32 * kSW;              // softmax threads
+constexpr uint32_t kWaitHintNs = 64;       // a parked mbarrier wait re-checks this often
 
 struct AttnTc {
   const __nv_bfloat16* q; const __nv_bfloat16* kv; const int32_t* idx; const int32_t* count;
@@ -63,7 +67,7 @@ struct AttnTc {
   int cluster;   // nsplit > 1: 1 = the splits of a query are one cluster and merge inside
                  // the kernel; 0 = fp32 partials go to the workspace and attn_merge_kernel
                  // combines them
-  uint8_t* part_bf;   // cluster mode: per item, bf16 O [512][64] (swizzled rows), max, sum
+  uint8_t* part_bf;   // cluster mode: per item, the scaled O as bf16 [512][64] (swizzled rows)
   float scale_log2;
 };
 
@@ -84,10 +88,10 @@ __device__ __forceinline__ QInfo query_info(const AttnTc& p, int qrow) {
 
 // Source row of list position pos, or nullptr for a padded / invalid row.
 __device__ __forceinline__ const __nv_bfloat16* row_src(const AttnTc& p, const QInfo& Q, int qrow,
-                                                        int pos) {
+                                                        int pos, int e_pre = INT_MIN) {
   if (pos >= Q.nrows) return nullptr;
   if (pos < Q.nsel) {
-    const int e = p.dense ? pos : p.idx[(size_t)qrow * p.k + pos];
+    const int e = p.dense ? pos : e_pre != INT_MIN ? e_pre : p.idx[(size_t)qrow * p.k + pos];
     if (e < 0 || e >= p.E_cap) return nullptr;
     return p.kv + ((size_t)Q.sb * p.E_cap + e) * kD;
   }
@@ -152,17 +156,15 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 constexpr int kMaxSplit = 16;         // splits of one query merged inside one cluster
 constexpr int kMaxSplitGlobal = 32;   // splits of one query merged through the workspace
 
-// Cluster merge.  Each split stores its unnormalised O (bf16 [512 dims][64 heads], the
-// 16-byte chunk c of dim d's row at chunk c ^ (d & 7)), its running max and sum to the
-// workspace with bulk stores; after a cluster barrier every rank bulk-loads, from every
-// split, the rows of the dims it merges.  Shared memory (KV / query tile area, free
-// once PV is done):
-//   [0, 64 KB)           this split's O, staged for the bulk store
+// Cluster merge.  Each split stores its O scaled by its log-sum-exp weight (bf16 [512
+// dims][64 heads], the 16-byte chunk c of dim d's row at chunk c ^ (d & 7)) to the
+// workspace with one bulk store; after a cluster barrier every rank bulk-loads, from
+// every split, the rows of the dims it owns and adds them.  Shared memory (KV / query
+// tile area, free once PV is done):
+//   [0, 64 KB)           this split's scaled O, staged for the bulk store
 //   [64 KB, 144 KB)      received slices: split j's rows of this rank's dims at slot j
-//   [144 KB, 152 KB)     received running maxima and sums: [split][2][64] fp32
 constexpr int kCmRecvO = 64 * 1024;
-constexpr int kCmRecvML = 144 * 1024;
-constexpr size_t kPartB = (size_t)kD * kH * 2 + 2 * kH * 4;   // one split's record
+constexpr size_t kPartB = (size_t)kD * kH * 2;   // one split's record
 __device__ __forceinline__ int cm_chunk(int d, int chunk) { return chunk ^ (d & 7); }
 
 __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_t bytes) {
@@ -179,6 +181,17 @@ __device__ __forceinline__ void bulk_load_g(void* sdst, const void* gsrc, uint32
 }
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+// Address of the same shared-memory object in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cl_map(const void* local, uint32_t rank) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(tc::smem_u32(local)), "r"(rank));
+  return ra;
+}
+// 8-byte store into another CTA's shared memory, counted (bytes) on that CTA's mbarrier.
+__device__ __forceinline__ void st_async8(uint32_t raddr, uint32_t a, uint32_t b, uint32_t rbar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v2.b32 [%0], {%1, %2}, [%3];"
+               ::"r"(raddr), "r"(a), "r"(b), "r"(rbar) : "memory");
 }
 
 // Dims of the output slice merged by cluster rank `rank`.
@@ -242,6 +255,7 @@ __device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool writ
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     for (int sp = 0; sp < ns; ++sp) {
       const float w = s_mw[sp * kH + h];
+      if (w == 0.f) continue;   // an empty split leaves its partial O unwritten
       const float* src = st + ((size_t)sp * dsl + dd) * kH + h;
 #pragma unroll
       for (int u = 0; u < 4; ++u) acc[u] = fmaf(src[u * kH], w, acc[u]);
@@ -256,13 +270,10 @@ __device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool writ
 }
 
 // Cluster merge of query `qrow` (every thread of the CTA joins).  Each split bulk-stores
-// its record to the workspace; after the cluster barrier rank r bulk-loads, from every
-// split, the rows of output dims [d0, d1) and the running maxima and sums, and combines
-// them: out = sum_j e^{m_j} O_j / (e^{sink} + sum_j e^{m_j} l_j).
+// its scaled O to the workspace; after the cluster barrier rank r bulk-loads, from every
+// split, the rows of output dims [d0, d1) and adds them.
 __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int item, int rank,
-                                              uint8_t* area, const float* s_M, const float* s_l,
-                                              float* s_mw, const float* s_sink2, uint64_t* bar_r,
-                                              bool ok) {
+                                              uint8_t* area, uint64_t* bar_r, bool ok) {
   const int tid = threadIdx.x;
   const int ns = p.nsplit;
   int d0, d1;
@@ -271,79 +282,42 @@ __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int ite
   const int dps = ((kD + ns - 1) / ns + 7) & ~7;
   // this split's record to the workspace (the rows were fenced for the async proxy)
   if (tid == 0) {
-    uint8_t* rec = p.part_bf + (size_t)item * kPartB;
-    bulk_store(rec, area, kD * kH * 2);
-    bulk_store(rec + kD * kH * 2, s_M, kH * 4);
-    bulk_store(rec + kD * kH * 2 + kH * 4, s_l, kH * 4);
+    bulk_store(p.part_bf + (size_t)item * kPartB, area, kD * kH * 2);
     bulk_store_commit_wait();
     fence_proxy_async_global();
   }
   cluster_sync_all();   // every split's record is in the workspace
   if (tid == 0) {
     fence_proxy_async_global();
-    tc::mbar_arrive_expect_tx(bar_r, (uint32_t)(ns * (dsl * kH * 2 + 2 * kH * 4)));
+    tc::mbar_arrive_expect_tx(bar_r, (uint32_t)(ns * dsl * kH * 2));
     const size_t it0 = (size_t)qrow * ns;
-    for (int j = 0; j < ns; ++j) {
-      const uint8_t* rec = p.part_bf + (it0 + j) * kPartB;
-      if (dsl > 0)
-        bulk_load_g(area + kCmRecvO + (size_t)j * dps * kH * 2, rec + (size_t)d0 * kH * 2,
-                    (uint32_t)(dsl * kH * 2), bar_r);
-      bulk_load_g(area + kCmRecvML + (size_t)j * 2 * kH * 4, rec + kD * kH * 2, 2 * kH * 4, bar_r);
-    }
+    if (dsl > 0)
+      for (int j = 0; j < ns; ++j)
+        bulk_load_g(area + kCmRecvO + (size_t)j * dps * kH * 2,
+                    p.part_bf + (it0 + j) * kPartB + (size_t)d0 * kH * 2, (uint32_t)(dsl * kH * 2),
+                    bar_r);
   }
-  const bool got = tc::mbar_wait(bar_r, 0, p.err);
-  const float* rml = reinterpret_cast<const float*>(area + kCmRecvML);
-  if (tid < kH) {
-    // maxima first (independent loads, four at a time), then the weights
-    const int h = tid;
-    const float sink2 = s_sink2[h];
-    float M = sink2;
-#pragma unroll 4
-    for (int j = 0; j < ns; ++j) M = fmaxf(M, rml[j * 2 * kH + h]);
-    float den = exp2f(sink2 - M);
-#pragma unroll 4
-    for (int j = 0; j < ns; ++j) {
-      const float mj = rml[j * 2 * kH + h];
-      const float e = mj == -INFINITY ? 0.f : exp2f(mj - M);
-      s_mw[j * kH + h] = e;
-      den = fmaf(rml[j * 2 * kH + kH + h], e, den);
-    }
-    const float inv = 1.f / den;
-#pragma unroll 4
-    for (int j = 0; j < ns; ++j) s_mw[j * kH + h] *= inv;
-    if (rank == 0 && p.lse) p.lse[(size_t)qrow * kH + h] = (M + log2f(den)) * 0.6931471805599453f;
-  }
-  __syncthreads();
+  // one thread waits for the slices and releases the others at a CTA barrier (threads
+  // parked in an mbarrier wait resume late)
+  const bool got = __syncthreads_and(tid == 0 ? tc::mbar_wait_hint(bar_r, 0, p.err, kWaitHintNs) : true);
   // thread = (chunk of 8 heads, dim); consecutive threads: consecutive dims, so each
   // split is one conflict-free 16-byte shared load per thread and each head's output
-  // run is a coalesced store.  Two splits' loads are in flight at a time.
+  // run is a coalesced store
   const __nv_bfloat16* recv = reinterpret_cast<const __nv_bfloat16*>(area + kCmRecvO);
   for (int x = tid; x < dsl * 8; x += blockDim.x) {
     const int c = x / dsl, dd = x - c * dsl;
     const int d = d0 + dd;
     const int off = dd * kH + cm_chunk(d, c) * 8;
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j0 = 0; j0 < ns; j0 += 2) {
-      uint4 v[2];
-      float4 wa[2], wb[2];
+#pragma unroll 4
+    for (int j = 0; j < ns; ++j) {
+      const uint4 v = *reinterpret_cast<const uint4*>(recv + (size_t)j * dps * kH + off);
+      const uint32_t q[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int j = min(j0 + u, ns - 1);
-        v[u] = *reinterpret_cast<const uint4*>(recv + (size_t)j * dps * kH + off);
-        wa[u] = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c);
-        wb[u] = *reinterpret_cast<const float4*>(s_mw + j * kH + 8 * c + 4);
-      }
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        if (j0 + u >= ns) break;
-        const float w[8] = {wa[u].x, wa[u].y, wa[u].z, wa[u].w, wb[u].x, wb[u].y, wb[u].z, wb[u].w};
-        const uint32_t q[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&q[e]);
-          acc[2 * e] = fmaf(__low2float(b2), w[2 * e], acc[2 * e]);
-          acc[2 * e + 1] = fmaf(__high2float(b2), w[2 * e + 1], acc[2 * e + 1]);
-        }
+      for (int e = 0; e < 4; ++e) {
+        const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&q[e]);
+        acc[2 * e] += __low2float(b2);
+        acc[2 * e + 1] += __high2float(b2);
       }
     }
     __nv_bfloat16* o = p.out + ((size_t)qrow * kH + 8 * c) * kD + d;
@@ -384,28 +358,18 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(s_flag + 4);
   uint64_t* bar_o = bar_s + 1;
   uint64_t* bar_r = bar_o + 1;                  // cluster merge: received slices
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_r + 1);
+  uint64_t* bar_st = bar_r + 1;                 // cluster merge: maxima and sums received
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_st + 1);
   const __nv_bfloat16** s_rows = reinterpret_cast<const __nv_bfloat16**>(tmem_holder + 2);  // [128]
-  float* s_mw = reinterpret_cast<float*>(                    // [kMaxSplit][kH] merge weights
+  float* s_stats = reinterpret_cast<float*>(                 // [kMaxSplit][kH][2]: (max, sum)
       (reinterpret_cast<uintptr_t>(s_rows + kRows) + 15) & ~(uintptr_t)15);
-  float* s_sink2 = s_mw + kMaxSplit * kH;                   // [kH] sink logits, log2 units
+  float* s_sink2 = s_stats + kMaxSplit * kH * 2;             // [kH] sink logits, log2 units
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int tid = threadIdx.x;
 
   pdl_launch_dependents();
-  if (tid < kH) s_sink2[tid] = p.sink[tid] * kLog2e;   // an input: read before the wait
-  if (tid == 0) {
-    tc::mbar_init(bar_s, 1);
-    tc::mbar_init(bar_o, 1);
-    tc::mbar_init(bar_r, 1);
-    tc::fence_barrier_init();
-  }
-  if (warp == 0) tc::tmem_alloc(tmem_holder, 512);
-  tc::tc_fence_before();
-  __syncthreads();
-  tc::tc_fence_after();
   // the first item's query heads are an input of this call: fetch them before waiting
   // on the preceding kernels (selections, positions and caches come from those)
   const bool q_pre = (int)blockIdx.x < p.rows_total * p.nsplit && warp < kSW;
@@ -413,6 +377,23 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
     const __nv_bfloat16* qb = p.q + (size_t)(blockIdx.x / p.nsplit) * kH * kD;
     gather_rows(sQ, kQBlkBytes, kH, warp, lane, [&](int h) { return qb + (size_t)h * kD; }, p.q);
   }
+  if (tid < kH) s_sink2[tid] = p.sink[tid] * kLog2e;   // an input: read before the wait
+  const int crank = p.cluster ? (int)cluster_rank() : 0;
+  if (tid == 0) {
+    tc::mbar_init(bar_s, 1);
+    tc::mbar_init(bar_o, 1);
+    tc::mbar_init(bar_r, 1);
+    tc::mbar_init(bar_st, 1);
+    tc::fence_barrier_init();
+    // one item per CTA in cluster mode: the bytes of maxima and sums every rank pushes here
+    if (p.cluster) tc::mbar_arrive_expect_tx(bar_st, (uint32_t)(p.nsplit * kH * 8));
+  }
+  if (warp == 0) tc::tmem_alloc(tmem_holder, 512);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  // every rank's barriers are initialised before any rank pushes into them
+  if (p.cluster) cluster_sync_all();
   pdl_wait();
   const uint32_t tmem = *tmem_holder;
   const uint32_t tS = tmem;            // columns [0, 64): S^T
@@ -426,6 +407,13 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   for (int item = blockIdx.x; item < items; item += gridDim.x) {
     const int qrow = item / p.nsplit;
     const int split = item % p.nsplit;
+    // the first tile's list entry of this thread's row is loaded alongside the query's
+    // position and selection count (all three come from the preceding kernels)
+    int e_pre = INT_MIN;
+    if (warp < 4 && !p.dense) {
+      const int pos0 = (item % p.nsplit) * p.rps + warp * 32 + lane;
+      if (pos0 < p.k) e_pre = p.idx[(size_t)qrow * p.k + pos0];
+    }
     const QInfo Q = query_info(p, qrow);
     // rows [rb, re) of the query's list, in sub-tiles of up to 128 rows
     const int rb = split * p.rps;
@@ -481,7 +469,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
     if (tid < kH) { s_M[tid] = -INFINITY; s_l[tid] = 0.f; }
     for (int j = jb; j < je; ++j) {
       if (j > jb) {                                  // previous PV done: KV, P and O are free
-        ok = ok && tc::mbar_wait(bar_o, no & 1, p.err);
+        ok = ok && tc::mbar_wait_hint(bar_o, no & 1, p.err, kWaitHintNs);
         ++no;
         tc::tc_fence_after();
       }
@@ -493,7 +481,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       // source of every row of the tile: one coalesced pass over the index list
       if (hf == 0) {
         const int pos = rb + j * kRows + r;
-        s_rows[r] = pos < re ? row_src(p, Q, qrow, pos) : nullptr;
+        s_rows[r] = pos < re ? row_src(p, Q, qrow, pos, j == jb ? e_pre : INT_MIN) : nullptr;
       }
       tc::named_bar(3, kST);
       gather_rows(sKV, kKVBlkBytes, kRows, warp, lane, [&](int rr) { return s_rows[rr]; }, p.kv);
@@ -503,7 +491,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       tc::named_bar(1, kThreadsA);
 
       // logits of row r for this thread's 32 heads
-      ok = ok && tc::mbar_wait(bar_s, ns & 1, p.err);
+      ok = ok && tc::mbar_wait_hint(bar_s, ns & 1, p.err, kWaitHintNs);
       ++ns;
       tc::tc_fence_after();
       if (j == je - 1 && p.nsplit == 1 && item + (int)gridDim.x < items) {
@@ -591,9 +579,33 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       tc::named_bar(2, kThreadsA);
     }
 
+    if (p.nsplit > 1 && p.cluster) {
+      // this split's running maxima and sums (final after its last softmax; an empty
+      // split keeps -inf and 0) to every rank while its PV still runs; with every rank's,
+      // each rank forms the same log-sum-exp denominators and its own weights
+      if (tid < kH) {
+        const float Mv = s_M[tid], lv = s_l[tid];
+        for (int j = 0; j < p.nsplit; ++j)
+          st_async8(cl_map(s_stats + (crank * kH + tid) * 2, (uint32_t)j), __float_as_uint(Mv),
+                    __float_as_uint(lv), cl_map(bar_st, (uint32_t)j));
+        const bool got = tc::mbar_wait_hint(bar_st, 0, p.err, kWaitHintNs);
+        const float sink2 = s_sink2[tid];
+        float M = sink2;
+        for (int j = 0; j < p.nsplit; ++j) M = fmaxf(M, s_stats[(j * kH + tid) * 2]);
+        float den = exp2f(sink2 - M);
+        for (int j = 0; j < p.nsplit; ++j) {
+          const float mj = s_stats[(j * kH + tid) * 2];
+          den = fmaf(s_stats[(j * kH + tid) * 2 + 1], mj == -INFINITY ? 0.f : exp2f(mj - M), den);
+        }
+        const float wme = Mv == -INFINITY ? 0.f : exp2f(Mv - M) / den;
+        s_alpha[tid] = (ok && got) ? wme : __int_as_float(0x7fc00000);
+        if (crank == 0 && p.lse) p.lse[(size_t)qrow * kH + tid] = (M + log2f(den)) * 0.6931471805599453f;
+      }
+    }
+
     if (je <= jb) {
       // empty split: nothing to add.  Cluster mode: its running max stays -inf (weight 0)
-      // and its O is zeroed so that the merge's 0 * O stays 0.
+      // and its O is zeroed so that the merge adds 0.
       if (p.nsplit > 1 && !p.cluster && tid < kH) {
         p.part_m[(size_t)item * kH + tid] = -INFINITY;
         p.part_l[(size_t)item * kH + tid] = 0.f;
@@ -604,7 +616,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         tc::fence_proxy_async();
       }
     } else {
-    ok = ok && tc::mbar_wait(bar_o, no & 1, p.err);
+    ok = ok && tc::mbar_wait_hint(bar_o, no & 1, p.err, kWaitHintNs);
     ++no;
     tc::tc_fence_after();
     tc::named_bar(3, kST);                           // s_l / s_M final
@@ -635,10 +647,17 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         }
       }
     } else if (p.cluster) {
-      // unnormalised O into shared memory (bf16) for the cluster merge (KV tile area, free now)
-      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
+      // O scaled by this split's weight (s_alpha, ordered by the barrier above) into shared
+      // memory (bf16) for the cluster merge (KV tile area, free now)
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+      for (int half = 0; half < 2; ++half) {
+        float wt[32];                         // this half's 32 head weights, in registers
+#pragma unroll
+        for (int h = 0; h < 32; h += 4) {
+          const float4 w4 = *reinterpret_cast<const float4*>(s_alpha + half * 32 + h);
+          wt[h] = w4.x; wt[h + 1] = w4.y; wt[h + 2] = w4.z; wt[h + 3] = w4.w;
+        }
+        for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
           uint32_t o[32];
           tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
           tc::tmem_ld_wait(o);
@@ -648,8 +667,10 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
             uint32_t w4[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(o[8 * c4 + 2 * e]),
-                                                              __uint_as_float(o[8 * c4 + 2 * e + 1]));
+              const int h0 = c4 * 8 + 2 * e;
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                  __uint_as_float(o[8 * c4 + 2 * e]) * wt[h0],
+                  __uint_as_float(o[8 * c4 + 2 * e + 1]) * wt[h0 + 1]);
               w4[e] = *reinterpret_cast<const uint32_t*>(&b2);
             }
             *reinterpret_cast<uint4*>(sKV + (size_t)d * kH * 2 + cm_chunk(d, half * 4 + c4) * 16) =
@@ -691,9 +712,8 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       // every split of this query has its O, max and sum in shared memory: merge one
       // slice of the dims, then keep this CTA's shared memory alive until all peers
       // have read it
-      if (tid < kH) tc::fence_proxy_async();   // s_M / s_l are read by the bulk stores too
       __syncthreads();
-      cluster_merge(p, qrow, item, (int)cluster_rank(), sKV, s_M, s_l, s_mw, s_sink2, bar_r, ok);
+      cluster_merge(p, qrow, item, crank, sKV, bar_r, ok);
     }
   }
 
@@ -705,9 +725,12 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   }
 }
 
+// alignment slack, KV tile, q, P^T, s_red + four per-head arrays, flag, four mbarriers,
+// TMEM holder, row-pointer table, 16-byte alignment, merge maxima / sums, sink logits
 constexpr size_t kSmemBytes = 1024 + 8 * kKVBlkBytes + 8 * kQBlkBytes + kRows * 128 +
-                              (4 * kH + 4 * kH) * 4 + 16 + 16 + 16 + kRows * 8 +
-                              16 + 16 + kMaxSplit * kH * 4 + kH * 4;
+                              (4 * kH + 4 * kH) * 4 + 16 + 4 * 8 + 8 + kRows * 8 + 16 +
+                              kMaxSplit * kH * 2 * 4 + kH * 4;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
 struct Plan {
   int nsplit, rps;   // splits per query and rows per split

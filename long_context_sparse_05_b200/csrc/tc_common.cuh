@@ -57,6 +57,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity) : "memory");
   return ok != 0;
 }
+// The same with a suspend-time hint: a thread parked in the wait re-checks the phase
+// at least every `hint_ns` nanoseconds.
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns) : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_hint(uint64_t* bar, uint32_t parity, int* err,
+                                               uint32_t hint_ns, uint64_t limit_ns = kWaitLimitNs) {
+  if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+    if (globaltimer() - t0 > limit_ns) {
+      atomicExch(err, CSA_ERR_TIMEOUT);
+      return false;
+    }
+  }
+}
 // Waits for the phase with the given parity; gives up after limit_ns, sets the
 // device error word *err and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err,

@@ -88,7 +88,8 @@ class DecodeState:
         self.out = torch.empty((w.b, w.H, w.c), dtype=dt, device=device)
         self.lse = torch.empty((w.b, w.H), dtype=torch.float32, device=device)
         self.ws_bytes = L.csa_decode_workspace_size(self.p)
-        self.ws = torch.empty((max(self.ws_bytes, 256),), dtype=torch.uint8, device=device)
+        # NaN bytes: a kernel that read workspace it had not written would show up
+        self.ws = torch.full((max(self.ws_bytes, 256),), 0xFF, dtype=torch.uint8, device=device)
 
     def build_caches(self, stream=None):
         w, x = self.w, self.x
@@ -137,7 +138,8 @@ class PrefillState:
         self.idx = torch.empty((w.b, w.n, w.k), dtype=torch.int32, device=device)
         self.count = torch.empty((w.b, w.n), dtype=torch.int32, device=device)
         self.ws_bytes = L.csa_prefill_workspace_size(self.p)
-        self.ws = torch.empty((max(self.ws_bytes, 256),), dtype=torch.uint8, device=device)
+        # NaN bytes: a kernel that read workspace it had not written would show up
+        self.ws = torch.full((max(self.ws_bytes, 256),), 0xFF, dtype=torch.uint8, device=device)
 
     def run(self, stream=None):
         x = self.x

@@ -67,7 +67,7 @@ def test_pool_topk_stage(fmt, H, d, T):
     pcnt[0, 0] = 50                               # fewer candidates than k
     p = L.IndexParams(H_I=H, d_I=d, m=m, qk_dtype=L.DTYPE[fmt], score_dtype=L.CSA_BF16)
     wsb = L.csa_pool_topk_workspace_size(p, b, T, P, k)
-    ws = torch.empty((wsb,), dtype=torch.uint8, device=DEV)
+    ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     idx = torch.empty((b, T, k), dtype=torch.int32, device=DEV)
     cnt = torch.empty((b, T), dtype=torch.int32, device=DEV)
     L.csa_pool_topk(p, _dev(x["q"]), _dev(x["qs"]), _dev(x["w"]), _dev(x["k"]), _dev(x["ks"]),

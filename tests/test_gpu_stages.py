@@ -271,7 +271,7 @@ def test_topk_1m_row():
     idx = torch.empty((1, 1, k), dtype=torch.int32, device=DEV)
     cnt = torch.empty((1, 1), dtype=torch.int32, device=DEV)
     wsb = L.csa_topk_workspace_size(L.CSA_BF16, 1, 1, E, k)
-    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    ws = torch.full((max(wsb, 256),), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_topk(st, L.CSA_BF16, qpos, m, 1, 1, E, k, idx, cnt, ws, wsb)
     torch.cuda.synchronize()
     ri, rc = csa.topk(f64(sc)[0], np.array([m * E - 1]), m, k)
@@ -292,7 +292,7 @@ def test_topk_chunked_rows_bit_exact(E, k, ties):
     idx = torch.empty((b, T, k), dtype=torch.int32, device=DEV)
     cnt = torch.empty((b, T), dtype=torch.int32, device=DEV)
     wsb = L.csa_topk_workspace_size(L.CSA_BF16, b, T, E, k)
-    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    ws = torch.full((max(wsb, 256),), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_topk(st, L.CSA_BF16, _dev(qpos), m, b, T, E, k, idx, cnt, ws, wsb)
     torch.cuda.synchronize()
     stored = f64(st)
@@ -346,7 +346,7 @@ def test_topk_cluster_rows_bit_exact(score, E, k, b):
     idx = torch.empty((b, 1, k), dtype=torch.int32, device=DEV)
     cnt = torch.empty((b, 1), dtype=torch.int32, device=DEV)
     wsb = L.csa_topk_workspace_size(L.DTYPE[score], b, 1, E, k)
-    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    ws = torch.full((max(wsb, 256),), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_topk(st, L.DTYPE[score], _dev(qpos), m, b, 1, E, k, idx, cnt, ws, wsb)
     torch.cuda.synchronize()
     stored = f64(st)
@@ -367,7 +367,7 @@ def test_topk_rows_beyond_a_cluster():
     cnt = torch.empty((b, 1), dtype=torch.int32, device=DEV)
     wsb = L.csa_topk_workspace_size(L.CSA_BF16, b, 1, E, k)
     assert wsb > 0
-    ws = torch.empty((wsb,), dtype=torch.uint8, device=DEV)
+    ws = torch.full((wsb,), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_topk(st, L.CSA_BF16, _dev(qpos), m, b, 1, E, k, idx, cnt, ws, wsb)
     torch.cuda.synchronize()
     stored = f64(st)
@@ -414,7 +414,7 @@ def test_sparse_attention(H, d, k, n_w, dtype, dense, T, E, n):
     p = L.AttnParams(H=H, d=d, n_w=n_w, scale=scale, m=c["m"], k=0 if dense else k,
                      dtype=L.DTYPE[dtype])
     wsb = L.csa_sparse_attn_workspace_size(p, b, T, E)
-    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    ws = torch.full((max(wsb, 256),), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_sparse_attn(p, c["q"], c["kv"], E, _dev(c["idx"]), _dev(c["cnt"]), c["win"], n,
                       _dev(c["qpos"]), c["sink"], b, T, out, lse, ws, wsb)
     torch.cuda.synchronize()
@@ -455,7 +455,7 @@ def test_attention_lazy_rescale_path(tile_of_spike):
     out = torch.empty((b, T, H, d), dtype=torch.bfloat16, device=DEV)
     p = L.AttnParams(H=H, d=d, n_w=n_w, scale=scale, m=c["m"], k=k, dtype=L.CSA_BF16)
     wsb = L.csa_sparse_attn_workspace_size(p, b, T, E)
-    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    ws = torch.full((max(wsb, 256),), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_sparse_attn(p, c["q"], c["kv"], E, _dev(c["idx"]), _dev(c["cnt"]), c["win"], n,
                       _dev(c["qpos"]), c["sink"], b, T, out, None, ws, wsb)
     torch.cuda.synchronize()

@@ -55,7 +55,7 @@ def _with_workspace(c):
     out = torch.empty((c["b"], 1, c["H"], c["d"]), dtype=torch.bfloat16, device=DEV)
     lse = torch.empty((c["b"], 1, c["H"]), dtype=torch.float32, device=DEV)
     wsb = L.csa_sparse_attn_workspace_size(c["p"], c["b"], 1, c["E"])
-    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device=DEV)
+    ws = torch.full((max(wsb, 256),), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_sparse_attn(c["p"], c["q"], c["kv"], c["E"], c["idx"], c["cnt"], c["win"], c["n"],
                       c["qpos"], c["sink"], c["b"], 1, out, lse, ws, wsb)
     return out, lse, wsb
