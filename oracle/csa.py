@@ -310,12 +310,47 @@ def window_rows(t, n_w):
     return np.arange(max(0, t - n_w + 1), t + 1)
 
 
-def sparse_attn(q, kv_comp, idx, cnt, kv_win, q_pos, sink, n_w, scale, m=None):
+def inverse_rope(o, t, d_rope, theta):
+    """Inverse RoPE on the last ``d_rope`` dims of every head's output, at query position t.
+
+    "DeepSeek V4 结构速览", section "CSA（c4a 路线）" (the last 64 output dims get
+    an inverse RoPE) and section "HCA（c128a 路线）" (the same there).  Read as
+    the rotation ``rope_partial`` applies at position t, undone: the pairs are
+    rotated by -t * theta^(-2j/d_rope).  The values (= keys) carry RoPE at their
+    entries' anchors p_s, so the output's rotary part becomes sum_s a_s R(p_s - t) v_s,
+    relative to the query.  o [H][d].
+    """
+    o = np.asarray(o, dtype=np.float64)
+    return rope_partial(o, np.full(o.shape[0], -float(t)), d_rope, theta)
+
+
+def grouped_out_proj(o, W):
+    """Grouped output projection: the H heads' outputs in g groups, each projected alone.
+
+    "DeepSeek-V4 技术解读", section 2.1 (分组输出投影: the output is split into g
+    groups that are projected separately, cutting the projection's cost g-fold).
+    Read as: o [T][H][d] -> group i = heads [i H/g, (i+1) H/g) concatenated
+    (H/g * d values); y[t, i] = W[i] @ group_i; the g results are concatenated.
+    W [g][d_g][H/g * d].  Returns y [T][g * d_g] in float64.
+    """
+    o = np.asarray(o, dtype=np.float64)
+    W = np.asarray(W, dtype=np.float64)
+    T, H, d = o.shape
+    g, d_g, K = W.shape
+    assert H % g == 0 and K == (H // g) * d
+    grouped = o.reshape(T, g, K)
+    y = np.einsum("tgk,gnk->tgn", grouped, W)
+    return y.reshape(T, g * d_g)
+
+
+def sparse_attn(q, kv_comp, idx, cnt, kv_win, q_pos, sink, n_w, scale, m=None, inv_rope=None):
     """CSA attention for T queries of one sequence.
 
     q [T][H][d]; kv_comp [E][d]; idx [T][k] / cnt [T] from ``topk`` (idx None
     means dense over all E(t) visible entries, the HCA case, which needs m);
-    kv_win [n][d] raw rows.  Returns (o [T][H][d], lse [T][H]) in float64.
+    kv_win [n][d] raw rows.  ``inv_rope`` = (d_rope, theta) applies ``inverse_rope``
+    to each query's output at its position.  Returns (o [T][H][d], lse [T][H]) in
+    float64.
     """
     q = np.asarray(q, dtype=np.float64)
     kv_comp = np.asarray(kv_comp, dtype=np.float64)
@@ -331,6 +366,8 @@ def sparse_attn(q, kv_comp, idx, cnt, kv_win, q_pos, sink, n_w, scale, m=None):
         rows = np.concatenate([kv_comp[sel],
                                np.asarray(kv_win[window_rows(t, n_w)], dtype=np.float64)], axis=0)
         o[r], lse[r] = attend(q[r], rows, sink, scale)
+        if inv_rope is not None:
+            o[r] = inverse_rope(o[r], t, inv_rope[0], inv_rope[1])
     return o, lse
 
 

@@ -49,14 +49,15 @@ def quantize_rows(x, idx_dtype):
 
 
 def csa_prefill(main, index, q, q_I, w, sink, *, m, d_rope, theta, eps, k, n_w, scale,
-                kv_dtype, idx_dtype, score_dtype, query_rows=None):
+                kv_dtype, idx_dtype, score_dtype, query_rows=None, inv_rope=False):
     """CSA prefill of one sequence: every token t = 0..n-1 is a query.
 
     main / index: dicts with C_a, Z_a, B_a, C_b, Z_b, B_b ([n][c], [m][c]).
     q [n][H][d]; q_I [n][H_I][d_I] (unquantised); w [n][H_I]; sink [H].
     The raw window rows are the main branch's C_a (the uncompressed latent).
     ``query_rows`` restricts the queries evaluated (all entries are still
-    compressed, as every query may select any visible entry).
+    compressed, as every query may select any visible entry).  ``inv_rope``
+    applies ``csa.inverse_rope`` (the last d_rope dims) to every output.
     Returns a dict of every intermediate.
     """
     n = main["C_a"].shape[0]
@@ -71,13 +72,14 @@ def csa_prefill(main, index, q, q_I, w, sink, *, m, d_rope, theta, eps, k, n_w, 
     qI_deq, _ = quantize_rows(q_I[rows], idx_dtype)
     scores = csa.index_scores(qI_deq, w[rows], kI_deq, rows, m, score_dtype)
     idx, cnt = csa.topk(scores, rows, m, k)
-    o, lse = csa.sparse_attn(q[rows], kv_st, idx, cnt, main["C_a"], rows, sink, n_w, scale)
+    o, lse = csa.sparse_attn(q[rows], kv_st, idx, cnt, main["C_a"], rows, sink, n_w, scale,
+                             inv_rope=(d_rope, theta) if inv_rope else None)
     return dict(kv=kv, kv_stored=kv_st, kI=kI, kI_deq=kI_deq, qI_deq=qI_deq, scores=scores,
                 idx=idx, cnt=cnt, out=round_out(o, kv_dtype), out_f64=o, lse=lse, rows=rows)
 
 
 def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k, n_w, scale,
-                   kv_dtype, idx_dtype, mode="full", idx_in=None, pool=None):
+                   kv_dtype, idx_dtype, mode="full", idx_in=None, pool=None, inv_rope=False):
     """One CSA decode step of one sequence with L tokens of context.
 
     The new token is t = L - 1; it completes block E - 1 (E = L / m), so the
@@ -95,6 +97,7 @@ def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k,
       "reindex" hierarchical indexer: only the entries of ``pool`` (entry ids,
                 -1 padded) are scored with this layer's q_I, and k kept
                 (``csa.pool_topk``).
+    ``inv_rope`` applies ``csa.inverse_rope`` (the last d_rope dims) to the output.
     """
     E = L // m
     t = L - 1
@@ -123,6 +126,8 @@ def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k,
     kv_sel_st = round_out(kv_sel, kv_dtype)
     rows = np.concatenate([kv_sel_st, np.asarray(main["C_a"][csa.window_rows(t, n_w)], dtype=np.float64)], axis=0)
     o, lse = csa.attend(np.asarray(q), rows, sink, scale)
+    if inv_rope:
+        o = csa.inverse_rope(o, t, d_rope, theta)
     new_entry = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
                                      main["B_b"], m, True, [E - 1], d_rope, theta, eps)[0]
     return dict(kI=kI, kI_deq=kI_deq, qI_deq=qI_deq, scores=scores[0], idx=idx[0], cnt=int(cnt[0]),
@@ -131,7 +136,7 @@ def csa_decode_seq(main, index, q, q_I, w, sink, *, L, m, d_rope, theta, eps, k,
 
 
 def hca_decode_seq(main, q, sink, *, L, m, d_rope, theta, eps, n_w, scale, kv_dtype,
-                   entries_needed=None):
+                   entries_needed=None, inv_rope=False):
     """One HCA decode step of one sequence: compress the completed block, attend densely.
 
     main holds C_a, Z_a, B_a (no previous-block branch in c128a).  The new
@@ -144,5 +149,7 @@ def hca_decode_seq(main, q, sink, *, L, m, d_rope, theta, eps, n_w, scale, kv_dt
     kv_st = round_out(kv, kv_dtype)
     rows = np.concatenate([kv_st, np.asarray(main["C_a"][csa.window_rows(t, n_w)], dtype=np.float64)], axis=0)
     o, lse = csa.attend(np.asarray(q), rows, sink, scale)
+    if inv_rope:
+        o = csa.inverse_rope(o, t, d_rope, theta)
     return dict(kv=kv, kv_stored=kv_st, new_entry=kv[E - 1], out=round_out(o, kv_dtype),
                 out_f64=o, lse=lse)
