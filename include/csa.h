@@ -288,6 +288,13 @@ typedef struct {
   int m;          /* compression rate (dense mode: E(t) = floor((t+1)/m)) */
   int k;          /* idx row length (ignored when idx == NULL) */
   int dtype;      /* CSA_F32 or CSA_BF16: q, kv_comp, kv_win and out */
+  int d_rope_out; /* inverse RoPE on the last d_rope_out dims of every head's output, at
+                     the query's position (even, <= d; 0 = none; the tensor-core path takes
+                     up to 64): "DeepSeek V4 结构速览", sections "CSA（c4a 路线）" and
+                     "HCA（c128a 路线）".  Each interleaved pair (o[d-r+2j], o[d-r+2j+1]) is
+                     rotated by -t * rope_theta^(-2j/d_rope_out), the angle formed in
+                     float64, undoing the rotation RoPE gives position t. */
+  double rope_theta;
 } csa_attn_params;
 
 /*
@@ -344,6 +351,28 @@ csa_status csa_sparse_attn_noalloc(const csa_attn_params* p, const void* q, cons
                                    cudaStream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Output epilogue: grouped output projection                                */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Source: "DeepSeek-V4 技术解读", section 2.1 (分组输出投影: the attention output is
+ * split into g groups, each projected on its own, which cuts the projection's work
+ * g-fold).  Group i holds heads [i*H/g, (i+1)*H/g), concatenated into K = H/g * d
+ * values; y[t][i*d_g + n] = sum_k o[t][i*K + k] * W[i][n][k] (float32 accumulation,
+ * bf16 result).
+ *   o   [T][H][d] bf16 (the attention output, inverse RoPE applied if wanted)
+ *   W   [g][d_g][K] bf16 (row n of group i's projection, K contiguous)
+ *   y   [T][g * d_g] bf16
+ *   ws  device scratch of csa_out_proj_workspace_size() bytes (non-zero only when a
+ *       few tokens leave SMs idle and the K dimension is split; NULL when 0)
+ * Requires H % g == 0, K a multiple of 64, d_g a multiple of 256, 16-byte aligned
+ * pointers; otherwise CSA_ERR_INVALID_ARG.
+ */
+size_t csa_out_proj_workspace_size(int T, int H, int d, int g, int d_g);
+csa_status csa_out_proj(const void* o, const void* W, int T, int H, int d, int g, int d_g,
+                        void* y, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Fused drivers                                                             */
 /* ------------------------------------------------------------------------ */
 
@@ -383,6 +412,7 @@ typedef struct {
   int E_cap;               /* entries each cache row-block holds (>= L/m) */
   int mode;                /* csa_decode_mode (CSA only; HCA takes CSA_MODE_FULL) */
   int P;                   /* CSA_MODE_REINDEX: pool row length */
+  int inv_rope;            /* 1: inverse RoPE on the last d_rope output dims (see csa_attn_params) */
 } csa_decode_params;
 
 typedef struct {
@@ -430,6 +460,7 @@ typedef struct {
   int kv_dtype;            /* CSA_BF16 or CSA_F32 */
   int idx_dtype;           /* CSA_FP8_E4M3, CSA_NVFP4 or CSA_F32 */
   int score_dtype;         /* CSA_BF16 or CSA_F32 */
+  int inv_rope;            /* 1: inverse RoPE on the last d_rope output dims (see csa_attn_params) */
 } csa_prefill_params;
 
 typedef struct {

@@ -38,7 +38,7 @@ class IndexParams(ctypes.Structure):
 
 class AttnParams(ctypes.Structure):
     _fields_ = [("H", c_int), ("d", c_int), ("n_w", c_int), ("scale", c_float), ("m", c_int),
-                ("k", c_int), ("dtype", c_int)]
+                ("k", c_int), ("dtype", c_int), ("d_rope_out", c_int), ("rope_theta", c_double)]
 
 
 class DecodeParams(ctypes.Structure):
@@ -46,7 +46,7 @@ class DecodeParams(ctypes.Structure):
                 ("c_I", c_int), ("H_I", c_int), ("d_rope", c_int), ("d_rope_I", c_int),
                 ("rope_theta", c_double), ("eps", c_float), ("k", c_int), ("n_w", c_int),
                 ("scale", c_float), ("kv_dtype", c_int), ("idx_dtype", c_int), ("hca", c_int),
-                ("E_cap", c_int), ("mode", c_int), ("P", c_int)]
+                ("E_cap", c_int), ("mode", c_int), ("P", c_int), ("inv_rope", c_int)]
 
 
 CSA_MODE_FULL, CSA_MODE_REUSE, CSA_MODE_REINDEX = 0, 1, 2
@@ -67,7 +67,7 @@ class PrefillParams(ctypes.Structure):
                 ("c_I", c_int), ("H_I", c_int), ("d_rope", c_int), ("d_rope_I", c_int),
                 ("rope_theta", c_double), ("eps", c_float), ("k", c_int), ("n_w", c_int),
                 ("scale", c_float), ("kv_dtype", c_int), ("idx_dtype", c_int),
-                ("score_dtype", c_int)]
+                ("score_dtype", c_int), ("inv_rope", c_int)]
 
 
 _PREFILL_TENSORS = ["C_a", "Z_a", "C_b", "Z_b", "B_a", "B_b", "CI_a", "ZI_a", "CI_b", "ZI_b",
@@ -99,6 +99,9 @@ _SIGS = {
                        c_void_p]),
     "csa_pool_topk_workspace_size": (c_size_t, [ctypes.POINTER(IndexParams), c_int, c_int, c_int,
                                                 c_int]),
+    "csa_out_proj": (c_int, [c_void_p, c_void_p] + [c_int] * 5 + [c_void_p, c_void_p, c_size_t,
+                                                                 c_void_p]),
+    "csa_out_proj_workspace_size": (c_size_t, [c_int] * 5),
     "csa_sparse_attn": (c_int, [ctypes.POINTER(AttnParams), c_void_p, c_void_p, c_int, c_void_p,
                                 c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_int, c_int,
                                 c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
@@ -212,6 +215,17 @@ def csa_pool_topk(p, q_I, q_scales, w, k_I, k_scales, q_pos, b, T, E_cap, E, poo
                                _ptr(k_scales), _ptr(q_pos), b, T, E_cap, E, _ptr(pool),
                                _ptr(pool_count), P, k, _ptr(idx), _ptr(count), _ptr(ws), ws_bytes,
                                _stream(stream)))
+
+
+def csa_out_proj_workspace_size(T, H, d, g, d_g):
+    return int(lib().csa_out_proj_workspace_size(T, H, d, g, d_g))
+
+
+def csa_out_proj(o, W, T, H, d, g, d_g, y, ws=None, ws_bytes=None, stream=None):
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size() if isinstance(ws, torch.Tensor) else 0
+    _check(lib().csa_out_proj(_ptr(o), _ptr(W), T, H, d, g, d_g, _ptr(y), _ptr(ws), ws_bytes,
+                              _stream(stream)))
 
 
 def csa_sparse_attn_workspace_size(p, b, T, E_cap):

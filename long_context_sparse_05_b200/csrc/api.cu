@@ -146,6 +146,8 @@ csa_status sparse_attn_impl(const csa_attn_params* p, const void* q, const void*
                             cudaStream_t stream, int pdl) {
   if (!p) return CSA_ERR_INVALID_ARG;
   if (p->H < 1 || p->d < 8 || p->d % 8 || p->n_w < 0 || p->m < 1) return CSA_ERR_INVALID_ARG;
+  if (p->d_rope_out < 0 || p->d_rope_out % 2 || p->d_rope_out > p->d) return CSA_ERR_INVALID_ARG;
+  if (p->d_rope_out > 0 && !(p->rope_theta > 0.0)) return CSA_ERR_INVALID_ARG;
   if (p->dtype != CSA_F32 && p->dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
   if (b < 0 || T < 0 || E_cap < 0 || n < 1) return CSA_ERR_INVALID_ARG;
   if (idx && (p->k < 1 || !count)) return CSA_ERR_INVALID_ARG;
@@ -158,6 +160,7 @@ csa_status sparse_attn_impl(const csa_attn_params* p, const void* q, const void*
   a.q = q; a.kv = kv_comp; a.idx = idx; a.count = count; a.win = kv_win; a.q_pos = q_pos;
   a.sink = sink; a.T = T; a.H = p->H; a.d = p->d; a.n_w = p->n_w; a.m = p->m; a.k = p->k;
   a.E_cap = E_cap; a.n = n; a.scale = p->scale; a.out = out; a.lse = lse; a.pdl = pdl;
+  a.d_rope_out = p->d_rope_out; a.theta = p->rope_theta;
   csa_status st = launch_attn_tc(a, b, p->dtype, ws, ws_bytes, stream);
   if (st != CSA_ERR_UNSUPPORTED) return st;
   return launch_attn_simt(a, b, p->dtype, stream);
@@ -282,6 +285,23 @@ csa_status csa_pool_topk(const csa_index_params* p, const void* q_I, const void*
 }
 
 // ---------------------------------------------------------------------------
+// grouped output projection
+// ---------------------------------------------------------------------------
+
+size_t csa_out_proj_workspace_size(int T, int H, int d, int g, int d_g) {
+  return out_proj_workspace_bytes(T, H, d, g, d_g);
+}
+
+csa_status csa_out_proj(const void* o, const void* W, int T, int H, int d, int g, int d_g,
+                        void* y, void* ws, size_t ws_bytes, cudaStream_t stream) {
+  if (T < 0 || H < 1 || d < 1 || g < 1 || d_g < 1) return CSA_ERR_INVALID_ARG;
+  if (!out_proj_supported(H, d, g, d_g)) return CSA_ERR_INVALID_ARG;
+  if (T == 0) return CSA_OK;
+  if (!o || !W || !y || !aligned16(o) || !aligned16(W) || !aligned16(y)) return CSA_ERR_INVALID_ARG;
+  return launch_out_proj(o, W, T, H, d, g, d_g, y, ws, ws_bytes, stream, false);
+}
+
+// ---------------------------------------------------------------------------
 // decode
 // ---------------------------------------------------------------------------
 
@@ -316,7 +336,8 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
       d.pool_ws = cv.take(d.pool_ws_bytes);
     }
   }
-  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype};
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype,
+                     p->inv_rope ? p->d_rope : 0, p->rope_theta};
   d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, b, 1, p->E_cap);
   d.attn_ws = cv.take(d.attn_ws_bytes);
   if (o) *o = d;
@@ -437,7 +458,8 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
     idx = io; cnt = co;
   }
   // 4. attention over the selection (or all entries) plus the window
-  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype};
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype,
+                     p->inv_rope ? p->d_rope : 0, p->rope_theta};
   return sparse_attn_impl(&ap, x->q, x->kv_cache, p->E_cap, idx, cnt, x->kv_win, p->L, d.qpos,
                           x->sink, b, 1, x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream, 1);
 }
@@ -469,7 +491,8 @@ size_t prefill_layout(const csa_prefill_params* p, void* ws, size_t cap, Prefill
   d.count = static_cast<int32_t*>(cv.take(rows * 4));
   d.topk_ws_bytes = topk_workspace_bytes((int)rows, E, p->k, p->score_dtype);
   d.topk_ws = cv.take(d.topk_ws_bytes);
-  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype};
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype,
+                     p->inv_rope ? p->d_rope : 0, p->rope_theta};
   d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, p->b, p->n, E);
   d.attn_ws = cv.take(d.attn_ws_bytes);
   if (o) *o = d;
@@ -529,7 +552,8 @@ csa_status csa_prefill(const csa_prefill_params* p, const csa_prefill_tensors* x
   st = topk_impl(d.scores, p->score_dtype, d.qpos, p->m, b, n, E, p->k, io, co, d.topk_ws,
                  d.topk_ws_bytes, stream, true);
   if (st) return st;
-  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype};
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->k, p->kv_dtype,
+                     p->inv_rope ? p->d_rope : 0, p->rope_theta};
   return sparse_attn_impl(&ap, x->q, x->kv_cache, E, io, co, x->kv_win, n, d.qpos, x->sink, b, n,
                           x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream, 1);
 }

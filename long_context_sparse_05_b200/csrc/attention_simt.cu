@@ -75,15 +75,28 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
     __syncthreads();
     const float inv = 1.f / den;
     T* oh = reinterpret_cast<T*>(a.out) + (qrow * a.H + h) * a.d;
-    for (int e = threadIdx.x; e < a.d; e += blockDim.x) {
-      float acc = 0.f;
+    // a thread per channel, or per rotary pair in the last d_rope_out channels (inverse
+    // RoPE at the query position)
+    const int base = a.d - a.d_rope_out;
+    for (int e = threadIdx.x; e < base + a.d_rope_out / 2; e += blockDim.x) {
+      const int c0 = e < base ? e : base + 2 * (e - base);
+      const int nc = e < base ? 1 : 2;
+      float acc[2] = {0.f, 0.f};
       for (int r = 0; r < R; ++r) {
         const int code = s_row[r];
         if (code == kSkipRow) continue;
         const T* row = code >= 0 ? kv + (size_t)code * a.d : win + (size_t)(-1 - code) * a.d;
-        acc = fmaf(s_l[r], to_f32(row[e]), acc);
+        for (int u = 0; u < nc; ++u) acc[u] = fmaf(s_l[r], to_f32(row[c0 + u]), acc[u]);
       }
-      oh[e] = from_f32<T>(acc * inv);
+      if (nc == 1) {
+        oh[c0] = from_f32<T>(acc[0] * inv);
+      } else {
+        float sn, cs;
+        rope_angle((double)t * pow(a.theta, -2.0 * (double)(e - base) / (double)a.d_rope_out), &sn, &cs);
+        const float x0 = acc[0] * inv, x1 = acc[1] * inv;
+        oh[c0] = from_f32<T>(inv_rope_elem(x0, x1, c0, a.d, a.d_rope_out, sn, cs));
+        oh[c0 + 1] = from_f32<T>(inv_rope_elem(x1, x0, c0 + 1, a.d, a.d_rope_out, sn, cs));
+      }
     }
     if (a.lse && threadIdx.x == 0) a.lse[qrow * a.H + h] = M + logf(den);
     __syncthreads();

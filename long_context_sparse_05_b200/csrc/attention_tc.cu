@@ -39,6 +39,7 @@
 #include "tc_common.cuh"
 
 #include <climits>
+#include <cmath>
 #include <mutex>
 
 namespace csa {
@@ -69,7 +70,17 @@ struct AttnTc {
                  // combines them
   uint8_t* part_bf;   // cluster mode: per item, the scaled O as bf16 [512][64] (swizzled rows)
   float scale_log2;
+  int d_rope_out;     // inverse RoPE on the last d_rope_out output dims at the query position
+  double inv_freq[kMaxOutRopePairs];   // theta^(-2j/d_rope_out)
 };
+
+// sin / cos of the inverse-RoPE angle of output dim d at position t (identity below the
+// rotary dims)
+__device__ __forceinline__ void out_rope_sincos(const AttnTc& p, int d, int t, float& sn, float& cs) {
+  sn = 0.f; cs = 1.f;
+  const int u = d - (kD - p.d_rope_out);
+  if (p.d_rope_out > 0 && u >= 0) rope_angle((double)t * p.inv_freq[u >> 1], &sn, &cs);
+}
 
 struct QInfo {
   int sb, t, nsel, w0, nrows;
@@ -260,6 +271,17 @@ __device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool writ
 #pragma unroll
       for (int u = 0; u < 4; ++u) acc[u] = fmaf(src[u * kH], w, acc[u]);
     }
+    if (p.d_rope_out > 0) {
+      const int t = query_info(p, qrow).t;
+#pragma unroll
+      for (int u = 0; u < 4; u += 2) {
+        float sn, cs;
+        out_rope_sincos(p, d0 + dd + u, t, sn, cs);
+        const float x0 = acc[u], x1 = acc[u + 1];
+        acc[u] = inv_rope_elem(x0, x1, d0 + dd + u, kD, p.d_rope_out, sn, cs);
+        acc[u + 1] = inv_rope_elem(x1, x0, d0 + dd + u + 1, kD, p.d_rope_out, sn, cs);
+      }
+    }
     __nv_bfloat162 lo = __floats2bfloat162_rn(acc[0], acc[1]);
     __nv_bfloat162 hi = __floats2bfloat162_rn(acc[2], acc[3]);
     uint2 u2;
@@ -318,6 +340,17 @@ __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int ite
         const __nv_bfloat162 b2 = *reinterpret_cast<const __nv_bfloat162*>(&q[e]);
         acc[2 * e] += __low2float(b2);
         acc[2 * e + 1] += __high2float(b2);
+      }
+    }
+    if (p.d_rope_out > 0) {
+      // dims d and d ^ 1 (a rotary pair) sit in lanes x and x ^ 1, both active
+      const unsigned mask = __activemask();
+      float sn, cs;
+      out_rope_sincos(p, d, query_info(p, qrow).t, sn, cs);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float y = __shfl_xor_sync(mask, acc[e], 1);
+        acc[e] = inv_rope_elem(acc[e], y, d, kD, p.d_rope_out, sn, cs);
       }
     }
     __nv_bfloat16* o = p.out + ((size_t)qrow * kH + 8 * c) * kD + d;
@@ -638,11 +671,19 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
           tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
           tc::tmem_ld_wait(o);
           const int d = mb * 128 + r;
+          // rotary output dims: the pair partner (dim d ^ 1) is in lane ^ 1; the condition
+          // is uniform over the warp's 32 dims when d_rope_out is a multiple of 32
+          const bool rot = p.d_rope_out > 0 && mb * 128 + qd * 32 + 31 >= kD - p.d_rope_out;
+          float sn, cs;
+          out_rope_sincos(p, d, Q.t, sn, cs);
 #pragma unroll
           for (int h = 0; h < 32; ++h) {
             const int hh = half * 32 + h;
-            const float val = ok ? __uint_as_float(o[h]) * s_inv[hh] : __int_as_float(0x7fc00000);
-            p.out[((size_t)qrow * kH + hh) * kD + d] = __float2bfloat16_rn(val);
+            float val = __uint_as_float(o[h]) * s_inv[hh];
+            if (rot) val = inv_rope_elem(val, __shfl_xor_sync(0xffffffffu, val, 1), d, kD,
+                                         p.d_rope_out, sn, cs);
+            p.out[((size_t)qrow * kH + hh) * kD + d] =
+                __float2bfloat16_rn(ok ? val : __int_as_float(0x7fc00000));
           }
         }
       }
@@ -828,6 +869,7 @@ size_t attn_tc_workspace_bytes(int H, int d, int k, int n_w, int b, int T, int E
 csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t ws_bytes,
                           cudaStream_t st) {
   if (!attn_tc_supported(a.H, a.d, dtype)) return CSA_ERR_UNSUPPORTED;
+  if (a.d_rope_out > 2 * kMaxOutRopePairs) return CSA_ERR_UNSUPPORTED;
   const bool dense = a.idx == nullptr;
   const int sms = sm_count();
   const Plan P = plan(dense ? 0 : a.k, a.n_w, b, a.T, a.E_cap, dense, sms);
@@ -844,6 +886,9 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
   p.rows_total = b * a.T; p.nsplit = P.nsplit; p.rps = P.rps; p.dense = dense ? 1 : 0;
   p.cluster = P.cluster;
   p.scale_log2 = a.scale * kLog2e;
+  p.d_rope_out = a.d_rope_out;
+  for (int j = 0; j < kMaxOutRopePairs; ++j)
+    p.inv_freq[j] = 2 * j < a.d_rope_out ? std::pow(a.theta, -2.0 * j / (double)a.d_rope_out) : 0.0;
   if (P.nsplit > 1 && P.cluster) {
     const size_t items = (size_t)b * a.T * P.nsplit;
     if (!ws || ws_bytes < items * kPartB || (reinterpret_cast<uintptr_t>(ws) & 15))

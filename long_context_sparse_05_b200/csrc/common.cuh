@@ -104,6 +104,27 @@ __host__ __device__ __forceinline__ size_t nvfp4_key_scale_seq_bytes(long long E
   return (size_t)((E_cap + 127) >> 7) * (size_t)(8 * c);
 }
 
+// Rotation angle p * inv_freq reduced to [-pi, pi] in float64 (Cody-Waite reduction
+// with 2*pi split into a head and a tail), then float32 sin / cos of the reduced angle.
+__device__ __forceinline__ void rope_angle(double ang, float* sn, float* cs) {
+  const double kTwoPiHi = 6.283185307179586;          // 2*pi rounded to float64
+  const double kTwoPiLo = 2.4492935982947064e-16;     // 2*pi - kTwoPiHi
+  const double k = rint(ang * (1.0 / 6.283185307179586));
+  double r = fma(-k, kTwoPiHi, ang);
+  r = fma(-k, kTwoPiLo, r);
+  sincosf((float)r, sn, cs);
+}
+
+// Inverse RoPE of one output element: dim d of a head whose last d_rope dims are rotary
+// (interleaved pairs), at query position t.  x is the element's value, y its pair
+// partner's; the pair is rotated by -t * inv_freq[j].
+__device__ __forceinline__ float inv_rope_elem(float x, float y, int d, int D, int d_rope,
+                                               float sn, float cs) {
+  const int u = d - (D - d_rope);
+  if (u < 0) return x;
+  return (u & 1) == 0 ? fmaf(x, cs, y * sn) : fmaf(x, cs, -y * sn);
+}
+
 // Visible entries of query position t: floor((t+1)/m), clamped to [0, E].
 __device__ __forceinline__ int visible_entries(int t, int m, int E) {
   int e = t < 0 ? 0 : (t + 1) / m;

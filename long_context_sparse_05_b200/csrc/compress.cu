@@ -45,17 +45,6 @@ __device__ __forceinline__ void load16(const InT* p, float* dst) {
 
 constexpr int kUnroll = 4;
 
-// Rotation angle p * inv_freq reduced to [-pi, pi] in float64 (Cody-Waite reduction
-// with 2*pi split into a head and a tail), then float32 sin / cos of the reduced angle.
-__device__ __forceinline__ void rope_angle(double ang, float* sn, float* cs) {
-  const double kTwoPiHi = 6.283185307179586;          // 2*pi rounded to float64
-  const double kTwoPiLo = 2.4492935982947064e-16;     // 2*pi - kTwoPiHi
-  const double k = rint(ang * (1.0 / 6.283185307179586));
-  double r = fma(-k, kTwoPiHi, ang);
-  r = fma(-k, kTwoPiLo, r);
-  sincosf((float)r, sn, cs);
-}
-
 // One compressed entry (entry i of sequence s) by the whole CTA; see compress_kernel.
 template <typename InT>
 __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int s, float* smem) {

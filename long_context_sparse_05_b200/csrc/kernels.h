@@ -43,7 +43,11 @@ struct AttnArgs {
   float scale;
   void* out; float* lse;
   int pdl;            // launch as a programmatic dependent of the preceding kernel
+  int d_rope_out;     // inverse RoPE on the last d_rope_out output dims (0: none)
+  double theta;       // its RoPE base
 };
+
+constexpr int kMaxOutRopePairs = 32;   // rotary pairs of the output with a host-built table
 
 csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry_count,
                            cudaStream_t st);
@@ -81,6 +85,13 @@ csa_status launch_pool_gather(int fmt, const int32_t* pool, const int32_t* pool_
                               cudaStream_t st, bool pdl);
 csa_status launch_pool_map(const void* ws, int fmt, int rows, int P, int d, int k, int32_t* idx,
                            const int32_t* count, cudaStream_t st, bool pdl);
+
+// Grouped output projection (tcgen05 bf16 GEMM per head group).
+bool out_proj_supported(int H, int d, int g, int d_g);
+size_t out_proj_workspace_bytes(int T, int H, int d, int g, int d_g);
+int out_proj_launch_count(int T, int H, int d, int g, int d_g);
+csa_status launch_out_proj(const void* o, const void* W, int T, int H, int d, int g, int d_g,
+                           void* y, void* ws, size_t ws_bytes, cudaStream_t st, bool pdl);
 
 // Small helpers.
 csa_status launch_fill_i32(int32_t* p, int count, int value, cudaStream_t st);

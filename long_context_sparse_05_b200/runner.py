@@ -48,14 +48,16 @@ def decode_params(w: Workload, E_cap=None):
                           d_rope=w.d_rope, d_rope_I=w.d_rope_I, rope_theta=w.theta, eps=w.eps,
                           k=max(w.k, 1), n_w=w.n_w, scale=w.scale, kv_dtype=L.DTYPE[w.dtype],
                           idx_dtype=L.DTYPE.get(w.idx_dtype, 0), hca=1 if hca else 0,
-                          E_cap=E_cap if E_cap is not None else w.E)
+                          E_cap=E_cap if E_cap is not None else w.E,
+                          inv_rope=1 if w.inv_rope else 0)
 
 
 def prefill_params(w: Workload):
     return L.PrefillParams(b=w.b, n=w.n, m=w.m, c=w.c, H=w.H, c_I=w.c_I, H_I=w.H_I,
                            d_rope=w.d_rope, d_rope_I=w.d_rope_I, rope_theta=w.theta, eps=w.eps,
                            k=w.k, n_w=w.n_w, scale=w.scale, kv_dtype=L.DTYPE[w.dtype],
-                           idx_dtype=L.DTYPE[w.idx_dtype], score_dtype=L.DTYPE[w.score_dtype])
+                           idx_dtype=L.DTYPE[w.idx_dtype], score_dtype=L.DTYPE[w.score_dtype],
+                           inv_rope=1 if w.inv_rope else 0)
 
 
 class DecodeState:

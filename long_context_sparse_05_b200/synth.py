@@ -24,7 +24,7 @@ import torch
 TENSOR_ID = {
     "C_a": 0, "Z_a": 1, "C_b": 2, "Z_b": 3, "B_a": 4, "B_b": 5,
     "CI_a": 6, "ZI_a": 7, "CI_b": 8, "ZI_b": 9, "BI_a": 10, "BI_b": 11,
-    "q": 12, "q_I": 13, "w": 14, "sink": 15,
+    "q": 12, "q_I": 13, "w": 14, "sink": 15, "W_o": 16,
 }
 
 _TORCH_DT = {"f32": torch.float32, "bf16": torch.bfloat16}

@@ -33,6 +33,7 @@ class Workload:
     score_dtype: str = "bf16"  # indexer score storage ("f32" | "bf16")
     w_div: float = 64.0  # indexer head weights ~ U(0,1) / w_div
     seed: int = 0
+    inv_rope: bool = False   # inverse RoPE on the last d_rope output dims
 
     @property
     def E(self):

@@ -55,8 +55,9 @@ def _check_attention(w, gpu_out, ref_out, same_sel, recheck, atol_bf16=2e-2):
             assert_abs_close(gpu_out, ref_out, 5e-2, "attention vs oracle selection")
 
 
-def test_tiny_prefill_f32_full():
-    w = workloads.TINY
+@pytest.mark.parametrize("inv_rope", [False, True])
+def test_tiny_prefill_f32_full(inv_rope):
+    w = workloads.shrink(workloads.TINY, inv_rope=inv_rope)
     inp = synth.make_inputs(w, device="cuda")
     st = runner.PrefillState(w, inp)
     st.run()
@@ -65,7 +66,8 @@ def test_tiny_prefill_f32_full():
     main, index = _branches(g)
     ref = pipeline.csa_prefill(main, index, g["q"], g["q_I"], g["w"], g["sink"], m=w.m,
                                d_rope=w.d_rope, theta=w.theta, eps=w.eps, k=w.k, n_w=w.n_w,
-                               scale=w.scale, kv_dtype="f32", idx_dtype="f32", score_dtype="f32")
+                               scale=w.scale, kv_dtype="f32", idx_dtype="f32", score_dtype="f32",
+                               inv_rope=w.inv_rope)
     assert_rel_close(f64(st.kv_cache[0]), ref["kv"], 1e-5, "kv cache")
     assert_rel_close(f64(st.kI_cache[0]), ref["kI"], 1e-5, "index keys")
     exact = csa.index_scores(ref["qI_deq"], g["w"], ref["kI_deq"], np.arange(w.n), w.m, "f64")
@@ -80,7 +82,8 @@ def test_tiny_prefill_f32_full():
 
         def recheck(t=t):
             o, _ = csa.sparse_attn(g["q"][t:t + 1], ref["kv_stored"], gi[t:t + 1], gc[t:t + 1],
-                                   g["C_a"], [t], g["sink"], w.n_w, w.scale)
+                                   g["C_a"], [t], g["sink"], w.n_w, w.scale,
+                                   inv_rope=(w.d_rope, w.theta) if w.inv_rope else None)
             return o[0]
         _check_attention(w, out[t], ref["out"][t], same, recheck)
     assert nd <= 2, nd
@@ -101,14 +104,14 @@ def _decode_case(w, seqs):
         if w.kind == "hca_decode":
             ref = pipeline.hca_decode_seq(main, q, g["sink"], L=w.n, m=w.m, d_rope=w.d_rope,
                                           theta=w.theta, eps=w.eps, n_w=w.n_w, scale=w.scale,
-                                          kv_dtype=w.dtype)
+                                          kv_dtype=w.dtype, inv_rope=w.inv_rope)
             assert_rel_close(f64(st.kv_cache[s]), ref["kv"], 2e-2, "hca cache (incl. new entry)")
             assert_abs_close(f64(st.out[s]), ref["out"], 2e-2, "hca attention")
             continue
         ref = pipeline.csa_decode_seq(main, index, q, g["q_I"][0], g["w"][0], g["sink"], L=w.n,
                                       m=w.m, d_rope=w.d_rope, theta=w.theta, eps=w.eps, k=w.k,
                                       n_w=w.n_w, scale=w.scale, kv_dtype=w.dtype,
-                                      idx_dtype=w.idx_dtype)
+                                      idx_dtype=w.idx_dtype, inv_rope=w.inv_rope)
         E = w.E
         assert_rel_close(f64(st.kv_cache[s, E - 1]), ref["new_entry"], 2e-2, "new latent entry")
         exact = csa.index_scores(ref["qI_deq"], g["w"][0][None], ref["kI_deq"], np.array([t]),
@@ -125,12 +128,15 @@ def _decode_case(w, seqs):
                                           w.theta, w.eps)
             rows = np.concatenate([pipeline.round_out(kv_sel, w.dtype),
                                    main["C_a"][csa.window_rows(t, w.n_w)]])
-            return csa.attend(q, rows, g["sink"], w.scale)[0]
+            o = csa.attend(q, rows, g["sink"], w.scale)[0]
+            return csa.inverse_rope(o, t, w.d_rope, w.theta) if w.inv_rope else o
         _check_attention(w, f64(st.out[s]), ref["out"], same, recheck)
 
 
-def test_csa_decode_fp8_small():
-    w = workloads.shrink(workloads.CSA_DECODE_64K, b=3, n=4100 - 4100 % 4)   # E = 1025: ragged tile
+@pytest.mark.parametrize("inv_rope", [False, True])
+def test_csa_decode_fp8_small(inv_rope):
+    w = workloads.shrink(workloads.CSA_DECODE_64K, b=3, n=4100 - 4100 % 4,   # E = 1025: ragged tile
+                         inv_rope=inv_rope)
     _decode_case(w, [0, 2])
 
 
@@ -139,8 +145,9 @@ def test_csa_decode_nvfp4_small():
     _decode_case(w, [1])
 
 
-def test_hca_decode_small():
-    w = workloads.shrink(workloads.HCA_DECODE_1M, b=2, n=128 * 70)
+@pytest.mark.parametrize("inv_rope", [False, True])
+def test_hca_decode_small(inv_rope):
+    w = workloads.shrink(workloads.HCA_DECODE_1M, b=2, n=128 * 70, inv_rope=inv_rope)
     _decode_case(w, [0, 1])
 
 

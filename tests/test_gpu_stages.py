@@ -399,20 +399,25 @@ def _attn_case(b, T, H, d, E, n, k, n_w, dtype, dense, seed):
     return dict(q=q, kv=kv, win=win, sink=sink, qpos=qpos, idx=idx_np, cnt=cnt_np, m=m, tdt=tdt)
 
 
-@pytest.mark.parametrize("H,d,k,n_w,dtype,dense,T,E,n", [
-    (64, 512, 512, 128, "bf16", False, 1, 1500, 6000),   # decode shape, ragged
-    (64, 512, 512, 128, "bf16", True, 1, 700, 2800),     # HCA-style dense, E(t) up to 700
-    (64, 512, 64, 128, "bf16", False, 9, 300, 1200),     # prefill shape, several queries
-    (4, 64, 16, 16, "f32", False, 40, 256, 1024),        # tiny fp32
+@pytest.mark.parametrize("H,d,k,n_w,dtype,dense,T,E,n,d_rope_out", [
+    (64, 512, 512, 128, "bf16", False, 1, 1500, 6000, 0),   # decode shape, ragged
+    (64, 512, 512, 128, "bf16", True, 1, 700, 2800, 0),     # HCA-style dense, E(t) up to 700
+    (64, 512, 64, 128, "bf16", False, 9, 300, 1200, 0),     # prefill shape, several queries
+    (4, 64, 16, 16, "f32", False, 40, 256, 1024, 0),        # tiny fp32
+    # inverse RoPE on the output's last dims: cluster merge, workspace merge, one split, SIMT
+    (64, 512, 512, 128, "bf16", False, 1, 1500, 6000, 64),
+    (64, 512, 512, 128, "bf16", True, 1, 700, 2800, 64),
+    (64, 512, 64, 128, "bf16", False, 9, 300, 1200, 64),
+    (4, 64, 16, 16, "f32", False, 40, 256, 1024, 16),
 ])
-def test_sparse_attention(H, d, k, n_w, dtype, dense, T, E, n):
+def test_sparse_attention(H, d, k, n_w, dtype, dense, T, E, n, d_rope_out):
     b = 2
     c = _attn_case(b, T, H, d, E, n, k, n_w, dtype, dense, 51)
     scale = 1.0 / math.sqrt(d)
     out = torch.empty((b, T, H, d), dtype=c["tdt"], device=DEV)
     lse = torch.empty((b, T, H), dtype=torch.float32, device=DEV)
     p = L.AttnParams(H=H, d=d, n_w=n_w, scale=scale, m=c["m"], k=0 if dense else k,
-                     dtype=L.DTYPE[dtype])
+                     dtype=L.DTYPE[dtype], d_rope_out=d_rope_out, rope_theta=1e4)
     wsb = L.csa_sparse_attn_workspace_size(p, b, T, E)
     ws = torch.full((max(wsb, 256),), 0xFF, dtype=torch.uint8, device=DEV)   # NaN bytes: no read before write
     L.csa_sparse_attn(p, c["q"], c["kv"], E, _dev(c["idx"]), _dev(c["cnt"]), c["win"], n,
@@ -421,7 +426,8 @@ def test_sparse_attention(H, d, k, n_w, dtype, dense, T, E, n):
     for s in range(b):
         o, l = csa.sparse_attn(f64(c["q"][s]), f64(c["kv"][s]),
                                None if dense else c["idx"][s], None if dense else c["cnt"][s],
-                               f64(c["win"][s]), c["qpos"][s], f64(c["sink"]), n_w, scale, m=c["m"])
+                               f64(c["win"][s]), c["qpos"][s], f64(c["sink"]), n_w, scale, m=c["m"],
+                               inv_rope=(d_rope_out, 1e4) if d_rope_out else None)
         if dtype == "bf16":
             assert_abs_close(f64(out[s]), o, 2e-2, "attention bf16")
         else:
