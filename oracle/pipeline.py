@@ -153,3 +153,63 @@ def hca_decode_seq(main, q, sink, *, L, m, d_rope, theta, eps, n_w, scale, kv_dt
         o = csa.inverse_rope(o, t, d_rope, theta)
     return dict(kv=kv, kv_stored=kv_st, new_entry=kv[E - 1], out=round_out(o, kv_dtype),
                 out_f64=o, lse=lse)
+
+
+def csa_decode_at(main, index, q, q_I, w, sink, *, t, m, d_rope, theta, eps, k, n_w, scale,
+                  kv_dtype, idx_dtype, inv_rope=False):
+    """One CSA decode step of a sequence whose newest token sits at any position t.
+
+    Variable-length batched decode ("DeepSeek-V4技术报告解读", section 3.2, the
+    heterogeneous KV cache: compressed blocks plus a per-request state of the
+    window and the not yet compressed tail) serves sequences at any t.  Token t
+    completes entry (t+1)/m - 1 when (t+1) % m == 0; in any case the query sees
+    the E(t) = floor((t+1)/m) entries whose blocks have ended, and the window
+    max(0, t-n_w+1)..t.  Rows after t are never read.  q [H][d]; q_I [H_I][d_I];
+    w [H_I].
+    """
+    Et = (t + 1) // m
+    qI_deq, _ = quantize_rows(np.asarray(q_I)[None], idx_dtype)
+    if Et > 0:
+        kI = csa.compress_range(index["C_a"], index["Z_a"], index["B_a"], index["C_b"],
+                                index["Z_b"], index["B_b"], m, True, 0, Et, d_rope, theta, eps,
+                                chunk_rows=1 << 16)
+        kI_deq, _ = quantize_rows(kI, idx_dtype)
+        scores = csa.index_scores(qI_deq, np.asarray(w)[None], kI_deq, np.array([t]), m, "bf16")
+        idx, cnt = csa.topk(scores, np.array([t]), m, k)
+    else:
+        kI = np.zeros((0, np.asarray(q_I).shape[-1]))
+        scores = np.zeros((1, 0))
+        idx, cnt = np.full((1, k), -1, dtype=np.int32), np.zeros(1, dtype=np.int32)
+    sel = idx[0, :cnt[0]].astype(np.int64)
+    kv_sel = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"], main["Z_b"],
+                                  main["B_b"], m, True, sel, d_rope, theta, eps)
+    rows = np.concatenate([round_out(kv_sel, kv_dtype).reshape(-1, np.asarray(q).shape[-1]),
+                           np.asarray(main["C_a"][csa.window_rows(t, n_w)], dtype=np.float64)], axis=0)
+    o, lse = csa.attend(np.asarray(q), rows, sink, scale)
+    if inv_rope:
+        o = csa.inverse_rope(o, t, d_rope, theta)
+    completes = (t + 1) % m == 0
+    new_entry = None
+    if completes:
+        new_entry = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], main["C_b"],
+                                         main["Z_b"], main["B_b"], m, True, [Et - 1], d_rope,
+                                         theta, eps)[0]
+    return dict(kI=kI, scores=scores[0], idx=idx[0], cnt=int(cnt[0]), new_entry=new_entry,
+                out=round_out(o, kv_dtype), out_f64=o, lse=lse)
+
+
+def hca_decode_at(main, q, sink, *, t, m, d_rope, theta, eps, n_w, scale, kv_dtype,
+                  inv_rope=False):
+    """One HCA decode step of a sequence whose newest token sits at any position t: dense
+    over the E(t) = floor((t+1)/m) completed entries plus the window."""
+    Et = (t + 1) // m
+    c = np.asarray(q).shape[-1]
+    kv = csa.compress_range(main["C_a"], main["Z_a"], main["B_a"], None, None, None, m, False,
+                            0, Et, d_rope, theta, eps, chunk_rows=1 << 16) if Et else np.zeros((0, c))
+    rows = np.concatenate([round_out(kv, kv_dtype).reshape(-1, c),
+                           np.asarray(main["C_a"][csa.window_rows(t, n_w)], dtype=np.float64)], axis=0)
+    o, lse = csa.attend(np.asarray(q), rows, sink, scale)
+    if inv_rope:
+        o = csa.inverse_rope(o, t, d_rope, theta)
+    new_entry = kv[Et - 1] if (t + 1) % m == 0 and Et else None
+    return dict(kv=kv, new_entry=new_entry, out=round_out(o, kv_dtype), out_f64=o, lse=lse)

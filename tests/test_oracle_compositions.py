@@ -208,3 +208,67 @@ def test_csa_pin_rejects_planted_mistakes(old, new):
     bad = mutant(pipeline.csa_decode_seq, old, new)
     with pytest.raises(Exception):
         csa_pin(bad)
+
+
+# ---------------------------------------------------------------------------
+# decode at any position (variable-length batches, paged state)
+# ---------------------------------------------------------------------------
+
+def _rand_inputs(n, c, cI, H, HI, m, seed):
+    rng = np.random.default_rng(seed)
+    br = lambda cc: dict(C_a=rng.normal(size=(n, cc)), Z_a=rng.normal(size=(n, cc)),  # noqa: E731
+                         B_a=rng.normal(0, 0.5, (m, cc)), C_b=rng.normal(size=(n, cc)),
+                         Z_b=rng.normal(size=(n, cc)), B_b=rng.normal(0, 0.5, (m, cc)))
+    return (br(c), br(cI), rng.normal(size=(n, H, c)), rng.normal(size=(n, HI, cI)),
+            rng.uniform(size=(n, HI)) / 4, rng.normal(size=H))
+
+
+def test_decode_at_any_position_equals_the_prefill_row():
+    n, m, c, cI, H, HI = 96, 4, 16, 8, 2, 2
+    main, index, q, qI, w, sink = _rand_inputs(n, c, cI, H, HI, m, 21)
+    kw = dict(m=m, d_rope=4, theta=1e4, eps=1e-6, k=5, n_w=6, scale=0.25, kv_dtype="f32",
+              idx_dtype="fp8")
+    pre = pipeline.csa_prefill(main, index, q, qI, w, sink, score_dtype="bf16", **kw)
+    for t in (0, 1, 2, 3, 4, 5, 22, 23, 24, 37, 63, 94, 95):
+        d = pipeline.csa_decode_at(main, index, q[t], qI[t], w[t], sink, t=t, **kw)
+        np.testing.assert_array_equal(d["idx"], pre["idx"][t])
+        np.testing.assert_allclose(d["out_f64"], pre["out_f64"][t], rtol=1e-12, atol=1e-14)
+        if (t + 1) % m == 0:
+            np.testing.assert_allclose(d["new_entry"], pre["kv"][(t + 1) // m - 1], rtol=1e-13)
+        else:
+            assert d["new_entry"] is None
+    # the block-completing last token is the whole-sequence decode step
+    L = n
+    full = pipeline.csa_decode_seq(main, index, q[L - 1], qI[L - 1], w[L - 1], sink, L=L, **kw)
+    at = pipeline.csa_decode_at(main, index, q[L - 1], qI[L - 1], w[L - 1], sink, t=L - 1, **kw)
+    np.testing.assert_allclose(at["out_f64"], full["out_f64"], rtol=1e-13)
+
+
+def test_decode_at_reads_nothing_after_t():
+    n, m, c, cI, H, HI = 64, 4, 8, 8, 2, 1
+    main, index, q, qI, w, sink = _rand_inputs(n, c, cI, H, HI, m, 22)
+    kw = dict(m=m, d_rope=2, theta=1e4, eps=1e-6, k=3, n_w=4, scale=0.3, kv_dtype="f32",
+              idx_dtype="f32")
+    t = 29
+    a = pipeline.csa_decode_at(main, index, q[t], qI[t], w[t], sink, t=t, **kw)
+    for br in (main, index):
+        for name in ("C_a", "Z_a", "C_b", "Z_b"):
+            br[name][t + 1:] = 1e3
+    b = pipeline.csa_decode_at(main, index, q[t], qI[t], w[t], sink, t=t, **kw)
+    np.testing.assert_array_equal(a["out_f64"], b["out_f64"])
+
+
+def test_hca_decode_at_any_position():
+    n, m, c, H = 4 * 16, 16, 8, 2
+    main, _, q, _, _, sink = _rand_inputs(n, c, 8, H, 1, m, 23)
+    kw = dict(m=m, d_rope=2, theta=1e4, eps=0.0, n_w=5, scale=0.3, kv_dtype="f32")
+    kv_all = csa.compress_entries(main["C_a"], main["Z_a"], main["B_a"], None, None, None, m, False,
+                                  np.arange(n // m), 2, 1e4, 0.0)
+    for t in (0, 14, 15, 16, 40, 63):
+        r = pipeline.hca_decode_at(main, q[t], sink, t=t, **kw)
+        o, _ = csa.dense_attn(q[t:t + 1], pipeline.round_out(kv_all, "f32"), main["C_a"], [t],
+                              sink, 5, 0.3, m)
+        np.testing.assert_allclose(r["out_f64"], o[0], rtol=1e-12, atol=1e-14)
+    full = pipeline.hca_decode_seq(main, q[n - 1], sink, L=n, **kw)
+    np.testing.assert_allclose(pipeline.hca_decode_at(main, q[n - 1], sink, t=n - 1, **kw)["out_f64"],
+                               full["out_f64"], rtol=1e-13)
