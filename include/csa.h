@@ -447,6 +447,77 @@ size_t csa_decode_workspace_size(const csa_decode_params* p);
 int csa_decode_launch_count(const csa_decode_params* p);
 
 /*
+ * Paged decode step for b sequences at any positions: the heterogeneous KV cache of
+ * "DeepSeek-V4技术报告解读", section 3.2 (异构 KV 缓存管理): a classical cache of
+ * fixed-size blocks of compressed entries per request, and a fixed-size state per
+ * request holding the sliding window and the raw rows not yet compressed.
+ *
+ * Classical cache: pages of CSA_PAGE_ENTRIES compressed entries (latent rows, index-key
+ * codes and scales share the page ids).  Entry e of sequence s lives in page
+ * block_table[s][e / CSA_PAGE_ENTRIES], row e % CSA_PAGE_ENTRIES:
+ *   kv_pages   [num_pages][CSA_PAGE_ENTRIES][c] kv_dtype
+ *   kI_pages   [num_pages][CSA_PAGE_ENTRIES][row] idx_dtype codes
+ *   kI_scales  FP8: float32 [num_pages][CSA_PAGE_ENTRIES]; NVFP4: the tiled key-scale
+ *              layout over num_pages * CSA_PAGE_ENTRIES entries (two tiles per page)
+ * (The pages speak of blocks covering 128 raw tokens; here a block is the
+ * tensor-core indexer's 256-entry stage, so that a stage is one page.)
+ * State (per sequence, fixed size, updated in place by every step):
+ *   win                    [b][n_w][c]: raw window row of token u at slot u % n_w
+ *   tail_C_a, tail_Z_a, ... [b][R][c]: raw rows of token u at slot u % R, R = 2m for
+ *                          c4a (the previous block joins), m for c128a; tail_CI_* the
+ *                          index branch [b][2m][c_I]
+ * Step inputs: pos[s] = t, the new token's position (any t, sequences may differ);
+ * the new token's raw rows new_* ([b][c] or [b][c_I]) and its window row new_win;
+ * q, q_I, w, sink as in csa_decode.  The step appends the new rows to the state, and
+ * for every sequence whose block the token completes ((t+1) % m == 0) compresses entry
+ * (t+1)/m - 1 into its page (the page must be in the block table).  It then scores
+ * the E(t) = floor((t+1)/m) visible entries, selects k (CSA) or takes all (HCA), and
+ * attends over them plus the window max(0, t-n_w+1)..t.  L_max bounds t + 1 over the
+ * batch (entries scored per sequence: floor(L_max / m)).  Page ids outside
+ * [0, num_pages) are read as page 0 by the indexer and skipped by the attention.
+ * The CSA index path must be FP8 or NVFP4 (tensor-core indexers); HCA has none.
+ */
+#define CSA_PAGE_ENTRIES 256
+typedef struct {
+  int b, m, c, H, c_I, H_I, d_rope, d_rope_I;
+  double rope_theta;
+  float eps;
+  int k, n_w;
+  float scale;
+  int kv_dtype, idx_dtype, hca;
+  int max_pages;      /* block-table row length */
+  int num_pages;      /* pages in kv_pages / kI_pages */
+  int L_max;          /* upper bound of pos[s] + 1 over the batch */
+  int inv_rope;       /* 1: inverse RoPE on the last d_rope output dims */
+} csa_paged_params;
+
+typedef struct {
+  void *kv_pages, *kI_pages, *kI_scales;
+  const int32_t* block_table;                        /* [b][max_pages] */
+  void* win;                                         /* [b][n_w][c] */
+  void *tail_C_a, *tail_Z_a, *tail_C_b, *tail_Z_b;   /* [b][R][c]; _b NULL for HCA */
+  void *tail_CI_a, *tail_ZI_a, *tail_CI_b, *tail_ZI_b; /* [b][2m][c_I] (CSA) */
+  const int32_t* pos;                                /* [b] */
+  const void *new_C_a, *new_Z_a, *new_C_b, *new_Z_b; /* [b][c] */
+  const void *new_CI_a, *new_ZI_a, *new_CI_b, *new_ZI_b; /* [b][c_I] (CSA) */
+  const void* new_win;                               /* [b][c] */
+  const float *B_a, *B_b, *BI_a, *BI_b;              /* [m][c], [m][c_I] */
+  const void* q;                                     /* [b][H][c] */
+  const void* q_I;                                   /* [b][H_I][c_I] (CSA) */
+  const float* w;                                    /* [b][H_I] (CSA) */
+  const float* sink;                                 /* [H] */
+  void* out;                                         /* [b][H][c] */
+  float* lse;                                        /* [b][H] or NULL */
+  int32_t* idx_out;                                  /* [b][k] or NULL (CSA) */
+  int32_t* count_out;                                /* [b] or NULL (CSA) */
+} csa_paged_tensors;
+
+csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* x, void* ws,
+                            size_t ws_bytes, cudaStream_t stream);
+size_t csa_decode_paged_workspace_size(const csa_paged_params* p);
+int csa_decode_paged_launch_count(const csa_paged_params* p);
+
+/*
  * CSA prefill of b sequences of n tokens; every token t = 0..n-1 is a query.
  * Compresses all E = n/m entries (latent and index branch) into the caches,
  * quantises q_I, scores every (t, s) pair, selects k per query and attends.

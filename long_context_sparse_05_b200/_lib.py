@@ -62,6 +62,28 @@ class DecodeTensors(ctypes.Structure):
     _fields_ = [(n, c_void_p) for n in _DECODE_TENSORS]
 
 
+class PagedParams(ctypes.Structure):
+    _fields_ = [("b", c_int), ("m", c_int), ("c", c_int), ("H", c_int), ("c_I", c_int),
+                ("H_I", c_int), ("d_rope", c_int), ("d_rope_I", c_int), ("rope_theta", c_double),
+                ("eps", c_float), ("k", c_int), ("n_w", c_int), ("scale", c_float),
+                ("kv_dtype", c_int), ("idx_dtype", c_int), ("hca", c_int), ("max_pages", c_int),
+                ("num_pages", c_int), ("L_max", c_int), ("inv_rope", c_int)]
+
+
+_PAGED_TENSORS = ["kv_pages", "kI_pages", "kI_scales", "block_table", "win", "tail_C_a",
+                  "tail_Z_a", "tail_C_b", "tail_Z_b", "tail_CI_a", "tail_ZI_a", "tail_CI_b",
+                  "tail_ZI_b", "pos", "new_C_a", "new_Z_a", "new_C_b", "new_Z_b", "new_CI_a",
+                  "new_ZI_a", "new_CI_b", "new_ZI_b", "new_win", "B_a", "B_b", "BI_a", "BI_b",
+                  "q", "q_I", "w", "sink", "out", "lse", "idx_out", "count_out"]
+
+
+class PagedTensors(ctypes.Structure):
+    _fields_ = [(n, c_void_p) for n in _PAGED_TENSORS]
+
+
+PAGE_ENTRIES = 256
+
+
 class PrefillParams(ctypes.Structure):
     _fields_ = [("b", c_int), ("n", c_int), ("m", c_int), ("c", c_int), ("H", c_int),
                 ("c_I", c_int), ("H_I", c_int), ("d_rope", c_int), ("d_rope_I", c_int),
@@ -116,6 +138,10 @@ _SIGS = {
                             c_void_p, c_size_t, c_void_p]),
     "csa_prefill_workspace_size": (c_size_t, [ctypes.POINTER(PrefillParams)]),
     "csa_decode_launch_count": (c_int, [ctypes.POINTER(DecodeParams)]),
+    "csa_decode_paged": (c_int, [ctypes.POINTER(PagedParams), ctypes.POINTER(PagedTensors),
+                                 c_void_p, c_size_t, c_void_p]),
+    "csa_decode_paged_workspace_size": (c_size_t, [ctypes.POINTER(PagedParams)]),
+    "csa_decode_paged_launch_count": (c_int, [ctypes.POINTER(PagedParams)]),
     "csa_prefill_launch_count": (c_int, [ctypes.POINTER(PrefillParams)]),
 }
 
@@ -290,3 +316,20 @@ def csa_decode_launch_count(p):
 
 def csa_prefill_launch_count(p):
     return int(lib().csa_prefill_launch_count(ctypes.byref(p)))
+
+
+def csa_decode_paged_workspace_size(p):
+    return int(lib().csa_decode_paged_workspace_size(ctypes.byref(p)))
+
+
+def csa_decode_paged_launch_count(p):
+    return int(lib().csa_decode_paged_launch_count(ctypes.byref(p)))
+
+
+def csa_decode_paged(p, tensors, ws, ws_bytes=None, stream=None):
+    """tensors: dict with the csa_paged_tensors field names (missing -> NULL)."""
+    x = _fill(PagedTensors, _PAGED_TENSORS, tensors)
+    if ws_bytes is None:
+        ws_bytes = ws.numel() * ws.element_size()
+    _check(lib().csa_decode_paged(ctypes.byref(p), ctypes.byref(x), _ptr(ws), ws_bytes,
+                                  _stream(stream)))

@@ -1,5 +1,6 @@
 // Host side of the C ABI declared in include/csa.h: argument checks, kernel
 // selection, launches, and the fused decode / prefill drivers.
+#include <algorithm>
 #include <cstring>
 
 #include "common.cuh"
@@ -462,6 +463,170 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
                      p->inv_rope ? p->d_rope : 0, p->rope_theta};
   return sparse_attn_impl(&ap, x->q, x->kv_cache, p->E_cap, idx, cnt, x->kv_win, p->L, d.qpos,
                           x->sink, b, 1, x->out, x->lse, d.attn_ws, d.attn_ws_bytes, stream, 1);
+}
+
+// ---------------------------------------------------------------------------
+// paged decode: classical paged caches + per-sequence state, any positions
+// ---------------------------------------------------------------------------
+
+namespace {
+
+struct PagedWs {
+  void* qI_codes; void* qI_scales; void* scores; int32_t* idx; int32_t* count; int32_t* qpos;
+  void* attn_ws; size_t attn_ws_bytes; void* topk_ws; size_t topk_ws_bytes;
+};
+
+size_t paged_layout(const csa_paged_params* p, void* ws, size_t cap, PagedWs* o) {
+  Carve cv(ws, cap);
+  PagedWs d{};
+  const int b = p->b;
+  const int E = p->L_max / p->m;
+  d.qpos = static_cast<int32_t*>(cv.take((size_t)b * 4));
+  if (!p->hca) {
+    if (p->idx_dtype != CSA_F32) {
+      d.qI_codes = cv.take((size_t)b * p->H_I * dtype_row_bytes(p->idx_dtype, p->c_I));
+      d.qI_scales = cv.take(p->idx_dtype == CSA_FP8_E4M3 ? (size_t)b * p->H_I * 4
+                                                          : (size_t)b * p->H_I * (p->c_I / 16));
+    }
+    d.idx = static_cast<int32_t*>(cv.take((size_t)b * p->k * 4));
+    d.count = static_cast<int32_t*>(cv.take((size_t)b * 4));
+    d.scores = cv.take((size_t)b * std::max(E, 1) * 2);
+    d.topk_ws_bytes = topk_workspace_bytes(b, E, p->k, CSA_BF16);
+    d.topk_ws = cv.take(d.topk_ws_bytes);
+  }
+  csa_attn_params ap{p->H, p->c, p->n_w, p->scale, p->m, p->hca ? 0 : p->k, p->kv_dtype,
+                     p->inv_rope ? p->d_rope : 0, p->rope_theta};
+  d.attn_ws_bytes = csa_sparse_attn_workspace_size(&ap, b, 1, p->max_pages * kPageEntries);
+  d.attn_ws = cv.take(d.attn_ws_bytes);
+  if (o) *o = d;
+  return cv.ok ? align256(cv.used) : 0;
+}
+
+}  // namespace
+
+size_t csa_decode_paged_workspace_size(const csa_paged_params* p) {
+  if (!p || p->b <= 0 || p->m < 1) return 0;
+  return paged_layout(p, nullptr, 0, nullptr);
+}
+
+int csa_decode_paged_launch_count(const csa_paged_params* p) {
+  if (!p || p->b <= 0 || p->m < 1) return 0;
+  int n = 1;
+  if (!p->hca) n += 1 + (topk_workspace_bytes(p->b, p->L_max / p->m, p->k, CSA_BF16) ? 2 : 1);
+  n += attn_launch_count(p->H, p->c, p->hca ? 0 : p->k, p->n_w, p->b, 1,
+                         p->max_pages * kPageEntries, p->kv_dtype);
+  return n;
+}
+
+csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* x, void* ws,
+                            size_t ws_bytes, cudaStream_t stream) {
+  if (!p || !x) return CSA_ERR_INVALID_ARG;
+  if (p->b < 0 || p->m < 1 || p->L_max < 1 || p->max_pages < 1 || p->num_pages < 1 || p->n_w < 1)
+    return CSA_ERR_INVALID_ARG;
+  if ((long long)p->max_pages * kPageEntries * p->m < p->L_max) return CSA_ERR_INVALID_ARG;
+  if (p->kv_dtype != CSA_BF16 && p->kv_dtype != CSA_F32) return CSA_ERR_INVALID_ARG;
+  if (p->c < 8 || p->c % 8 || p->d_rope < 0 || p->d_rope % 2 || p->d_rope > p->c)
+    return CSA_ERR_INVALID_ARG;
+  if (!p->hca && (p->k < 1 || p->c_I < 16 || p->c_I % 16 || p->H_I < 1 || p->d_rope_I < 0 ||
+                  p->d_rope_I % 2 || p->d_rope_I > p->c_I))
+    return CSA_ERR_INVALID_ARG;
+  if (!p->hca && p->idx_dtype != CSA_FP8_E4M3 && p->idx_dtype != CSA_NVFP4)
+    return CSA_ERR_UNSUPPORTED;   // the paged key cache is read by the tensor-core indexers
+  if (!p->hca && p->idx_dtype == CSA_NVFP4 && p->c_I % 64) return CSA_ERR_INVALID_ARG;
+  if (p->b == 0) return CSA_OK;
+  PagedWs d{};
+  if (paged_layout(p, ws, ws_bytes, &d) == 0 || !ws || ws_bytes < csa_decode_paged_workspace_size(p))
+    return CSA_ERR_INVALID_ARG;
+  if (!x->kv_pages || !x->block_table || !x->win || !x->tail_C_a || !x->tail_Z_a || !x->pos ||
+      !x->new_C_a || !x->new_Z_a || !x->new_win || !x->B_a || !x->q || !x->sink || !x->out)
+    return CSA_ERR_INVALID_ARG;
+  if (!p->hca && (!x->tail_C_b || !x->tail_Z_b || !x->new_C_b || !x->new_Z_b || !x->B_b ||
+                  !x->kI_pages || !x->kI_scales || !x->tail_CI_a || !x->tail_ZI_a ||
+                  !x->tail_CI_b || !x->tail_ZI_b || !x->new_CI_a || !x->new_ZI_a ||
+                  !x->new_CI_b || !x->new_ZI_b || !x->BI_a || !x->BI_b || !x->q_I || !x->w))
+    return CSA_ERR_INVALID_ARG;
+  const void* ptrs16[] = {x->kv_pages, x->win, x->tail_C_a, x->tail_Z_a, x->new_C_a, x->new_Z_a,
+                          x->new_win, x->q, x->out};
+  for (const void* q : ptrs16)
+    if (!aligned16(q)) return CSA_ERR_INVALID_ARG;
+  if (!p->hca) {
+    const void* more[] = {x->tail_C_b, x->tail_Z_b, x->new_C_b, x->new_Z_b, x->kI_pages,
+                          x->kI_scales, x->tail_CI_a, x->tail_ZI_a, x->tail_CI_b, x->tail_ZI_b,
+                          x->new_CI_a, x->new_ZI_a, x->new_CI_b, x->new_ZI_b};
+    for (const void* q : more)
+      if (!aligned16(q)) return CSA_ERR_INVALID_ARG;
+  }
+  const int b = p->b;
+  const int E = p->L_max / p->m;
+  const int ring = p->hca ? p->m : 2 * p->m;
+  const size_t eb = p->kv_dtype == CSA_F32 ? 4 : 2;
+  if ((size_t)p->c * eb % 16 || (!p->hca && (size_t)p->c_I * eb % 16)) return CSA_ERR_INVALID_ARG;
+
+  // 1. prologue: append the new token's rows to the state, compress the entries the new
+  //    tokens complete into their pages, quantise the index queries, copy the positions
+  PrologueArgs pa{};
+  CompressArgs& mc = pa.main;
+  mc.C_a = x->tail_C_a; mc.Z_a = x->tail_Z_a; mc.B_a = x->B_a;
+  mc.C_b = x->tail_C_b; mc.Z_b = x->tail_Z_b; mc.B_b = x->B_b;
+  mc.n = ring; mc.m = p->m; mc.overlap = p->hca ? 0 : 1; mc.c = p->c; mc.d_rope = p->d_rope;
+  mc.apply_norm = 1; mc.out_dtype = p->kv_dtype; mc.entry_begin = 0;
+  mc.out_E = p->max_pages * kPageEntries; mc.theta = p->rope_theta; mc.eps = p->eps;
+  mc.out = x->kv_pages; mc.out_scales = nullptr;
+  mc.ring = ring; mc.pos = x->pos;
+  mc.new_C_a = x->new_C_a; mc.new_Z_a = x->new_Z_a; mc.new_C_b = x->new_C_b; mc.new_Z_b = x->new_Z_b;
+  mc.block_table = x->block_table; mc.max_pages = p->max_pages;
+  pa.nbranch = p->hca ? 1 : 2;
+  pa.b = b; pa.t = 0; pa.qpos = d.qpos;
+  pa.paged = 1; pa.win = x->win; pa.new_win = x->new_win; pa.win_ring = p->n_w;
+  const void* qI = x->q_I;
+  const void* qs = nullptr;
+  if (!p->hca) {
+    CompressArgs& ic = pa.index;
+    ic = mc;
+    ic.C_a = x->tail_CI_a; ic.Z_a = x->tail_ZI_a; ic.B_a = x->BI_a;
+    ic.C_b = x->tail_CI_b; ic.Z_b = x->tail_ZI_b; ic.B_b = x->BI_b;
+    ic.c = p->c_I; ic.d_rope = p->d_rope_I; ic.out_dtype = p->idx_dtype;
+    ic.out = x->kI_pages; ic.out_scales = x->kI_scales;
+    ic.new_C_a = x->new_CI_a; ic.new_Z_a = x->new_ZI_a; ic.new_C_b = x->new_CI_b; ic.new_Z_b = x->new_ZI_b;
+    pa.q_in = x->q_I; pa.q_rows = b * p->H_I; pa.q_d = p->c_I; pa.q_dtype = p->idx_dtype;
+    pa.q_codes = static_cast<uint8_t*>(d.qI_codes); pa.q_scales = d.qI_scales;
+    qI = d.qI_codes; qs = d.qI_scales;
+  }
+  csa_status st = launch_decode_prologue(pa, p->kv_dtype, stream);
+  if (st) return st;
+  const int32_t* idx = nullptr;
+  const int32_t* cnt = nullptr;
+  if (!p->hca) {
+    // 2. score the visible entries of every sequence (their pages through the block table)
+    IndexArgs a{};
+    a.q = qI; a.q_scales = qs; a.w = x->w; a.k = x->kI_pages; a.k_scales = x->kI_scales;
+    a.q_pos = d.qpos; a.T = 1; a.H = p->H_I; a.d = p->c_I; a.m = p->m; a.qk_dtype = p->idx_dtype;
+    a.score_dtype = CSA_BF16; a.E_cap = p->max_pages * kPageEntries; a.E = std::max(E, 1);
+    a.scores = d.scores; a.pdl = 1; a.all_visible = 0; a.dep_entry = -1;
+    a.block_table = x->block_table; a.max_pages = p->max_pages; a.num_pages = p->num_pages;
+    st = launch_index_scores_tc(a, b, stream);
+    if (st == CSA_ERR_UNSUPPORTED) st = launch_index_scores_fp4_tc(a, b, stream);
+    if (st) return st;
+    // 3. top-k of each sequence's visible entries
+    int32_t* io = x->idx_out ? x->idx_out : d.idx;
+    int32_t* co = x->count_out ? x->count_out : d.count;
+    st = topk_impl(d.scores, CSA_BF16, d.qpos, p->m, b, 1, std::max(E, 1), p->k, io, co,
+                   d.topk_ws, d.topk_ws_bytes, stream, true);
+    if (st) return st;
+    idx = io; cnt = co;
+  }
+  // 4. attention over the selection (or every visible entry) plus the window ring
+  AttnArgs a{};
+  a.q = x->q; a.kv = x->kv_pages; a.idx = idx; a.count = cnt; a.win = x->win; a.q_pos = d.qpos;
+  a.sink = x->sink; a.T = 1; a.H = p->H; a.d = p->c; a.n_w = p->n_w; a.m = p->m;
+  a.k = p->hca ? 0 : p->k; a.E_cap = p->max_pages * kPageEntries; a.n = p->L_max;
+  a.scale = p->scale; a.out = x->out; a.lse = x->lse; a.pdl = 1;
+  a.d_rope_out = p->inv_rope ? p->d_rope : 0; a.theta = p->rope_theta;
+  a.block_table = x->block_table; a.max_pages = p->max_pages; a.num_pages = p->num_pages;
+  a.win_ring = p->n_w;
+  st = launch_attn_tc(a, b, p->kv_dtype, d.attn_ws, d.attn_ws_bytes, stream);
+  if (st == CSA_ERR_UNSUPPORTED) st = launch_attn_simt(a, b, p->kv_dtype, stream);
+  return st;
 }
 
 // ---------------------------------------------------------------------------

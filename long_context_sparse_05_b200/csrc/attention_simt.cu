@@ -35,14 +35,21 @@ __global__ void __launch_bounds__(256) attn_simt_kernel(AttnArgs a) {
   float* s_l = s_q + a.d;          // [R]
   int* s_row = reinterpret_cast<int*>(s_l + R);   // [R] encoded row: >=0 cache entry, <0 window token
   float* s_red = reinterpret_cast<float*>(s_row + R);   // [32]
-  const T* kv = reinterpret_cast<const T*>(a.kv) + (size_t)sb * a.E_cap * a.d;
-  const T* win = reinterpret_cast<const T*>(a.win) + (size_t)sb * a.n * a.d;
+  // entry e / window token u of this sequence (paged entries, ring window as the args say)
+  const T* kv = reinterpret_cast<const T*>(a.kv) + (a.block_table ? 0 : (size_t)sb * a.E_cap * a.d);
+  const T* win = reinterpret_cast<const T*>(a.win) +
+                 (size_t)sb * (a.win_ring ? a.win_ring : a.n) * a.d;
   for (int r = threadIdx.x; r < R; r += blockDim.x) {
     if (r < nsel) {
-      const int e = a.idx ? a.idx[qrow * a.k + r] : r;
-      s_row[r] = (e >= 0 && e < a.E_cap) ? e : kSkipRow;
+      int e = a.idx ? a.idx[qrow * a.k + r] : r;
+      if (e >= 0 && e < a.E_cap && a.block_table) {
+        const int pg = a.block_table[(size_t)sb * a.max_pages + e / kPageEntries];
+        e = (unsigned)pg < (unsigned)a.num_pages ? pg * kPageEntries + e % kPageEntries : -1;
+      }
+      s_row[r] = (e >= 0 && (a.block_table || e < a.E_cap)) ? e : kSkipRow;
     } else {
-      s_row[r] = -1 - (w0 + (r - nsel));
+      const int u = w0 + (r - nsel);
+      s_row[r] = -1 - (a.win_ring ? u % a.win_ring : u);
     }
   }
   __syncthreads();

@@ -72,6 +72,8 @@ struct AttnTc {
   float scale_log2;
   int d_rope_out;     // inverse RoPE on the last d_rope_out output dims at the query position
   double inv_freq[kMaxOutRopePairs];   // theta^(-2j/d_rope_out)
+  const int32_t* block_table;   // paged entries (see AttnArgs)
+  int max_pages, num_pages, win_ring;
 };
 
 // sin / cos of the inverse-RoPE angle of output dim d at position t (identity below the
@@ -104,9 +106,15 @@ __device__ __forceinline__ const __nv_bfloat16* row_src(const AttnTc& p, const Q
   if (pos < Q.nsel) {
     const int e = p.dense ? pos : e_pre != INT_MIN ? e_pre : p.idx[(size_t)qrow * p.k + pos];
     if (e < 0 || e >= p.E_cap) return nullptr;
+    if (p.block_table) {
+      const int pg = p.block_table[(size_t)Q.sb * p.max_pages + e / kPageEntries];
+      if ((unsigned)pg >= (unsigned)p.num_pages) return nullptr;
+      return p.kv + ((size_t)pg * kPageEntries + e % kPageEntries) * kD;
+    }
     return p.kv + ((size_t)Q.sb * p.E_cap + e) * kD;
   }
   const int u = Q.w0 + (pos - Q.nsel);
+  if (p.win_ring) return p.win + ((size_t)Q.sb * p.win_ring + u % p.win_ring) * kD;
   return p.win + ((size_t)Q.sb * p.n + u) * kD;
 }
 
@@ -887,6 +895,8 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
   p.cluster = P.cluster;
   p.scale_log2 = a.scale * kLog2e;
   p.d_rope_out = a.d_rope_out;
+  p.block_table = a.block_table; p.max_pages = a.max_pages; p.num_pages = a.num_pages;
+  p.win_ring = a.win_ring;
   for (int j = 0; j < kMaxOutRopePairs; ++j)
     p.inv_freq[j] = 2 * j < a.d_rope_out ? std::pow(a.theta, -2.0 * j / (double)a.d_rope_out) : 0.0;
   if (P.nsplit > 1 && P.cluster) {

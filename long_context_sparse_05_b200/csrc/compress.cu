@@ -29,7 +29,7 @@ template <> struct Vec16<__nv_bfloat16> { static constexpr int N = 8; };
 
 template <typename InT>
 __device__ __forceinline__ void load16(const InT* p, float* dst) {
-  uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
+  uint4 v = __ldcg(reinterpret_cast<const uint4*>(p));   // L2: rings are rewritten every step
   if constexpr (sizeof(InT) == 4) {
     dst[0] = __uint_as_float(v.x); dst[1] = __uint_as_float(v.y);
     dst[2] = __uint_as_float(v.z); dst[3] = __uint_as_float(v.w);
@@ -58,10 +58,18 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
   const int m = a.m;
   const int R = a.overlap ? 2 * m : m;
 
-  const InT* Ca = reinterpret_cast<const InT*>(a.C_a) + (size_t)s * a.n * c;
-  const InT* Za = reinterpret_cast<const InT*>(a.Z_a) + (size_t)s * a.n * c;
-  const InT* Cb = a.overlap ? reinterpret_cast<const InT*>(a.C_b) + (size_t)s * a.n * c : nullptr;
-  const InT* Zb = a.overlap ? reinterpret_cast<const InT*>(a.Z_b) + (size_t)s * a.n * c : nullptr;
+  const size_t seq_rows = a.ring ? (size_t)a.ring : (size_t)a.n;
+  const InT* Ca = reinterpret_cast<const InT*>(a.C_a) + (size_t)s * seq_rows * c;
+  const InT* Za = reinterpret_cast<const InT*>(a.Z_a) + (size_t)s * seq_rows * c;
+  const InT* Cb = a.overlap ? reinterpret_cast<const InT*>(a.C_b) + (size_t)s * seq_rows * c : nullptr;
+  const InT* Zb = a.overlap ? reinterpret_cast<const InT*>(a.Z_b) + (size_t)s * seq_rows * c : nullptr;
+  // paged state: the newest token's rows come from the step's inputs, the rest from the rings
+  const int t_new = a.ring ? a.pos[s] : -1;
+  auto rowp = [&](const InT* base, const void* fresh, int row) -> const InT* {
+    if (!a.ring) return base + (size_t)row * c;
+    if (row == t_new) return reinterpret_cast<const InT*>(fresh) + (size_t)s * c;
+    return base + (size_t)(row % a.ring) * c;
+  };
 
   float mx[VEC], sum[VEC], acc[VEC];
 #pragma unroll
@@ -88,8 +96,9 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
           }
         }
         if (live[u]) {
-          load16<InT>(Z + (size_t)row * c + cc * VEC, zv[u]);
-          load16<InT>(C + (size_t)row * c + cc * VEC, cv[u]);
+          const bool cur = Z == Za;
+          load16<InT>(rowp(Z, cur ? a.new_Z_a : a.new_Z_b, row) + cc * VEC, zv[u]);
+          load16<InT>(rowp(C, cur ? a.new_C_a : a.new_C_b, row) + cc * VEC, cv[u]);
 #pragma unroll
           for (int v = 0; v < VEC; ++v) bv[u][v] = __ldg(B + cc * VEC + v);
         }
@@ -171,7 +180,10 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
   }
   __syncthreads();
 
-  const size_t orow = (size_t)s * a.out_E + i;
+  // physical output row (paged: the page of entry i from the sequence's block table)
+  const size_t orow = a.block_table
+      ? (size_t)a.block_table[(size_t)s * a.max_pages + i / kPageEntries] * kPageEntries + i % kPageEntries
+      : (size_t)s * a.out_E + i;
   if (a.out_dtype == CSA_F32) {
     float* o = reinterpret_cast<float*>(a.out) + orow * c;
     for (int ch = tid; ch < c; ch += blockDim.x) o[ch] = s_x[ch];
@@ -189,7 +201,10 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
     if (tid == 0) reinterpret_cast<float*>(a.out_scales)[orow] = scale;
   } else {  // CSA_NVFP4
     uint8_t* o = reinterpret_cast<uint8_t*>(a.out) + orow * (c / 2);
-    uint8_t* so = reinterpret_cast<uint8_t*>(a.out_scales) + (size_t)s * nvfp4_key_scale_seq_bytes(a.out_E, c);
+    // the tiled key-scale layout of the sequence, or (paged) of all pages as one array
+    uint8_t* so = reinterpret_cast<uint8_t*>(a.out_scales) +
+                  (a.block_table ? (size_t)0 : (size_t)s * nvfp4_key_scale_seq_bytes(a.out_E, c));
+    const long long srow = a.block_table ? (long long)orow : (long long)i;
     for (int blk = tid; blk < c / 16; blk += blockDim.x) {
       float am = 0.f;
 #pragma unroll
@@ -202,7 +217,7 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
             ? f32x2_to_e2m1x2(s_x[blk * 16 + e] / sv, s_x[blk * 16 + e + 1] / sv)
             : (uint8_t)0;
       }
-      so[nvfp4_key_scale_offset(i, blk, c)] = sc;
+      so[nvfp4_key_scale_offset(srow, blk, c)] = sc;
     }
   }
 }
@@ -280,6 +295,17 @@ __global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int 
 // Decode prologue in one launch: CTAs [0, b) compress the latent entry of each
 // sequence, [b, 2b) its index-key entry (CSA), the rest quantise the index queries
 // (8 rows per CTA); CTA 0 of that range also writes the query positions.
+// Appends row `src` ([b][c] of InT, sequence s) to slot `slot` of the ring `dst`
+// ([b][ring][c]), 16 bytes per thread.
+template <typename InT>
+__device__ __forceinline__ void ring_append(void* dst, const void* src, int s, int ring, int slot,
+                                            int c) {
+  const int n16 = c * (int)sizeof(InT) / 16;
+  const uint4* in = reinterpret_cast<const uint4*>(reinterpret_cast<const InT*>(src) + (size_t)s * c);
+  uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<InT*>(dst) + ((size_t)s * ring + slot) * c);
+  for (int x = threadIdx.x; x < n16; x += blockDim.x) out[x] = in[x];
+}
+
 template <typename InT>
 __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
   extern __shared__ float smem[];
@@ -287,12 +313,32 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
   const int blk = blockIdx.x;
   if (blk < a.b * a.nbranch) {
     const int br = blk / a.b;
-    compress_body<InT>(br == 0 ? a.main : a.index, br == 0 ? a.main.entry_begin : a.index.entry_begin,
-                       blk % a.b, smem);
+    const int s = blk % a.b;
+    const CompressArgs& ca = br == 0 ? a.main : a.index;
+    if (!a.paged) {
+      compress_body<InT>(ca, ca.entry_begin, s, smem);
+      return;
+    }
+    // paged state: the entry the newest token completes (if it completes one), then the
+    // token's raw rows into the rings (no row this step reads sits in the slot written:
+    // the 2m rows of an entry occupy distinct slots and the newest comes from the inputs)
+    const int t = a.main.pos[s];
+    if (t >= 0 && (t + 1) % ca.m == 0) compress_body<InT>(ca, (t + 1) / ca.m - 1, s, smem);
+    if (t >= 0) {
+      const int slot = t % ca.ring;
+      ring_append<InT>(const_cast<void*>(ca.C_a), ca.new_C_a, s, ca.ring, slot, ca.c);
+      ring_append<InT>(const_cast<void*>(ca.Z_a), ca.new_Z_a, s, ca.ring, slot, ca.c);
+      if (ca.overlap) {
+        ring_append<InT>(const_cast<void*>(ca.C_b), ca.new_C_b, s, ca.ring, slot, ca.c);
+        ring_append<InT>(const_cast<void*>(ca.Z_b), ca.new_Z_b, s, ca.ring, slot, ca.c);
+      }
+      if (br == 0) ring_append<InT>(a.win, a.new_win, s, a.win_ring, t % a.win_ring, ca.c);
+    }
     return;
   }
   const int qb = blk - a.b * a.nbranch;
-  if (qb == 0 && threadIdx.x < a.b) a.qpos[threadIdx.x] = a.t;
+  if (qb == 0)
+    for (int i = threadIdx.x; i < a.b; i += blockDim.x) a.qpos[i] = a.paged ? a.main.pos[i] : a.t;
   const int row = qb * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (row < a.q_rows)
     quantize_row<InT>(reinterpret_cast<const InT*>(a.q_in), row, a.q_d, a.q_dtype, a.q_codes,
@@ -534,7 +580,7 @@ csa_status launch_compress_split(CompressArgs& a, int in_dtype, int b, int32_t* 
 }
 
 csa_status launch_decode_prologue(PrologueArgs& a, int in_dtype, cudaStream_t st) {
-  if (a.nbranch == 1 && a.q_rows == 0 && !a.main.overlap && a.main.m >= 64) {
+  if (!a.paged && a.nbranch == 1 && a.q_rows == 0 && !a.main.overlap && a.main.m >= 64) {
     // c128a: the block's rows over a cluster (the query positions come from the caller)
     const csa_status r = launch_compress_split(a.main, in_dtype, a.b, a.qpos, a.t, st, false);
     if (r != CSA_ERR_UNSUPPORTED) return r;

@@ -79,6 +79,7 @@ constexpr uint32_t kSfaCol = NACC * kAccCols;    // 384: NACC x (kTPS x 8) key-s
 constexpr uint32_t kSfbCol = kSfaCol + NACC * kTPS * 8;   // 432: 2 x 8 query-scale columns
 static_assert(kSfbCol + 16 <= kTmemCols, "TMEM budget");
 static_assert(kStage % 1024 == 0, "stages must keep the swizzle alignment");
+static_assert(kStageE == kPageEntries, "a stage of the paged key cache is one page");
 
 struct IdxFp4 {
   void* scores;
@@ -90,6 +91,8 @@ struct IdxFp4 {
   int score_f32;
   int all_visible;   // every query sees all E entries: q_pos is not read
   int dep_stage;     // stages >= dep_stage hold entries the preceding kernel writes
+  const int32_t* block_table;   // paged keys (one query per sequence: a stage is one page)
+  int max_pages, num_pages;
 };
 
 // Query buffer: codes | raw scales | rearranged scales | weights, padded to 1 KB so
@@ -247,6 +250,16 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         const int j0 = js * kTPS;                                // first tile of the stage
         const int nsf = min(kTPS, sf_seq - j0);                  // scale tiles inside the sequence
         uint8_t* st = sStage + slot * kStage;
+        if (p.block_table) {
+          // a stage is one page: its keys and its whole scale tiles
+          const int pg0 = p.block_table[(size_t)sb * p.max_pages + js];
+          const int pg = (unsigned)pg0 < (unsigned)p.num_pages ? pg0 : 0;
+          tc::mbar_arrive_expect_tx(&full[slot], kKeyB + kTPS * kSfTileB);
+          tc::tma_load_2d(st, &tmK, 0, pg * kStageE, &full[slot]);
+          bulk_load(st + kKeyB, p.k_scales + (size_t)pg * kTPS * kSfTileB, kTPS * kSfTileB,
+                    &full[slot]);
+          return;
+        }
         tc::mbar_arrive_expect_tx(&full[slot], kKeyB + nsf * kSfTileB);
         tc::tma_load_2d(st, &tmK, 0, sb * p.E_cap + j0 * kTileE, &full[slot]);
         bulk_load(st + kKeyB, p.k_scales + ((size_t)sb * sf_seq + j0) * kSfTileB,
@@ -479,7 +492,8 @@ csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st
       (reinterpret_cast<uintptr_t>(a.w) & 15))
     return CSA_ERR_INVALID_ARG;   // the TMA copies need 16-byte aligned rows and scale runs
   CUtensorMap tmK, tmQ, tmQS, tmW;
-  const uint64_t krows = (uint64_t)b * a.E_cap, qrows = (uint64_t)b * a.T * kHeads;
+  const uint64_t krows = a.block_table ? (uint64_t)a.num_pages * kPageEntries : (uint64_t)b * a.E_cap;
+  const uint64_t qrows = (uint64_t)b * a.T * kHeads;
   if (!make_tmap_2d_u8_swz(&tmK, a.k, kRowB, krows, kRowB, kStageE, 64) ||
       !make_tmap_2d_u8_swz(&tmQ, a.q, kRowB, qrows, kRowB, kHeads, 64) ||
       !make_tmap_2d_u8_swz(&tmQS, a.q_scales, 16, qrows / 2, 16, kHeads / 2, 0) ||
@@ -507,6 +521,7 @@ csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st
   p.units = (int)units;
   p.score_f32 = a.score_dtype == CSA_F32;
   p.all_visible = a.all_visible;
+  p.block_table = a.block_table; p.max_pages = a.max_pages; p.num_pages = a.num_pages;
   p.dep_stage = a.dep_entry < 0 ? 0 : a.dep_entry / kStageE;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;

@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(128) index_scores_simt_kernel(IndexArgs a) {
 }
 
 csa_status launch_index_scores_simt(const IndexArgs& a, int b, cudaStream_t st) {
+  if (a.block_table) return CSA_ERR_UNSUPPORTED;   // paged keys: tensor-core shapes only
   if (a.T == 0 || a.E == 0 || b == 0) return CSA_OK;
   const size_t smem = ((size_t)a.H * a.d + a.H) * sizeof(float);
   if (smem > 200 * 1024) return CSA_ERR_UNSUPPORTED;

@@ -62,6 +62,8 @@ struct IdxTc {
   int score_f32;
   int all_visible;   // every query sees all E entries: q_pos is not read
   int dep_stage;     // stages >= dep_stage hold entries the preceding kernel writes
+  const int32_t* block_table;   // paged keys (one query per sequence: a stage is one page)
+  int max_pages, num_pages;
 };
 
 template <int QG>
@@ -162,7 +164,11 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       auto load_stage = [&](int slot, int sb, int js) {
-        const int row0 = sb * p.E_cap + js * kStageE;
+        int row0 = sb * p.E_cap + js * kStageE;
+        if (p.block_table) {
+          const int pg = p.block_table[(size_t)sb * p.max_pages + js];
+          row0 = ((unsigned)pg < (unsigned)p.num_pages ? pg : 0) * kStageE;
+        }
         tc::mbar_arrive_expect_tx(&full[slot], LY::kStageKeyB + kStageE * 4);
         tc::tma_load_2d(sA + slot * LY::kStageKeyB, &tmK, 0, row0, &full[slot]);
         tc::tma_load_1d(sKS + slot * kStageE, &tmKS, row0, &full[slot]);
@@ -368,9 +374,10 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   using LY = Layout<QG>;
   CUtensorMap tmK, tmQ, tmKS, tmW, tmQS;
   const uint64_t qrows = (uint64_t)b * a.T * kHeads;
-  if (!make_tmap_2d_u8(&tmK, a.k, kDim, (uint64_t)b * a.E_cap, kDim, LY::kStageE) ||
+  const uint64_t krows = a.block_table ? (uint64_t)a.num_pages * kPageEntries : (uint64_t)b * a.E_cap;
+  if (!make_tmap_2d_u8(&tmK, a.k, kDim, krows, kDim, LY::kStageE) ||
       !make_tmap_2d_u8(&tmQ, a.q, kDim, qrows, kDim, LY::N) ||
-      !make_tmap_1d_f32(&tmKS, a.k_scales, (uint64_t)b * a.E_cap, LY::kStageE) ||
+      !make_tmap_1d_f32(&tmKS, a.k_scales, krows, LY::kStageE) ||
       !make_tmap_1d_f32(&tmW, a.w, qrows, LY::N) ||
       !make_tmap_1d_f32(&tmQS, a.q_scales, qrows, LY::N))
     return CSA_ERR_CUDA;
@@ -397,6 +404,7 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   p.score_f32 = a.score_dtype == CSA_F32;
   p.all_visible = a.all_visible;
   p.dep_stage = a.dep_entry < 0 ? 0 : a.dep_entry / LY::kStageE;
+  p.block_table = a.block_table; p.max_pages = a.max_pages; p.num_pages = a.num_pages;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
@@ -417,6 +425,7 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
 
 csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st) {
   if (a.qk_dtype != CSA_FP8_E4M3 || a.H != kHeads || a.d != kDim) return CSA_ERR_UNSUPPORTED;
+  if (a.block_table && (a.T != 1 || Layout<1>::kStageE != kPageEntries)) return CSA_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.q) & 15) ||
       (reinterpret_cast<uintptr_t>(a.k_scales) & 15) || (reinterpret_cast<uintptr_t>(a.w) & 15) ||
       (reinterpret_cast<uintptr_t>(a.q_scales) & 15) || (a.E_cap % 4))

@@ -16,13 +16,29 @@ struct CompressArgs {
   void* out;
   void* out_scales;
   double inv_freq[kMaxRopePairs];   // theta^(-2j/d_rope) in float64, filled by the launcher
+  // Paged state-cache mode (ring != 0): raw row u of sequence s is slot u % ring of the
+  // per-sequence ring buffers C_* / Z_* ([b][ring][c]), except the newest token's row
+  // (u = pos[s]), which comes from new_* ([b][c]); entry i is written at physical row
+  // block_table[s][i / kPageEntries] * kPageEntries + i % kPageEntries of out / out_scales.
+  int ring;
+  const int32_t* pos;
+  const void *new_C_a, *new_Z_a, *new_C_b, *new_Z_b;
+  const int32_t* block_table;
+  int max_pages;
 };
+
+constexpr int kPageEntries = CSA_PAGE_ENTRIES;   // compressed entries per page of the paged caches
 
 struct PrologueArgs {
   CompressArgs main, index;        // index used when nbranch == 2
   int nbranch, b, t;
-  int32_t* qpos;                   // [b] <- t
+  int32_t* qpos;                   // [b] <- t (or <- pos[s] in paged mode)
   const void* q_in; int q_rows, q_d, q_dtype; uint8_t* q_codes; void* q_scales;
+  // paged mode: the step appends the newest token's raw rows to the state rings
+  // (ring slot pos[s] % main.ring; window ring slot pos[s] % win_ring) and compresses
+  // an entry only for sequences whose block the token completes
+  int paged;
+  void* win; const void* new_win; int win_ring;
 };
 
 struct IndexArgs {
@@ -34,6 +50,10 @@ struct IndexArgs {
   int all_visible;    // every query sees all E entries (decode at t = L-1): q_pos is not read
   int dep_entry;      // first entry the preceding kernel writes (tiles before it may be
                       // fetched before waiting on that kernel); -1: all depend
+  // paged keys (one query per sequence): stage js of sequence s is page
+  // block_table[s][js] of kPageEntries rows; pages outside [0, num_pages) read as page 0
+  const int32_t* block_table;
+  int max_pages, num_pages;
 };
 
 struct AttnArgs {
@@ -45,6 +65,11 @@ struct AttnArgs {
   int pdl;            // launch as a programmatic dependent of the preceding kernel
   int d_rope_out;     // inverse RoPE on the last d_rope_out output dims (0: none)
   double theta;       // its RoPE base
+  // paged entries: entry e of sequence s is row e % kPageEntries of page
+  // block_table[s][e / kPageEntries] (pages outside [0, num_pages) are skipped);
+  // win_ring > 0: window token u of sequence s is slot u % win_ring of win ([b][win_ring][d])
+  const int32_t* block_table;
+  int max_pages, num_pages, win_ring;
 };
 
 constexpr int kMaxOutRopePairs = 32;   // rotary pairs of the output with a host-built table

@@ -197,3 +197,144 @@ def decode_launches_per_step(w: Workload):
 
 def prefill_launches(w: Workload):
     return L.csa_prefill_launch_count(prefill_params(w))
+
+
+def paged_params(w: Workload, max_pages, num_pages, L_max):
+    hca = w.kind == "hca_decode"
+    return L.PagedParams(b=w.b, m=w.m, c=w.c, H=w.H, c_I=w.c_I, H_I=w.H_I, d_rope=w.d_rope,
+                         d_rope_I=w.d_rope_I, rope_theta=w.theta, eps=w.eps, k=max(w.k, 1),
+                         n_w=w.n_w, scale=w.scale, kv_dtype=L.DTYPE[w.dtype],
+                         idx_dtype=L.DTYPE.get(w.idx_dtype, 0), hca=1 if hca else 0,
+                         max_pages=max_pages, num_pages=num_pages, L_max=L_max,
+                         inv_rope=1 if w.inv_rope else 0)
+
+
+class PagedDecodeState:
+    """Paged caches and per-sequence state of one decode workload, for csa_decode_paged.
+
+    ``positions[s]`` is the position t of sequence s's new token (default n - 1 for all).
+    Set-up (untimed) compresses every entry completed before t into the pages of the
+    sequence (consecutive pages per sequence, then the pages are shuffled and the block
+    table follows them), fills the rings of the state with the raw rows before t and
+    stages the new token's rows as the step's inputs.
+    """
+
+    def __init__(self, w: Workload, inputs, positions=None, device="cuda", shuffle_seed=0):
+        self.w, self.x, self.device = w, inputs, device
+        b, m, PE = w.b, w.m, L.PAGE_ENTRIES
+        self.hca = w.kind == "hca_decode"
+        pos = [w.n - 1] * b if positions is None else list(positions)
+        self.positions = pos
+        self.pos = torch.tensor(pos, dtype=torch.int32, device=device)
+        E_fin = [(t + 1) // m for t in pos]
+        npages = [max(1, (e + PE - 1) // PE) for e in E_fin]
+        self.max_pages = max(npages)
+        self.num_pages = sum(npages) + 1                      # one spare page
+        first = [sum(npages[:s]) for s in range(b)]
+        dt = _TDT[w.dtype]
+        rows_total = self.num_pages * PE
+        self.kv_pages = torch.zeros((rows_total, w.c), dtype=dt, device=device)
+        if not self.hca:
+            self.kI_pages, self.kI_scales = alloc_index_cache(1, rows_total, w.c_I, w.idx_dtype,
+                                                              device)
+            self.kI_pages = self.kI_pages[0]
+            self.kI_scales = self.kI_scales[0]
+        else:
+            self.kI_pages = self.kI_scales = None
+        # entries completed before each sequence's new token, compressed into its pages
+        for s in range(b):
+            E0 = pos[s] // m
+            if E0 == 0:
+                continue
+            cap = npages[s] * PE
+            sl = slice(first[s] * PE, first[s] * PE + cap)
+            xs = {k: (v[s:s + 1] if v.dim() >= 3 else v) for k, v in inputs.items()}
+            L.csa_compress(compress_params(w, "main"), xs["C_a"], xs["Z_a"], xs["B_a"],
+                           xs.get("C_b"), xs.get("Z_b"), xs.get("B_b"), 1, w.n, 0, E0, cap,
+                           self.kv_pages[sl], None)
+            if not self.hca:
+                sc = self.kI_scales[sl] if w.idx_dtype == "fp8" else self.kI_scales[sl]
+                L.csa_compress(compress_params(w, "index"), xs["CI_a"], xs["ZI_a"], xs["BI_a"],
+                               xs["CI_b"], xs["ZI_b"], xs["BI_b"], 1, w.n, 0, E0, cap,
+                               self.kI_pages[sl], sc)
+        # shuffle the physical pages; the block table follows
+        g = torch.Generator(device="cpu").manual_seed(shuffle_seed)
+        perm = torch.randperm(self.num_pages, generator=g)     # new page of old page i
+        inv = torch.empty_like(perm)
+        inv[perm] = torch.arange(self.num_pages)
+        def shuffle(t):
+            v = t.reshape(self.num_pages, -1)
+            return v[inv.to(device)].reshape(t.shape).contiguous()
+        self.kv_pages = shuffle(self.kv_pages)
+        if not self.hca:
+            self.kI_pages = shuffle(self.kI_pages)
+            self.kI_scales = shuffle(self.kI_scales)
+        bt = torch.full((b, self.max_pages), -1, dtype=torch.int32)
+        for s in range(b):
+            for j in range(npages[s]):
+                bt[s, j] = int(perm[first[s] + j])
+        self.block_table = bt.to(device)
+        # state rings: raw rows of the tokens before t
+        R = m if self.hca else 2 * m
+        self.ring = R
+        def ring_of(name, c):
+            r = torch.zeros((b, R, c), dtype=dt, device=device)
+            for s in range(b):
+                us = [u for u in range(max(0, pos[s] - R + 1), pos[s])]
+                if us:
+                    ui = torch.tensor(us, device=device)
+                    r[s, ui % R] = inputs[name][s, ui]
+            return r
+        names = ["C_a", "Z_a"] + ([] if self.hca else ["C_b", "Z_b"])
+        self.tails = {"tail_" + n: ring_of(n, w.c) for n in names}
+        if not self.hca:
+            for n in ("CI_a", "ZI_a", "CI_b", "ZI_b"):
+                self.tails["tail_" + n] = ring_of(n, w.c_I)
+        self.win = torch.zeros((b, w.n_w, w.c), dtype=dt, device=device)
+        for s in range(b):
+            us = [u for u in range(max(0, pos[s] - w.n_w + 1), pos[s])]
+            if us:
+                ui = torch.tensor(us, device=device)
+                self.win[s, ui % w.n_w] = inputs["C_a"][s, ui]
+        # the new token's rows (the step's inputs)
+        ti = self.pos.long()
+        ar = torch.arange(b, device=device)
+        self.new = {"new_" + n: inputs[n][ar, ti].contiguous() for n in names}
+        if not self.hca:
+            for n in ("CI_a", "ZI_a", "CI_b", "ZI_b"):
+                self.new["new_" + n] = inputs[n][ar, ti].contiguous()
+        self.new["new_win"] = inputs["C_a"][ar, ti].contiguous()
+        self.L_max = max(pos) + 1
+        self.p = paged_params(w, self.max_pages, self.num_pages, self.L_max)
+        self.out = torch.empty((b, w.H, w.c), dtype=dt, device=device)
+        self.lse = torch.empty((b, w.H), dtype=torch.float32, device=device)
+        if not self.hca:
+            self.idx = torch.empty((b, w.k), dtype=torch.int32, device=device)
+            self.count = torch.empty((b,), dtype=torch.int32, device=device)
+        else:
+            self.idx = self.count = None
+        self.ws_bytes = L.csa_decode_paged_workspace_size(self.p)
+        # NaN bytes: a kernel that read workspace it had not written would show up
+        self.ws = torch.full((max(self.ws_bytes, 256),), 0xFF, dtype=torch.uint8, device=device)
+
+    def tensors(self, q=None, q_I=None, w_=None, new=None):
+        x = self.x
+        d = dict(kv_pages=self.kv_pages, block_table=self.block_table, win=self.win,
+                 pos=self.pos, B_a=x["B_a"], B_b=x.get("B_b"), sink=x["sink"],
+                 q=q if q is not None else x["q"], out=self.out, lse=self.lse)
+        d.update(self.tails)
+        d.update(new if new is not None else self.new)
+        if not self.hca:
+            d.update(kI_pages=self.kI_pages, kI_scales=self.kI_scales, BI_a=x["BI_a"],
+                     BI_b=x["BI_b"], q_I=q_I if q_I is not None else x["q_I"],
+                     w=w_ if w_ is not None else x["w"], idx_out=self.idx, count_out=self.count)
+        return d
+
+    def step(self, stream=None, **over):
+        L.csa_decode_paged(self.p, self.tensors(**over), self.ws, self.ws_bytes, stream)
+        return self.out
+
+    def entry_row(self, s, e):
+        """Physical row of entry e of sequence s in the pages."""
+        PE = L.PAGE_ENTRIES
+        return int(self.block_table[s, e // PE]) * PE + e % PE

@@ -42,6 +42,11 @@ def test_binding_covers_every_declared_symbol():
     assert set(declared_functions()) <= set(L._SIGS), set(declared_functions()) - set(L._SIGS)
 
 
+def test_page_size_matches_header():
+    m = re.search(r"#define\s+CSA_PAGE_ENTRIES\s+(\d+)", open(HEADER).read())
+    assert m and int(m.group(1)) == L.PAGE_ENTRIES
+
+
 def test_noalloc_scratch_size_matches_header():
     """The binding's copy of the fixed scratch size is the header's (the tests rely on it)."""
     m = re.search(r"#define\s+CSA_NOALLOC_SCRATCH_BYTES\s+\(\(size_t\)(\d+)\s*<<\s*(\d+)\)",
@@ -54,6 +59,7 @@ def test_struct_layouts_match_c():
     structs = {"csa_compress_params": L.CompressParams, "csa_index_params": L.IndexParams,
                "csa_attn_params": L.AttnParams, "csa_decode_params": L.DecodeParams,
                "csa_decode_tensors": L.DecodeTensors, "csa_prefill_params": L.PrefillParams,
+               "csa_paged_params": L.PagedParams, "csa_paged_tensors": L.PagedTensors,
                "csa_prefill_tensors": L.PrefillTensors}
     prog = ["#include <stdio.h>", "#include <stddef.h>", '#include "csa.h"', "int main(void){"]
     for cname, py in structs.items():
