@@ -340,22 +340,18 @@ def stage_times_decode(w, st, steps, flush, stream):
 
 
 def e2e_decode(w, st, steps, flush, stream, world=1):
-    """Same step through the public API with host inputs: every step copies its new
-    inputs (q, q_I, w and the m raw rows of the completing block of every C / Z
-    tensor) from one pinned host buffer to one device staging buffer (a single H2D
-    copy), places the raw rows into the sequence tensors with device-to-device
-    copies, runs the decode call on the staged q / q_I / w, and reads the output back
-    (one D2H copy).  Whole-job throughput: all ranks' tokens over the slowest rank's
-    time."""
-    x = st.x
-    t = w.n - 1
-    r0 = t - (w.m - 1)
-    names = ["C_a", "Z_a", "C_b", "Z_b", "CI_a", "ZI_a", "CI_b", "ZI_b"]
-    names = [n for n in names if n in x]
-    parts = [("q", x["q"])]
-    if "q_I" in x:
-        parts += [("q_I", x["q_I"]), ("w", x["w"])]
-    parts += [(n, x[n][:, r0:t + 1]) for n in names]
+    """The decode step through the public serving call, csa_decode_paged, with host inputs.
+
+    The caches live in pages and the per-sequence state (window and raw tail rings) on
+    the device, as a server keeps them; each step copies only what a new token brings
+    (its raw C / Z rows of both branches, its window row, q, q_I, w and the positions)
+    from one pinned host buffer to one device staging buffer (a single H2D copy), runs
+    the step on the staged tensors and reads the output back (one D2H copy).
+    Whole-job throughput: all ranks' tokens over the slowest rank's time."""
+    ps = runner.PagedDecodeState(w, st.x)
+    parts = [("pos", ps.pos)] + [(k, v) for k, v in ps.new.items()] + [("q", st.x["q"])]
+    if "q_I" in st.x:
+        parts += [("q_I", st.x["q_I"]), ("w", st.x["w"])]
     # one staging layout shared by host and device: each part 256-byte aligned
     offs, off = {}, 0
     for n, v in parts:
@@ -370,27 +366,34 @@ def e2e_decode(w, st, steps, flush, stream, world=1):
 
     for n, v in parts:
         view(hstage, n, v).copy_(v.contiguous().cpu())
-    dviews = {n: view(dstage, n, v) for n, v in parts}
-    hout = torch.empty(st.out.shape, dtype=st.out.dtype).pin_memory()
+    dv = {n: view(dstage, n, v) for n, v in parts}
+    ps.pos = dv["pos"]
+    new = {k: dv[k] for k in ps.new}
+    hout = torch.empty(ps.out.shape, dtype=ps.out.dtype).pin_memory()
     h2d = sum(v.numel() * v.element_size() for _, v in parts)
     d2h = hout.numel() * hout.element_size()
 
     def one():
         dstage.copy_(hstage, non_blocking=True)
-        for n in names:
-            x[n][:, r0:t + 1].copy_(dviews[n])
-        st.step(stream, q=dviews["q"], q_I=dviews.get("q_I"), w_=dviews.get("w"))
-        hout.copy_(st.out, non_blocking=True)
+        ps.step(stream, q=dv["q"], q_I=dv.get("q_I"), w_=dv.get("w"), new=new)
+        hout.copy_(ps.out, non_blocking=True)
 
     for _ in range(3):
         one()
     torch.cuda.synchronize()
+    dev_times = timed_loop(lambda: ps.step(stream, q=dv["q"], q_I=dv.get("q_I"), w_=dv.get("w"),
+                                           new=new), steps, flush, stream)
     barrier(world)
     times = timed_loop(one, steps, flush, stream)
     ms, _, value = aggregate(float(np.mean(times)), w.b, world)   # whole job, slowest rank
-    return {"value": value, "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
-            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
-            "copies_per_step": {"h2d": 1, "d2d": len(names), "d2h": 1}}
+    res = {"value": value, "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
+           "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
+           "copies_per_step": {"h2d": 1, "d2h": 1},
+           "call": "csa_decode_paged (pages of %d entries, state rings)" % L.PAGE_ENTRIES,
+           "device_ms_per_step": round(float(np.mean(dev_times)), 4),
+           "gpu_launches_per_step": L.csa_decode_paged_launch_count(ps.p)}
+    del ps
+    return res
 
 
 # ---------------------------------------------------------------------------
@@ -660,6 +663,40 @@ def cpu_baseline(w, budget_s=20.0):
 
 SUB_WORKLOADS = (workloads.CSA_DECODE_1M, workloads.HCA_DECODE_1M, workloads.CSA_PREFILL_32K)
 
+# Grouped output projection (an output epilogue of the attention): 64 heads x 512 in 8
+# groups, each projected to 1024 outputs, for the 64K decode batch and the 32K prefill.
+OUT_PROJ = dict(H=64, d=512, g=8, d_g=1024)
+
+
+def bench_out_proj(args, peaks, world):
+    """Event-timed csa_out_proj at the decode batch (16 tokens: the 64 MB of bf16 weights
+    bound it, HBM roofline) and at the prefill length (32768 tokens: tensor roofline)."""
+    H, d, g, d_g = OUT_PROJ["H"], OUT_PROJ["d"], OUT_PROJ["g"], OUT_PROJ["d_g"]
+    K = (H // g) * d
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    W = synth.draw("W_o", (g, d_g, K), 7, "cuda", "bf16", spread=1.0 / math.sqrt(K))
+    res = {}
+    for label, T in (("decode_16_tokens", workloads.CSA_DECODE_64K.b),
+                     ("prefill_32768_tokens", workloads.CSA_PREFILL_32K.n)):
+        o = synth.draw("q", (T, H, d), 8, "cuda", "bf16")
+        y = torch.empty((T, g * d_g), dtype=torch.bfloat16, device="cuda")
+        wsb = L.csa_out_proj_workspace_size(T, H, d, g, d_g)
+        ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device="cuda")
+        fn = lambda: L.csa_out_proj(o, W, T, H, d, g, d_g, y, ws, wsb, stream)  # noqa: E731
+        us = float(np.mean(timed_loop(fn, max(3, min(args.steps, 10)), flush, stream, warm=3))) * 1e3
+        if T <= 64:
+            nbytes = W.numel() * 2 + o.numel() * 2 + y.numel() * 2
+            res[label] = kernel_record(us, nbytes, peaks["hbm"])
+        else:
+            res[label] = kernel_record(us, 2.0 * T * K * d_g * g, peaks["bf16"], "TFLOP/s", "tensor")
+        res[label]["launches"] = L.lib().csa_out_proj_workspace_size(T, H, d, g, d_g) and 2 or 1
+        del o, y, ws
+    del W, flush
+    torch.cuda.empty_cache()
+    res["config"] = dict(OUT_PROJ)
+    return res
+
 
 def run_workload(w, args, world, rank, peaks, min_span_s, cpu_budget_s):
     """One workload's record: throughput, rooflines, per-kernel fractions, clocks, e2e and (rank
@@ -736,6 +773,7 @@ def main():
     if args.workload is None and not args.context and not args.batch:
         for w2 in SUB_WORKLOADS:
             subs[w2.name] = run_workload(w2, args, world, rank, peaks, 0.5, 10.0)
+        subs["grouped_out_proj"] = bench_out_proj(args, peaks, world)
     if rank == 0:
         line = {"metric": METRIC, "value": head["value"], "unit": "tok/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],

@@ -600,24 +600,25 @@ csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* 
     // 2. score the visible entries of every sequence (their pages through the block table)
     IndexArgs a{};
     a.q = qI; a.q_scales = qs; a.w = x->w; a.k = x->kI_pages; a.k_scales = x->kI_scales;
-    a.q_pos = d.qpos; a.T = 1; a.H = p->H_I; a.d = p->c_I; a.m = p->m; a.qk_dtype = p->idx_dtype;
+    a.q_pos = x->pos; a.T = 1; a.H = p->H_I; a.d = p->c_I; a.m = p->m; a.qk_dtype = p->idx_dtype;
     a.score_dtype = CSA_BF16; a.E_cap = p->max_pages * kPageEntries; a.E = std::max(E, 1);
     a.scores = d.scores; a.pdl = 1; a.all_visible = 0; a.dep_entry = -1;
     a.block_table = x->block_table; a.max_pages = p->max_pages; a.num_pages = p->num_pages;
+    a.pos_input = 1;
     st = launch_index_scores_tc(a, b, stream);
     if (st == CSA_ERR_UNSUPPORTED) st = launch_index_scores_fp4_tc(a, b, stream);
     if (st) return st;
     // 3. top-k of each sequence's visible entries
     int32_t* io = x->idx_out ? x->idx_out : d.idx;
     int32_t* co = x->count_out ? x->count_out : d.count;
-    st = topk_impl(d.scores, CSA_BF16, d.qpos, p->m, b, 1, std::max(E, 1), p->k, io, co,
+    st = topk_impl(d.scores, CSA_BF16, x->pos, p->m, b, 1, std::max(E, 1), p->k, io, co,
                    d.topk_ws, d.topk_ws_bytes, stream, true);
     if (st) return st;
     idx = io; cnt = co;
   }
   // 4. attention over the selection (or every visible entry) plus the window ring
   AttnArgs a{};
-  a.q = x->q; a.kv = x->kv_pages; a.idx = idx; a.count = cnt; a.win = x->win; a.q_pos = d.qpos;
+  a.q = x->q; a.kv = x->kv_pages; a.idx = idx; a.count = cnt; a.win = x->win; a.q_pos = x->pos;
   a.sink = x->sink; a.T = 1; a.H = p->H; a.d = p->c; a.n_w = p->n_w; a.m = p->m;
   a.k = p->hca ? 0 : p->k; a.E_cap = p->max_pages * kPageEntries; a.n = p->L_max;
   a.scale = p->scale; a.out = x->out; a.lse = x->lse; a.pdl = 1;

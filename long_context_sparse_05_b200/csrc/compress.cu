@@ -63,8 +63,9 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
   const InT* Za = reinterpret_cast<const InT*>(a.Z_a) + (size_t)s * seq_rows * c;
   const InT* Cb = a.overlap ? reinterpret_cast<const InT*>(a.C_b) + (size_t)s * seq_rows * c : nullptr;
   const InT* Zb = a.overlap ? reinterpret_cast<const InT*>(a.Z_b) + (size_t)s * seq_rows * c : nullptr;
-  // paged state: the newest token's rows come from the step's inputs, the rest from the rings
-  const int t_new = a.ring ? a.pos[s] : -1;
+  // paged state: the newest token's rows come from the step's inputs, the rest from the
+  // rings; an entry is compressed only by the token that completes it, m (i + 1) - 1
+  const int t_new = a.ring ? m * (i + 1) - 1 : -1;
   auto rowp = [&](const InT* base, const void* fresh, int row) -> const InT* {
     if (!a.ring) return base + (size_t)row * c;
     if (row == t_new) return reinterpret_cast<const InT*>(fresh) + (size_t)s * c;
@@ -293,18 +294,10 @@ __global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int 
 }
 
 // Decode prologue in one launch: CTAs [0, b) compress the latent entry of each
-// sequence, [b, 2b) its index-key entry (CSA), the rest quantise the index queries
-// (8 rows per CTA); CTA 0 of that range also writes the query positions.
-// Appends row `src` ([b][c] of InT, sequence s) to slot `slot` of the ring `dst`
-// ([b][ring][c]), 16 bytes per thread.
-template <typename InT>
-__device__ __forceinline__ void ring_append(void* dst, const void* src, int s, int ring, int slot,
-                                            int c) {
-  const int n16 = c * (int)sizeof(InT) / 16;
-  const uint4* in = reinterpret_cast<const uint4*>(reinterpret_cast<const InT*>(src) + (size_t)s * c);
-  uint4* out = reinterpret_cast<uint4*>(reinterpret_cast<InT*>(dst) + ((size_t)s * ring + slot) * c);
-  for (int x = threadIdx.x; x < n16; x += blockDim.x) out[x] = in[x];
-}
+// sequence, [b, 2b) its index-key entry (CSA), in paged mode the next b append the new
+// token's rows to the state rings, the rest quantise the index queries (16 rows per CTA);
+// CTA 0 of that range also writes the query positions.
+constexpr int kQRowsPerWarp = 2;   // index-query rows quantised by one warp of the prologue
 
 template <typename InT>
 __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
@@ -319,30 +312,71 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
       compress_body<InT>(ca, ca.entry_begin, s, smem);
       return;
     }
-    // paged state: the entry the newest token completes (if it completes one), then the
-    // token's raw rows into the rings (no row this step reads sits in the slot written:
-    // the 2m rows of an entry occupy distinct slots and the newest comes from the inputs)
+    // paged state: the entry the newest token completes, if it completes one
     const int t = a.main.pos[s];
     if (t >= 0 && (t + 1) % ca.m == 0) compress_body<InT>(ca, (t + 1) / ca.m - 1, s, smem);
-    if (t >= 0) {
+    return;
+  }
+  if (a.paged && blk < a.b * (a.nbranch + 1)) {
+    // paged state: the token's raw rows into the rings, by CTAs of their own, alongside
+    // the compression (no row the compression reads sits in a slot written here: the 2m
+    // rows of an entry occupy distinct slots and the newest comes from the inputs)
+    const int s = blk - a.b * a.nbranch;
+    const int t = a.main.pos[s];
+    if (t < 0) return;
+    // up to nine rows (C, Z of both blocks of both branches, the window row): every
+    // thread loads all its 16-byte pieces first, then stores them (one memory round trip)
+    const uint4* src[9];
+    uint4* dst[9];
+    int n16[9], nr = 0;
+    auto add = [&](void* ring, const void* fresh, int ringlen, int slot, int c) {
+      src[nr] = reinterpret_cast<const uint4*>(reinterpret_cast<const InT*>(fresh) + (size_t)s * c);
+      dst[nr] = reinterpret_cast<uint4*>(reinterpret_cast<InT*>(ring) + ((size_t)s * ringlen + slot) * c);
+      n16[nr] = c * (int)sizeof(InT) / 16;
+      ++nr;
+    };
+    for (int br = 0; br < a.nbranch; ++br) {
+      const CompressArgs& ca = br == 0 ? a.main : a.index;
       const int slot = t % ca.ring;
-      ring_append<InT>(const_cast<void*>(ca.C_a), ca.new_C_a, s, ca.ring, slot, ca.c);
-      ring_append<InT>(const_cast<void*>(ca.Z_a), ca.new_Z_a, s, ca.ring, slot, ca.c);
+      add(const_cast<void*>(ca.C_a), ca.new_C_a, ca.ring, slot, ca.c);
+      add(const_cast<void*>(ca.Z_a), ca.new_Z_a, ca.ring, slot, ca.c);
       if (ca.overlap) {
-        ring_append<InT>(const_cast<void*>(ca.C_b), ca.new_C_b, s, ca.ring, slot, ca.c);
-        ring_append<InT>(const_cast<void*>(ca.Z_b), ca.new_Z_b, s, ca.ring, slot, ca.c);
+        add(const_cast<void*>(ca.C_b), ca.new_C_b, ca.ring, slot, ca.c);
+        add(const_cast<void*>(ca.Z_b), ca.new_Z_b, ca.ring, slot, ca.c);
       }
-      if (br == 0) ring_append<InT>(a.win, a.new_win, s, a.win_ring, t % a.win_ring, ca.c);
+    }
+    add(a.win, a.new_win, a.win_ring, t % a.win_ring, a.main.c);
+    int total = 0;
+    for (int r = 0; r < nr; ++r) total += n16[r];
+    for (int x0 = threadIdx.x; x0 < total; x0 += 4 * blockDim.x) {
+      uint4 v[4];
+      uint4* d[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        int x = x0 + u * blockDim.x;
+        d[u] = nullptr;
+        if (x >= total) continue;
+        int r = 0;
+        while (x >= n16[r]) { x -= n16[r]; ++r; }
+        v[u] = src[r][x];
+        d[u] = dst[r] + x;
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        if (d[u]) *d[u] = v[u];
     }
     return;
   }
-  const int qb = blk - a.b * a.nbranch;
+  const int qb = blk - a.b * (a.nbranch + (a.paged ? 1 : 0));
   if (qb == 0)
     for (int i = threadIdx.x; i < a.b; i += blockDim.x) a.qpos[i] = a.paged ? a.main.pos[i] : a.t;
-  const int row = qb * (blockDim.x / 32) + (threadIdx.x >> 5);
-  if (row < a.q_rows)
-    quantize_row<InT>(reinterpret_cast<const InT*>(a.q_in), row, a.q_d, a.q_dtype, a.q_codes,
-                      a.q_scales);
+  // kQRowsPerWarp rows per warp, so that the whole prologue fits in one wave of CTAs
+  for (int j = 0; j < kQRowsPerWarp; ++j) {
+    const int row = (qb * (blockDim.x / 32) + (threadIdx.x >> 5)) * kQRowsPerWarp + j;
+    if (row < a.q_rows)
+      quantize_row<InT>(reinterpret_cast<const InT*>(a.q_in), row, a.q_d, a.q_dtype, a.q_codes,
+                        a.q_scales);
+  }
 }
 
 // One entry of a long non-overlapped block (c128a: m = 128 rows) split over the CTAs of
@@ -596,8 +630,9 @@ csa_status launch_decode_prologue(PrologueArgs& a, int in_dtype, cudaStream_t st
     smem = std::max(smem, compress_smem_bytes(a.index, in_dtype, nt));
   }
   if (smem > 200 * 1024) return CSA_ERR_UNSUPPORTED;
-  const int qblocks = std::max(1, (a.q_rows + 7) / 8);
-  const int grid = a.b * a.nbranch + qblocks;
+  const int qrows_per_cta = 8 * kQRowsPerWarp;
+  const int qblocks = std::max(1, (a.q_rows + qrows_per_cta - 1) / qrows_per_cta);
+  const int grid = a.b * (a.nbranch + (a.paged ? 1 : 0)) + qblocks;
   if (in_dtype == CSA_F32) {
     cudaFuncSetAttribute(decode_prologue_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     decode_prologue_kernel<float><<<grid, nt, smem, st>>>(a);

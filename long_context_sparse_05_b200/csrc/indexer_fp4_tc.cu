@@ -50,6 +50,8 @@
 #include "kernels.h"
 #include "tc_common.cuh"
 
+#include <climits>
+
 namespace csa {
 
 namespace {
@@ -69,6 +71,7 @@ constexpr int kPermBytes = 2 * 512;              // query scales in the tcgen05.
 constexpr int NACC = 3;                          // accumulators of kTPS x 64 columns
 constexpr int S = 8;                             // stages
 constexpr int kMaxLocalUnits = 256;
+constexpr int kPagedSlots = 1024;    // page ids of the stages a CTA loads, kept in shared memory
 constexpr int kEpiGroups = 3;                    // one epilogue warpgroup per accumulator
 constexpr int kThreads = 96 + 128 * kEpiGroups;   // producer, MMA, 12 epilogue, waiter
 constexpr int kWaitWarp = kThreads / 32 - 1;       // warp 14
@@ -93,6 +96,7 @@ struct IdxFp4 {
   int dep_stage;     // stages >= dep_stage hold entries the preceding kernel writes
   const int32_t* block_table;   // paged keys (one query per sequence: a stage is one page)
   int max_pages, num_pages;
+  int pos_input;     // q_pos is an input: read before the wait; per-sequence dependent stage
 };
 
 // Query buffer: codes | raw scales | rearranged scales | weights, padded to 1 KB so
@@ -202,11 +206,25 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(tempty + NACC);
   int* s_vis = reinterpret_cast<int*>(tmem_holder + 4);      // [kMaxLocalUnits] visible stages
   int* s_ev = s_vis + kMaxLocalUnits;                         // [kMaxLocalUnits] visible entries
+  int* s_pg = s_ev + kMaxLocalUnits;                          // [kPagedSlots] page of each stage
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   pdl_launch_dependents();
-  if (!p.all_visible) pdl_wait();   // the query positions come from the preceding kernel
+  if (p.block_table) {
+    // page ids of every stage of every unit this CTA walks, [local unit][stage of the
+    // chunk]: inputs of the call, fetched at once while the CTA sets up instead of one
+    // dependent load before each stage's copy
+    const int nloc = min(kMaxLocalUnits, (p.units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x);
+    for (int x = threadIdx.x; x < nloc * p.chunk && x < kPagedSlots; x += blockDim.x) {
+      const int i = x / p.chunk, j = x % p.chunk;
+      const int u = blockIdx.x + i * gridDim.x;
+      const int sb = u / p.n_chunks;
+      const int js = (u % p.n_chunks) * p.chunk + j;
+      s_pg[x] = js < p.max_pages ? p.block_table[(size_t)sb * p.max_pages + js] : -1;
+    }
+  }
+  if (!p.all_visible && !p.pos_input) pdl_wait();   // the positions come from the preceding kernel
 
   for (int i = threadIdx.x; i * (int)gridDim.x + (int)blockIdx.x < p.units && i < kMaxLocalUnits;
        i += blockDim.x) {
@@ -245,14 +263,16 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     if (lane == 0) {
       // ---------------------------------------------------------------- producer
       const int sf_seq = p.sf_tiles_cap;
-      auto load_stage = [&](int slot, int row, int js) {
+      auto load_stage = [&](int slot, int row, int js, int li) {
         const int sb = row / p.T;
         const int j0 = js * kTPS;                                // first tile of the stage
         const int nsf = min(kTPS, sf_seq - j0);                  // scale tiles inside the sequence
         uint8_t* st = sStage + slot * kStage;
         if (p.block_table) {
           // a stage is one page: its keys and its whole scale tiles
-          const int pg0 = p.block_table[(size_t)sb * p.max_pages + js];
+          const uint32_t fl = (uint32_t)(li * p.chunk + js % p.chunk);
+          const int pg0 = fl < (uint32_t)kPagedSlots ? s_pg[fl]
+                                                       : p.block_table[(size_t)sb * p.max_pages + js];
           const int pg = (unsigned)pg0 < (unsigned)p.num_pages ? pg0 : 0;
           tc::mbar_arrive_expect_tx(&full[slot], kKeyB + kTPS * kSfTileB);
           tc::tma_load_2d(st, &tmK, 0, pg * kStageE, &full[slot]);
@@ -271,8 +291,13 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         int row, js0, js1, nc;
         unit(u, i, row, js0, js1, nc);
         if (nc == 0) continue;
-        for (int js = js0; js < js0 + nc && (int)npre < S && js < p.dep_stage; ++js, ++npre)
-          load_stage(npre, row, js);
+        int dep = p.dep_stage;
+        if (p.pos_input) {   // the stage holding the entry the sequence's new token completes
+          const int t = p.q_pos[row];
+          dep = (t + 1) % p.m == 0 ? ((t + 1) / p.m - 1) / kStageE : INT_MAX;
+        }
+        for (int js = js0; js < js0 + nc && (int)npre < S && js < dep; ++js, ++npre)
+          load_stage(npre, row, js, i);
         break;
       }
       pdl_wait();
@@ -295,7 +320,7 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           const int s = it % S;
           ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
           if (!ok) break;
-          load_stage(s, row, js);
+          load_stage(s, row, js, i);
         }
         ++ul;
       }
@@ -522,12 +547,13 @@ csa_status launch_index_scores_fp4_tc(const IndexArgs& a, int b, cudaStream_t st
   p.score_f32 = a.score_dtype == CSA_F32;
   p.all_visible = a.all_visible;
   p.block_table = a.block_table; p.max_pages = a.max_pages; p.num_pages = a.num_pages;
+  p.pos_input = a.pos_input;
   p.dep_stage = a.dep_entry < 0 ? 0 : a.dep_entry / kStageE;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
   const size_t smem = 1024 + (size_t)S * kStage + 2 * (size_t)kQBuf + (2 * S + 4 + 2 * NACC) * 8 +
-                      16 + (size_t)kMaxLocalUnits * 2 * 4;
+                      16 + (size_t)kMaxLocalUnits * 2 * 4 + (size_t)kPagedSlots * 4;
   if (cudaFuncSetAttribute(index_scores_fp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem) != cudaSuccess)
     return CSA_ERR_CUDA;

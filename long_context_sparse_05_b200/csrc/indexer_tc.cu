@@ -41,6 +41,8 @@
 #include "kernels.h"
 #include "tc_common.cuh"
 
+#include <climits>
+
 namespace csa {
 
 namespace {
@@ -50,6 +52,7 @@ constexpr int kHeads = 64;           // index heads
 constexpr int kDim = 128;            // index dim (bytes per FP8 row)
 constexpr int kTileBytes = kTileE * kDim;
 constexpr int kMaxLocalUnits = 256;  // units one CTA walks (grid is sized to respect it)
+constexpr int kPagedSlots = 1024;    // page ids of the stages a CTA loads, kept in shared memory
 constexpr int kEpiGroups = 2;        // epilogue warpgroups, alternating stages
 constexpr int kThreads = 64 + 128 * kEpiGroups;
 
@@ -64,6 +67,7 @@ struct IdxTc {
   int dep_stage;     // stages >= dep_stage hold entries the preceding kernel writes
   const int32_t* block_table;   // paged keys (one query per sequence: a stage is one page)
   int max_pages, num_pages;
+  int pos_input;     // q_pos is an input: read before the wait; per-sequence dependent stage
 };
 
 template <int QG>
@@ -108,11 +112,25 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   float* s_wq = reinterpret_cast<float*>(tmem_holder + 4);    // [kEpiGroups][N] w * qs of the unit
   int* s_vis = reinterpret_cast<int*>(s_wq + kEpiGroups * N); // [kMaxLocalUnits] visible stages
   int* s_ev = s_vis + kMaxLocalUnits;                         // [kMaxLocalUnits][QG] visible entries
+  int* s_pg = s_ev + kMaxLocalUnits * QG;                     // [kPagedSlots] page of each stage
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   pdl_launch_dependents();
-  if (!p.all_visible) pdl_wait();   // the query positions come from the preceding kernel
+  if (p.block_table) {
+    // page ids of every stage of every unit this CTA walks, [local unit][stage of the
+    // chunk]: inputs of the call, fetched at once while the CTA sets up instead of one
+    // dependent load before each stage's copy
+    const int nloc = min(kMaxLocalUnits, (p.units - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x);
+    for (int x = threadIdx.x; x < nloc * p.chunk && x < kPagedSlots; x += blockDim.x) {
+      const int i = x / p.chunk, j = x % p.chunk;
+      const int u = blockIdx.x + i * gridDim.x;
+      const int sb = (u / p.n_chunks) / p.n_qg;
+      const int js = (u % p.n_chunks) * p.chunk + j;
+      s_pg[x] = js < p.max_pages ? p.block_table[(size_t)sb * p.max_pages + js] : -1;
+    }
+  }
+  if (!p.all_visible && !p.pos_input) pdl_wait();   // the positions come from the preceding kernel
 
   // causal extent of every unit this CTA will walk
   for (int i = threadIdx.x; i * (int)gridDim.x + (int)blockIdx.x < p.units && i < kMaxLocalUnits;
@@ -163,10 +181,12 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
-      auto load_stage = [&](int slot, int sb, int js) {
+      auto load_stage = [&](int slot, int sb, int js, int li) {
         int row0 = sb * p.E_cap + js * kStageE;
         if (p.block_table) {
-          const int pg = p.block_table[(size_t)sb * p.max_pages + js];
+          const uint32_t fl = (uint32_t)(li * p.chunk + js % p.chunk);
+          const int pg = fl < (uint32_t)kPagedSlots ? s_pg[fl]
+                                                      : p.block_table[(size_t)sb * p.max_pages + js];
           row0 = ((unsigned)pg < (unsigned)p.num_pages ? pg : 0) * kStageE;
         }
         tc::mbar_arrive_expect_tx(&full[slot], LY::kStageKeyB + kStageE * 4);
@@ -180,8 +200,13 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
         int sb, g, js0, js1, nc, nq;
         unit(u, i, sb, g, js0, js1, nc, nq);
         if (nc == 0) continue;
-        for (int js = js0; js < js0 + nc && (int)npre < S && js < p.dep_stage; ++js, ++npre)
-          load_stage(npre, sb, js);
+        int dep = p.dep_stage;
+        if (p.pos_input) {   // the stage holding the entry the sequence's new token completes
+          const int t = p.q_pos[sb];
+          dep = (t + 1) % p.m == 0 ? ((t + 1) / p.m - 1) / kStageE : INT_MAX;
+        }
+        for (int js = js0; js < js0 + nc && (int)npre < S && js < dep; ++js, ++npre)
+          load_stage(npre, sb, js, i);
         break;
       }
       pdl_wait();
@@ -204,7 +229,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
           const int s = it % S;
           ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
           if (!ok) break;
-          load_stage(s, sb, js);
+          load_stage(s, sb, js, i);
         }
         ++ul;
       }
@@ -405,12 +430,14 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   p.all_visible = a.all_visible;
   p.dep_stage = a.dep_entry < 0 ? 0 : a.dep_entry / LY::kStageE;
   p.block_table = a.block_table; p.max_pages = a.max_pages; p.num_pages = a.num_pages;
+  p.pos_input = a.pos_input;
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
   const size_t smem = 1024 + (size_t)S * (LY::kStageKeyB + LY::kStageE * 4) + 2 * (size_t)LY::kQBytes +
                       4 * (size_t)LY::N * 4 + (2 * S + 4 + 2 * LY::NACC) * 8 + 16 +
-                      kEpiGroups * (size_t)LY::N * 4 + (size_t)kMaxLocalUnits * (1 + QG) * 4;
+                      kEpiGroups * (size_t)LY::N * 4 + (size_t)kMaxLocalUnits * (1 + QG) * 4 +
+                      (size_t)kPagedSlots * 4;
   auto kern = index_scores_tc_kernel<QG, S>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
       cudaSuccess)

@@ -54,6 +54,10 @@ struct IndexArgs {
   // block_table[s][js] of kPageEntries rows; pages outside [0, num_pages) read as page 0
   const int32_t* block_table;
   int max_pages, num_pages;
+  // q_pos is an input of the call (not written by the preceding kernel): it is read
+  // before waiting, and only the page of the entry the token completes, (t+1)/m - 1 when
+  // (t+1) % m == 0, is written by the preceding kernel
+  int pos_input;
 };
 
 struct AttnArgs {
