@@ -99,10 +99,14 @@ csa_status csa_quantize(int in_dtype, int out_dtype, const void* x, int rows, in
 
 namespace {
 
+// q_raw: bf16 index queries the FP8 tensor-core kernel quantises itself (decode, one query
+// per sequence); q_I and q_scales are then unused.  There is no other kernel for it.
 csa_status index_scores_impl(const csa_index_params* p, const void* q_I, const void* q_scales,
                              const float* w, const void* k_I, const void* k_scales,
                              const int32_t* q_pos, int b, int T, int E_cap, int E, void* scores,
-                             cudaStream_t stream, int pdl, int all_visible, int dep_entry) {
+                             cudaStream_t stream, int pdl, int all_visible, int dep_entry,
+                             const void* q_raw = nullptr) {
+  if (q_raw) { q_I = q_raw; q_scales = k_scales; }
   if (!p) return CSA_ERR_INVALID_ARG;
   if (p->H_I < 1 || p->d_I < 16 || p->d_I % 16 || p->m < 1) return CSA_ERR_INVALID_ARG;
   if (p->qk_dtype < CSA_F32 || p->qk_dtype > CSA_NVFP4 || p->qk_dtype == CSA_BF16)
@@ -117,9 +121,9 @@ csa_status index_scores_impl(const csa_index_params* p, const void* q_I, const v
   a.q = q_I; a.q_scales = q_scales; a.w = w; a.k = k_I; a.k_scales = k_scales; a.q_pos = q_pos;
   a.T = T; a.H = p->H_I; a.d = p->d_I; a.m = p->m; a.qk_dtype = p->qk_dtype;
   a.score_dtype = p->score_dtype; a.E_cap = E_cap; a.E = E; a.scores = scores;
-  a.pdl = pdl; a.all_visible = all_visible; a.dep_entry = dep_entry;
+  a.pdl = pdl; a.all_visible = all_visible; a.dep_entry = dep_entry; a.q_raw = q_raw;
   csa_status st = launch_index_scores_tc(a, b, stream);
-  if (st != CSA_ERR_UNSUPPORTED) return st;
+  if (st != CSA_ERR_UNSUPPORTED || q_raw) return st;
   st = launch_index_scores_fp4_tc(a, b, stream);
   if (st != CSA_ERR_UNSUPPORTED) return st;
   return launch_index_scores_simt(a, b, stream);
@@ -347,6 +351,14 @@ size_t decode_layout(const csa_decode_params* p, void* ws, size_t cap, DecodeWs*
 
 }  // namespace
 
+namespace {
+// The FP8 tensor-core indexer quantises the bf16 index queries itself (so the prologue
+// does not, and the indexer does not wait for it except for the key page it writes).
+bool indexer_takes_raw_q(int hca, int idx_dtype, int kv_dtype, int H_I, int c_I) {
+  return !hca && idx_dtype == CSA_FP8_E4M3 && kv_dtype == CSA_BF16 && H_I == 64 && c_I == 128;
+}
+}  // namespace
+
 int csa_decode_launch_count(const csa_decode_params* p) {
   if (!p || p->b <= 0) return 0;
   int n = 1;                                   // prologue: compressors, quantiser, positions
@@ -413,13 +425,15 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
   pa.b = b; pa.t = t; pa.qpos = d.qpos;
   const void* qI = x->q_I;
   const void* qs = nullptr;
+  const bool raw_q = p->mode == CSA_MODE_FULL &&
+                     indexer_takes_raw_q(p->hca, p->idx_dtype, p->kv_dtype, p->H_I, p->c_I);
   if (!p->hca) {
     pa.index = pa.main;
     pa.index.C_a = x->CI_a; pa.index.Z_a = x->ZI_a; pa.index.B_a = x->BI_a;
     pa.index.C_b = x->CI_b; pa.index.Z_b = x->ZI_b; pa.index.B_b = x->BI_b;
     pa.index.c = p->c_I; pa.index.d_rope = p->d_rope_I; pa.index.out_dtype = p->idx_dtype;
     pa.index.out = x->kI_cache; pa.index.out_scales = x->kI_scales;
-    if (p->idx_dtype != CSA_F32) {
+    if (p->idx_dtype != CSA_F32 && !raw_q) {
       pa.q_in = x->q_I; pa.q_rows = b * p->H_I; pa.q_d = p->c_I; pa.q_dtype = p->idx_dtype;
       pa.q_codes = static_cast<uint8_t*>(d.qI_codes); pa.q_scales = d.qI_scales;
       qI = d.qI_codes; qs = d.qI_scales;
@@ -448,7 +462,7 @@ csa_status csa_decode(const csa_decode_params* p, const csa_decode_tensors* x, v
     //  predecessor drains and waits for it only where it reads its outputs)
     csa_index_params ip{p->H_I, p->c_I, p->m, p->idx_dtype, CSA_BF16};
     st = index_scores_impl(&ip, qI, qs, x->w, x->kI_cache, x->kI_scales, d.qpos, b, 1, p->E_cap,
-                           E, d.scores, stream, 1, 1, E - 1);
+                           E, d.scores, stream, 1, 1, E - 1, raw_q ? x->q_I : nullptr);
     if (st) return st;
     // 4. top-k
     int32_t* io = x->idx_out ? x->idx_out : d.idx;
@@ -580,6 +594,7 @@ csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* 
   pa.paged = 1; pa.win = x->win; pa.new_win = x->new_win; pa.win_ring = p->n_w;
   const void* qI = x->q_I;
   const void* qs = nullptr;
+  const bool raw_q = indexer_takes_raw_q(p->hca, p->idx_dtype, p->kv_dtype, p->H_I, p->c_I);
   if (!p->hca) {
     CompressArgs& ic = pa.index;
     ic = mc;
@@ -588,9 +603,11 @@ csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* 
     ic.c = p->c_I; ic.d_rope = p->d_rope_I; ic.out_dtype = p->idx_dtype;
     ic.out = x->kI_pages; ic.out_scales = x->kI_scales;
     ic.new_C_a = x->new_CI_a; ic.new_Z_a = x->new_ZI_a; ic.new_C_b = x->new_CI_b; ic.new_Z_b = x->new_ZI_b;
-    pa.q_in = x->q_I; pa.q_rows = b * p->H_I; pa.q_d = p->c_I; pa.q_dtype = p->idx_dtype;
-    pa.q_codes = static_cast<uint8_t*>(d.qI_codes); pa.q_scales = d.qI_scales;
-    qI = d.qI_codes; qs = d.qI_scales;
+    if (!raw_q) {
+      pa.q_in = x->q_I; pa.q_rows = b * p->H_I; pa.q_d = p->c_I; pa.q_dtype = p->idx_dtype;
+      pa.q_codes = static_cast<uint8_t*>(d.qI_codes); pa.q_scales = d.qI_scales;
+      qI = d.qI_codes; qs = d.qI_scales;
+    }
   }
   csa_status st = launch_decode_prologue(pa, p->kv_dtype, stream);
   if (st) return st;
@@ -599,14 +616,16 @@ csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* 
   if (!p->hca) {
     // 2. score the visible entries of every sequence (their pages through the block table)
     IndexArgs a{};
-    a.q = qI; a.q_scales = qs; a.w = x->w; a.k = x->kI_pages; a.k_scales = x->kI_scales;
+    a.q = raw_q ? x->q_I : qI; a.q_scales = raw_q ? x->kI_scales : qs; a.w = x->w;
+    a.q_raw = raw_q ? x->q_I : nullptr;
+    a.k = x->kI_pages; a.k_scales = x->kI_scales;
     a.q_pos = x->pos; a.T = 1; a.H = p->H_I; a.d = p->c_I; a.m = p->m; a.qk_dtype = p->idx_dtype;
     a.score_dtype = CSA_BF16; a.E_cap = p->max_pages * kPageEntries; a.E = std::max(E, 1);
     a.scores = d.scores; a.pdl = 1; a.all_visible = 0; a.dep_entry = -1;
     a.block_table = x->block_table; a.max_pages = p->max_pages; a.num_pages = p->num_pages;
     a.pos_input = 1;
     st = launch_index_scores_tc(a, b, stream);
-    if (st == CSA_ERR_UNSUPPORTED) st = launch_index_scores_fp4_tc(a, b, stream);
+    if (st == CSA_ERR_UNSUPPORTED && !raw_q) st = launch_index_scores_fp4_tc(a, b, stream);
     if (st) return st;
     // 3. top-k of each sequence's visible entries
     int32_t* io = x->idx_out ? x->idx_out : d.idx;

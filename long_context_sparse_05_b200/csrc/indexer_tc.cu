@@ -24,7 +24,11 @@
 //   warp 0  TMA producer: per stage one 2-D box of 128 TPS key rows (128-byte
 //           swizzle) and their fp32 key scales into an S-stage ring; per work unit
 //           the query group (64 QG x 128 B), its head weights and query scales
-//           into one of two buffers;
+//           into one of two buffers.  Decode with bf16 index queries: the
+//           epilogue warps quantise each unit's 64 query rows (FP8, one scale per
+//           row) into the buffer, a unit ahead, and the producer brings only the
+//           head weights, so that only the key stage holding the entry the
+//           preceding kernel writes waits for that kernel;
 //   warp 1  MMA issuer (one thread): 4 TPS x tcgen05.mma kind::f8f6f4 per stage
 //           into one of NACC TMEM accumulators;
 //   warps 2-9 epilogue, two warpgroups taking alternate stages (warps w and w+4
@@ -68,7 +72,53 @@ struct IdxTc {
   const int32_t* block_table;   // paged keys (one query per sequence: a stage is one page)
   int max_pages, num_pages;
   int pos_input;     // q_pos is an input: read before the wait; per-sequence dependent stage
+  const __nv_bfloat16* q_raw;   // QG = 1: bf16 index queries quantised here (else q by TMA)
 };
+
+// Raw index queries (bf16 [row][128]) of one warp's 8 rows r0 .. r0 + 7, four lanes per
+// row: lane l holds row r0 + l / 4, elements 32 (l % 4) .. 32 (l % 4) + 31.
+struct QRows { uint4 v[4]; };
+__device__ __forceinline__ void qrows_load(QRows& q, const __nv_bfloat16* row0, int lane) {
+  const uint4* src = reinterpret_cast<const uint4*>(row0 + (size_t)(lane >> 2) * kDim) + (lane & 3) * 4;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) q.v[j] = __ldg(src + j);
+}
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// FP8 quantisation of those rows (scale = amax / 448 per row, code = e4m3(x / scale), the
+// arithmetic of the stand-alone quantiser) into the 128-byte-swizzled B tile and the row
+// scales.  The code loop is rolled (it runs a few times per CTA, so its code is fetched
+// once); the register rows move to the front instead of being indexed.
+__device__ __noinline__ void qrows_quantise(QRows q, uint8_t* tile, float* scales, int r0, int lane) {
+  float am = 0.f;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t w[4] = {q.v[j].x, q.v[j].y, q.v[j].z, q.v[j].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) am = fmaxf(am, fmaxf(fabsf(bf16_lo(w[e])), fabsf(bf16_hi(w[e]))));
+  }
+  am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+  am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+  const float sc = am / 448.f;
+  const int row = r0 + (lane >> 2), qq = lane & 3;
+#pragma unroll 1
+  for (int j = 0; j < 4; ++j) {   // eight elements -> eight codes
+    const uint32_t w[4] = {q.v[0].x, q.v[0].y, q.v[0].z, q.v[0].w};
+    uint32_t c2[2] = {0u, 0u};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t lo = sc > 0.f ? (uint32_t)f32_to_e4m3(bf16_lo(w[e]) / sc) : 0u;
+      const uint32_t hi = sc > 0.f ? (uint32_t)f32_to_e4m3(bf16_hi(w[e]) / sc) : 0u;
+      c2[e >> 1] |= (lo | (hi << 8)) << (16 * (e & 1));
+    }
+    const int chunk = 2 * qq + (j >> 1);   // 16-byte chunk of the row
+    *reinterpret_cast<uint2*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4) + (j & 1) * 8) =
+        make_uint2(c2[0], c2[1]);
+    q.v[0] = q.v[1]; q.v[1] = q.v[2]; q.v[2] = q.v[3];
+  }
+  if (qq == 0) scales[row] = sc;
+}
 
 template <int QG>
 struct Layout {
@@ -117,6 +167,13 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   pdl_launch_dependents();
+  // raw index queries: the epilogue warps fetch their rows of the CTA's first unit now, so
+  // that the memory round trip overlaps the set-up (an input of the call)
+  QRows qfirst;
+  if (QG == 1 && p.q_raw && warp >= 2 && (int)blockIdx.x < p.units) {
+    const int sb0 = ((int)blockIdx.x / p.n_chunks) / p.n_qg, g0 = ((int)blockIdx.x / p.n_chunks) % p.n_qg;
+    qrows_load(qfirst, p.q_raw + ((size_t)(sb0 * p.T + g0 * QG) * kHeads + 8 * (warp - 2)) * kDim, lane);
+  }
   if (p.block_table) {
     // page ids of every stage of every unit this CTA walks, [local unit][stage of the
     // chunk]: inputs of the call, fetched at once while the CTA sets up instead of one
@@ -151,7 +208,7 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   if (threadIdx.x == 0) {
     for (int i = 0; i < S; ++i) { tc::mbar_init(&full[i], 1); tc::mbar_init(&empty[i], 1 + 4); }
     for (int i = 0; i < 2; ++i) {
-      tc::mbar_init(&bfull[i], 1);
+      tc::mbar_init(&bfull[i], 1 + (p.q_raw ? 4 * kEpiGroups : 0));
       tc::mbar_init(&bempty[i], 1 + 4 * kEpiGroups);
     }
     for (int i = 0; i < NACC; ++i) { tc::mbar_init(&tfull[i], 1); tc::mbar_init(&tempty[i], 4); }
@@ -179,60 +236,82 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
   };
 
   if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    // (lane 0 issues the copies; with raw index queries the whole warp quantises them)
+    auto load_stage = [&](int slot, int sb, int js, int li) {
+      int row0 = sb * p.E_cap + js * kStageE;
+      if (p.block_table) {
+        const uint32_t fl = (uint32_t)(li * p.chunk + js % p.chunk);
+        const int pg = fl < (uint32_t)kPagedSlots ? s_pg[fl]
+                                                    : p.block_table[(size_t)sb * p.max_pages + js];
+        row0 = ((unsigned)pg < (unsigned)p.num_pages ? pg : 0) * kStageE;
+      }
+      tc::mbar_arrive_expect_tx(&full[slot], LY::kStageKeyB + kStageE * 4);
+      tc::tma_load_2d(sA + slot * LY::kStageKeyB, &tmK, 0, row0, &full[slot]);
+      tc::tma_load_1d(sKS + slot * kStageE, &tmKS, row0, &full[slot]);
+    };
+    // first stage of sequence sb holding an entry the preceding kernel writes
+    auto dep_of = [&](int sb) {
+      if (!p.pos_input) return p.dep_stage;
+      const int t = p.q_pos[sb];   // the stage holding the entry the new token completes
+      return (t + 1) % p.m == 0 ? ((t + 1) / p.m - 1) / kStageE : INT_MAX;
+    };
+    // Key stages the preceding kernel does not write are fetched before waiting on it,
+    // into the first free slots, so that HBM streaming overlaps that kernel.
+    uint32_t npre = 0;
     if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      auto load_stage = [&](int slot, int sb, int js, int li) {
-        int row0 = sb * p.E_cap + js * kStageE;
-        if (p.block_table) {
-          const uint32_t fl = (uint32_t)(li * p.chunk + js % p.chunk);
-          const int pg = fl < (uint32_t)kPagedSlots ? s_pg[fl]
-                                                      : p.block_table[(size_t)sb * p.max_pages + js];
-          row0 = ((unsigned)pg < (unsigned)p.num_pages ? pg : 0) * kStageE;
-        }
-        tc::mbar_arrive_expect_tx(&full[slot], LY::kStageKeyB + kStageE * 4);
-        tc::tma_load_2d(sA + slot * LY::kStageKeyB, &tmK, 0, row0, &full[slot]);
-        tc::tma_load_1d(sKS + slot * kStageE, &tmKS, row0, &full[slot]);
-      };
-      // Key stages the preceding kernel does not write are fetched before waiting on it,
-      // into the first free slots, so that HBM streaming overlaps that kernel.
-      uint32_t npre = 0;
       for (int u = blockIdx.x, i = 0; u < p.units && npre == 0; u += gridDim.x, ++i) {
         int sb, g, js0, js1, nc, nq;
         unit(u, i, sb, g, js0, js1, nc, nq);
         if (nc == 0) continue;
-        int dep = p.dep_stage;
-        if (p.pos_input) {   // the stage holding the entry the sequence's new token completes
-          const int t = p.q_pos[sb];
-          dep = (t + 1) % p.m == 0 ? ((t + 1) / p.m - 1) / kStageE : INT_MAX;
-        }
+        const int dep = dep_of(sb);
         for (int js = js0; js < js0 + nc && (int)npre < S && js < dep; ++js, ++npre)
           load_stage(npre, sb, js, i);
         break;
       }
-      pdl_wait();
-      uint32_t it = 0, ul = 0;
-      bool ok = true;
-      for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
-        int sb, g, js0, js1, nc, nq;
-        unit(u, i, sb, g, js0, js1, nc, nq);
-        if (nc == 0) continue;
-        const int bb = ul & 1;
-        ok = tc::mbar_wait(&bempty[bb], ((ul >> 1) & 1) ^ 1, p.err);
-        if (!ok) break;
-        const int qrow0 = (sb * p.T + g * QG) * kHeads;
+    }
+    npre = __shfl_sync(0xffffffffu, npre, 0);
+    // quantised queries from the preceding kernel: wait for it before the first unit
+    bool waited = p.q_raw == nullptr;
+    if (waited) pdl_wait();
+    uint32_t it = 0, ul = 0;
+    bool ok = true;
+    for (int u = blockIdx.x, i = 0; u < p.units && ok; u += gridDim.x, ++i) {
+      int sb, g, js0, js1, nc, nq;
+      unit(u, i, sb, g, js0, js1, nc, nq);
+      if (nc == 0) continue;
+      const int bb = ul & 1;
+      if (lane == 0) ok = tc::mbar_wait(&bempty[bb], ((ul >> 1) & 1) ^ 1, p.err);
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+      if (!ok) break;
+      const int qrow0 = (sb * p.T + g * QG) * kHeads;
+      if (p.q_raw) {                  // the codes and scales come from the epilogue warps
+        if (lane == 0) {
+          tc::mbar_arrive_expect_tx(&bfull[bb], N * 4);
+          tc::tma_load_1d(sW + bb * N, &tmW, qrow0, &bfull[bb]);
+        }
+      } else if (lane == 0) {
         tc::mbar_arrive_expect_tx(&bfull[bb], kQBytes + 2 * N * 4);
         tc::tma_load_2d(sB + bb * kQBytes, &tmQ, 0, qrow0, &bfull[bb]);
         tc::tma_load_1d(sW + bb * N, &tmW, qrow0, &bfull[bb]);
         tc::tma_load_1d(sQS + bb * N, &tmQS, qrow0, &bfull[bb]);
-        for (int js = js0; js < js0 + nc; ++js, ++it) {
-          if (it < npre) continue;                       // fetched before the wait
-          const int s = it % S;
-          ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
-          if (!ok) break;
-          load_stage(s, sb, js, i);
-        }
-        ++ul;
       }
+      const int dep = waited ? INT_MAX : dep_of(sb);
+      for (int js = js0; js < js0 + nc; ++js, ++it) {
+        if (it < npre) continue;                       // fetched before the wait
+        if (js >= dep && !waited) {                    // this stage holds an entry the
+          pdl_wait();                                  // preceding kernel writes
+          waited = true;
+        }
+        const int s = it % S;
+        if (lane == 0) {
+          ok = tc::mbar_wait(&empty[s], ((it / S) & 1) ^ 1, p.err);
+          if (ok) load_stage(s, sb, js, i);
+        }
+        ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+        if (!ok) break;
+      }
+      ++ul;
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -284,11 +363,38 @@ index_scores_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_con
     float wq1[QG == 1 ? kHeads : 1];         // one query: its 64 weights live in registers
     uint32_t c = 0, ul = 0;                  // computed stages seen, units with work seen
     bool ok = true;
+    // raw index queries: this warp's 8 rows of the unit with work `nth` after (u, i), into
+    // buffer bb once its previous use is over (QG = 1)
+    auto quantise_unit = [&](int u, int i, int nth, uint32_t unit_no) {
+      for (; u < p.units; u += gridDim.x, ++i) {
+        int sb, g, js0, js1, nc, nq;
+        unit(u, i, sb, g, js0, js1, nc, nq);
+        if (nc == 0) continue;
+        if (nth-- > 0) continue;
+        const int bb = unit_no & 1;
+        ok = ok && tc::mbar_wait(&bempty[bb], ((unit_no >> 1) & 1) ^ 1, p.err);
+        const int r0 = 8 * ew;
+        QRows q = qfirst;                              // fetched at kernel start
+        if (u != (int)blockIdx.x)
+          qrows_load(q, p.q_raw + ((size_t)(sb * p.T + g * QG) * kHeads + r0) * kDim, lane);
+        qrows_quantise(q, sB + bb * kQBytes, sQS + bb * N, r0, lane);
+        tc::fence_proxy_async();   // the MMA reads the codes through the async proxy
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(&bfull[bb]);
+        return;
+      }
+    };
+    if (QG == 1 && p.q_raw) {        // the first two units' queries, one per buffer
+      quantise_unit(blockIdx.x, 0, 0, 0);
+      quantise_unit(blockIdx.x, 0, 1, 1);
+    }
     for (int u = blockIdx.x, i = 0; u < p.units; u += gridDim.x, ++i) {
       int sb, g, js0, js1, nc, nq;
       unit(u, i, sb, g, js0, js1, nc, nq);
       if (nc > 0) {
         const int bb = ul & 1;
+        // the queries of the unit after this one, into the buffer the previous unit freed
+        if (QG == 1 && p.q_raw && ul >= 1) quantise_unit(u, i, 1, ul + 1);
         tc::named_bar(1 + grp, 128);                   // previous unit's my_wq no longer read
         ok = ok && tc::mbar_wait(&bfull[bb], (ul >> 1) & 1, p.err);
         for (int x = gtid; x < N; x += 128) my_wq[x] = sW[bb * N + x] * sQS[bb * N + x];
@@ -401,11 +507,16 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   const uint64_t qrows = (uint64_t)b * a.T * kHeads;
   const uint64_t krows = a.block_table ? (uint64_t)a.num_pages * kPageEntries : (uint64_t)b * a.E_cap;
   if (!make_tmap_2d_u8(&tmK, a.k, kDim, krows, kDim, LY::kStageE) ||
-      !make_tmap_2d_u8(&tmQ, a.q, kDim, qrows, kDim, LY::N) ||
       !make_tmap_1d_f32(&tmKS, a.k_scales, krows, LY::kStageE) ||
-      !make_tmap_1d_f32(&tmW, a.w, qrows, LY::N) ||
-      !make_tmap_1d_f32(&tmQS, a.q_scales, qrows, LY::N))
+      !make_tmap_1d_f32(&tmW, a.w, qrows, LY::N))
     return CSA_ERR_CUDA;
+  if (a.q_raw) {           // quantised in the kernel: the query maps are not read
+    tmQ = tmK;
+    tmQS = tmKS;
+  } else if (!make_tmap_2d_u8(&tmQ, a.q, kDim, qrows, kDim, LY::N) ||
+             !make_tmap_1d_f32(&tmQS, a.q_scales, qrows, LY::N)) {
+    return CSA_ERR_CUDA;
+  }
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -431,6 +542,7 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
   p.dep_stage = a.dep_entry < 0 ? 0 : a.dep_entry / LY::kStageE;
   p.block_table = a.block_table; p.max_pages = a.max_pages; p.num_pages = a.num_pages;
   p.pos_input = a.pos_input;
+  p.q_raw = reinterpret_cast<const __nv_bfloat16*>(a.q_raw);
   long long grid = units < sms ? units : sms;
   const long long min_grid = (units + kMaxLocalUnits - 1) / kMaxLocalUnits;
   if (grid < min_grid) grid = min_grid;
@@ -453,9 +565,12 @@ csa_status launch_qg(const IndexArgs& a, int b, cudaStream_t st) {
 csa_status launch_index_scores_tc(const IndexArgs& a, int b, cudaStream_t st) {
   if (a.qk_dtype != CSA_FP8_E4M3 || a.H != kHeads || a.d != kDim) return CSA_ERR_UNSUPPORTED;
   if (a.block_table && (a.T != 1 || Layout<1>::kStageE != kPageEntries)) return CSA_ERR_UNSUPPORTED;
-  if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(a.q) & 15) ||
+  if (a.q_raw && a.T != 1) return CSA_ERR_UNSUPPORTED;
+  const void* qp = a.q_raw ? a.q_raw : a.q;
+  const void* qsp = a.q_raw ? a.k_scales : a.q_scales;
+  if ((reinterpret_cast<uintptr_t>(a.k) & 15) || (reinterpret_cast<uintptr_t>(qp) & 15) ||
       (reinterpret_cast<uintptr_t>(a.k_scales) & 15) || (reinterpret_cast<uintptr_t>(a.w) & 15) ||
-      (reinterpret_cast<uintptr_t>(a.q_scales) & 15) || (a.E_cap % 4))
+      (reinterpret_cast<uintptr_t>(qsp) & 15) || (a.E_cap % 4))
     return CSA_ERR_INVALID_ARG;   // the TMA copies need 16-byte aligned rows and scale runs
   if (a.T >= 4) return launch_qg<4, 4>(a, b, st);
   return launch_qg<1, 5>(a, b, st);

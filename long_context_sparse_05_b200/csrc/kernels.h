@@ -58,6 +58,10 @@ struct IndexArgs {
   // before waiting, and only the page of the entry the token completes, (t+1)/m - 1 when
   // (t+1) % m == 0, is written by the preceding kernel
   int pos_input;
+  // FP8 tensor-core path, one query per sequence: the index queries as bf16 [rows][128],
+  // quantised inside the kernel (q and q_scales unused).  An input of the call, so the
+  // key stages the preceding kernel does not write are scored without waiting for it.
+  const void* q_raw;
 };
 
 struct AttnArgs {

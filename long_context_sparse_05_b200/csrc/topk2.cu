@@ -19,14 +19,15 @@
 // the high 16) writes the selection in ascending entry order.
 //
 // Few long rows (decode: one query per sequence) spread each row over a thread-block
-// cluster of 2..16 CTAs, each holding a contiguous slice.  The search there splits
-// the candidate range into 16 power-of-two buckets per round (about 3 rounds for a
-// bf16 row), and every count is a cluster sum: warp 0 of each CTA pushes its 16
-// bucket counts into every CTA's shared memory with st.async, counted on the
-// receiver's mbarrier, so a round costs one one-way message instead of a cluster
-// barrier plus remote reads.  The final counts of keys above / equal to tau give
-// each CTA its exclusive prefix over the lower ranks, so the selection still comes
-// out in ascending entry order.
+// cluster of 2..16 CTAs, each holding a contiguous slice, and every count is a cluster
+// sum: warp 0 of each CTA pushes its counts into every CTA's shared memory with
+// st.async, counted on the receiver's mbarrier, so a round costs one one-way message
+// instead of a cluster barrier plus remote reads.  bf16 rows take two rounds of 256
+// buckets (the top byte of the 16-bit key, then the low byte) when each thread holds 8
+// keys, and the two histograms of every rank also give each CTA the keys above / equal
+// to tau of the lower ranks; otherwise (fp32 rows, 32 keys per thread) the candidate
+// range splits into 16 power-of-two buckets per round and those counts are exchanged
+// once more at the end.  Either way the selection comes out in ascending entry order.
 //
 // Rows longer than a cluster holds (16 x 16384) are cut into chunks: every chunk
 // keeps its own top-k (the global top-k is contained in the union, and since chunks
@@ -606,6 +607,256 @@ __global__ void __launch_bounds__(kNT) topk_cluster_kernel(
   cl_wait();
 }
 
+// bf16 rows over a cluster, in two rounds of 256 buckets: the top byte of the 16-bit key
+// over all visible keys, then the low byte over the keys whose top byte is the chosen
+// one, give the exact k-th key tau.  Each round's message is a CTA's 256 bucket counts
+// (16 bits each), pushed into every CTA of the cluster, so every CTA keeps every CTA's
+// two histograms: the keys above / equal to tau of the lower ranks (for the ascending
+// output) follow from them without a further exchange.
+constexpr int kHistWords = 128;   // 256 counts of 16 bits
+
+// Bucket counts of this warp into its own histogram s_wh (zeroed; shared atomics, so
+// only lanes of one warp contend).  Round A (top < 0): bucket = key >> 8 over the
+// visible keys; round B: bucket = key & 255 over the visible keys with key >> 8 == top.
+template <int EPT>
+__device__ __forceinline__ void hist256(const uint32_t (&key)[EPT], int j0, int n, int top,
+                                        uint32_t* s_wh) {
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const uint32_t kk = key[e];
+    const bool act = j0 + e < n && (top < 0 || (int)(kk >> 8) == top);
+    if (act) atomicAdd(&s_wh[top < 0 ? (kk >> 8) : (kk & 255u)], 1u);
+  }
+}
+// CTA histogram s_hist[b] = sum over the warps' histograms, each warp's zeroed again.
+__device__ __forceinline__ void sum_warp_hists(uint32_t* s_wh, uint32_t* s_hist, int nw) {
+  for (int b = threadIdx.x; b < 256; b += blockDim.x) {
+    uint32_t t = 0;
+    for (int w = 0; w < nw; ++w) { t += s_wh[w * 256 + b]; s_wh[w * 256 + b] = 0u; }
+    s_hist[b] = t;
+  }
+}
+
+// Warp 0: this CTA's histogram (16-bit counts, lane l: buckets 8l .. 8l + 7) into row
+// `rank` of slot `slot` of every CTA of the cluster, counted on that CTA's s_bar[slot].
+__device__ __forceinline__ void push_hist(const uint32_t* s_hist, uint32_t* s_msg, uint64_t* s_bar,
+                                          int slot, uint32_t cs, uint32_t rank) {
+  const int lane = threadIdx.x & 31;
+  const uint4 a = *reinterpret_cast<const uint4*>(s_hist + 8 * lane);
+  const uint4 b = *reinterpret_cast<const uint4*>(s_hist + 8 * lane + 4);
+  const uint4 v = make_uint4(a.x | (a.y << 16), a.z | (a.w << 16), b.x | (b.y << 16), b.z | (b.w << 16));
+  uint32_t* row = s_msg + (slot * kMaxClusterRanks + rank) * kHistWords + 4 * lane;
+  for (uint32_t r = 0; r < cs; ++r) st_async16(cl_map(row, r), v, cl_map(&s_bar[slot], r));
+}
+
+// Warp 0, after slot `slot` holds all cs histograms: the bucket B holding the krem-th
+// largest key (buckets above it hold fewer than krem keys, B and above at least krem)
+// and the count of keys in the buckets above B (every lane gets both).
+__device__ __forceinline__ void pick_bucket(const uint32_t* s_msg, int slot, uint32_t cs,
+                                            uint32_t krem, uint32_t& B, uint32_t& above_B) {
+  const int lane = threadIdx.x & 31;
+  uint32_t t[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  for (uint32_t r = 0; r < cs; ++r) {
+    const uint4 v = *reinterpret_cast<const uint4*>(s_msg + (slot * kMaxClusterRanks + r) * kHistWords + 4 * lane);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) { t[2 * i] += w[i] & 0xffffu; t[2 * i + 1] += w[i] >> 16; }
+  }
+  uint32_t tot = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) tot += t[i];
+  uint32_t suf = tot;                              // keys in the buckets of lanes >= this one
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_down_sync(0xffffffffu, suf, o);
+    if (lane + o < 32) suf += y;
+  }
+  const uint32_t higher = suf - tot;               // keys in the buckets of lanes above
+  uint32_t b_here = 0, above_here = 0;
+  const bool mine = higher < krem && suf >= krem;
+  if (mine) {
+    uint32_t s = higher;
+#pragma unroll
+    for (int i = 7; i >= 0; --i) {
+      if (s + t[i] >= krem) { b_here = 8 * lane + i; above_here = s; break; }
+      s += t[i];
+    }
+  }
+  const uint32_t who = __ballot_sync(0xffffffffu, mine);
+  const int src = who ? __ffs(who) - 1 : 0;
+  B = __shfl_sync(0xffffffffu, b_here, src);
+  above_B = __shfl_sync(0xffffffffu, above_here, src);
+}
+
+template <int EPT>
+__global__ void __launch_bounds__(kNT) topk_cluster256_kernel(
+    const __nv_bfloat16* __restrict__ scores, const int32_t* __restrict__ q_pos, int m, int E, int k,
+    int per, int32_t* __restrict__ idx, int32_t* __restrict__ count, int* err) {
+  using K = Keys<__nv_bfloat16>;
+  static_assert(EPT % 8 == 0, "keys are loaded in groups of 8");
+  __shared__ __align__(16) uint32_t s_hist[256];
+  __shared__ __align__(16) uint32_t s_wh[kNT / 32 * 256];                     // per-warp histograms
+  __shared__ __align__(16) uint32_t s_msg[2 * kMaxClusterRanks * kHistWords];
+  __shared__ __align__(8) uint64_t s_bar[2];
+  __shared__ uint32_t s_sc[32];
+  __shared__ uint32_t s_sel[4];
+  const uint32_t cs = cl_size(), rank = cl_rank();
+  const int tid = threadIdx.x, NT = blockDim.x;
+  const int lane = tid & 31, wid = tid >> 5, nw = NT >> 5;
+  if (tid == 0) {
+    // each slot is used once: both expect every rank's histogram
+    tc::mbar_init(&s_bar[0], 1);
+    tc::mbar_init(&s_bar[1], 1);
+    tc::fence_barrier_init();
+    tc::mbar_arrive_expect_tx(&s_bar[0], cs * kHistWords * 4);
+    tc::mbar_arrive_expect_tx(&s_bar[1], cs * kHistWords * 4);
+  }
+  for (int i = tid; i < nw * 256; i += NT) s_wh[i] = 0u;
+  cl_arrive();                                   // barriers initialised before any push
+  pdl_launch_dependents();
+  pdl_wait();
+  const int row = blockIdx.x / cs;
+  const int base = (int)rank * per;
+  const uint16_t* bits = reinterpret_cast<const uint16_t*>(scores + (size_t)row * E + base);
+  const int nl = max(0, min(E - base, per));     // entries of this slice in the row
+  const int j0 = tid * EPT;
+
+  uint32_t key[EPT];
+  const bool vec = ((reinterpret_cast<uintptr_t>(bits + j0) & 15) == 0) && j0 + EPT <= nl;
+  if (vec) {
+#pragma unroll
+    for (int v = 0; v < EPT / 8; ++v) {
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(bits + j0) + v);
+      const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        key[v * 8 + 2 * i] = w[i] & 0xffffu;
+        key[v * 8 + 2 * i + 1] = w[i] >> 16;
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < EPT; ++e) key[e] = j0 + e < nl ? bits[j0 + e] : 0u;
+  }
+  const int ev = visible_entries(q_pos[row], m, E);
+  const int n = max(0, min(ev - base, per));     // this CTA's visible entries
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) key[e] = j0 + e < n ? K::key(key[e]) : 0u;
+
+  int32_t* out = idx + (size_t)row * k;
+  if (ev <= k) {                                 // everything visible is kept
+    for (int j = (int)rank * NT + tid; j < k; j += (int)cs * NT) out[j] = j < ev ? j : -1;
+    if (rank == 0 && tid == 0) count[row] = ev;
+    cl_wait();
+    return;
+  }
+
+  // round A: the top byte
+  __syncthreads();                               // the warp histograms are zeroed
+  hist256<EPT>(key, j0, n, -1, s_wh + wid * 256);
+  __syncthreads();
+  sum_warp_hists(s_wh, s_hist, nw);
+  __syncthreads();
+  cl_wait();                                     // every CTA's barriers are initialised
+  if (wid == 0) push_hist(s_hist, s_msg, s_bar, 0, cs, rank);
+  if (wid == 0) {
+    const bool got = tc::mbar_wait(&s_bar[0], 0, err);
+    uint32_t B0, aboveA;
+    pick_bucket(s_msg, 0, cs, (uint32_t)k, B0, aboveA);
+    if (lane == 0) { s_sel[0] = got ? B0 : 0u; s_sel[1] = aboveA; }
+  }
+  __syncthreads();
+  const uint32_t B0 = s_sel[0], aboveA = s_sel[1];
+  // round B: the low byte among the keys with top byte B0
+  hist256<EPT>(key, j0, n, (int)B0, s_wh + wid * 256);
+  __syncthreads();
+  sum_warp_hists(s_wh, s_hist, nw);
+  __syncthreads();
+  if (wid == 0) push_hist(s_hist, s_msg, s_bar, 1, cs, rank);
+  if (wid == 0) {
+    const bool got = tc::mbar_wait(&s_bar[1], 0, err);
+    uint32_t B1, aboveB;
+    pick_bucket(s_msg, 1, cs, (uint32_t)k - aboveA, B1, aboveB);
+    // keys above / equal to tau of the ranks below this one, from their histograms
+    uint32_t G = 0, Q = 0;
+    for (uint32_t r = 0; r < rank; ++r) {
+      const uint4 a = *reinterpret_cast<const uint4*>(s_msg + (0 * kMaxClusterRanks + r) * kHistWords + 4 * lane);
+      const uint4 b = *reinterpret_cast<const uint4*>(s_msg + (1 * kMaxClusterRanks + r) * kHistWords + 4 * lane);
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w}, wb[4] = {b.x, b.y, b.z, b.w};
+      uint32_t g = 0, q = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t bin = 8 * lane + i;
+        const uint32_t ca = (i & 1) ? (wa[i >> 1] >> 16) : (wa[i >> 1] & 0xffffu);
+        const uint32_t cb = (i & 1) ? (wb[i >> 1] >> 16) : (wb[i >> 1] & 0xffffu);
+        g += (bin > B0 ? ca : 0u) + (bin > B1 ? cb : 0u);
+        q += bin == B1 ? cb : 0u;
+      }
+      G += __reduce_add_sync(0xffffffffu, g);
+      Q += __reduce_add_sync(0xffffffffu, q);
+    }
+    if (lane == 0) {
+      s_sel[0] = got ? ((B0 << 8) | B1) : 0xffffffffu;
+      s_sel[1] = aboveA + aboveB;                // keys above tau in the row
+      s_sel[2] = G;
+      s_sel[3] = Q;
+    }
+  }
+  __syncthreads();
+  cl_arrive();                                   // every push into this CTA has landed
+  const uint32_t tau = s_sel[0];
+  const int need = k - (int)s_sel[1];            // keys equal to tau to take, lowest first
+  const int G = (int)s_sel[2], Q = (int)s_sel[3];
+
+  uint32_t gt_mask = 0, eq_mask = 0;
+#pragma unroll
+  for (int e = 0; e < EPT; ++e) {
+    const bool v = j0 + e < n;
+    gt_mask |= (v && key[e] > tau ? 1u : 0u) << e;
+    eq_mask |= (v && key[e] == tau ? 1u : 0u) << e;
+  }
+  const uint32_t n_gt = __popc(gt_mask), n_eq = __popc(eq_mask);
+  const uint32_t packed = n_gt | (n_eq << 16);
+  uint32_t x = packed;                           // inclusive warp scan, warp totals to s_sc
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_sc[wid] = x;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t w = lane < nw ? s_sc[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    if (lane < nw) s_sc[lane] = w;
+  }
+  __syncthreads();
+  const uint32_t excl = (wid > 0 ? s_sc[wid - 1] : 0u) + x - packed;
+  const int gt_before = G + (int)(excl & 0xffffu);
+  const int eq_before = Q + (int)(excl >> 16);
+  const int take_eq = min(max(need - eq_before, 0), (int)n_eq);
+  uint32_t eq_take = 0, rest = eq_mask;
+  for (int i = 0; i < take_eq; ++i) {
+    const uint32_t low = rest & (0u - rest);
+    eq_take |= low;
+    rest ^= low;
+  }
+  uint32_t sel = gt_mask | eq_take;
+  int pos = gt_before + min(eq_before, need);
+  while (sel) {
+    const int e = __ffs(sel) - 1;
+    sel &= sel - 1;
+    if (pos >= 0 && pos < k) out[pos] = base + j0 + e;
+    ++pos;
+  }
+  if (rank == 0 && tid == 0) count[row] = k;
+  cl_wait();
+}
+
 int threads_for(int n) {
   const int nt = (n + kEPT - 1) / kEPT;
   return nt <= 128 ? 128 : (nt <= 256 ? 256 : 512);
@@ -620,11 +871,20 @@ int sm_count() {
   return sms;
 }
 
+// The cluster kernel of a score type and slice: two 256-bucket rounds for bf16 slices of
+// 8 keys per thread; the 16-bucket search for fp32 and for 32 keys per thread (there
+// the per-warp histograms of the first round contend more than the extra rounds cost).
+template <typename S, int EPT> struct ClusterKernel {
+  static constexpr auto fn = topk_cluster_kernel<S, EPT>;
+};
+template <> struct ClusterKernel<__nv_bfloat16, 8> {
+  static constexpr auto fn = topk_cluster256_kernel<8>;
+};
+
 template <typename S, int EPT>
 cudaError_t prep_cluster_kernel(int cs) {
   if (cs > 8)
-    return cudaFuncSetAttribute(topk_cluster_kernel<S, EPT>,
-                                cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    return cudaFuncSetAttribute(ClusterKernel<S, EPT>::fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   return cudaSuccess;
 }
 
@@ -651,13 +911,13 @@ bool cluster_fits(int cs, int nt, bool bf, int ept) {
   if (bf) {
     e = ept == 32 ? prep_cluster_kernel<__nv_bfloat16, 32>(cs) : prep_cluster_kernel<__nv_bfloat16, 8>(cs);
     if (e == cudaSuccess)
-      e = ept == 32 ? cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<__nv_bfloat16, 32>, &cfg)
-                    : cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<__nv_bfloat16, 8>, &cfg);
+      e = ept == 32 ? cudaOccupancyMaxActiveClusters(&n, ClusterKernel<__nv_bfloat16, 32>::fn, &cfg)
+                    : cudaOccupancyMaxActiveClusters(&n, ClusterKernel<__nv_bfloat16, 8>::fn, &cfg);
   } else {
     e = ept == 32 ? prep_cluster_kernel<float, 32>(cs) : prep_cluster_kernel<float, 8>(cs);
     if (e == cudaSuccess)
-      e = ept == 32 ? cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<float, 32>, &cfg)
-                    : cudaOccupancyMaxActiveClusters(&n, topk_cluster_kernel<float, 8>, &cfg);
+      e = ept == 32 ? cudaOccupancyMaxActiveClusters(&n, ClusterKernel<float, 32>::fn, &cfg)
+                    : cudaOccupancyMaxActiveClusters(&n, ClusterKernel<float, 8>::fn, &cfg);
   }
   if (e != cudaSuccess) { cudaGetLastError(); n = 0; }
   c = n > 0 ? 2 : 1;
@@ -744,9 +1004,9 @@ csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t
     cudaError_t e;
     if (bf) {
       const auto* sc = reinterpret_cast<const __nv_bfloat16*>(scores);
-      e = pl.ept == 32 ? cudaLaunchKernelEx(&cfg, topk_cluster_kernel<__nv_bfloat16, 32>, sc, q_pos, m,
+      e = pl.ept == 32 ? cudaLaunchKernelEx(&cfg, ClusterKernel<__nv_bfloat16, 32>::fn, sc, q_pos, m,
                                             E, k, pl.per, idx, count, err)
-                       : cudaLaunchKernelEx(&cfg, topk_cluster_kernel<__nv_bfloat16, 8>, sc, q_pos, m,
+                       : cudaLaunchKernelEx(&cfg, ClusterKernel<__nv_bfloat16, 8>::fn, sc, q_pos, m,
                                             E, k, pl.per, idx, count, err);
     } else {
       const auto* sc = reinterpret_cast<const float*>(scores);

@@ -188,3 +188,53 @@ def test_csa_prefill_fp8_sampled():
                                    g["C_a"], [t], g["sink"], w.n_w, w.scale)
             return o[0]
         _check_attention(w, out[t], ref["out"][j], same, recheck)
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_fused_fp8_decode_selection_equals_stage_calls(paged):
+    """The fused FP8 decode quantises the bf16 index queries inside the indexer (so that
+    only the key page the step writes waits for the compressor).  The same arithmetic as
+    csa_quantize: the selection is bit for bit the one of the stage calls (csa_quantize,
+    csa_index_scores, csa_topk) on the updated cache."""
+    from long_context_sparse_05_b200 import _lib as L
+    w = workloads.shrink(workloads.CSA_DECODE_64K, b=3, n=4100 - 4100 % 4)
+    inp = synth.make_inputs(w, device="cuda")
+    if paged:
+        st = runner.PagedDecodeState(w, inp, shuffle_seed=9)
+        st.step()
+        # each sequence's key rows in entry order, gathered from its pages
+        e = torch.arange(w.E, device="cuda")
+        PE = L.PAGE_ENTRIES
+        rows = st.block_table[:, e // PE].long() * PE + e % PE
+        kI = st.kI_pages[rows]
+        ks = st.kI_scales[rows]
+    else:
+        st = runner.DecodeState(w, inp)
+        st.build_caches()
+        st.step()
+        kI = st.kI_cache[:, :w.E].contiguous()
+        ks = st.kI_scales[:, :w.E].contiguous()
+    torch.cuda.synchronize()
+    E = w.E
+    E_cap = (E + 3) // 4 * 4
+    kIp = torch.zeros((w.b, E_cap, kI.shape[-1]), dtype=torch.uint8, device="cuda")
+    kIp[:, :E] = kI
+    ksp = torch.zeros((w.b, E_cap), dtype=torch.float32, device="cuda")
+    ksp[:, :E] = ks
+    rows_q = w.b * w.H_I
+    codes = torch.empty((rows_q, w.c_I), dtype=torch.uint8, device="cuda")
+    scales = torch.empty((rows_q,), dtype=torch.float32, device="cuda")
+    L.csa_quantize(L.CSA_BF16, L.CSA_FP8_E4M3, inp["q_I"], rows_q, w.c_I, codes, scales)
+    qpos = torch.full((w.b, 1), w.n - 1, dtype=torch.int32, device="cuda")
+    ip = L.IndexParams(H_I=w.H_I, d_I=w.c_I, m=w.m, qk_dtype=L.CSA_FP8_E4M3, score_dtype=L.CSA_BF16)
+    scores = torch.empty((w.b, 1, E), dtype=torch.bfloat16, device="cuda")
+    L.csa_index_scores(ip, codes, scales, inp["w"], kIp, ksp, qpos, w.b, 1, E_cap, E, scores)
+    idx = torch.empty((w.b, 1, w.k), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((w.b, 1), dtype=torch.int32, device="cuda")
+    wsb = L.csa_topk_workspace_size(L.CSA_BF16, w.b, 1, E, w.k)
+    ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device="cuda")
+    L.csa_topk(scores, L.CSA_BF16, qpos, w.m, w.b, 1, E, w.k, idx, cnt, ws, wsb)
+    torch.cuda.synchronize()
+    assert L.csa_device_error() == 0
+    assert torch.equal(cnt.view(-1), st.count.view(-1))
+    assert torch.equal(idx.view(w.b, -1), st.idx.view(w.b, -1))
