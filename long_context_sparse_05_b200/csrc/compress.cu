@@ -46,7 +46,9 @@ __device__ __forceinline__ void load16(const InT* p, float* dst) {
 constexpr int kUnroll = 4;
 
 // One compressed entry (entry i of sequence s) by the whole CTA; see compress_kernel.
-template <typename InT>
+// U rows per thread are loaded together (one memory round trip); the decode prologue,
+// which runs this code once per CTA, takes U = 2 so that less code is fetched.
+template <typename InT, int U = kUnroll>
 __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int s, float* smem) {
   constexpr int VEC = Vec16<InT>::N;
   const int c = a.c;
@@ -77,11 +79,11 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
   for (int v = 0; v < VEC; ++v) { mx[v] = -INFINITY; sum[v] = 0.f; acc[v] = 0.f; }
 
   if (g < rg) {
-    for (int r0 = g; r0 < R; r0 += rg * kUnroll) {
-      float zv[kUnroll][VEC], cv[kUnroll][VEC], bv[kUnroll][VEC];
-      bool live[kUnroll];
+    for (int r0 = g; r0 < R; r0 += rg * U) {
+      float zv[U][VEC], cv[U][VEC], bv[U][VEC];
+      bool live[U];
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int r = r0 + u * rg;
         live[u] = r < R;
         const InT *Z = nullptr, *C = nullptr;
@@ -100,12 +102,20 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
           const bool cur = Z == Za;
           load16<InT>(rowp(Z, cur ? a.new_Z_a : a.new_Z_b, row) + cc * VEC, zv[u]);
           load16<InT>(rowp(C, cur ? a.new_C_a : a.new_C_b, row) + cc * VEC, cv[u]);
+          if ((reinterpret_cast<uintptr_t>(B) & 15) == 0) {   // rows of c floats, c % 8 == 0
 #pragma unroll
-          for (int v = 0; v < VEC; ++v) bv[u][v] = __ldg(B + cc * VEC + v);
+            for (int v = 0; v < VEC; v += 4) {
+              const float4 b4 = __ldg(reinterpret_cast<const float4*>(B + cc * VEC + v));
+              bv[u][v] = b4.x; bv[u][v + 1] = b4.y; bv[u][v + 2] = b4.z; bv[u][v + 3] = b4.w;
+            }
+          } else {
+#pragma unroll
+            for (int v = 0; v < VEC; ++v) bv[u][v] = __ldg(B + cc * VEC + v);
+          }
         }
       }
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < U; ++u) {
         if (!live[u]) continue;
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
@@ -309,12 +319,12 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
     const int s = blk % a.b;
     const CompressArgs& ca = br == 0 ? a.main : a.index;
     if (!a.paged) {
-      compress_body<InT>(ca, ca.entry_begin, s, smem);
+      compress_body<InT, 2>(ca, ca.entry_begin, s, smem);
       return;
     }
     // paged state: the entry the newest token completes, if it completes one
     const int t = a.main.pos[s];
-    if (t >= 0 && (t + 1) % ca.m == 0) compress_body<InT>(ca, (t + 1) / ca.m - 1, s, smem);
+    if (t >= 0 && (t + 1) % ca.m == 0) compress_body<InT, 2>(ca, (t + 1) / ca.m - 1, s, smem);
     return;
   }
   if (a.paged && blk < a.b * (a.nbranch + 1)) {
