@@ -205,21 +205,28 @@ def timed_region(fn, steps, flush, stream, world, min_span_s, max_repeats=4000):
     return out, t0, t1
 
 
-# DRAM bytes (read + write) per processed key entry of a kernel, from the ncu captures under
-# profiles/ (ncu_full_csa_decode_64k_fp8_b4.md: the FP8 indexer at batch 4, 16384 entries per
-# sequence; ncu_full_index_scores_fp4_ctx256k_b2.md: the NVFP4 indexer at 256K context, batch
-# 2, 65536 entries per sequence).  The traffic is linear in the entries, so one launch's figure
-# is this times b * E of the launch timed.  A kernel changed after its capture has no entry
+# DRAM bytes (read + write) of one launch, from the ncu captures under profiles/, per unit the
+# launch processes, so that the figure scales to the launch timed:
+#   FP8 indexer: per key entry (ncu_full_index_scores_tc_csa_decode_64k_b4.md: batch 4,
+#     16384 entries per sequence); NVFP4 indexer: per key entry
+#     (ncu_full_index_scores_fp4_ctx256k_b2.md: batch 2, 65536 entries per sequence);
+#   decode attention of the 64K workload: per query (ncu_full_attn_tc_csa_decode_64k_b4.md:
+#     batch 4, 640 rows per query).
+# The traffic is linear in those units.  A kernel changed after its capture has no entry
 # here (its traffic is then reported as null).
-PROFILED_TRAFFIC_PER_ENTRY = {
-    ("index_scores", "fp8"): 8717056 / (4 * 16384),
-    ("index_scores", "nvfp4"): 9491712 / (2 * 65536),
+PROFILED_TRAFFIC = {
+    ("index_scores", "fp8"): ("entries", 8773376 / (4 * 16384)),
+    ("index_scores", "nvfp4"): ("entries", 9491712 / (2 * 65536)),
+    ("sparse_attn", "csa_decode_64k_fp8"): ("queries", 2978304 / 4),
 }
 
 
 def profiled_traffic(w, kernel):
-    per = PROFILED_TRAFFIC_PER_ENTRY.get((kernel, w.idx_dtype))
-    return None if per is None else round(per * w.b * w.E)
+    rec = PROFILED_TRAFFIC.get((kernel, w.idx_dtype)) or PROFILED_TRAFFIC.get((kernel, w.name))
+    if rec is None:
+        return None
+    unit, per = rec
+    return round(per * w.b * (w.E if unit == "entries" else 1))
 
 
 def kernel_record(us, amount, peak, unit="GB/s", bound="hbm"):
@@ -339,6 +346,9 @@ def stage_times_decode(w, st, steps, flush, stream):
     return {k: float(v) for k, v in res.items()}
 
 
+L2_BYTES = 126 * 1024 * 1024
+
+
 def e2e_decode(w, st, steps, flush, stream, world=1):
     """The decode step through the public serving call, csa_decode_paged, with host inputs.
 
@@ -347,52 +357,93 @@ def e2e_decode(w, st, steps, flush, stream, world=1):
     (its raw C / Z rows of both branches, its window row, q, q_I, w and the positions)
     from one pinned host buffer to one device staging buffer (a single H2D copy), runs
     the step on the staged tensors and reads the output back (one D2H copy).
-    Whole-job throughput: all ranks' tokens over the slowest rank's time."""
-    ps = runner.PagedDecodeState(w, st.x)
-    parts = [("pos", ps.pos)] + [(k, v) for k, v in ps.new.items()] + [("q", st.x["q"])]
-    if "q_I" in st.x:
-        parts += [("q_I", st.x["q_I"]), ("w", st.x["w"])]
-    # one staging layout shared by host and device: each part 256-byte aligned
-    offs, off = {}, 0
-    for n, v in parts:
-        offs[n] = off
-        off += (v.numel() * v.element_size() + 255) // 256 * 256
-    hstage = torch.empty(off, dtype=torch.uint8).pin_memory()
-    dstage = torch.empty(off, dtype=torch.uint8, device="cuda")
 
-    def view(buf, n, v):
-        nb = v.numel() * v.element_size()
-        return buf[offs[n]:offs[n] + nb].view(v.dtype).view(v.shape)
+    As a server overlaps the transfers of one batch with the compute of another, the
+    timed loop cycles through R independent batches (their own pages, state and staging
+    buffers) on three streams: H2D of step i, compute of step i, D2H of step i, each
+    ordered after what it depends on by events.  R is chosen so that the other batches'
+    steps touch more than twice the L2 between two uses of one batch (inputs larger than
+    L2, no flush inside the timed region).  Whole-job throughput: all ranks' tokens over
+    the slowest rank's time."""
+    step_bytes = runner.decode_bytes_per_step(w)
+    R = max(4, math.ceil(2 * L2_BYTES / max(step_bytes, 1)) + 1)
+    batches = []
+    for _ in range(R):
+        ps = runner.PagedDecodeState(w, st.x)
+        parts = [("pos", ps.pos)] + [(k, v) for k, v in ps.new.items()] + [("q", st.x["q"])]
+        if "q_I" in st.x:
+            parts += [("q_I", st.x["q_I"]), ("w", st.x["w"])]
+        # one staging layout shared by host and device: each part 256-byte aligned
+        offs, off = {}, 0
+        for n, v in parts:
+            offs[n] = off
+            off += (v.numel() * v.element_size() + 255) // 256 * 256
+        hstage = torch.empty(off, dtype=torch.uint8).pin_memory()
+        dstage = torch.empty(off, dtype=torch.uint8, device="cuda")
 
-    for n, v in parts:
-        view(hstage, n, v).copy_(v.contiguous().cpu())
-    dv = {n: view(dstage, n, v) for n, v in parts}
-    ps.pos = dv["pos"]
-    new = {k: dv[k] for k in ps.new}
-    hout = torch.empty(ps.out.shape, dtype=ps.out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for _, v in parts)
-    d2h = hout.numel() * hout.element_size()
+        def view(buf, n, v, offs=offs):
+            nb = v.numel() * v.element_size()
+            return buf[offs[n]:offs[n] + nb].view(v.dtype).view(v.shape)
 
-    def one():
-        dstage.copy_(hstage, non_blocking=True)
-        ps.step(stream, q=dv["q"], q_I=dv.get("q_I"), w_=dv.get("w"), new=new)
-        hout.copy_(ps.out, non_blocking=True)
+        for n, v in parts:
+            view(hstage, n, v).copy_(v.contiguous().cpu())
+        dv = {n: view(dstage, n, v) for n, v in parts}
+        ps.pos = dv["pos"]
+        new = {k: dv[k] for k in ps.new}
+        hout = torch.empty(ps.out.shape, dtype=ps.out.dtype).pin_memory()
+        ev = {k: torch.cuda.Event() for k in ("h2d", "done", "d2h")}
+        batches.append(dict(ps=ps, dv=dv, new=new, hstage=hstage, dstage=dstage, hout=hout, ev=ev))
+    h2d = batches[0]["hstage"].numel()          # the staging buffer crosses whole (256-byte parts)
+    d2h = batches[0]["hout"].numel() * batches[0]["hout"].element_size()
+    s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
 
-    for _ in range(3):
-        one()
-    torch.cuda.synchronize()
-    dev_times = timed_loop(lambda: ps.step(stream, q=dv["q"], q_I=dv.get("q_I"), w_=dv.get("w"),
-                                           new=new), steps, flush, stream)
+    def step_of(bt):
+        dv = bt["dv"]
+        bt["ps"].step(stream, q=dv["q"], q_I=dv.get("q_I"), w_=dv.get("w"), new=bt["new"])
+
+    def one(i):
+        bt = batches[i % R]
+        e = bt["ev"]
+        s_h2d.wait_event(e["done"])              # the batch's previous step has read its staging
+        with torch.cuda.stream(s_h2d):
+            bt["dstage"].copy_(bt["hstage"], non_blocking=True)
+        e["h2d"].record(s_h2d)
+        stream.wait_event(e["h2d"])
+        stream.wait_event(e["d2h"])              # its previous output has been read back
+        step_of(bt)
+        e["done"].record(stream)
+        s_d2h.wait_event(e["done"])
+        with torch.cuda.stream(s_d2h):
+            bt["hout"].copy_(bt["ps"].out, non_blocking=True)
+        e["d2h"].record(s_d2h)
+
+    def run(n):
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        t0.record(stream)
+        s_h2d.wait_event(t0)
+        for i in range(n):
+            one(i)
+        stream.wait_stream(s_d2h)
+        t1.record(stream)
+        torch.cuda.synchronize()
+        return t0.elapsed_time(t1) / n
+
+    run(2 * R)                                   # warm-up
+    dev_times = timed_loop(lambda: step_of(batches[0]), steps, flush, stream)
     barrier(world)
-    times = timed_loop(one, steps, flush, stream)
-    ms, _, value = aggregate(float(np.mean(times)), w.b, world)   # whole job, slowest rank
+    n = max(steps, 4 * R)
+    ms_local = float(np.median([run(n) for _ in range(3)]))
+    ms, _, value = aggregate(ms_local, w.b, world)   # whole job, slowest rank
     res = {"value": value, "unit": "tok/s", "h2d_bytes_per_step": int(h2d),
            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
            "copies_per_step": {"h2d": 1, "d2h": 1},
            "call": "csa_decode_paged (pages of %d entries, state rings)" % L.PAGE_ENTRIES,
+           "pipeline": "%d batches in rotation; H2D, step and D2H on three streams, "
+                       "ordered by events; no L2 flush (the batches' data exceed L2)" % R,
            "device_ms_per_step": round(float(np.mean(dev_times)), 4),
-           "gpu_launches_per_step": L.csa_decode_paged_launch_count(ps.p)}
-    del ps
+           "gpu_launches_per_step": L.csa_decode_paged_launch_count(batches[0]["ps"].p)}
+    del batches
     return res
 
 
