@@ -523,9 +523,20 @@ size_t csa_decode_paged_workspace_size(const csa_paged_params* p) {
   return paged_layout(p, nullptr, 0, nullptr);
 }
 
+namespace {
+// Paged c128a: the entry is compressed by the cluster-split kernel after the prologue
+// (which then only appends the rows and copies the positions).
+bool paged_split(const csa_paged_params* p) {
+  if (!p->hca) return false;
+  CompressArgs a{};
+  a.c = p->c; a.m = p->m; a.overlap = 0; a.out_dtype = p->kv_dtype; a.d_rope = p->d_rope;
+  return compress_split_supported(a, p->kv_dtype);
+}
+}  // namespace
+
 int csa_decode_paged_launch_count(const csa_paged_params* p) {
   if (!p || p->b <= 0 || p->m < 1) return 0;
-  int n = 1;
+  int n = 1 + (paged_split(p) ? 1 : 0);
   if (!p->hca) n += 1 + (topk_workspace_bytes(p->b, p->L_max / p->m, p->k, CSA_BF16) ? 2 : 1);
   n += attn_launch_count(p->H, p->c, p->hca ? 0 : p->k, p->n_w, p->b, 1,
                          p->max_pages * kPageEntries, p->kv_dtype);
@@ -609,8 +620,14 @@ csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* 
       qI = d.qI_codes; qs = d.qI_scales;
     }
   }
+  const bool split = paged_split(p);
+  pa.skip_compress = split ? 1 : 0;
   csa_status st = launch_decode_prologue(pa, p->kv_dtype, stream);
   if (st) return st;
+  if (split) {   // c128a: the block's 128 rows pooled over a cluster of CTAs
+    st = launch_compress_split(pa.main, p->kv_dtype, b, nullptr, 0, stream, true);
+    if (st) return st;
+  }
   const int32_t* idx = nullptr;
   const int32_t* cnt = nullptr;
   if (!p->hca) {

@@ -315,6 +315,7 @@ __global__ void __launch_bounds__(256) decode_prologue_kernel(PrologueArgs a) {
   pdl_launch_dependents();   // the indexer may start fetching the unchanged key tiles
   const int blk = blockIdx.x;
   if (blk < a.b * a.nbranch) {
+    if (a.skip_compress) return;   // the split kernel that follows compresses
     const int br = blk / a.b;
     const int s = blk % a.b;
     const CompressArgs& ca = br == 0 ? a.main : a.index;
@@ -425,15 +426,30 @@ __global__ void __launch_bounds__(256) compress_split_kernel(CompressArgs a, int
   const int CS = gridDim.x;
   const int rank = (int)cs_rank();
   const int s = blockIdx.y;
-  const int i = a.entry_begin;
   const int rpr = m / CS;
   pdl_launch_dependents();
-  pdl_wait();
+  // paged state: the entry the sequence's new token completes, if it completes one (the
+  // same for every CTA of the cluster); the preceding kernel (ring appends, positions) is
+  // waited for at the end, so that this kernel's completion implies its completion
+  int i = a.entry_begin, t_new = -1;
+  if (a.ring) {
+    const int tp = a.pos[s];
+    if (tp < 0 || (tp + 1) % m != 0) { pdl_wait(); return; }
+    i = (tp + 1) / m - 1;
+    t_new = tp;
+  } else {
+    pdl_wait();
+  }
   if (qpos && blockIdx.x == 0 && blockIdx.y == 0)
     for (int x = tid; x < nq; x += blockDim.x) qpos[x] = t;   // query positions of the step
-
-  const InT* Ca = reinterpret_cast<const InT*>(a.C_a) + (size_t)s * a.n * c;
-  const InT* Za = reinterpret_cast<const InT*>(a.Z_a) + (size_t)s * a.n * c;
+  const size_t seq_rows = a.ring ? (size_t)a.ring : (size_t)a.n;
+  const InT* Ca = reinterpret_cast<const InT*>(a.C_a) + (size_t)s * seq_rows * c;
+  const InT* Za = reinterpret_cast<const InT*>(a.Z_a) + (size_t)s * seq_rows * c;
+  auto rowp = [&](const InT* base, const void* fresh, size_t row) -> const InT* {
+    if (!a.ring) return base + row * c;
+    if ((long long)row == t_new) return reinterpret_cast<const InT*>(fresh) + (size_t)s * c;
+    return base + (row % a.ring) * c;
+  };
   float mx[VEC], sum[VEC], acc[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) { mx[v] = -INFINITY; sum[v] = 0.f; acc[v] = 0.f; }
@@ -448,8 +464,8 @@ __global__ void __launch_bounds__(256) compress_split_kernel(CompressArgs a, int
         if (live[u]) {
           const int r = rank * rpr + q;             // row inside the block
           const size_t row = (size_t)m * i + r;
-          load16<InT>(Za + row * c + cc * VEC, zv[u]);
-          load16<InT>(Ca + row * c + cc * VEC, cv[u]);
+          load16<InT>(rowp(Za, a.new_Z_a, row) + cc * VEC, zv[u]);
+          load16<InT>(rowp(Ca, a.new_C_a, row) + cc * VEC, cv[u]);
 #pragma unroll
           for (int v = 0; v < VEC; ++v) bv[u][v] = __ldg(a.B_a + (size_t)r * c + cc * VEC + v);
         }
@@ -547,7 +563,9 @@ __global__ void __launch_bounds__(256) compress_split_kernel(CompressArgs a, int
   }
   // RMSNorm + RoPE on this rank's channels (pairs stay inside a rank: cpr is even)
   const int rope0 = c - a.d_rope;
-  const size_t orow = (size_t)s * a.out_E + i;
+  const size_t orow = a.block_table
+      ? (size_t)a.block_table[(size_t)s * a.max_pages + i / kPageEntries] * kPageEntries + i % kPageEntries
+      : (size_t)s * a.out_E + i;
   for (int pj = tid; pj < cpr / 2; pj += blockDim.x) {
     const int ch = ch0 + 2 * pj;
     float x0 = s_x[ch] * inv, x1 = s_x[ch + 1] * inv;
@@ -570,6 +588,7 @@ __global__ void __launch_bounds__(256) compress_split_kernel(CompressArgs a, int
     }
   }
   cs_sync();   // peers are done reading this CTA's shared memory
+  if (a.ring) pdl_wait();
 }
 
 void fill_inv_freq(CompressArgs& a) {
@@ -585,19 +604,26 @@ size_t compress_smem_bytes(const CompressArgs& a, int in_dtype, int nt) {
 }
 
 // Split launch for one long non-overlapped block per sequence (c128a decode).
+constexpr int kSplitCS = 8;
+constexpr int kSplitThreads = 256;
+size_t split_smem_bytes(const CompressArgs& a, int in_dtype) {
+  const int cols = a.c / (in_dtype == CSA_F32 ? 4 : 8);
+  return (size_t)(3 * (kSplitThreads / cols) * a.c + a.c + 32 + 4) * sizeof(float);
+}
+bool compress_split_supported(const CompressArgs& a, int in_dtype) {
+  const int cols = a.c / (in_dtype == CSA_F32 ? 4 : 8);
+  return cols <= kSplitThreads && a.m % kSplitCS == 0 && a.c % (2 * kSplitCS) == 0 && !a.overlap &&
+         (a.out_dtype == CSA_F32 || a.out_dtype == CSA_BF16) && (a.c - a.d_rope) % 2 == 0 &&
+         split_smem_bytes(a, in_dtype) <= 200 * 1024;
+}
+
 csa_status launch_compress_split(CompressArgs& a, int in_dtype, int b, int32_t* qpos, int t,
                                  cudaStream_t st, bool pdl) {
-  constexpr int CS = 8;
-  const int nt = 256;
-  const int vec = in_dtype == CSA_F32 ? 4 : 8;
-  const int cols = a.c / vec;
-  if (cols > nt || a.m % CS || a.c % (2 * CS) || a.overlap) return CSA_ERR_UNSUPPORTED;
-  if (a.out_dtype != CSA_F32 && a.out_dtype != CSA_BF16) return CSA_ERR_UNSUPPORTED;
-  if ((a.c - a.d_rope) % 2) return CSA_ERR_UNSUPPORTED;
+  constexpr int CS = kSplitCS;
+  const int nt = kSplitThreads;
+  if (!compress_split_supported(a, in_dtype)) return CSA_ERR_UNSUPPORTED;
   fill_inv_freq(a);
-  const int rg = nt / cols;
-  const size_t smem = (size_t)(3 * rg * a.c + a.c + 32 + 4) * sizeof(float);
-  if (smem > 200 * 1024) return CSA_ERR_UNSUPPORTED;
+  const size_t smem = split_smem_bytes(a, in_dtype);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(CS, b);
   cfg.blockDim = dim3(nt);

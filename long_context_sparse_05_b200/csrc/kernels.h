@@ -39,6 +39,8 @@ struct PrologueArgs {
   // an entry only for sequences whose block the token completes
   int paged;
   void* win; const void* new_win; int win_ring;
+  // paged c128a: the entries are compressed by the cluster-split kernel launched next
+  int skip_compress;
 };
 
 struct IndexArgs {
@@ -85,6 +87,12 @@ constexpr int kMaxOutRopePairs = 32;   // rotary pairs of the output with a host
 csa_status launch_compress(const CompressArgs& a, int in_dtype, int b, int entry_count,
                            cudaStream_t st);
 csa_status launch_decode_prologue(PrologueArgs& a, int in_dtype, cudaStream_t st);
+// One long non-overlapped block (c128a) per sequence over a cluster of CTAs.  With a.ring
+// (paged state) it compresses only for sequences whose new token completes a block and
+// waits for the preceding kernel at its end, so that its completion implies that kernel's.
+bool compress_split_supported(const CompressArgs& a, int in_dtype);
+csa_status launch_compress_split(CompressArgs& a, int in_dtype, int b, int32_t* qpos, int t,
+                                 cudaStream_t st, bool pdl);
 csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
                            void* codes, void* scales, cudaStream_t st);
 csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
