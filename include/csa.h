@@ -133,6 +133,9 @@ typedef struct {
   int apply_norm;     /* 1: RMSNorm with unit gain; 0: skip (identity checks) */
   int in_dtype;       /* CSA_F32 or CSA_BF16: type of C_* and Z_* */
   int out_dtype;      /* CSA_F32, CSA_BF16, CSA_FP8_E4M3 or CSA_NVFP4 */
+  int out_entry_offset; /* entry i is written at row i - out_entry_offset of each sequence's
+                           out (a shard of the entries, as in context-parallel decode); 0 for
+                           a whole cache; a multiple of 128 for NVFP4 output */
 } csa_compress_params;
 
 /*
@@ -559,6 +562,57 @@ csa_status csa_prefill(const csa_prefill_params* p, const csa_prefill_tensors* x
 size_t csa_prefill_workspace_size(const csa_prefill_params* p);
 /* Number of kernel launches one csa_prefill call makes with these parameters; host only. */
 int csa_prefill_launch_count(const csa_prefill_params* p);
+
+/* ------------------------------------------------------------------------ */
+/* Context-parallel decode: each sequence's compressed entries sharded       */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Source: "DeepSeek Technical Reports", section DSA (the k best index scores of a query
+ * select the entries it attends to).  A long cache is split into contiguous shards of
+ * entries, one per rank; rank r holds entries [entry_offset, entry_offset + E_local) of
+ * every sequence.  A decode step then runs:
+ *   1. csa_index_scores and csa_topk on the rank's shard, with the query positions
+ *      shifted by -m * entry_offset (the entries visible to t are those below
+ *      E(t) - entry_offset in the shard);
+ *   2. csa_cp_candidates: the rank's top-k as (bf16 score, global entry) pairs;
+ *   3. an all-gather of the candidates over the ranks (the caller's collective), rank r's
+ *      block at index r;
+ *   4. csa_cp_merge: the top-k of the gathered candidates, which is exactly the top-k of
+ *      the whole cache (every entry of the global top-k is among its shard's k best under
+ *      the same order: score descending, entry ascending); entries ascending, -1 padded;
+ *   5. csa_cp_pack_rows: the selected rows this rank holds, into their selection slots
+ *      (zeros elsewhere), then a sum over the ranks (the caller's all-reduce) gathers
+ *      the selected rows on every rank;
+ *   6. csa_sparse_attn over the gathered rows (E_cap = k, selection rows_idx) and the
+ *      window, which every rank holds.
+ * The pages speak of no context parallelism; this follows from the top-k's definition.
+ * All pointers are device memory, all calls asynchronous on the stream.
+ */
+
+/* cand_scores [b][k] bf16 and cand_idx [b][k] int32 from the rank's scores ([b][E_local]
+ * bf16) and its top-k (idx [b][k] local entries, count [b]): the score and the global
+ * entry (entry_offset + local) of each selected entry; -inf and -1 past count. */
+csa_status csa_cp_candidates(const void* scores, int E_local, const int32_t* idx,
+                             const int32_t* count, int b, int k, int entry_offset,
+                             void* cand_scores, int32_t* cand_idx, cudaStream_t stream);
+
+/* Top-k of G ranks' candidates: cand_scores [G][b][k] bf16, cand_idx [G][b][k] (rank r's
+ * entries all below rank r + 1's).  Writes idx [b][k] (global entries, ascending, -1
+ * padded), count [b] and rows_idx [b][k] (0 .. count - 1, then -1: the selection of the
+ * gathered rows).  ws: csa_cp_merge_workspace_size() bytes, 256-byte aligned. */
+size_t csa_cp_merge_workspace_size(int G, int b, int k);
+csa_status csa_cp_merge(const void* cand_scores, const int32_t* cand_idx, int G, int b, int k,
+                        int32_t* idx, int32_t* count, int32_t* rows_idx, void* ws, size_t ws_bytes,
+                        cudaStream_t stream);
+
+/* rows [b][k][c] (kv_dtype): slot j of sequence s is row (idx[s][j] - entry_offset) of
+ * the rank's shard kv_local ([b][E_cap_local][c]) when entry_offset <= idx[s][j] <
+ * entry_offset + E_local and j < count[s]; zeros otherwise.  c * element size must be a
+ * multiple of 16; kv_local and rows 16-byte aligned. */
+csa_status csa_cp_pack_rows(const void* kv_local, int E_cap_local, int E_local, int entry_offset,
+                            int c, int kv_dtype, const int32_t* idx, const int32_t* count, int b,
+                            int k, void* rows, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

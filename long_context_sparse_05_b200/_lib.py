@@ -28,7 +28,7 @@ class CsaError(RuntimeError):
 class CompressParams(ctypes.Structure):
     _fields_ = [("m", c_int), ("overlap", c_int), ("c", c_int), ("d_rope", c_int),
                 ("rope_theta", c_double), ("eps", c_float), ("apply_norm", c_int),
-                ("in_dtype", c_int), ("out_dtype", c_int)]
+                ("in_dtype", c_int), ("out_dtype", c_int), ("out_entry_offset", c_int)]
 
 
 class IndexParams(ctypes.Structure):
@@ -143,6 +143,13 @@ _SIGS = {
     "csa_decode_paged_workspace_size": (c_size_t, [ctypes.POINTER(PagedParams)]),
     "csa_decode_paged_launch_count": (c_int, [ctypes.POINTER(PagedParams)]),
     "csa_prefill_launch_count": (c_int, [ctypes.POINTER(PrefillParams)]),
+    "csa_cp_candidates": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_int,
+                                  c_void_p, c_void_p, c_void_p]),
+    "csa_cp_merge_workspace_size": (c_size_t, [c_int, c_int, c_int]),
+    "csa_cp_merge": (c_int, [c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p,
+                             c_void_p, c_size_t, c_void_p]),
+    "csa_cp_pack_rows": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_int, c_void_p, c_void_p,
+                                 c_int, c_int, c_void_p, c_void_p]),
 }
 
 
@@ -333,3 +340,27 @@ def csa_decode_paged(p, tensors, ws, ws_bytes=None, stream=None):
         ws_bytes = ws.numel() * ws.element_size()
     _check(lib().csa_decode_paged(ctypes.byref(p), ctypes.byref(x), _ptr(ws), ws_bytes,
                                   _stream(stream)))
+
+
+# ---------------------------------------------------------------- context-parallel decode
+
+def csa_cp_candidates(scores, E_local, idx, count, b, k, entry_offset, cand_scores, cand_idx,
+                      stream=None):
+    _check(lib().csa_cp_candidates(_ptr(scores), E_local, _ptr(idx), _ptr(count), b, k,
+                                   entry_offset, _ptr(cand_scores), _ptr(cand_idx),
+                                   _stream(stream)))
+
+
+def csa_cp_merge_workspace_size(G, b, k):
+    return int(lib().csa_cp_merge_workspace_size(G, b, k))
+
+
+def csa_cp_merge(cand_scores, cand_idx, G, b, k, idx, count, rows_idx, ws, ws_bytes, stream=None):
+    _check(lib().csa_cp_merge(_ptr(cand_scores), _ptr(cand_idx), G, b, k, _ptr(idx), _ptr(count),
+                              _ptr(rows_idx), _ptr(ws), ws_bytes, _stream(stream)))
+
+
+def csa_cp_pack_rows(kv_local, E_cap_local, E_local, entry_offset, c, kv_dtype, idx, count, b, k,
+                     rows, stream=None):
+    _check(lib().csa_cp_pack_rows(_ptr(kv_local), E_cap_local, E_local, entry_offset, c, kv_dtype,
+                                  _ptr(idx), _ptr(count), b, k, _ptr(rows), _stream(stream)))

@@ -68,7 +68,10 @@ csa_status csa_compress(const csa_compress_params* p, const void* C_a, const voi
   if (p->in_dtype == CSA_F32 && p->c % 4) return CSA_ERR_INVALID_ARG;
   if (b < 0 || n < 0 || entry_begin < 0 || entry_count < 0) return CSA_ERR_INVALID_ARG;
   if ((long long)p->m * (entry_begin + entry_count) > n) return CSA_ERR_INVALID_ARG;
-  if (entry_begin + entry_count > out_entries_per_seq) return CSA_ERR_INVALID_ARG;
+  const int off = p->out_entry_offset;
+  if (off < 0 || entry_begin < off || entry_begin + entry_count - off > out_entries_per_seq)
+    return CSA_ERR_INVALID_ARG;
+  if (p->out_dtype == CSA_NVFP4 && off % 128) return CSA_ERR_INVALID_ARG;
   if (b == 0 || entry_count == 0) return CSA_OK;
   if (!C_a || !Z_a || !B_a || !out) return CSA_ERR_INVALID_ARG;
   if (p->overlap && (!C_b || !Z_b || !B_b)) return CSA_ERR_INVALID_ARG;
@@ -81,7 +84,7 @@ csa_status csa_compress(const csa_compress_params* p, const void* C_a, const voi
   a.n = n; a.m = p->m; a.overlap = p->overlap ? 1 : 0; a.c = p->c; a.d_rope = p->d_rope;
   a.apply_norm = p->apply_norm; a.out_dtype = p->out_dtype; a.entry_begin = entry_begin;
   a.out_E = out_entries_per_seq; a.theta = p->rope_theta; a.eps = p->eps;
-  a.out = out; a.out_scales = out_scales;
+  a.out = out; a.out_scales = out_scales; a.out_off = off;
   return launch_compress(a, p->in_dtype, b, entry_count, stream);
 }
 
@@ -664,6 +667,51 @@ csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* 
   st = launch_attn_tc(a, b, p->kv_dtype, d.attn_ws, d.attn_ws_bytes, stream);
   if (st == CSA_ERR_UNSUPPORTED) st = launch_attn_simt(a, b, p->kv_dtype, stream);
   return st;
+}
+
+// ---------------------------------------------------------------------------
+// context-parallel decode (entries sharded over ranks)
+// ---------------------------------------------------------------------------
+
+csa_status csa_cp_candidates(const void* scores, int E_local, const int32_t* idx,
+                             const int32_t* count, int b, int k, int entry_offset,
+                             void* cand_scores, int32_t* cand_idx, cudaStream_t stream) {
+  if (b < 0 || k < 1 || E_local < 0 || entry_offset < 0) return CSA_ERR_INVALID_ARG;
+  if (b == 0) return CSA_OK;
+  if (!scores || !idx || !count || !cand_scores || !cand_idx) return CSA_ERR_INVALID_ARG;
+  return launch_cp_candidates(scores, E_local, idx, count, b, k, entry_offset, cand_scores, cand_idx,
+                              stream);
+}
+
+size_t csa_cp_merge_workspace_size(int G, int b, int k) {
+  if (G < 1 || b < 0 || k < 1) return 0;
+  return cp_merge_bytes(G, b, k, topk_workspace_bytes(b, G * k, k, CSA_BF16)) + 256;
+}
+
+csa_status csa_cp_merge(const void* cand_scores, const int32_t* cand_idx, int G, int b, int k,
+                        int32_t* idx, int32_t* count, int32_t* rows_idx, void* ws, size_t ws_bytes,
+                        cudaStream_t stream) {
+  if (G < 1 || b < 0 || k < 1 || (long long)G * k > (1 << 30)) return CSA_ERR_INVALID_ARG;
+  if (b == 0) return CSA_OK;
+  if (!cand_scores || !cand_idx || !idx || !count || !rows_idx || !ws) return CSA_ERR_INVALID_ARG;
+  if (ws_bytes < csa_cp_merge_workspace_size(G, b, k) || (reinterpret_cast<uintptr_t>(ws) & 255))
+    return CSA_ERR_INVALID_ARG;
+  return launch_cp_merge(cand_scores, cand_idx, G, b, k, idx, count, rows_idx, ws, ws_bytes, stream);
+}
+
+csa_status csa_cp_pack_rows(const void* kv_local, int E_cap_local, int E_local, int entry_offset,
+                            int c, int kv_dtype, const int32_t* idx, const int32_t* count, int b,
+                            int k, void* rows, cudaStream_t stream) {
+  if (b < 0 || k < 1 || c < 8 || E_local < 0 || E_local > E_cap_local || entry_offset < 0)
+    return CSA_ERR_INVALID_ARG;
+  if (kv_dtype != CSA_F32 && kv_dtype != CSA_BF16) return CSA_ERR_INVALID_ARG;
+  const size_t row_bytes = (size_t)c * (kv_dtype == CSA_F32 ? 4 : 2);
+  if (row_bytes % 16) return CSA_ERR_INVALID_ARG;
+  if (b == 0) return CSA_OK;
+  if (!kv_local || !idx || !count || !rows || !aligned16(kv_local) || !aligned16(rows))
+    return CSA_ERR_INVALID_ARG;
+  return launch_cp_pack(kv_local, E_cap_local, E_local, entry_offset, row_bytes, idx, count, b, k,
+                        rows, stream);
 }
 
 // ---------------------------------------------------------------------------

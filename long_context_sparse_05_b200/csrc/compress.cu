@@ -191,10 +191,11 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
   }
   __syncthreads();
 
-  // physical output row (paged: the page of entry i from the sequence's block table)
+  // physical output row (paged: the page of entry i from the sequence's block table; a
+  // shard of the entries: row i - out_off)
   const size_t orow = a.block_table
       ? (size_t)a.block_table[(size_t)s * a.max_pages + i / kPageEntries] * kPageEntries + i % kPageEntries
-      : (size_t)s * a.out_E + i;
+      : (size_t)s * a.out_E + (i - a.out_off);
   if (a.out_dtype == CSA_F32) {
     float* o = reinterpret_cast<float*>(a.out) + orow * c;
     for (int ch = tid; ch < c; ch += blockDim.x) o[ch] = s_x[ch];
@@ -215,7 +216,7 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
     // the tiled key-scale layout of the sequence, or (paged) of all pages as one array
     uint8_t* so = reinterpret_cast<uint8_t*>(a.out_scales) +
                   (a.block_table ? (size_t)0 : (size_t)s * nvfp4_key_scale_seq_bytes(a.out_E, c));
-    const long long srow = a.block_table ? (long long)orow : (long long)i;
+    const long long srow = a.block_table ? (long long)orow : (long long)(i - a.out_off);
     for (int blk = tid; blk < c / 16; blk += blockDim.x) {
       float am = 0.f;
 #pragma unroll

@@ -25,6 +25,8 @@ struct CompressArgs {
   const void *new_C_a, *new_Z_a, *new_C_b, *new_Z_b;
   const int32_t* block_table;
   int max_pages;
+  // entry i goes to row i - out_off of its sequence (a shard of the entries); 0: row i
+  int out_off;
 };
 
 constexpr int kPageEntries = CSA_PAGE_ENTRIES;   // compressed entries per page of the paged caches
@@ -95,6 +97,19 @@ csa_status launch_compress_split(CompressArgs& a, int in_dtype, int b, int32_t* 
                                  cudaStream_t st, bool pdl);
 csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows, int d,
                            void* codes, void* scales, cudaStream_t st);
+// Context-parallel decode (cp.cu): a rank's top-k as (score, global entry) candidates; the
+// top-k of every rank's candidates (workspace of cp_merge_bytes); the selected rows a rank
+// holds packed into their selection slots.
+csa_status launch_cp_candidates(const void* scores, int E_local, const int32_t* idx,
+                                const int32_t* count, int b, int k, int offset, void* cand_s,
+                                int32_t* cand_i, cudaStream_t st);
+size_t cp_merge_bytes(int G, int b, int k, size_t topk_ws);
+csa_status launch_cp_merge(const void* cand_s, const int32_t* cand_i, int G, int b, int k,
+                           int32_t* idx, int32_t* count, int32_t* rows_idx, void* ws,
+                           size_t ws_bytes, cudaStream_t st);
+csa_status launch_cp_pack(const void* kv, int E_cap_local, int E_local, int offset, size_t row_bytes,
+                          const int32_t* idx, const int32_t* count, int b, int k, void* rows,
+                          cudaStream_t st);
 csa_status launch_topk_search(const void* scores, int score_dtype, const int32_t* q_pos, int m,
                               int rows, int E, int k, int32_t* idx, int32_t* count, void* ws,
                               size_t ws_bytes, cudaStream_t st, bool pdl = false);
