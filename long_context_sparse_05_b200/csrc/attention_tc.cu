@@ -554,6 +554,17 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         lgb[h] = __float_as_uint(l);
         v[h] = l;
       }
+      // After the first tile, the common case: no logit exceeds the running maximum by more
+      // than the rescale threshold, so the running maximum stays this tile's reference
+      // (p <= 2^8) and no maximum pass or rescale is needed; otherwise the exact pass.
+      bool exact = j == jb;
+      if (!exact) {
+        bool big = false;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) big |= __uint_as_float(lgb[h]) > s_M[32 * hf + h] + kRescaleThresh;
+        exact = tc::bar_red_or(3, kST, big);
+      }
+      if (exact) {
       xpose_reduce32<true>(v, lane);
       if (tid == 0) s_flag[0] = 0;   // every read of the previous tile's flag is behind two barriers
       s_red[qd * kH + 32 * hf + lane] = v[0];
@@ -571,7 +582,8 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         if (resc) atomicOr(&s_flag[0], 1);
       }
       tc::named_bar(3, kST);
-      if (s_flag[0] && j > jb) {
+      }
+      if (exact && s_flag[0] && j > jb) {
         // rescale the O^T accumulator: column h of this thread's two blocks times alpha[h]
         for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
 #pragma unroll
@@ -613,7 +625,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       tc::named_bar(3, kST);
       if (tid < kH) {
         const float ts = s_red[tid] + s_red[kH + tid] + s_red[2 * kH + tid] + s_red[3 * kH + tid];
-        s_l[tid] = (j == jb ? 0.f : s_l[tid] * s_alpha[tid]) + ts;
+        s_l[tid] = (j == jb ? 0.f : exact ? s_l[tid] * s_alpha[tid] : s_l[tid]) + ts;
       }
       tc::fence_proxy_async();
       tc::tc_fence_before();

@@ -143,16 +143,6 @@ __device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdes
 }
 
 // 16 consecutive 32-bit TMEM columns of this warp's lane quarter from registers.
-// Named-barrier rendezvous of `n` threads that also ORs a predicate across them.
-__device__ __forceinline__ bool bar_red_or(int id, int n, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r) : "r"(v ? 1u : 0u), "r"(id), "r"(n) : "memory");
-  return r != 0;
-}
-
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
@@ -355,7 +345,7 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
         // the waiter has seen this stage's accumulator free (with its key scales) and
         // its key codes landed (bar.red is warp-aligned: the warp reconverges first)
         __syncwarp();
-        const bool failed = bar_red_or(1, 64, false);
+        const bool failed = tc::bar_red_or(1, 64, false);
         ok = ok && !failed;
         if (!ok || lane != 0) continue;
         tc::tc_fence_after();
@@ -392,7 +382,7 @@ index_scores_fp4_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
           ok = tc::mbar_wait(&tempty[it % NACC], (it / NACC) & 1, p.err) &&
                tc::mbar_wait(&full[it % S], (it / S) & 1, p.err);
         ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-        bar_red_or(1, 64, !ok);
+        tc::bar_red_or(1, 64, !ok);
       }
     }
   } else {

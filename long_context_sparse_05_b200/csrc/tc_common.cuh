@@ -248,6 +248,15 @@ __device__ __forceinline__ void fence_proxy_async() {
 __device__ __forceinline__ void named_bar(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
+// Named-barrier rendezvous of `n` threads that also ORs a predicate across them.
+__device__ __forceinline__ bool bar_red_or(int id, int n, bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r) : "r"(v ? 1u : 0u), "r"(id), "r"(n) : "memory");
+  return r != 0;
+}
 
 }  // namespace tc
 
