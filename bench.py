@@ -397,9 +397,33 @@ def e2e_decode(w, st, steps, flush, stream, world=1):
     d2h = batches[0]["hout"].numel() * batches[0]["hout"].element_size()
     s_h2d, s_d2h = torch.cuda.Stream(), torch.cuda.Stream()
 
-    def step_of(bt):
+    def step_of(bt, st=None):
         dv = bt["dv"]
-        bt["ps"].step(stream, q=dv["q"], q_I=dv.get("q_I"), w_=dv.get("w"), new=bt["new"])
+        bt["ps"].step(stream if st is None else st, q=dv["q"], q_I=dv.get("q_I"), w_=dv.get("w"),
+                      new=bt["new"])
+
+    # each batch's step (its kernel launches) captured once as a CUDA graph, so the host
+    # issues one graph launch per step instead of the step's launches
+    graphs = None
+    try:
+        cap = torch.cuda.Stream()
+        gs = []
+        for bt in batches:
+            bt["dstage"].copy_(bt["hstage"])     # the step's inputs (positions included)
+        torch.cuda.synchronize()
+        for bt in batches:
+            step_of(bt, cap)                     # warm the launch path on the capture stream
+        torch.cuda.synchronize()
+        for bt in batches:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="relaxed"):
+                step_of(bt, cap)
+            gs.append(g)
+        torch.cuda.synchronize()
+        graphs = gs
+    except Exception:   # a launch path that cannot be captured: plain launches
+        torch.cuda.synchronize()
+        graphs = None
 
     def one(i):
         bt = batches[i % R]
@@ -410,7 +434,11 @@ def e2e_decode(w, st, steps, flush, stream, world=1):
         e["h2d"].record(s_h2d)
         stream.wait_event(e["h2d"])
         stream.wait_event(e["d2h"])              # its previous output has been read back
-        step_of(bt)
+        if graphs is not None:
+            with torch.cuda.stream(stream):
+                graphs[i % R].replay()
+        else:
+            step_of(bt)
         e["done"].record(stream)
         s_d2h.wait_event(e["done"])
         with torch.cuda.stream(s_d2h):
@@ -439,8 +467,9 @@ def e2e_decode(w, st, steps, flush, stream, world=1):
            "d2h_bytes_per_step": int(d2h), "ms_per_step": round(ms, 4),
            "copies_per_step": {"h2d": 1, "d2h": 1},
            "call": "csa_decode_paged (pages of %d entries, state rings)" % L.PAGE_ENTRIES,
-           "pipeline": "%d batches in rotation; H2D, step and D2H on three streams, "
-                       "ordered by events; no L2 flush (the batches' data exceed L2)" % R,
+           "pipeline": "%d batches in rotation; H2D, step%s and D2H on three streams, "
+                       "ordered by events; no L2 flush (the batches' data exceed L2)"
+                       % (R, " (one CUDA graph per batch)" if graphs is not None else ""),
            "device_ms_per_step": round(float(np.mean(dev_times)), 4),
            "gpu_launches_per_step": L.csa_decode_paged_launch_count(batches[0]["ps"].p)}
     del batches

@@ -602,7 +602,7 @@ csa_status csa_decode_paged(const csa_paged_params* p, const csa_paged_tensors* 
   mc.out = x->kv_pages; mc.out_scales = nullptr;
   mc.ring = ring; mc.pos = x->pos;
   mc.new_C_a = x->new_C_a; mc.new_Z_a = x->new_Z_a; mc.new_C_b = x->new_C_b; mc.new_Z_b = x->new_Z_b;
-  mc.block_table = x->block_table; mc.max_pages = p->max_pages;
+  mc.block_table = x->block_table; mc.max_pages = p->max_pages; mc.num_pages = p->num_pages;
   pa.nbranch = p->hca ? 1 : 2;
   pa.b = b; pa.t = 0; pa.qpos = d.qpos;
   pa.paged = 1; pa.win = x->win; pa.new_win = x->new_win; pa.win_ring = p->n_w;

@@ -74,6 +74,14 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
     return base + (size_t)(row % a.ring) * c;
   };
 
+  // paged output: an entry past the sequence's block table, or whose page is not in the
+  // pool, is not written (positions are device data; the kernel does not trust them)
+  if (a.block_table) {
+    if (i / kPageEntries >= a.max_pages) return;
+    const int pg = a.block_table[(size_t)s * a.max_pages + i / kPageEntries];
+    if ((unsigned)pg >= (unsigned)a.num_pages) return;
+  }
+
   float mx[VEC], sum[VEC], acc[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) { mx[v] = -INFINITY; sum[v] = 0.f; acc[v] = 0.f; }
@@ -438,6 +446,13 @@ __global__ void __launch_bounds__(256) compress_split_kernel(CompressArgs a, int
     if (tp < 0 || (tp + 1) % m != 0) { pdl_wait(); return; }
     i = (tp + 1) / m - 1;
     t_new = tp;
+    // an entry past the block table, or whose page is not in the pool, is not written
+    bool bad = i / kPageEntries >= a.max_pages;
+    if (!bad && a.block_table) {
+      const int pg = a.block_table[(size_t)s * a.max_pages + i / kPageEntries];
+      bad = (unsigned)pg >= (unsigned)a.num_pages;
+    }
+    if (bad) { pdl_wait(); return; }
   } else {
     pdl_wait();
   }

@@ -27,6 +27,7 @@ struct CompressArgs {
   int max_pages;
   // entry i goes to row i - out_off of its sequence (a shard of the entries); 0: row i
   int out_off;
+  int num_pages;   // paged: pages in the pool (an entry whose page is outside it is skipped)
 };
 
 constexpr int kPageEntries = CSA_PAGE_ENTRIES;   // compressed entries per page of the paged caches
