@@ -190,45 +190,45 @@ def test_csa_prefill_fp8_sampled():
         _check_attention(w, out[t], ref["out"][j], same, recheck)
 
 
-@pytest.mark.parametrize("paged", [False, True])
-def test_fused_fp8_decode_selection_equals_stage_calls(paged):
-    """The fused FP8 decode quantises the bf16 index queries inside the indexer (so that
-    only the key page the step writes waits for the compressor).  The same arithmetic as
-    csa_quantize: the selection is bit for bit the one of the stage calls (csa_quantize,
-    csa_index_scores, csa_topk) on the updated cache."""
+@pytest.mark.parametrize("fmt,paged", [("fp8", False), ("fp8", True), ("nvfp4", False)])
+def test_fused_decode_selection_equals_stage_calls(fmt, paged):
+    """The fused decode quantises the bf16 index queries with the arithmetic of
+    csa_quantize (FP8: inside the indexer, so that only the key page the step writes waits
+    for the compressor; NVFP4: in the prologue): the selection is bit for bit the one of
+    the stage calls (csa_quantize, csa_index_scores, csa_topk) on the updated cache."""
     from long_context_sparse_05_b200 import _lib as L
-    w = workloads.shrink(workloads.CSA_DECODE_64K, b=3, n=4100 - 4100 % 4)
+    base = workloads.CSA_DECODE_64K if fmt == "fp8" else workloads.CSA_DECODE_1M
+    w = workloads.shrink(base, b=3, n=4100 - 4100 % 4)
     inp = synth.make_inputs(w, device="cuda")
+    E = w.E
     if paged:
         st = runner.PagedDecodeState(w, inp, shuffle_seed=9)
         st.step()
-        # each sequence's key rows in entry order, gathered from its pages
-        e = torch.arange(w.E, device="cuda")
+        # each sequence's key rows in entry order, gathered from its pages (FP8 scales are
+        # one float per row)
+        e = torch.arange(E, device="cuda")
         PE = L.PAGE_ENTRIES
         rows = st.block_table[:, e // PE].long() * PE + e % PE
-        kI = st.kI_pages[rows]
-        ks = st.kI_scales[rows]
+        E_cap = (E + 3) // 4 * 4
+        kI = torch.zeros((w.b, E_cap, w.c_I), dtype=torch.uint8, device="cuda")
+        kI[:, :E] = st.kI_pages[rows]
+        ks = torch.zeros((w.b, E_cap), dtype=torch.float32, device="cuda")
+        ks[:, :E] = st.kI_scales[rows]
     else:
         st = runner.DecodeState(w, inp)
         st.build_caches()
         st.step()
-        kI = st.kI_cache[:, :w.E].contiguous()
-        ks = st.kI_scales[:, :w.E].contiguous()
+        kI, ks, E_cap = st.kI_cache, st.kI_scales, st.E_cap
     torch.cuda.synchronize()
-    E = w.E
-    E_cap = (E + 3) // 4 * 4
-    kIp = torch.zeros((w.b, E_cap, kI.shape[-1]), dtype=torch.uint8, device="cuda")
-    kIp[:, :E] = kI
-    ksp = torch.zeros((w.b, E_cap), dtype=torch.float32, device="cuda")
-    ksp[:, :E] = ks
     rows_q = w.b * w.H_I
-    codes = torch.empty((rows_q, w.c_I), dtype=torch.uint8, device="cuda")
-    scales = torch.empty((rows_q,), dtype=torch.float32, device="cuda")
-    L.csa_quantize(L.CSA_BF16, L.CSA_FP8_E4M3, inp["q_I"], rows_q, w.c_I, codes, scales)
+    codes = torch.empty((rows_q, runner.row_bytes(fmt, w.c_I)), dtype=torch.uint8, device="cuda")
+    sc = (torch.empty((rows_q,), dtype=torch.float32, device="cuda") if fmt == "fp8" else
+          torch.empty((rows_q, w.c_I // 16), dtype=torch.uint8, device="cuda"))
+    L.csa_quantize(L.CSA_BF16, L.DTYPE[fmt], inp["q_I"], rows_q, w.c_I, codes, sc)
     qpos = torch.full((w.b, 1), w.n - 1, dtype=torch.int32, device="cuda")
-    ip = L.IndexParams(H_I=w.H_I, d_I=w.c_I, m=w.m, qk_dtype=L.CSA_FP8_E4M3, score_dtype=L.CSA_BF16)
+    ip = L.IndexParams(H_I=w.H_I, d_I=w.c_I, m=w.m, qk_dtype=L.DTYPE[fmt], score_dtype=L.CSA_BF16)
     scores = torch.empty((w.b, 1, E), dtype=torch.bfloat16, device="cuda")
-    L.csa_index_scores(ip, codes, scales, inp["w"], kIp, ksp, qpos, w.b, 1, E_cap, E, scores)
+    L.csa_index_scores(ip, codes, sc, inp["w"], kI, ks, qpos, w.b, 1, E_cap, E, scores)
     idx = torch.empty((w.b, 1, w.k), dtype=torch.int32, device="cuda")
     cnt = torch.empty((w.b, 1), dtype=torch.int32, device="cuda")
     wsb = L.csa_topk_workspace_size(L.CSA_BF16, w.b, 1, E, w.k)
