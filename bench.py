@@ -216,7 +216,7 @@ def timed_region(fn, steps, flush, stream, world, min_span_s, max_repeats=4000):
 # here (its traffic is then reported as null).
 PROFILED_TRAFFIC = {
     ("index_scores", "fp8"): ("entries", 8773376 / (4 * 16384)),
-    ("index_scores", "nvfp4"): ("entries", 9491712 / (2 * 65536)),
+    ("index_scores", "nvfp4"): ("entries", 9498368 / (2 * 65536)),
     ("sparse_attn", "csa_decode_64k_fp8"): ("queries", 2978304 / 4),
 }
 
