@@ -34,7 +34,10 @@
 // CTA (288 threads): warps 0-7 gather, read TMEM and run the softmax, two warps per
 // TMEM lane quarter (warp w owns lanes 32 (w % 4).., 32 heads each); warp 8 lane 0
 // issues every MMA.  Ordering uses named barriers (tile ready, P ready) and
-// mbarriers signalled by tcgen05.commit (S ready, O ready).
+// mbarriers signalled by tcgen05.commit (S ready; PV done per 128-dim block).  Within an
+// item, the next tile is gathered column-block pair by pair as soon as the current PV
+// has read that pair, and its S^T MMAs start on each pair as it lands, so the gather of
+// tile j + 1 runs under the PV of tile j.
 #include "kernels.h"
 #include "tc_common.cuh"
 
@@ -136,6 +139,29 @@ __device__ __forceinline__ void gather_rows(uint8_t* dst, int blk_bytes, int nro
   }
 }
 
+// Copy dims 128 mb .. 128 mb + 127 (column blocks 2 mb, 2 mb + 1) of the tile's rows:
+// half a warp per row (256 contiguous source bytes), rows 2 w, 2 w + 1, 2 w + 16, ... for
+// gather warp w.
+__device__ __forceinline__ void gather_pair(uint8_t* dst, int mb, int gw, int lane,
+                                            const __nv_bfloat16* const* rows, const void* dummy) {
+  const int c = 16 * mb + (lane & 15);          // 16-byte chunk of the row
+  const int cb = c >> 3, cc = c & 7;
+  for (int r = 2 * gw + (lane >> 4); r < kRows; r += 2 * kSW) {
+    const __nv_bfloat16* src = rows[r];
+    uint8_t* d = dst + cb * kKVBlkBytes + r * 128 + ((cc ^ (r & 7)) << 4);
+    if (src) tc::cp_async16(d, src + c * 8, 16);
+    else tc::cp_async16(d, dummy, 0);
+  }
+}
+
+// This thread's copies of a pair have landed: publish them to the tensor core and arrive
+// at the pair's named barrier (the MMA warp syncs on it).
+__device__ __forceinline__ void pair_landed(int id) {
+  tc::fence_proxy_async();
+  tc::tc_fence_before();
+  tc::named_bar_arrive(id, kThreadsA);
+}
+
 // One halving step of the transpose-reduction: lanes with bit `OFF` set keep the
 // upper half of their HALF live values, the others the lower half, and each
 // combines what it keeps with what its partner sends.
@@ -190,8 +216,12 @@ __device__ __forceinline__ void bulk_store(void* gdst, const void* ssrc, uint32_
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
                ::"l"(gdst), "r"(tc::smem_u32(ssrc)), "r"(bytes) : "memory");
 }
-__device__ __forceinline__ void bulk_store_commit_wait() {
-  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Waits until this thread's committed bulk copies have completed (their writes performed).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_load_g(void* sdst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
   asm volatile(
@@ -303,17 +333,25 @@ __device__ void merge_slice(const AttnTc& p, int qrow, int d0, int d1, bool writ
 // its scaled O to the workspace; after the cluster barrier rank r bulk-loads, from every
 // split, the rows of output dims [d0, d1) and adds them.
 __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int item, int rank,
-                                              uint8_t* area, uint64_t* bar_r, bool ok) {
+                                              uint8_t* area, uint64_t* bar_r, bool ok,
+                                              bool blocks_stored) {
   const int tid = threadIdx.x;
   const int ns = p.nsplit;
   int d0, d1;
   cm_slice(ns, rank, d0, d1);
   const int dsl = d1 - d0;
   const int dps = ((kD + ns - 1) / ns + 7) & ~7;
-  // this split's record to the workspace (the rows were fenced for the async proxy)
-  if (tid == 0) {
-    bulk_store(p.part_bf + (size_t)item * kPartB, area, kD * kH * 2);
-    bulk_store_commit_wait();
+  // this split's record to the workspace (the rows were fenced for the async proxy): in
+  // one copy, or already in flight as four blocks issued by threads 0 and kST / 2
+  if (!blocks_stored) {
+    if (tid == 0) {
+      bulk_store(p.part_bf + (size_t)item * kPartB, area, kD * kH * 2);
+      bulk_commit();
+      bulk_wait_all();
+      fence_proxy_async_global();
+    }
+  } else if (tid == 0 || tid == kST / 2) {
+    bulk_wait_all();
     fence_proxy_async_global();
   }
   cluster_sync_all();   // every split's record is in the workspace
@@ -397,8 +435,8 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   float* s_l = s_alpha + kH;                    // running sum
   int* s_flag = reinterpret_cast<int*>(s_l + kH);
   uint64_t* bar_s = reinterpret_cast<uint64_t*>(s_flag + 4);
-  uint64_t* bar_o = bar_s + 1;
-  uint64_t* bar_r = bar_o + 1;                  // cluster merge: received slices
+  uint64_t* bar_pv = bar_s + 1;                 // [4]: PV of dim block mb done (3: all of O)
+  uint64_t* bar_r = bar_pv + 4;                 // cluster merge: received slices
   uint64_t* bar_st = bar_r + 1;                 // cluster merge: maxima and sums received
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(bar_st + 1);
   const __nv_bfloat16** s_rows = reinterpret_cast<const __nv_bfloat16**>(tmem_holder + 2);  // [128]
@@ -422,7 +460,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   const int crank = p.cluster ? (int)cluster_rank() : 0;
   if (tid == 0) {
     tc::mbar_init(bar_s, 1);
-    tc::mbar_init(bar_o, 1);
+    for (int i = 0; i < 4; ++i) tc::mbar_init(bar_pv + i, 1);
     tc::mbar_init(bar_r, 1);
     tc::mbar_init(bar_st, 1);
     tc::fence_barrier_init();
@@ -441,7 +479,8 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   const uint32_t tO = tmem + 64;       // columns [64, 320): O^T, 4 blocks of 64
 
   const int items = p.rows_total * p.nsplit;
-  uint32_t ns = 0, no = 0;             // commits waited on bar_s / bar_o
+  uint32_t ns = 0;                     // commits waited on bar_s
+  uint32_t npv = 0;                    // tiles whose PV commits were waited on (bar_pv)
   bool ok = true;
   bool q_ready = false;                // softmax warps: this item's query heads are on their way
 
@@ -467,20 +506,25 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       constexpr uint32_t idS = tc::instr_desc(128, kH, 1, 1, 0, 0);   // bf16 K-major x K-major
       constexpr uint32_t idO = tc::instr_desc(128, kH, 1, 1, 1, 1);   // bf16 MN-major x MN-major
       for (int j = jb; j < je; ++j) {
-        tc::named_bar(1, kThreadsA);                 // tile (and q) in shared memory
-        if (lane == 0) {
-          tc::tc_fence_after();
-          for (int kb = 0; kb < 8; ++kb) {
+        // S^T by column-block pairs (dims 128 mb ..): the item's first tile (and q) arrives
+        // whole, every later tile pair by pair as the previous tile's PV frees the pairs
+        for (int mb = 0; mb < 4; ++mb) {
+          if (j > jb) tc::named_bar(4 + mb, kThreadsA);
+          else if (mb == 0) tc::named_bar(1, kThreadsA);
+          if (lane == 0) {
+            tc::tc_fence_after();
+            for (int kb = 2 * mb; kb < 2 * mb + 2; ++kb) {
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t a = tc::smem_desc_sw128(tc::smem_u32(sKV + kb * kKVBlkBytes + kk * 32), 16, 1024);
-              const uint64_t b = tc::smem_desc_sw128(tc::smem_u32(sQ + kb * kQBlkBytes + kk * 32), 16, 1024);
-              tc::mma_f16(tS, a, b, idS, (kb | kk) != 0);
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t a = tc::smem_desc_sw128(tc::smem_u32(sKV + kb * kKVBlkBytes + kk * 32), 16, 1024);
+                const uint64_t b = tc::smem_desc_sw128(tc::smem_u32(sQ + kb * kQBlkBytes + kk * 32), 16, 1024);
+                tc::mma_f16(tS, a, b, idS, (kb | kk) != 0);
+              }
             }
+            if (mb == 3) tc::mma_commit(bar_s);
           }
-          tc::mma_commit(bar_s);
+          __syncwarp();
         }
-        __syncwarp();
         tc::named_bar(2, kThreadsA);                 // P^T in shared memory, O rescaled
         if (lane == 0) {
           tc::tc_fence_after();
@@ -492,8 +536,9 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
               const uint64_t b = tc::smem_desc_sw128(tc::smem_u32(sP + kk * 2048), 8192, 1024);
               tc::mma_f16(tO + mb * kH, a, b, idO, (j > jb) || (kk > 0));
             }
+            // every MMA so far is tracked: KV column blocks 2 mb, 2 mb + 1 are free once it fires
+            tc::mma_commit(bar_pv + mb);
           }
-          tc::mma_commit(bar_o);
         }
         __syncwarp();
       }
@@ -508,21 +553,17 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
     const bool have_q = (q_pre && item == (int)blockIdx.x) || q_ready;
     q_ready = false;
     if (tid < kH) { s_M[tid] = -INFINITY; s_l[tid] = 0.f; }
-    for (int j = jb; j < je; ++j) {
-      if (j > jb) {                                  // previous PV done: KV, P and O are free
-        ok = ok && tc::mbar_wait_hint(bar_o, no & 1, p.err, kWaitHintNs);
-        ++no;
-        tc::tc_fence_after();
-      }
-      if (j == jb && !have_q) {
+    if (je > jb) {
+      // the item's first tile, whole (the previous item's O has been read: KV and P are free)
+      if (!have_q) {
         const __nv_bfloat16* qb = p.q + (size_t)qrow * kH * kD;
         gather_rows(sQ, kQBlkBytes, kH, warp, lane,
                     [&](int h) { return qb + (size_t)h * kD; }, p.kv);
       }
       // source of every row of the tile: one coalesced pass over the index list
       if (hf == 0) {
-        const int pos = rb + j * kRows + r;
-        s_rows[r] = pos < re ? row_src(p, Q, qrow, pos, j == jb ? e_pre : INT_MIN) : nullptr;
+        const int pos = rb + jb * kRows + r;
+        s_rows[r] = pos < re ? row_src(p, Q, qrow, pos, e_pre) : nullptr;
       }
       tc::named_bar(3, kST);
       gather_rows(sKV, kKVBlkBytes, kRows, warp, lane, [&](int rr) { return s_rows[rr]; }, p.kv);
@@ -530,6 +571,14 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       tc::fence_proxy_async();
       tc::tc_fence_before();
       tc::named_bar(1, kThreadsA);
+    }
+    for (int j = jb; j < je; ++j) {
+      // the next tile's list entry of this thread's row, loaded behind this tile's S^T
+      int e_nxt = INT_MIN;
+      if (hf == 0 && !p.dense && j + 1 < je) {
+        const int pn = rb + (j + 1) * kRows + r;
+        if (pn < p.k) e_nxt = p.idx[(size_t)qrow * p.k + pn];
+      }
 
       // logits of row r for this thread's 32 heads
       ok = ok && tc::mbar_wait_hint(bar_s, ns & 1, p.err, kWaitHintNs);
@@ -630,6 +679,31 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       tc::fence_proxy_async();
       tc::tc_fence_before();
       tc::named_bar(2, kThreadsA);
+      if (j + 1 < je) {
+        // the next tile, column-block pair by pair as this tile's PV frees the pairs; the
+        // MMA warp starts its S^T on each pair as soon as it has landed.  Every read of
+        // this tile's row table is behind the barrier above.
+        if (hf == 0) {
+          const int pos = rb + (j + 1) * kRows + r;
+          s_rows[r] = pos < re ? row_src(p, Q, qrow, pos, e_nxt) : nullptr;
+        }
+        tc::named_bar(3, kST);
+        for (int mb = 0; mb < 4; ++mb) {
+          ok = ok && tc::mbar_wait_hint(bar_pv + mb, npv & 1, p.err, kWaitHintNs);
+          tc::tc_fence_after();
+          gather_pair(sKV, mb, warp, lane, s_rows, p.kv);
+          tc::cp_async_commit();
+        }
+        ++npv;
+        tc::cp_async_wait_group<3>();
+        pair_landed(4);
+        tc::cp_async_wait_group<2>();
+        pair_landed(5);
+        tc::cp_async_wait_group<1>();
+        pair_landed(6);
+        tc::cp_async_wait_group<0>();
+        pair_landed(7);
+      }
     }
 
     if (p.nsplit > 1 && p.cluster) {
@@ -668,9 +742,51 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         for (int x = tid; x < kD * kH * 2 / 16; x += kST) z[x] = make_uint4(0u, 0u, 0u, 0u);
         tc::fence_proxy_async();
       }
+    } else if (p.nsplit > 1 && p.cluster) {
+      // O scaled by this split's weight into shared memory (bf16 record rows, dims 128 mb ..
+      // at bytes 16 KB mb: the KV column block that PV block mb / 2 has already read).  Each
+      // half of the warps stages its two dim blocks as soon as the PV of the block is done,
+      // and one thread of the half bulk-stores the block to the workspace, so the staging and
+      // the stores run under the remaining PV.
+      tc::named_bar(3, kST);                         // weights (s_alpha) final
+      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
+        ok = ok && tc::mbar_wait_hint(bar_pv + mb, npv & 1, p.err, kWaitHintNs);
+        tc::tc_fence_after();
+        const int d = mb * 128 + r;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
+          tc::tmem_ld_wait(o);
+#pragma unroll
+          for (int c4 = 0; c4 < 4; ++c4) {    // 8 heads = one 16-byte chunk
+            const float4 wa = *reinterpret_cast<const float4*>(s_alpha + half * 32 + c4 * 8);
+            const float4 wb = *reinterpret_cast<const float4*>(s_alpha + half * 32 + c4 * 8 + 4);
+            const float wt[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                  __uint_as_float(o[8 * c4 + 2 * e]) * wt[2 * e],
+                  __uint_as_float(o[8 * c4 + 2 * e + 1]) * wt[2 * e + 1]);
+              w4[e] = *reinterpret_cast<const uint32_t*>(&b2);
+            }
+            *reinterpret_cast<uint4*>(sKV + (size_t)d * kH * 2 + cm_chunk(d, half * 4 + c4) * 16) =
+                make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+        tc::fence_proxy_async();   // the bulk copy reads these rows through the async proxy
+        tc::named_bar(4 + hf, kST / 2);
+        if (qd == 0 && lane == 0) {
+          const size_t off = (size_t)mb * 128 * kH * 2;
+          bulk_store(p.part_bf + (size_t)item * kPartB + off, sKV + off, 128 * kH * 2);
+          bulk_commit();
+        }
+      }
+      ++npv;
     } else {
-    ok = ok && tc::mbar_wait_hint(bar_o, no & 1, p.err, kWaitHintNs);
-    ++no;
+    ok = ok && tc::mbar_wait_hint(bar_pv + 3, npv & 1, p.err, kWaitHintNs);
+    ++npv;
     tc::tc_fence_after();
     tc::named_bar(3, kST);                           // s_l / s_M final
     // finalise: thread owns dims d = 128 mb + r of every head, mb in {2 hf, 2 hf + 1}
@@ -707,39 +823,6 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
           }
         }
       }
-    } else if (p.cluster) {
-      // O scaled by this split's weight (s_alpha, ordered by the barrier above) into shared
-      // memory (bf16) for the cluster merge (KV tile area, free now)
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        float wt[32];                         // this half's 32 head weights, in registers
-#pragma unroll
-        for (int h = 0; h < 32; h += 4) {
-          const float4 w4 = *reinterpret_cast<const float4*>(s_alpha + half * 32 + h);
-          wt[h] = w4.x; wt[h + 1] = w4.y; wt[h + 2] = w4.z; wt[h + 3] = w4.w;
-        }
-        for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
-          uint32_t o[32];
-          tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
-          tc::tmem_ld_wait(o);
-          const int d = mb * 128 + r;
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {    // 8 heads = one 16-byte chunk
-            uint32_t w4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int h0 = c4 * 8 + 2 * e;
-              const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                  __uint_as_float(o[8 * c4 + 2 * e]) * wt[h0],
-                  __uint_as_float(o[8 * c4 + 2 * e + 1]) * wt[h0 + 1]);
-              w4[e] = *reinterpret_cast<const uint32_t*>(&b2);
-            }
-            *reinterpret_cast<uint4*>(sKV + (size_t)d * kH * 2 + cm_chunk(d, half * 4 + c4) * 16) =
-                make_uint4(w4[0], w4[1], w4[2], w4[3]);
-          }
-        }
-      }
-      tc::fence_proxy_async();   // the bulk copies read these rows through the async proxy
     } else {
       for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
 #pragma unroll
@@ -774,7 +857,7 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       // slice of the dims, then keep this CTA's shared memory alive until all peers
       // have read it
       __syncthreads();
-      cluster_merge(p, qrow, item, crank, sKV, bar_r, ok);
+      cluster_merge(p, qrow, item, crank, sKV, bar_r, ok, je > jb);
     }
   }
 
@@ -786,10 +869,10 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
   }
 }
 
-// alignment slack, KV tile, q, P^T, s_red + four per-head arrays, flag, four mbarriers,
+// alignment slack, KV tile, q, P^T, s_red + four per-head arrays, flag, seven mbarriers,
 // TMEM holder, row-pointer table, 16-byte alignment, merge maxima / sums, sink logits
 constexpr size_t kSmemBytes = 1024 + 8 * kKVBlkBytes + 8 * kQBlkBytes + kRows * 128 +
-                              (4 * kH + 4 * kH) * 4 + 16 + 4 * 8 + 8 + kRows * 8 + 16 +
+                              (4 * kH + 4 * kH) * 4 + 16 + 7 * 8 + 8 + kRows * 8 + 16 +
                               kMaxSplit * kH * 2 * 4 + kH * 4;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 
