@@ -411,15 +411,16 @@ __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int ite
 constexpr int kMergeDims = 16;
 __global__ void __launch_bounds__(128) attn_merge_kernel(AttnTc p) {
   extern __shared__ __align__(16) float mm_smem[];
-  float* s_ml = mm_smem;                                  // [2][kMaxSplitGlobal][kH]
-  float* s_mw = s_ml + 2 * kMaxSplitGlobal * kH;          // [kMaxSplitGlobal][kH]
-  uint8_t* stage = reinterpret_cast<uint8_t*>(s_mw + kMaxSplitGlobal * kH);
+  const int cap = p.nsplit;                               // shared memory sized for it
+  float* s_ml = mm_smem;                                  // [2][cap][kH]
+  float* s_mw = s_ml + 2 * cap * kH;                      // [cap][kH]
+  uint8_t* stage = reinterpret_cast<uint8_t*>(s_mw + cap * kH);
   pdl_launch_dependents();
   pdl_wait();
   const int qrow = blockIdx.x;
   const int d0 = blockIdx.y * kMergeDims;
   merge_slice(p, qrow, d0, min(kD, d0 + kMergeDims), blockIdx.y == 0, stage, s_ml, s_mw,
-              kMaxSplitGlobal, p.q);
+              cap, p.q);
 }
 
 __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
@@ -784,13 +785,41 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         }
       }
       ++npv;
+    } else if (p.nsplit > 1) {
+      // fp32 partials for the workspace merge, each 128-dim block as soon as its PV is done;
+      // this thread's heads' running max and sum are its own (tid < kH) writes
+      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
+        ok = ok && tc::mbar_wait_hint(bar_pv + mb, npv & 1, p.err, kWaitHintNs);
+        tc::tc_fence_after();
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
+          tc::tmem_ld_wait(o);
+          const int d = mb * 128 + r;
+          float4* dst = reinterpret_cast<float4*>(&p.part_o[((size_t)item * kD + d) * kH + half * 32]);
+#pragma unroll
+          for (int h4 = 0; h4 < 8; ++h4) {
+            float4 v = make_float4(__uint_as_float(o[4 * h4]), __uint_as_float(o[4 * h4 + 1]),
+                                   __uint_as_float(o[4 * h4 + 2]), __uint_as_float(o[4 * h4 + 3]));
+            if (!ok) v = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
+                                     __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
+            dst[h4] = v;
+          }
+        }
+      }
+      ++npv;
+      if (tid < kH) {
+        p.part_m[(size_t)item * kH + tid] = s_M[tid];
+        p.part_l[(size_t)item * kH + tid] = s_l[tid];
+      }
     } else {
-    ok = ok && tc::mbar_wait_hint(bar_pv + 3, npv & 1, p.err, kWaitHintNs);
-    ++npv;
-    tc::tc_fence_after();
-    tc::named_bar(3, kST);                           // s_l / s_M final
-    // finalise: thread owns dims d = 128 mb + r of every head, mb in {2 hf, 2 hf + 1}
-    if (p.nsplit == 1) {
+      // one split: the normalised output.  Thread owns dims d = 128 mb + r of every head,
+      // mb in {2 hf, 2 hf + 1}
+      ok = ok && tc::mbar_wait_hint(bar_pv + 3, npv & 1, p.err, kWaitHintNs);
+      ++npv;
+      tc::tc_fence_after();
+      tc::named_bar(3, kST);                         // s_l / s_M final
       // one reciprocal denominator per head (the sink joins it), kept where the
       // per-tile rescale factors were
       float* s_inv = s_alpha;
@@ -823,30 +852,6 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
           }
         }
       }
-    } else {
-      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t o[32];
-          tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
-          tc::tmem_ld_wait(o);
-          const int d = mb * 128 + r;
-          float4* dst = reinterpret_cast<float4*>(&p.part_o[((size_t)item * kD + d) * kH + half * 32]);
-#pragma unroll
-          for (int h4 = 0; h4 < 8; ++h4) {
-            float4 v = make_float4(__uint_as_float(o[4 * h4]), __uint_as_float(o[4 * h4 + 1]),
-                                   __uint_as_float(o[4 * h4 + 2]), __uint_as_float(o[4 * h4 + 3]));
-            if (!ok) v = make_float4(__int_as_float(0x7fc00000), __int_as_float(0x7fc00000),
-                                     __int_as_float(0x7fc00000), __int_as_float(0x7fc00000));
-            dst[h4] = v;
-          }
-        }
-      }
-      if (tid < kH) {
-        p.part_m[(size_t)item * kH + tid] = s_M[tid];
-        p.part_l[(size_t)item * kH + tid] = s_l[tid];
-      }
-    }
     }
     tc::tc_fence_before();
     tc::named_bar(3, kST);                           // s_M / s_l reads done before the next item
@@ -944,8 +949,9 @@ Plan plan(int k, int n_w, int b, int T, int E_cap, bool dense, int sms) {
   return P;
 }
 
-size_t merge_smem_bytes() {
-  return (size_t)3 * kMaxSplitGlobal * kH * 4 + (size_t)kMaxSplitGlobal * kMergeDims * kH * 4;
+// Shared memory of attn_merge_kernel for ns splits (several CTAs fit on an SM).
+size_t merge_smem_bytes(int ns) {
+  return (size_t)3 * ns * kH * 4 + (size_t)ns * kMergeDims * kH * 4;
 }
 
 }  // namespace
@@ -1019,7 +1025,7 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
         cudaSuccess)
       return CSA_ERR_CUDA;
     if (P.nsplit > 1) {
-      const size_t msm = merge_smem_bytes();
+      const size_t msm = merge_smem_bytes(P.nsplit);
       if (cudaFuncSetAttribute(attn_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)msm) != cudaSuccess)
         return CSA_ERR_CUDA;
