@@ -814,44 +814,44 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         p.part_l[(size_t)item * kH + tid] = s_l[tid];
       }
     } else {
-      // one split: the normalised output.  Thread owns dims d = 128 mb + r of every head,
-      // mb in {2 hf, 2 hf + 1}
-      ok = ok && tc::mbar_wait_hint(bar_pv + 3, npv & 1, p.err, kWaitHintNs);
-      ++npv;
-      tc::tc_fence_after();
-      tc::named_bar(3, kST);                         // s_l / s_M final
-      // one reciprocal denominator per head (the sink joins it), kept where the
-      // per-tile rescale factors were
-      float* s_inv = s_alpha;
-      if (tid < kH) {
+      // one split: the normalised output, the sink in the denominator.  Every warp takes
+      // the four 128-dim blocks of O one after another, each as soon as its PV is done
+      // (the later blocks' PV still runs): thread = dim d = 128 mb + r, heads of its half hf.
+      // Every read of s_alpha / s_l / s_M by the last softmax is behind its closing barrier.
+      if (tid < kH) {   // one reciprocal denominator per head, where the rescale factors were
         const float den = s_l[tid] + exp2f(s_sink2[tid] - s_M[tid]);
-        s_inv[tid] = 1.f / den;
+        s_alpha[tid] = 1.f / den;
         if (p.lse) p.lse[(size_t)qrow * kH + tid] = (s_M[tid] + log2f(den)) * 0.6931471805599453f;
       }
       tc::named_bar(3, kST);
-      for (int mb = 2 * hf; mb < 2 * hf + 2; ++mb) {
+      float inv[32];                                 // this half's 32 head denominators
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t o[32];
-          tc::tmem_ld32(tO + mb * kH + half * 32 + lane_addr, o);
-          tc::tmem_ld_wait(o);
-          const int d = mb * 128 + r;
-          // rotary output dims: the pair partner (dim d ^ 1) is in lane ^ 1; the condition
-          // is uniform over the warp's 32 dims when d_rope_out is a multiple of 32
-          const bool rot = p.d_rope_out > 0 && mb * 128 + qd * 32 + 31 >= kD - p.d_rope_out;
-          float sn, cs;
-          out_rope_sincos(p, d, Q.t, sn, cs);
+      for (int h = 0; h < 32; h += 4) {
+        const float4 w4 = *reinterpret_cast<const float4*>(s_alpha + 32 * hf + h);
+        inv[h] = w4.x; inv[h + 1] = w4.y; inv[h + 2] = w4.z; inv[h + 3] = w4.w;
+      }
+      for (int mb = 0; mb < 4; ++mb) {
+        ok = ok && tc::mbar_wait_hint(bar_pv + mb, npv & 1, p.err, kWaitHintNs);
+        tc::tc_fence_after();
+        uint32_t o[32];
+        tc::tmem_ld32(tO + mb * kH + 32 * hf + lane_addr, o);
+        tc::tmem_ld_wait(o);
+        const int d = mb * 128 + r;
+        // rotary output dims: the pair partner (dim d ^ 1) is in lane ^ 1; the condition
+        // is uniform over the warp's 32 dims when d_rope_out is a multiple of 32
+        const bool rot = p.d_rope_out > 0 && mb * 128 + qd * 32 + 31 >= kD - p.d_rope_out;
+        float sn, cs;
+        out_rope_sincos(p, d, Q.t, sn, cs);
 #pragma unroll
-          for (int h = 0; h < 32; ++h) {
-            const int hh = half * 32 + h;
-            float val = __uint_as_float(o[h]) * s_inv[hh];
-            if (rot) val = inv_rope_elem(val, __shfl_xor_sync(0xffffffffu, val, 1), d, kD,
-                                         p.d_rope_out, sn, cs);
-            p.out[((size_t)qrow * kH + hh) * kD + d] =
-                __float2bfloat16_rn(ok ? val : __int_as_float(0x7fc00000));
-          }
+        for (int h = 0; h < 32; ++h) {
+          float val = __uint_as_float(o[h]) * inv[h];
+          if (rot) val = inv_rope_elem(val, __shfl_xor_sync(0xffffffffu, val, 1), d, kD,
+                                       p.d_rope_out, sn, cs);
+          p.out[((size_t)qrow * kH + 32 * hf + h) * kD + d] =
+              __float2bfloat16_rn(ok ? val : __int_as_float(0x7fc00000));
         }
       }
+      ++npv;
     }
     tc::tc_fence_before();
     tc::named_bar(3, kST);                           // s_M / s_l reads done before the next item
