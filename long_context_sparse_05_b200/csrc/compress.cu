@@ -242,11 +242,13 @@ __device__ __forceinline__ void compress_body(const CompressArgs& a, int i, int 
   }
 }
 
-// Layout of the work: one CTA per (entry, sequence); see compress_body.
-template <typename InT>
+// Layout of the work: one CTA per (entry, sequence); see compress_body.  U = rows a thread
+// loads at once: the rows per thread of the launch, at most kUnroll (fewer registers, more
+// CTAs resident per SM when each thread has only one or two rows).
+template <typename InT, int U>
 __global__ void __launch_bounds__(512) compress_kernel(CompressArgs a) {
   extern __shared__ float smem[];
-  compress_body<InT>(a, a.entry_begin + blockIdx.x, blockIdx.y, smem);
+  compress_body<InT, U>(a, a.entry_begin + blockIdx.x, blockIdx.y, smem);
 }
 
 // One row of the index-path quantiser by one warp: FP8 (per-row scale) or NVFP4 (per-16 scale).
@@ -310,6 +312,56 @@ __global__ void quantize_kernel(const InT* __restrict__ x, int rows, int d, int 
   const int row = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
   if (row >= rows) return;
   quantize_row<InT>(x, row, d, out_dtype, codes, scales);
+}
+
+// The same quantisers for bf16 rows of 128 (index queries): a warp takes kQ128Rows rows,
+// loads all of them first (8 bytes per lane and row, one coalesced 256-byte row per
+// instruction) and keeps them in registers for the scale and the codes, so enough bytes
+// are in flight to stream at HBM speed.  Element arithmetic as in quantize_row.
+constexpr int kQ128Rows = 4;
+__global__ void __launch_bounds__(256) quantize128_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          int rows, int out_dtype,
+                                                          uint8_t* __restrict__ codes,
+                                                          void* __restrict__ scales) {
+  const int lane = threadIdx.x & 31;
+  const int row0 = (blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5)) * kQ128Rows;
+  if (row0 >= rows) return;
+  uint2 raw[kQ128Rows];
+#pragma unroll
+  for (int i = 0; i < kQ128Rows; ++i)
+    raw[i] = row0 + i < rows ? __ldg(reinterpret_cast<const uint2*>(x + (size_t)(row0 + i) * 128) + lane)
+                             : make_uint2(0u, 0u);
+#pragma unroll
+  for (int i = 0; i < kQ128Rows; ++i) {
+    const int row = row0 + i;
+    if (row >= rows) break;
+    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw[i].x);
+    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw[i].y);
+    const float v[4] = {__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi)};
+    float am = 0.f;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(v[e]));
+    if (out_dtype == CSA_FP8_E4M3) {
+      am = warp_max(am);
+      const float scale = am / 448.f;
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        packed |= (scale > 0.f ? f32_to_e4m3(v[e] / scale) : 0u) << (8 * e);
+      reinterpret_cast<uint32_t*>(codes + (size_t)row * 128)[lane] = packed;
+      if (lane == 0) reinterpret_cast<float*>(scales)[row] = scale;
+    } else {
+      // NVFP4: 4 lanes x 4 elements = one 16-element block
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 1));
+      am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, 2));
+      const uint8_t sc = f32_to_e4m3(am / 6.f);
+      const float sv = e4m3_to_f32(sc);
+      const uint8_t p0 = sv > 0.f ? f32x2_to_e2m1x2(v[0] / sv, v[1] / sv) : (uint8_t)0;
+      const uint8_t p1 = sv > 0.f ? f32x2_to_e2m1x2(v[2] / sv, v[3] / sv) : (uint8_t)0;
+      reinterpret_cast<uint16_t*>(codes + (size_t)row * 64)[lane] = (uint16_t)(p0 | (p1 << 8));
+      if ((lane & 3) == 0) reinterpret_cast<uint8_t*>(scales)[(size_t)row * 8 + lane / 4] = sc;
+    }
+  }
 }
 
 // Decode prologue in one launch: CTAs [0, b) compress the latent entry of each
@@ -713,12 +765,19 @@ csa_status launch_compress(const CompressArgs& a_in, int in_dtype, int b, int en
   const size_t smem = (size_t)(3 * (nt / cols) * a.c + a.c + 32) * sizeof(float);
   if (smem > 200 * 1024) return CSA_ERR_UNSUPPORTED;
   dim3 grid(entry_count, b);
+  const int rows_per_thread = (R + rg - 1) / rg;
+  auto go = [&](auto kern) {
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    kern<<<grid, nt, smem, st>>>(a);
+  };
   if (in_dtype == CSA_F32) {
-    cudaFuncSetAttribute(compress_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    compress_kernel<float><<<grid, nt, smem, st>>>(a);
+    if (rows_per_thread <= 1) go(compress_kernel<float, 1>);
+    else if (rows_per_thread <= 2) go(compress_kernel<float, 2>);
+    else go(compress_kernel<float, kUnroll>);
   } else {
-    cudaFuncSetAttribute(compress_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    compress_kernel<__nv_bfloat16><<<grid, nt, smem, st>>>(a);
+    if (rows_per_thread <= 1) go(compress_kernel<__nv_bfloat16, 1>);
+    else if (rows_per_thread <= 2) go(compress_kernel<__nv_bfloat16, 2>);
+    else go(compress_kernel<__nv_bfloat16, kUnroll>);
   }
   CSA_CHECK_LAUNCH();
   return CSA_OK;
@@ -728,6 +787,17 @@ csa_status launch_quantize(int in_dtype, int out_dtype, const void* x, int rows,
                            void* codes, void* scales, cudaStream_t st) {
   if (rows == 0) return CSA_OK;
   const int warps = 8;
+  if (in_dtype == CSA_BF16 && d == 128 && (reinterpret_cast<uintptr_t>(x) & 7) == 0 &&
+      (out_dtype == CSA_FP8_E4M3 || out_dtype == CSA_NVFP4) &&
+      (out_dtype != CSA_NVFP4 || (reinterpret_cast<uintptr_t>(codes) & 1) == 0) &&
+      (out_dtype != CSA_FP8_E4M3 || (reinterpret_cast<uintptr_t>(codes) & 3) == 0)) {
+    const int rows_per_cta = warps * kQ128Rows;
+    quantize128_kernel<<<(rows + rows_per_cta - 1) / rows_per_cta, warps * 32, 0, st>>>(
+        reinterpret_cast<const __nv_bfloat16*>(x), rows, out_dtype, reinterpret_cast<uint8_t*>(codes),
+        scales);
+    CSA_CHECK_LAUNCH();
+    return CSA_OK;
+  }
   dim3 grid((rows + warps - 1) / warps);
   if (in_dtype == CSA_F32)
     quantize_kernel<float><<<grid, warps * 32, 0, st>>>(
