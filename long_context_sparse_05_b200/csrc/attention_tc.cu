@@ -506,6 +506,11 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
       // ---------------------------------------------------------------- MMA issuer
       constexpr uint32_t idS = tc::instr_desc(128, kH, 1, 1, 0, 0);   // bf16 K-major x K-major
       constexpr uint32_t idO = tc::instr_desc(128, kH, 1, 1, 1, 1);   // bf16 MN-major x MN-major
+      // base descriptors; each MMA's operands are a constant byte offset from them
+      const uint64_t dS_a = tc::smem_desc_sw128(tc::smem_u32(sKV), 16, 1024);
+      const uint64_t dS_b = tc::smem_desc_sw128(tc::smem_u32(sQ), 16, 1024);
+      const uint64_t dO_a = tc::smem_desc_sw128(tc::smem_u32(sKV), kKVBlkBytes, 1024);
+      const uint64_t dO_b = tc::smem_desc_sw128(tc::smem_u32(sP), 8192, 1024);
       for (int j = jb; j < je; ++j) {
         // S^T by column-block pairs (dims 128 mb ..): the item's first tile (and q) arrives
         // whole, every later tile pair by pair as the previous tile's PV frees the pairs
@@ -514,11 +519,12 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
           else if (mb == 0) tc::named_bar(1, kThreadsA);
           if (lane == 0) {
             tc::tc_fence_after();
+#pragma unroll
             for (int kb = 2 * mb; kb < 2 * mb + 2; ++kb) {
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = tc::smem_desc_sw128(tc::smem_u32(sKV + kb * kKVBlkBytes + kk * 32), 16, 1024);
-                const uint64_t b = tc::smem_desc_sw128(tc::smem_u32(sQ + kb * kQBlkBytes + kk * 32), 16, 1024);
+                const uint64_t a = tc::desc_advance(dS_a, kb * kKVBlkBytes + kk * 32);
+                const uint64_t b = tc::desc_advance(dS_b, kb * kQBlkBytes + kk * 32);
                 tc::mma_f16(tS, a, b, idS, (kb | kk) != 0);
               }
             }
@@ -529,12 +535,12 @@ __global__ void __launch_bounds__(kThreadsA, 1) attn_tc_kernel(AttnTc p) {
         tc::named_bar(2, kThreadsA);                 // P^T in shared memory, O rescaled
         if (lane == 0) {
           tc::tc_fence_after();
+#pragma unroll
           for (int mb = 0; mb < 4; ++mb) {
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t a = tc::smem_desc_sw128(
-                  tc::smem_u32(sKV + 2 * mb * kKVBlkBytes + kk * 2048), kKVBlkBytes, 1024);
-              const uint64_t b = tc::smem_desc_sw128(tc::smem_u32(sP + kk * 2048), 8192, 1024);
+              const uint64_t a = tc::desc_advance(dO_a, 2 * mb * kKVBlkBytes + kk * 2048);
+              const uint64_t b = tc::desc_advance(dO_b, kk * 2048);
               tc::mma_f16(tO + mb * kH, a, b, idO, (j > jb) || (kk > 0));
             }
             // every MMA so far is tracked: KV column blocks 2 mb, 2 mb + 1 are free once it fires

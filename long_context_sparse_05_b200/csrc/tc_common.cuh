@@ -149,6 +149,14 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   return d;
 }
 
+// The descriptor of the same layout `bytes` (a multiple of 16) further on: the start
+// address field holds address / 16 in 14 bits and shared addresses stay below 2^18, so
+// the field never carries into the next one and one 32-bit add of the low word suffices.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)d + (bytes >> 4);
+  return ((d >> 32) << 32) | lo;
+}
+
 // kind::f16 / kind::f8f6f4 instruction descriptor; D = f32.
 // fmt codes: kind::f16 -> 0 f16, 1 bf16; kind::f8f6f4 -> 0 e4m3, 1 e5m2, 5 e2m1.
 __host__ __device__ constexpr uint32_t instr_desc(int M, int N, int a_fmt, int b_fmt, int a_mn,
