@@ -154,7 +154,7 @@ def aggregate(ms_local, tokens_local, world):
     return ms, tokens, tokens / (ms * 1e-3)
 
 
-HOST_LEAD_CYCLES = 400_000   # device spin per timed step before the loop (~0.2 ms at 1.9 GHz)
+HOST_LEAD_CYCLES = 100_000   # device spin per timed step before the loop (~50 us at 1.9 GHz)
 
 
 def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
@@ -173,7 +173,7 @@ def timed_loop(fn, steps, flush_buf, stream, warm=0, nvtx=None):
         torch.cuda.synchronize()
         if nvtx:
             torch.cuda.nvtx.range_push(nvtx)
-        # the device first spins for ~0.2 ms per step (outside every event pair), so that the
+        # the device first spins for ~50 us per step (outside every event pair), so that the
         # host has queued each call before its start event fires: the events then time the
         # device work, not the host's Python and ctypes overhead per call
         torch.cuda._sleep(int(steps * HOST_LEAD_CYCLES))
@@ -194,6 +194,8 @@ def timed_region(fn, steps, flush, stream, world, min_span_s, max_repeats=4000):
     (its wall time is maxed over the ranks, so every rank repeats equally often).
     Returns (mean ms per step of each repeat, host time at start, at end)."""
     barrier(world)
+    torch.cuda.synchronize()
+    timed_loop(fn, steps, flush, stream)   # one-time costs of the loop itself (events, first calls)
     torch.cuda.synchronize()
     c0 = time.time()
     timed_loop(fn, steps, flush, stream)
@@ -217,11 +219,14 @@ def timed_region(fn, steps, flush, stream, world, min_span_s, max_repeats=4000):
 #   FP8 indexer: per key entry (ncu_full_index_scores_tc_csa_decode_64k_b4.md: batch 4,
 #     16384 entries per sequence); NVFP4 indexer: per key entry
 #     (ncu_full_index_scores_fp4_ctx256k_b2.md: batch 2, 65536 entries per sequence);
+#   decode attention of the 64K workload: per query (ncu_full_attn_tc_csa_decode_64k_b4.md:
+#     batch 4, 640 rows per query).
 # The traffic is linear in those units.  A kernel changed after its capture has no entry
 # here (its traffic is then reported as null).
 PROFILED_TRAFFIC = {
     ("index_scores", "fp8"): ("entries", 8773376 / (4 * 16384)),
     ("index_scores", "nvfp4"): ("entries", 9498368 / (2 * 65536)),
+    ("sparse_attn", "csa_decode_64k_fp8"): ("queries", 3032576 / 4),
 }
 
 

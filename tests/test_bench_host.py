@@ -35,14 +35,16 @@ def test_profiled_traffic_per_entry_is_close_to_the_algorithmic_bytes():
 
 def test_profiled_attention_traffic_is_per_query_and_near_the_rows_read():
     # 64K decode attention: 640 rows of 1 KiB and the 64 KiB query heads per query (the
-    # output's writes stay in L2 in the capture)
+    # output's writes stay in L2 in the capture), plus a few percent: the query's selection
+    # list, and the lines of the merge records (written to L2 just before the cluster
+    # barrier) that the cold-cache capture reads back from DRAM
     w = workloads.CSA_DECODE_64K
     if ("sparse_attn", w.name) not in bench.PROFILED_TRAFFIC:
         pytest.skip("no capture of the current attention kernel")
     unit, per = bench.PROFILED_TRAFFIC[("sparse_attn", w.name)]
     assert unit == "queries"
     alg = 640 * 1024 + 64 * 1024
-    assert 0.97 * alg <= per <= 1.05 * alg
+    assert 0.97 * alg <= per <= 1.08 * alg
     assert bench.profiled_traffic(w, "sparse_attn") == round(per * w.b)
     assert abs(bench.profiled_traffic(workloads.shrink(w, b=4), "sparse_attn") - 4 * per) <= 1
 
