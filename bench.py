@@ -787,6 +787,108 @@ def bench_out_proj(args, peaks, world):
     return res
 
 
+def bench_csa2(args, peaks, world, w):
+    """CSA2 decode modes at a CSA decode workload, each a whole csa_decode call timed with
+    events (L2 flushed before each): Full (indexer over every entry, top-k), Reuse (an
+    earlier layer's selection: no indexer, no top-k) and Reindex (the indexer and top-k over
+    a candidate pool of P = 2k entries per sequence, the earlier layer's top-P)."""
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    inp = synth.make_inputs(w, device="cuda")
+    st = runner.DecodeState(w, inp)
+    st.build_caches(stream)
+    st.step(stream)                                   # layer 1: its selection and caches
+    torch.cuda.synchronize()
+    idx1, cnt1 = st.idx.clone(), st.count.clone()
+    E, P = w.E, 2 * w.k
+    # layer 1's top-P of its own scores: the Reindex pool
+    ip = L.IndexParams(H_I=w.H_I, d_I=w.c_I, m=w.m, qk_dtype=L.DTYPE[w.idx_dtype],
+                       score_dtype=L.CSA_BF16)
+    codes = torch.empty((w.b * w.H_I, runner.row_bytes(w.idx_dtype, w.c_I)), dtype=torch.uint8,
+                        device="cuda")
+    qs = (torch.empty((w.b * w.H_I,), dtype=torch.float32, device="cuda") if w.idx_dtype == "fp8"
+          else torch.empty((w.b * w.H_I, w.c_I // 16), dtype=torch.uint8, device="cuda"))
+    L.csa_quantize(L.DTYPE[w.dtype], L.DTYPE[w.idx_dtype], inp["q_I"], w.b * w.H_I, w.c_I, codes,
+                   qs, stream)
+    qpos = torch.full((w.b, 1), w.n - 1, dtype=torch.int32, device="cuda")
+    sc1 = torch.empty((w.b, 1, E), dtype=torch.bfloat16, device="cuda")
+    L.csa_index_scores(ip, codes, qs, inp["w"], st.kI_cache, st.kI_scales, qpos, w.b, 1, st.E_cap,
+                       E, sc1, stream)
+    pool = torch.empty((w.b, 1, P), dtype=torch.int32, device="cuda")
+    pcnt = torch.empty((w.b, 1), dtype=torch.int32, device="cuda")
+    tkb = L.csa_topk_workspace_size(L.CSA_BF16, w.b, 1, E, P)
+    tkws = torch.empty((max(tkb, 256),), dtype=torch.uint8, device="cuda")
+    L.csa_topk(sc1, L.CSA_BF16, qpos, w.m, w.b, 1, E, P, pool, pcnt, tkws, tkb, stream)
+    res = {}
+    for label, mode in (("full", L.CSA_MODE_FULL), ("reuse", L.CSA_MODE_REUSE),
+                        ("reindex", L.CSA_MODE_REINDEX)):
+        p = runner.decode_params(w, st.E_cap)
+        p.mode, p.P = mode, (P if mode == L.CSA_MODE_REINDEX else 0)
+        t = st.tensors()
+        t["out"] = torch.empty_like(st.out)
+        t["idx_out"] = torch.empty((w.b, w.k), dtype=torch.int32, device="cuda")
+        t["count_out"] = torch.empty((w.b,), dtype=torch.int32, device="cuda")
+        if mode == L.CSA_MODE_REUSE:
+            t["idx_in"], t["count_in"] = idx1, cnt1
+        if mode == L.CSA_MODE_REINDEX:
+            t["pool"], t["pool_count"] = pool.reshape(w.b, P), pcnt.reshape(w.b)
+        wsb = L.csa_decode_workspace_size(p)
+        ws = torch.empty((max(wsb, 256),), dtype=torch.uint8, device="cuda")
+        fn = lambda: L.csa_decode(p, t, ws, wsb, stream)  # noqa: E731
+        us = float(np.median(timed_loop(fn, max(5, min(args.steps, 20)), flush, stream, warm=3))) * 1e3
+        res[label] = {"us_per_step": round(us, 2), "tok_s": round(w.b / (us * 1e-6), 1),
+                      "launches": L.csa_decode_launch_count(p)}
+        del ws
+    if L.csa_device_error():
+        raise RuntimeError("device error word set during the CSA2 measurement")
+    del st, inp, flush
+    torch.cuda.empty_cache()
+    res["config"] = {"workload": w.name, "batch": w.b, "context": w.n, "top_k": w.k, "pool": P}
+    return res
+
+
+def bench_cp(args, peaks, world, G=8):
+    """One rank's share of a context-parallel 1M CSA decode over G ranks (1M workload, the
+    entries of every sequence split into G shards), timed on this GPU phase by phase with
+    events (L2 flushed before each): the local phase (compress the new entry on the rank that
+    holds it, quantise, score the shard, its top-k, candidates), the merge of the gathered
+    candidates and the packing of the rows this rank holds, and the attention over the k
+    gathered rows and the window.  The two collectives between them move the bytes given in
+    `exchange_bytes` (all-gather of the candidates, all-reduce of the packed rows); one GPU
+    does not measure them."""
+    from long_context_sparse_05_b200 import cp as cpmod
+    w = workloads.CSA_DECODE_1M
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    inp = synth.make_inputs(w, device="cuda")
+    full = runner.DecodeState(w, inp)
+    full.build_caches(stream)
+    torch.cuda.synchronize()
+    shard = cpmod.CPShard(w, inp, G - 1, G, full)     # the rank that completes the new entry
+    del full
+    torch.cuda.empty_cache()
+    shard.phase_local(stream)
+    for r in range(G):                                # every rank's candidates: this rank's
+        shard.gath_s[r].copy_(shard.cand_s)
+        shard.gath_i[r].copy_(shard.cand_i)
+    steps = max(5, min(args.steps, 20))
+    res = {}
+    for label, fn in (("local", lambda: shard.phase_local(stream)),
+                      ("merge_pack", lambda: shard.phase_merge(stream)),
+                      ("attend", lambda: shard.phase_attend(stream))):
+        res[label + "_us"] = round(float(np.median(timed_loop(fn, steps, flush, stream, warm=3))) * 1e3, 2)
+    if L.csa_device_error():
+        raise RuntimeError("device error word set during the context-parallel measurement")
+    res["rank_us_without_collectives"] = round(res["local_us"] + res["merge_pack_us"] + res["attend_us"], 2)
+    res["exchange_bytes"] = {"all_gather_candidates": G * w.b * w.k * (2 + 4),
+                             "all_reduce_rows": w.b * w.k * w.c * 2}
+    res["config"] = {"workload": w.name, "ranks": G, "rank": G - 1, "shard_entries": shard.n_local,
+                     "batch": w.b, "context": w.n, "top_k": w.k}
+    del shard, inp, flush
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_workload(w, args, world, rank, peaks, min_span_s, cpu_budget_s):
     """One workload's record: throughput, rooflines, per-kernel fractions, clocks, e2e and (rank
     0 of a single-GPU run) the oracle's rate on this host."""
@@ -863,6 +965,9 @@ def main():
         for w2 in SUB_WORKLOADS:
             subs[w2.name] = run_workload(w2, args, world, rank, peaks, 0.5, 10.0)
         subs["grouped_out_proj"] = bench_out_proj(args, peaks, world)
+        subs["csa2_modes_64k"] = bench_csa2(args, peaks, world, workloads.CSA_DECODE_64K)
+        subs["csa2_modes_1m"] = bench_csa2(args, peaks, world, workloads.CSA_DECODE_1M)
+        subs["context_parallel_1m_rank"] = bench_cp(args, peaks, world)
     if rank == 0:
         line = {"metric": METRIC, "value": head["value"], "unit": "tok/s", "n_gpus": world,
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": head["ms_per_step"],

@@ -8,12 +8,13 @@
 // The pool of every query row is gathered into a key set of its own, so that the
 // tensor-core indexer scores it unchanged (one "sequence" of P entries per query
 // row, one query each) and the top-k selects positions in it:
-//   pool_gather_kernel  CTA per query row: compacts the pool entries visible to the
-//                       row's position (a block scan keeps their order), copies their
-//                       index-key rows and scales (FP8: one float per row; NVFP4: the
-//                       tiled key-scale layout, re-tiled for the new positions), zeroes
-//                       the rest of the last 256-entry stage, and writes the position
-//                       m * count - 1 whose causal range is exactly the compacted pool;
+//   pool_gather_kernel  CTA per (query row, 256 pool slots): compacts the pool entries
+//                       visible to the row's position (counts and a block scan keep their
+//                       order), copies their index-key rows and scales (FP8: one float per
+//                       row; NVFP4: the tiled key-scale layout, re-tiled for the new
+//                       positions), zeroes the rest of the last 256-entry stage, and writes
+//                       the position m * count - 1 whose causal range is exactly the
+//                       compacted pool;
 //   pool_map_kernel     replaces each selected position by the entry it holds
 //                       (ascending positions of an ascending pool are ascending entries).
 #include "common.cuh"
@@ -57,73 +58,104 @@ struct PoolArgs {
   int T, P, P_cap, E_cap, E, m, row_bytes, d, fmt;   // fmt: CSA_F32, CSA_FP8_E4M3 or CSA_NVFP4
 };
 
+// Sums of a and b over the CTA (every thread gets both).
+__device__ __forceinline__ void block_sum2_i(int& a, int& b, int* s_warp) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  a = __reduce_add_sync(0xffffffffu, a);
+  b = __reduce_add_sync(0xffffffffu, b);
+  __syncthreads();
+  if (lane == 0) { s_warp[wid] = a; s_warp[16 + wid] = b; }
+  __syncthreads();
+  a = 0; b = 0;
+  for (int w = 0; w < nw; ++w) { a += s_warp[w]; b += s_warp[16 + w]; }
+  __syncthreads();
+}
+
+// CTA (query row r, chunk c of kGatherThreads pool slots), one slot per thread.  The
+// entries the row sees keep their order: an entry's compacted position is the count of
+// kept entries before its chunk (every CTA counts them itself, in one coalesced pass over
+// the pool) plus its rank among its chunk's kept entries.  Each thread then copies its
+// entry's key row and scales, and zeroes position j0 + tid if that lies between the
+// compacted count and the end of its 256-entry stage; chunk 0 writes the position
+// m * count - 1 whose causal range is exactly the compacted pool.
 __global__ void __launch_bounds__(kGatherThreads) pool_gather_kernel(PoolArgs a) {
   __shared__ int s_warp[32];
-  __shared__ int s_base;
   pdl_launch_dependents();
   pdl_wait();   // the pool, the positions and the newest key may come from preceding kernels
   const int r = blockIdx.x;
+  const int j0 = blockIdx.y * kGatherThreads;
   const int sb = r / a.T;
   const int ev = visible_entries(a.q_pos[r], a.m, a.E);
   const int pc = min(a.pool_count[r], a.P);
   const int32_t* pl = a.pool + (size_t)r * a.P;
-  int32_t* gp = a.gpool + (size_t)r * a.P;
-  if (threadIdx.x == 0) s_base = 0;
-  __syncthreads();
-  for (int j0 = 0; j0 < pc; j0 += kGatherThreads) {
-    const int j = j0 + threadIdx.x;
-    const int e = j < pc ? pl[j] : -1;
+  int before = 0, cnt = 0;
+  for (int j = threadIdx.x; j < pc; j += kGatherThreads) {
+    const int e = pl[j];
     const int keep = (e >= 0 && e < ev) ? 1 : 0;
-    int tot;
-    const int off = block_excl_scan_i(keep, s_warp, tot);
-    if (keep) gp[s_base + off] = e;
-    __syncthreads();
-    if (threadIdx.x == 0) s_base += tot;
-    __syncthreads();
+    cnt += keep;
+    before += j < j0 ? keep : 0;
   }
-  const int cnt = s_base;
-  if (threadIdx.x == 0) a.gpos[r] = a.m * cnt - 1;
-  // key rows of the compacted pool, 16 bytes at a time; the rest of the last stage zeroed
-  const int cpr = a.row_bytes / 16;
+  block_sum2_i(before, cnt, s_warp);
+  const int j = j0 + threadIdx.x;
+  const int e = j < pc ? pl[j] : -1;
+  const int keep = (e >= 0 && e < ev) ? 1 : 0;
+  int tot;
+  const int pos = before + block_excl_scan_i(keep, s_warp, tot);
+  if (blockIdx.y == 0 && threadIdx.x == 0) a.gpos[r] = a.m * cnt - 1;
+  const int rb = a.row_bytes, cpr = rb / 16;
+  const uint8_t* kseq = a.k + (size_t)sb * a.E_cap * rb;
+  uint8_t* gkr = a.gk + (size_t)r * a.P_cap * rb;
   const int zend = min(a.P_cap, (cnt + 255) / 256 * 256);
-  const uint8_t* kseq = a.k + (size_t)sb * a.E_cap * a.row_bytes;
-  uint8_t* gkr = a.gk + (size_t)r * a.P_cap * a.row_bytes;
-  for (int x = threadIdx.x; x < zend * cpr; x += kGatherThreads) {
-    const int j = x / cpr, c = x % cpr;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (j < cnt) v = *reinterpret_cast<const uint4*>(kseq + (size_t)gp[j] * a.row_bytes + c * 16);
-    *reinterpret_cast<uint4*>(gkr + (size_t)j * a.row_bytes + c * 16) = v;
+  const bool zero = j >= cnt && j < zend;       // slot j of the compacted pool is padding
+  if (keep) {
+    a.gpool[(size_t)r * a.P + pos] = e;
+    const uint4* src = reinterpret_cast<const uint4*>(kseq + (size_t)e * rb);
+    uint4* dst = reinterpret_cast<uint4*>(gkr + (size_t)pos * rb);
+    for (int x0 = 0; x0 < cpr; x0 += 8) {       // up to eight 16-byte loads in flight
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (x0 + u < cpr) v[u] = __ldg(src + x0 + u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (x0 + u < cpr) dst[x0 + u] = v[u];
+    }
   }
-  if (a.fmt == CSA_F32) {
-    // no scales: the rows are the values
-  } else if (a.fmt == CSA_FP8_E4M3) {
+  if (zero) {
+    uint4* dst = reinterpret_cast<uint4*>(gkr + (size_t)j * rb);
+    for (int x = 0; x < cpr; ++x) dst[x] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (a.fmt == CSA_FP8_E4M3) {
     const float* ks = static_cast<const float*>(a.k_scales) + (size_t)sb * a.E_cap;
     float* g = static_cast<float*>(a.gks) + (size_t)r * a.P_cap;
-    for (int j = threadIdx.x; j < zend; j += kGatherThreads) g[j] = j < cnt ? ks[gp[j]] : 0.f;
-  } else {
+    if (keep) g[pos] = ks[e];
+    if (zero) g[j] = 0.f;
+  } else if (a.fmt == CSA_NVFP4) {
     const int nb = a.d / 16;
     const uint8_t* ks = static_cast<const uint8_t*>(a.k_scales) +
                         (size_t)sb * nvfp4_key_scale_seq_bytes(a.E_cap, a.d);
     uint8_t* g = static_cast<uint8_t*>(a.gks) + (size_t)r * nvfp4_key_scale_seq_bytes(a.P_cap, a.d);
-    for (int x = threadIdx.x; x < zend * nb; x += kGatherThreads) {
-      const int j = x / nb, blk = x % nb;
-      g[nvfp4_key_scale_offset(j, blk, a.d)] =
-          j < cnt ? ks[nvfp4_key_scale_offset(gp[j], blk, a.d)] : (uint8_t)0;
+    for (int blk = 0; blk < nb; ++blk) {
+      if (keep) g[nvfp4_key_scale_offset(pos, blk, a.d)] = ks[nvfp4_key_scale_offset(e, blk, a.d)];
+      if (zero) g[nvfp4_key_scale_offset(j, blk, a.d)] = 0;
     }
   }
 }
 
-__global__ void pool_map_kernel(const int32_t* gpool, int P, int k, int32_t* idx,
-                                const int32_t* count) {
+// CTA (query row, chunk of kGatherThreads selection slots): each slot's position in the
+// compacted pool is replaced by the entry it holds.
+__global__ void __launch_bounds__(kGatherThreads) pool_map_kernel(const int32_t* gpool, int P,
+                                                                  int k, int32_t* idx,
+                                                                  const int32_t* count) {
   pdl_launch_dependents();
   pdl_wait();
   const int r = blockIdx.x;
+  const int j = blockIdx.y * kGatherThreads + threadIdx.x;
+  if (j >= k) return;
   const int c = count[r];
   int32_t* o = idx + (size_t)r * k;
-  for (int j = threadIdx.x; j < k; j += blockDim.x) {
-    const int pos = o[j];
-    o[j] = (j < c && pos >= 0 && pos < P) ? gpool[(size_t)r * P + pos] : -1;
-  }
+  const int pos = o[j];
+  o[j] = (j < c && pos >= 0 && pos < P) ? gpool[(size_t)r * P + pos] : -1;
 }
 
 }  // namespace
@@ -164,8 +196,8 @@ csa_status launch_pool_gather(int fmt, const int32_t* pool, const int32_t* pool_
   a.gpos = reinterpret_cast<int32_t*>(w + o_ps);
   a.T = T; a.P = P; a.P_cap = (P + 255) / 256 * 256; a.E_cap = E_cap; a.E = E; a.m = m;
   a.row_bytes = pool_row_bytes(fmt, d); a.d = d; a.fmt = fmt;
-  if (csa_launch(pool_gather_kernel, dim3(rows), dim3(kGatherThreads), 0, st, pdl, a) !=
-      cudaSuccess)
+  if (csa_launch(pool_gather_kernel, dim3(rows, a.P_cap / kGatherThreads), dim3(kGatherThreads), 0,
+                 st, pdl, a) != cudaSuccess)
     return CSA_ERR_CUDA;
   return CSA_OK;
 }
@@ -176,8 +208,8 @@ csa_status launch_pool_map(const void* ws, int fmt, int rows, int P, int d, int 
   size_t o_pl;
   pool_gather_bytes(fmt, rows, P, d, nullptr, &o_pl, nullptr);
   const int32_t* gpool = reinterpret_cast<const int32_t*>(static_cast<const uint8_t*>(ws) + o_pl);
-  if (csa_launch(pool_map_kernel, dim3(rows), dim3(128), 0, st, pdl, gpool, P, k, idx, count) !=
-      cudaSuccess)
+  if (csa_launch(pool_map_kernel, dim3(rows, (k + kGatherThreads - 1) / kGatherThreads),
+                 dim3(kGatherThreads), 0, st, pdl, gpool, P, k, idx, count) != cudaSuccess)
     return CSA_ERR_CUDA;
   return CSA_OK;
 }
