@@ -331,10 +331,10 @@ size_t csa_sparse_attn_workspace_size(const csa_attn_params* p, int b, int T, in
  * method on the pages has no counterpart of this; it only changes where the
  * scratch lives.
  *
- *  - The first call on a device (with that device current) looks up the
- *    array's device address and keeps it for the process; make that first call
- *    before any stream capture.  The address is not looked up again, so do not
- *    use this entry point on a device after cudaDeviceReset there.
+ *  - Every call looks up the array's device address in the current device's
+ *    context (a runtime query, no allocation), so a context recreated after
+ *    cudaDeviceReset is served too.  The first call on a device may load the
+ *    library's module there: make it before any stream capture.
  *  - A problem whose workspace (csa_sparse_attn_workspace_size) exceeds
  *    CSA_NOALLOC_SCRATCH_BYTES is rejected with CSA_ERR_INVALID_ARG and
  *    nothing is launched.

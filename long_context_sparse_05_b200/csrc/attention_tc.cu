@@ -43,7 +43,6 @@
 
 #include <climits>
 #include <cmath>
-#include <mutex>
 
 namespace csa {
 
@@ -1076,24 +1075,13 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[CSA_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device.  In host code the
-// array's name is only a host-side stand-in, so the address must come from the
-// runtime; it is looked up once per device.
+// Device address of the scratch array in the current device's context.  In host code the
+// array's name is only a host-side stand-in, so the address comes from the runtime, on
+// every call: a context recreated after a device reset places the array anew.
 csa_status noalloc_scratch(void** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return CSA_ERR_CUDA;
-  if (dev < 0 || dev >= kMaxDevices) return CSA_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* ptr = nullptr;
-    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return CSA_ERR_CUDA;
-    g_noalloc_ptr[dev] = ptr;
-  }
-  *out = g_noalloc_ptr[dev];
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return CSA_ERR_CUDA;
+  *out = ptr;
   return CSA_OK;
 }
 

@@ -178,3 +178,11 @@ def test_product_path_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(L, "LIB_PATH", "/nonexistent/libcsa.so")
     with pytest.raises(L.CsaError):
         L.lib()
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    # the binding's copy of the no-alloc scratch size is the header's CSA_NOALLOC_SCRATCH_BYTES
+    hdr = open(HEADER).read()
+    m = re.search(r"#define CSA_NOALLOC_SCRATCH_BYTES \(\(size_t\)(\d+) << (\d+)\)", hdr)
+    assert m, "CSA_NOALLOC_SCRATCH_BYTES not found in csa.h"
+    assert int(m.group(1)) << int(m.group(2)) == L.NOALLOC_SCRATCH_BYTES
