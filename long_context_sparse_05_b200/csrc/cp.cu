@@ -17,6 +17,8 @@
 //                         gathered rows;
 //   cp_pack_kernel        the selected rows this rank holds into their selection slots
 //                         (zeros elsewhere), so that a sum over the ranks gathers them.
+// Each is launched as a programmatic dependent of the kernel before it on the stream and
+// waits for that kernel before it reads anything.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -30,6 +32,8 @@ __global__ void __launch_bounds__(kCpThreads) cp_candidates_kernel(
     const __nv_bfloat16* __restrict__ scores, int E_local, const int32_t* __restrict__ idx,
     const int32_t* __restrict__ count, int k, int offset, __nv_bfloat16* __restrict__ cand_s,
     int32_t* __restrict__ cand_i) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int q = blockIdx.x;
   const int n = count[q];
   for (int j = threadIdx.x; j < k; j += blockDim.x) {
@@ -44,6 +48,8 @@ __global__ void __launch_bounds__(kCpThreads) cp_candidates_kernel(
 __global__ void __launch_bounds__(kCpThreads) cp_permute_kernel(
     const __nv_bfloat16* __restrict__ cand_s, const int32_t* __restrict__ cand_i, int G, int b,
     int k, __nv_bfloat16* __restrict__ row_s, int32_t* __restrict__ row_i, int32_t* __restrict__ pos) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int q = blockIdx.x;
   const int n = G * k;
   for (int x = threadIdx.x; x < n; x += blockDim.x) {
@@ -86,6 +92,8 @@ __global__ void __launch_bounds__(kCpThreads) cp_map_kernel(
     const int32_t* __restrict__ row_i, int n, int k, int32_t* __restrict__ idx,
     int32_t* __restrict__ count, int32_t* __restrict__ rows_idx) {
   __shared__ int s_warp[32];
+  pdl_launch_dependents();
+  pdl_wait();
   const int q = blockIdx.x;
   const int ns = sel_cnt[q];
   int base = 0;
@@ -112,6 +120,8 @@ __global__ void __launch_bounds__(kCpThreads) cp_pack_kernel(
     const uint8_t* __restrict__ kv, int E_cap_local, int E_local, int offset, size_t row_bytes,
     const int32_t* __restrict__ idx, const int32_t* __restrict__ count, int k,
     uint8_t* __restrict__ rows) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int q = blockIdx.y;
   const int warps = blockDim.x >> 5, lane = threadIdx.x & 31;
   const int j = blockIdx.x * warps + (threadIdx.x >> 5);
@@ -130,10 +140,10 @@ __global__ void __launch_bounds__(kCpThreads) cp_pack_kernel(
 csa_status launch_cp_candidates(const void* scores, int E_local, const int32_t* idx,
                                 const int32_t* count, int b, int k, int offset, void* cand_s,
                                 int32_t* cand_i, cudaStream_t st) {
-  cp_candidates_kernel<<<b, kCpThreads, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(scores),
-                                                 E_local, idx, count, k, offset,
-                                                 static_cast<__nv_bfloat16*>(cand_s), cand_i);
-  CSA_CHECK_LAUNCH();
+  if (csa_launch(cp_candidates_kernel, dim3(b), dim3(kCpThreads), 0, st, true,
+                 reinterpret_cast<const __nv_bfloat16*>(scores), E_local, idx, count, k, offset,
+                 static_cast<__nv_bfloat16*>(cand_s), cand_i) != cudaSuccess)
+    return CSA_ERR_CUDA;
   return CSA_OK;
 }
 
@@ -158,15 +168,17 @@ csa_status launch_cp_merge(const void* cand_s, const int32_t* cand_i, int G, int
   auto* sel = reinterpret_cast<int32_t*>(p);              p += al((size_t)b * k * 4);
   auto* sel_cnt = reinterpret_cast<int32_t*>(p);          p += al((size_t)b * 4);
   void* tws = topk_ws ? p : nullptr;
-  cp_permute_kernel<<<b, kCpThreads, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(cand_s), cand_i,
-                                              G, b, k, row_s, row_i, pos);
-  CSA_CHECK_LAUNCH();
+  if (csa_launch(cp_permute_kernel, dim3(b), dim3(kCpThreads), 0, st, true,
+                 reinterpret_cast<const __nv_bfloat16*>(cand_s), cand_i, G, b, k, row_s, row_i,
+                 pos) != cudaSuccess)
+    return CSA_ERR_CUDA;
   csa_status r = launch_topk_search(row_s, CSA_BF16, pos, 1, b, n, k, sel, sel_cnt, tws, topk_ws, st,
-                                    false);
+                                    true);
   if (r == CSA_ERR_UNSUPPORTED) r = launch_topk(row_s, CSA_BF16, pos, 1, b, n, k, sel, sel_cnt, st);
   if (r) return r;
-  cp_map_kernel<<<b, kCpThreads, 0, st>>>(sel, sel_cnt, row_i, n, k, idx, count, rows_idx);
-  CSA_CHECK_LAUNCH();
+  if (csa_launch(cp_map_kernel, dim3(b), dim3(kCpThreads), 0, st, true, sel, sel_cnt, row_i, n, k,
+                 idx, count, rows_idx) != cudaSuccess)
+    return CSA_ERR_CUDA;
   return CSA_OK;
 }
 
@@ -175,10 +187,10 @@ csa_status launch_cp_pack(const void* kv, int E_cap_local, int E_local, int offs
                           cudaStream_t st) {
   const int warps = kCpThreads / 32;
   dim3 grid((k + warps - 1) / warps, b);
-  cp_pack_kernel<<<grid, kCpThreads, 0, st>>>(static_cast<const uint8_t*>(kv), E_cap_local, E_local,
-                                              offset, row_bytes, idx, count, k,
-                                              static_cast<uint8_t*>(rows));
-  CSA_CHECK_LAUNCH();
+  if (csa_launch(cp_pack_kernel, grid, dim3(kCpThreads), 0, st, true,
+                 static_cast<const uint8_t*>(kv), E_cap_local, E_local, offset, row_bytes, idx, count,
+                 k, static_cast<uint8_t*>(rows)) != cudaSuccess)
+    return CSA_ERR_CUDA;
   return CSA_OK;
 }
 
