@@ -408,7 +408,8 @@ __device__ __forceinline__ void cluster_merge(const AttnTc& p, int qrow, int ite
 // Workspace merge (dense decode with more splits than a cluster holds): CTA per
 // (query, slice of 16 dims).
 constexpr int kMergeDims = 16;
-__global__ void __launch_bounds__(128) attn_merge_kernel(AttnTc p) {
+constexpr int kMergeThreads = 256;
+__global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(AttnTc p) {
   extern __shared__ __align__(16) float mm_smem[];
   const int cap = p.nsplit;                               // shared memory sized for it
   float* s_ml = mm_smem;                                  // [2][cap][kH]
@@ -1034,7 +1035,7 @@ csa_status launch_attn_tc(const AttnArgs& a, int b, int dtype, void* ws, size_t 
       if (cudaFuncSetAttribute(attn_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                (int)msm) != cudaSuccess)
         return CSA_ERR_CUDA;
-      if (csa_launch(attn_merge_kernel, dim3(b * a.T, kD / kMergeDims), dim3(128), msm, st,
+      if (csa_launch(attn_merge_kernel, dim3(b * a.T, kD / kMergeDims), dim3(kMergeThreads), msm, st,
                      a.pdl != 0, p) != cudaSuccess)
         return CSA_ERR_CUDA;
     }
