@@ -59,24 +59,6 @@ __device__ __forceinline__ float warp_max(float v) {
 }
 
 // Block-wide sum / max; every thread gets the result.  `red` needs blockDim/32 floats.
-// FP8 E4M3 quantisation of one row of 128 elements held by a warp, four per lane (lane l:
-// elements 4l .. 4l+3): scale = amax / 448 over the row, code = e4m3(x / scale) (round to
-// nearest even, saturating); a zero row has scale 0 and zero codes.  Returns the lane's
-// four codes packed little-endian; every lane gets the scale.
-__device__ __forceinline__ uint32_t fp8_quant_row128(const float (&v)[4], float* scale) {
-  float am = 0.f;
-#pragma unroll
-  for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(v[e]));
-  am = warp_max(am);
-  const float sc = am / 448.f;
-  uint32_t packed = 0;
-#pragma unroll
-  for (int e = 0; e < 4; ++e)
-    packed |= (sc > 0.f ? (uint32_t)f32_to_e4m3(v[e] / sc) : 0u) << (8 * e);
-  *scale = sc;
-  return packed;
-}
-
 __device__ __forceinline__ float block_sum(float v, float* red) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = blockDim.x >> 5;
   v = warp_sum(v);
