@@ -79,8 +79,3 @@ def make_inputs(w, device="cpu", T=None, b=None):
     d["q"] = draw("q", (b, T, w.H, w.c), w.seed, device, dt)
     d["sink"] = draw("sink", (w.H,), w.seed, device, "f32")
     return d
-
-
-def to_f64(x):
-    """A torch tensor (any device) as a float64 numpy array, for the oracle."""
-    return x.detach().to("cpu", torch.float64).numpy()
